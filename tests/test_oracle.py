@@ -1,0 +1,402 @@
+"""Pins for the CPU oracle (CPU only, no GPU, no CUDA library).
+
+Each test ties an oracle function to something other than the oracle itself:
+values the pages print (fixtures under tests/golden/, each citing its source),
+closed forms, independent library routines (stdlib/scipy quantiles, torch's
+float8 and bf16 casts), brute force on tiny inputs and finite differences.
+"""
+from __future__ import annotations
+
+import math
+import os
+import statistics
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import nf4_oracle as o
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden_lines(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return [ln.strip() for ln in f if ln.strip() and not ln.startswith("#")]
+
+
+def _golden_table(name):
+    out = {}
+    for ln in _golden_lines(name):
+        k, v, tol = ln.split()
+        out[k] = (float(v), float(tol))
+    return out
+
+
+# --------------------------------------------------------------------------
+# Codebook
+# --------------------------------------------------------------------------
+def test_codebook_matches_printed_digits():
+    codes, _ = o.nf4_codebook()
+    for ln in _golden_lines("nf4_printed_codes.txt"):
+        i, v = ln.split()
+        assert abs(float(codes[int(i)]) - float(v)) <= 5e-5, (i, codes[int(i)], v)
+
+
+def test_codebook_structure():
+    codes, mids = o.nf4_codebook()
+    assert codes.dtype == np.float32 and codes.shape == (16,)
+    assert np.all(np.diff(codes) > 0)
+    assert codes[7] == 0.0 and codes[0] == -1.0 and codes[15] == 1.0
+    # 8 levels on the negative side and 9 on the positive side, sharing zero
+    assert (codes < 0).sum() == 7 and (codes > 0).sum() == 8
+    assert mids.shape == (15,)
+    assert np.all(mids > codes[:-1]) and np.all(mids < codes[1:])
+
+
+@pytest.mark.parametrize("ppf", [statistics.NormalDist().inv_cdf,
+                                 pytest.importorskip("scipy.special").ndtri])
+def test_codebook_independent_quantile_routines(ppf):
+    ours = o.nf4_codebook()[0]
+    theirs = o.nf4_levels_fp64(ppf=lambda p: float(ppf(p))).astype(np.float32)
+    assert np.array_equal(ours.view(np.uint32), theirs.view(np.uint32))
+
+
+def test_norm_ppf_closed_forms():
+    assert o.norm_ppf(0.5) == pytest.approx(0.0, abs=1e-15)
+    # Phi(1.959963984540054) = 0.975 (textbook value)
+    assert o.norm_ppf(0.975) == pytest.approx(1.959963984540054, abs=1e-13)
+    assert o.norm_ppf(0.025) == pytest.approx(-1.959963984540054, abs=1e-13)
+
+
+def test_codebook_alternative_offsets_fail_printed_digits():
+    """The offset reading is pinned: the two single-sided offsets miss."""
+    printed = {int(a): float(b) for a, b in (ln.split() for ln in _golden_lines("nf4_printed_codes.txt"))}
+    for delta in (1 - 1 / 30, 1 - 1 / 32):
+        pos = [o.norm_ppf(delta - i * (delta - 0.5) / 8) for i in range(8)]
+        neg = [-o.norm_ppf(delta - j * (delta - 0.5) / 7) for j in range(7)]
+        lv = np.array(sorted(neg + [0.0] + pos)) / o.norm_ppf(delta)
+        assert max(abs(lv[i] - v) for i, v in printed.items()) > 5e-5
+
+
+def test_midpoints_are_rounded_exact_averages():
+    codes, mids = o.nf4_codebook()
+    for i in range(15):
+        exact = (float(codes[i]) + float(codes[i + 1])) / 2
+        m = float(mids[i])
+        below = float(np.nextafter(mids[i], np.float32(-2)))
+        above = float(np.nextafter(mids[i], np.float32(2)))
+        assert abs(m - exact) <= abs(below - exact) and abs(m - exact) <= abs(above - exact)
+
+
+# --------------------------------------------------------------------------
+# Blockwise quantisation
+# --------------------------------------------------------------------------
+def _worked():
+    d = {}
+    for ln in _golden_lines("worked_example_block8.txt"):
+        k, v = ln.split(":")
+        d[k] = [float(t) for t in v.split()]
+    return d
+
+
+def test_worked_example_block_of_eight():
+    d = _worked()
+    codes, mids = o.nf4_codebook()
+    w = np.array(d["weights"], dtype=np.float32)
+    c = o.block_absmax(w, block=8)
+    assert c.shape == (1,) and abs(c[0] - d["absmax"][0]) < 1e-7
+    x = o.normalise_blocks(w, c, block=8)
+    assert np.allclose(x, d["normalised"], atol=5e-4)
+    idx = o.nearest_code_index(x, mids)
+    assert idx.tolist() == [int(v) for v in d["indices"]]
+    rec = codes[idx] * c[0]
+    assert np.allclose(rec, d["reconstructed"], atol=5e-5)
+    assert np.allclose(np.abs(rec - w), d["abs_error"], atol=5e-5)
+    assert rec[3] == w[3]        # the absmax element is reconstructed exactly
+
+
+def test_nearest_index_agrees_with_brute_force():
+    rng = np.random.default_rng(1)
+    codes, mids = o.nf4_codebook()
+    x = rng.uniform(-1, 1, 20000).astype(np.float32)
+    x = np.concatenate([x, codes, -np.abs(codes)])
+    fast = o.nearest_code_index(x, mids)
+    brute = o.brute_nearest_index(x, codes)
+    on_mid = np.isin(x, mids)
+    assert np.array_equal(fast[~on_mid], brute[~on_mid])
+
+
+def test_tie_rule_goes_to_lower_code():
+    codes, mids = o.nf4_codebook()
+    for i, m in enumerate(mids):
+        assert o.nearest_code_index(np.array([m]), mids)[0] == i
+        up = np.nextafter(m, np.float32(2))
+        dn = np.nextafter(m, np.float32(-2))
+        assert o.nearest_code_index(np.array([up]), mids)[0] == i + 1
+        assert o.nearest_code_index(np.array([dn]), mids)[0] == i
+
+
+def test_roundtrip_of_exact_codes():
+    """Blocks made of codes times a power of two, each holding a +-1, quantise
+    back to the very indices they were built from."""
+    rng = np.random.default_rng(2)
+    codes, mids = o.nf4_codebook()
+    idx = rng.integers(0, 16, size=(40, 64)).astype(np.uint8)
+    idx[:, 5] = np.where(rng.random(40) < 0.5, 0, 15)
+    scale = (2.0 ** rng.integers(-20, 5, size=(40, 1))).astype(np.float32)
+    w = (codes[idx] * scale).astype(np.float32)
+    packed, _, _ = o.quantize(w)
+    got = o.unpack_nibbles(packed, w.size).reshape(40, 64)
+    assert np.array_equal(got, idx)
+
+
+def test_error_bound_half_local_gap():
+    rng = np.random.default_rng(3)
+    codes, mids = o.nf4_codebook()
+    w = rng.normal(0, 0.02, 64 * 500).astype(np.float32)
+    c = o.block_absmax(w)
+    x = o.normalise_blocks(w, c)
+    idx = o.nearest_code_index(x, mids)
+    q = codes[idx].astype(np.float64)
+    lo = codes[np.maximum(idx.astype(int) - 1, 0)]
+    hi = codes[np.minimum(idx.astype(int) + 1, 15)]
+    gap = np.maximum(q - lo, hi - q)
+    ulp = np.spacing(np.abs(x).astype(np.float32)).astype(np.float64)
+    assert np.all(np.abs(x - q) <= 0.5 * gap + ulp)
+    err = np.abs(w.astype(np.float64) - q * np.repeat(c, 64))
+    assert np.all(err <= (0.5 * gap + 2 * ulp) * np.repeat(c, 64))
+
+
+def test_pack_nibble_order_and_padding():
+    idx = np.array([1, 2, 3, 4, 15, 0, 9], dtype=np.uint8)
+    p = o.pack_nibbles(idx)
+    assert p.tolist() == [0x21, 0x43, 0x0F, 0x79]
+    assert o.unpack_nibbles(p, 7).tolist() == idx.tolist()
+
+
+def test_zero_block_and_partial_tail():
+    w = np.zeros(64 * 3 + 10, dtype=np.float32)
+    w[64:128] = np.linspace(-1, 1, 64, dtype=np.float32)
+    w[-3] = 0.5
+    packed, sc, meta = o.quantize(w)
+    nb, ng = 4, 1
+    assert packed.size == nb * 32 and sc.size == nb and meta.size == ng
+    idx = o.unpack_nibbles(packed, nb * 64)
+    assert np.all(idx[:64] == 7)                       # zero block -> zero code
+    assert np.all(idx[192 + 10:] == 7)                 # padding -> zero code
+    deq = o.bf16_bits_to_float(o.dequantize_bits(packed, sc, meta, w.size))
+    assert np.all(deq[:64] == 0)
+    assert deq[-3] > 0
+
+
+def test_all_zero_tensor():
+    packed, sc, meta = o.quantize(np.zeros((4, 64), np.float32))
+    assert np.all(packed == 0x77) and np.all(sc == 0) and np.all(meta == 0)
+
+
+def test_nonfinite_rejected():
+    w = np.ones(128, np.float32)
+    for bad in (np.nan, np.inf, -np.inf):
+        w2 = w.copy()
+        w2[7] = bad
+        with pytest.raises(o.NonFiniteWeight):
+            o.quantize(w2)
+
+
+def test_quantize_against_per_element_loop():
+    """Brute force on a tiny tensor, one element at a time in plain Python."""
+    rng = np.random.default_rng(4)
+    codes, _ = o.nf4_codebook()
+    w = rng.normal(0, 0.02, (3, 128)).astype(np.float32)
+    w[1, 7] *= 10
+    packed, _, _ = o.quantize(w)
+    flat = w.reshape(-1)
+    got = o.unpack_nibbles(packed, flat.size)
+    for b in range(flat.size // 64):
+        blk = flat[b * 64:(b + 1) * 64]
+        c = max(abs(float(v)) for v in blk)
+        for j, v in enumerate(blk):
+            xv = float(np.float32(v) / np.float32(c))
+            dist = [abs(xv - float(q)) for q in codes]
+            best = min(range(16), key=lambda i: (dist[i], i))
+            assert got[b * 64 + j] == best
+
+
+# --------------------------------------------------------------------------
+# FP8 scales and bf16
+# --------------------------------------------------------------------------
+def test_e4m3_encode_matches_torch_cast():
+    rng = np.random.default_rng(5)
+    vals = np.concatenate([
+        o.e4m3_value_table().astype(np.float32),
+        ((o.e4m3_value_table()[:-1] + o.e4m3_value_table()[1:]) / 2).astype(np.float32),
+        rng.uniform(0, 464, 3000).astype(np.float32),
+        (2.0 ** rng.uniform(-12, -5, 1000)).astype(np.float32),
+        np.array([0.0, 2 ** -10, 3 * 2 ** -10, 448.0, 460.0, 464.0], np.float32),
+    ])
+    ours = o.e4m3_encode(vals)
+    theirs = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, theirs)
+    assert o.e4m3_encode(np.array([465.0, 1e30], np.float32)).tolist() == [0x7E, 0x7E]
+
+
+def test_e4m3_decode_matches_torch():
+    c = np.arange(127, dtype=np.uint8)
+    theirs = torch.from_numpy(c).view(torch.float8_e4m3fn).to(torch.float32).numpy()
+    assert np.array_equal(o.e4m3_decode(c), theirs)
+    assert o.e4m3_decode(np.array([0x7E], np.uint8))[0] == 448.0
+
+
+def test_bf16_rounding_matches_torch():
+    rng = np.random.default_rng(6)
+    x = np.concatenate([rng.normal(0, 1, 20000), rng.normal(0, 1e-30, 100),
+                        [1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -(1.0 + 2 ** -8), 0.0]]).astype(np.float32)
+    theirs = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(o.bf16_bits(x), theirs)
+
+
+def test_double_quant_properties():
+    rng = np.random.default_rng(7)
+    c = np.abs(rng.normal(0, 0.05, 1000)).astype(np.float32)
+    c[512:768] = 0                                    # one all-zero group
+    codes, meta = o.double_quantize(c)
+    assert codes.size == 1000 and meta.size == 4
+    ct = o.dequantize_scales(codes, meta)
+    g = np.arange(1000) // 256
+    for gi in range(4):
+        sel = g == gi
+        if meta[gi] == 0:
+            assert np.all(codes[sel] == 0) and np.all(ct[sel] == 0)
+            continue
+        big = c[sel] >= meta[gi] * 2 ** -6           # normal E4M3 range
+        rel = np.abs(ct[sel][big] - c[sel][big]) / c[sel][big]
+        assert np.all(rel <= 2 ** -4 + 1e-6)
+        assert codes[sel].max() == 0x7E               # the group max maps to 448
+    assert meta[0] == np.float32(c[:256].max()) / np.float32(448)
+
+
+def test_dequantize_bits_against_per_element_torch():
+    rng = np.random.default_rng(8)
+    w = rng.normal(0, 0.02, (2, 256)).astype(np.float32)
+    packed, sc, meta = o.quantize(w)
+    codes, _ = o.nf4_codebook()
+    bits = o.dequantize_bits(packed, sc, meta, w.size)
+    idx = o.unpack_nibbles(packed, w.size)
+    for e in range(w.size):
+        b = e // 64
+        cdec = torch.tensor([int(sc[b])], dtype=torch.uint8).view(torch.float8_e4m3fn).float()
+        ct = (cdec * torch.tensor([float(meta[b // 256])], dtype=torch.float32))
+        v = (torch.tensor([float(codes[idx[e]])], dtype=torch.float32) * ct).to(torch.bfloat16)
+        assert int(v.view(torch.int16).item()) & 0xFFFF == int(bits[e])
+
+
+def test_storage_closed_forms():
+    t = _golden_table("toy_statistics.txt")
+    assert o.storage_bits_per_param() == 4.126953125
+    assert abs(o.storage_bits_per_param() - t["bits_b64_dq"][0]) <= t["bits_b64_dq"][1]
+    assert abs(o.storage_bits_per_param(16) - t["bits_b16_dq"][0]) <= t["bits_b16_dq"][1]
+    assert o.storage_bits_per_param(16, double_quant=False) == t["bits_b16_nodq"][0]
+    saving = o.storage_bits_per_param(64, double_quant=False) - o.storage_bits_per_param()
+    assert abs(saving - t["dq_saving_b64"][0]) <= t["dq_saving_b64"][1]
+    for n, k in ((4096, 4096), (11008, 4096), (28672, 8192)):
+        p, s, m = o.quantized_nbytes(n * k)
+        assert p + s + m == n * k // 2 + n * k // 64 + 4 * math.ceil(n * k / 16384)
+        assert 8 * (p + s + m) / (n * k) == pytest.approx(4.126953125, abs=1e-4)
+
+
+# --------------------------------------------------------------------------
+# The page's toy statistics
+# --------------------------------------------------------------------------
+def _relmse(w, cb, B):
+    r = o.single_quant_roundtrip(w, cb, B).astype(np.float64)
+    return 100 * np.mean((r - w) ** 2) / np.mean(w.astype(np.float64) ** 2)
+
+
+def test_toy_statistics_reproduce():
+    t = _golden_table("toy_statistics.txt")
+    rng = np.random.default_rng(0)
+    w = rng.normal(0, 0.02, 2 ** 20).astype(np.float32)
+    nf4, _ = o.nf4_codebook()
+    fp4, int4 = o.fp4_e2m1_codebook(), o.int4_codebook()
+    got = {
+        "gauss_nf4_b64": _relmse(w, nf4, 64),
+        "gauss_fp4_b64": _relmse(w, fp4, 64),
+        "gauss_int4_b64": _relmse(w, int4, 64),
+        "gauss_nf4_b16": _relmse(w, nf4, 16),
+        "gauss_nf4_b4096": _relmse(w, nf4, 4096),
+    }
+    got["sqnr_nf4_db"] = 10 * math.log10(100 / got["gauss_nf4_b64"])
+    got["sqnr_fp4_db"] = 10 * math.log10(100 / got["gauss_fp4_b64"])
+    got["sqnr_int4_db"] = 10 * math.log10(100 / got["gauss_int4_b64"])
+    s = (rng.standard_t(5, 2 ** 20) * 0.02 / math.sqrt(5 / 3)).astype(np.float32)
+    got["student5_nf4_b64"] = _relmse(s, nf4, 64)
+    got["student5_fp4_b64"] = _relmse(s, fp4, 64)
+    got["student5_int4_b64"] = _relmse(s, int4, 64)
+    for k, v in got.items():
+        ref, tol = t[k]
+        assert abs(v - ref) <= tol, (k, v, ref)
+
+
+def test_residual_is_close_to_full_rank():
+    t = _golden_table("toy_statistics.txt")
+    nf4, _ = o.nf4_codebook()
+    W = np.random.default_rng(0).normal(0, 0.02, (1024, 1024)).astype(np.float32)
+    R = (W - o.single_quant_roundtrip(W, nf4, 64).reshape(W.shape)).astype(np.float64)
+    e = np.linalg.svd(R, compute_uv=False) ** 2
+    for k in (16, 64, 256):
+        ref, tol = t[f"residual_rank{k}"]
+        assert abs(100 * e[:k].sum() / e.sum() - ref) <= tol
+
+
+# --------------------------------------------------------------------------
+# The adapted linear layer
+# --------------------------------------------------------------------------
+def _tiny_linear(seed=9, M=3, N=4, K=5, r=2):
+    rng = np.random.default_rng(seed)
+    return (rng.normal(size=(M, K)), rng.normal(size=(N, K)), rng.normal(size=(r, K)),
+            rng.normal(size=(N, r)), rng.normal(size=(M, N)), 1.75)
+
+
+def test_linear_forward_elementwise_loops():
+    X, W, A, B, dY, g = _tiny_linear()
+    Y, T = o.linear_forward(X, W, A, B, g)
+    M, K = X.shape
+    N, r = B.shape
+    for m in range(M):
+        for j in range(r):
+            assert T[m, j] == pytest.approx(sum(X[m, k] * A[j, k] for k in range(K)), abs=1e-12)
+        for n in range(N):
+            base = sum(X[m, k] * W[n, k] for k in range(K))
+            lora = sum(sum(X[m, k] * A[j, k] for k in range(K)) * B[n, j] for j in range(r))
+            assert Y[m, n] == pytest.approx(base + g * lora, abs=1e-12)
+
+
+def test_linear_backward_finite_differences():
+    """Gradients of L = <dY, Y> by central differences in fp64."""
+    X, W, A, B, dY, g = _tiny_linear()
+    dX, dA, dB, _ = o.linear_backward(dY, X, W, A, B, g)
+
+    def loss(X_, A_, B_):
+        return float(np.sum(dY * o.linear_forward(X_, W, A_, B_, g)[0]))
+
+    h = 1e-6
+    for arr, grad, which in ((X, dX, 0), (A, dA, 1), (B, dB, 2)):
+        num = np.zeros_like(arr)
+        for i in np.ndindex(arr.shape):
+            p, m = arr.copy(), arr.copy()
+            p[i] += h
+            m[i] -= h
+            args_p = [X, A, B]
+            args_m = [X, A, B]
+            args_p[which], args_m[which] = p, m
+            num[i] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        assert np.allclose(num, grad, atol=1e-6), which
+
+
+def test_no_lora_reduces_to_plain_product():
+    X, W, A, B, dY, g = _tiny_linear()
+    Y, _ = o.linear_forward(X, W, A, np.zeros_like(B), g)
+    assert np.allclose(Y, np.einsum("mk,nk->mn", X, W))
+    dX, dA, dB, _ = o.linear_backward(dY, X, W, A, np.zeros_like(B), g)
+    assert np.allclose(dX, np.einsum("mn,nk->mk", dY, W)) and np.allclose(dA, 0)
