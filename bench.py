@@ -1,0 +1,436 @@
+"""Benchmark of the QLoRA NF4 linear layer on B200.
+
+One step = forward (Y, T saved) + backward (dX, dA, dB) of the Llama-7B-shaped
+attention projection: W 4096 x 4096 NF4 (+ double quant), 4096 tokens, LoRA
+r = 16, alpha = 32, synthetic seeded inputs already resident in HBM.  Metric:
+algorithmic TFLOP/s, 4MNK + 6Mr(N+K) flops per step.  Two input sets are
+alternated so that consecutive steps never reuse L2 (each set is ~140 MB,
+over the 126 MB L2).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+--impl reference times the CPU oracle on the host instead (a bounded token
+sample of the same workload).  Under torchrun every rank runs its own
+replica (weak scaling) and all-reduces its adapter gradients; the time is the
+max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WORKLOAD = "llama7b_attn_proj_4096x4096_m4096_r16"
+GEMV_WORKLOAD = "decode_gemv_28672x8192_m1"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Kernels the library launches per step (forward: LoRA T product, its
+# finalize, B padding, dequant-GEMM; backward: gamma*T conversion, U product
+# + finalize, dB product + finalize, A padding, dequant-GEMM dX, dA product +
+# finalize).  The memsets of the workspace error word are runtime memsets.
+LAUNCHES_PER_STEP = 4 + 9
+# ncu DRAM traffic (read + write bytes) of one dequant-GEMM launch of this
+# workload, valid only for the source it was captured on.
+GEMM_TRAFFIC = {"source_sha": None, "fwd_bytes": None, "dx_bytes": None}
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def _source_sha():
+    p = os.path.join(ROOT, "bit_nf4_quantised_b200", "csrc", "gemm_sm100.cu")
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for ln in f:
+                p = [x.strip() for x in ln.split(",")]
+                if len(p) < 9:
+                    continue
+                try:
+                    sm.append(float(p[1]))
+                    smax.append(float(p[2]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, p[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ GPU arm
+def _setup_layer(q, syn, lin, device):
+    d = syn.make_layer(lin)
+    w = q.qlora_quantize(torch.from_numpy(d["W"]).to(device))
+    g = {k: d[k].to(device) for k in ("X", "A", "B", "dY")}
+    return d, w, g
+
+
+def _step(q, lin, w, g, bufs, ws, events=None):
+    """forward + backward of one layer; events = (fwd_b, fwd_e, bwd_b, bwd_e)."""
+    ev_f = (events[0], events[1]) if events else None
+    ev_b = (events[2], events[3]) if events else None
+    q.qlora_linear_forward(g["X"], w, g["A"], g["B"], lin.gamma, Y=bufs["Y"], T_save=bufs["T"],
+                           ws=ws, events=ev_f)
+    q.qlora_linear_backward(g["dY"], g["X"], w, g["A"], g["B"], lin.gamma, T_saved=bufs["T"],
+                            dX=bufs["dX"], dA=bufs["dA"], dB=bufs["dB"], ws=ws, events=ev_b)
+
+
+def _bufs(lin, device):
+    return {"Y": torch.empty(lin.M, lin.N, dtype=torch.bfloat16, device=device),
+            "T": torch.empty(lin.M, lin.r, dtype=torch.float32, device=device),
+            "dX": torch.empty(lin.M, lin.K, dtype=torch.bfloat16, device=device),
+            "dA": torch.empty(lin.r, lin.K, dtype=torch.float32, device=device),
+            "dB": torch.empty(lin.N, lin.r, dtype=torch.float32, device=device)}
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def _gemv_measure(q, syn, device, reps=20):
+    """Decode GEMV (M = 1, 28672 x 8192): GB/s of algorithmic bytes of the
+    forward call, weights rotated over enough copies to exceed 2x L2."""
+    lin = syn.WORKLOADS[GEMV_WORKLOAD].layers[0]
+    d = syn.make_layer(lin, with_grad=False)
+    W0 = torch.from_numpy(d["W"]).to(device)
+    copies = [q.qlora_quantize(W0) for _ in range(3)]          # 3 x 121 MB stored
+    del W0
+    X, A, B = (d[k].to(device) for k in ("X", "A", "B"))
+    Y = torch.empty(lin.M, lin.N, dtype=torch.bfloat16, device=device)
+    ws = q.workspace(lin.M, lin.N, lin.K, lin.r, device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(reps)]
+    for i in range(3):
+        q.qlora_linear_forward(X, copies[i % 3], A, B, lin.gamma, Y=Y, ws=ws)
+    torch.cuda.synchronize()
+    call_b = torch.cuda.Event(enable_timing=True)
+    call_e = torch.cuda.Event(enable_timing=True)
+    call_b.record()
+    for i in range(reps):
+        q.qlora_linear_forward(X, copies[i % 3], A, B, lin.gamma, Y=Y, ws=ws, events=evs[i])
+    call_e.record()
+    torch.cuda.synchronize()
+    kern_ms = sum(b.elapsed_time(e) for b, e in evs) / reps
+    call_ms = call_b.elapsed_time(call_e) / reps
+    wbytes = copies[0].nbytes
+    act = lin.M * lin.K * 2 + lin.r * lin.K * 2 + lin.N * lin.r * 2 + lin.M * lin.N * 2
+    return {"workload": GEMV_WORKLOAD, "kernel_us": kern_ms * 1e3, "call_us": call_ms * 1e3,
+            "algorithmic_bytes": wbytes + act,
+            "kernel_GBps": (wbytes + lin.M * lin.K * 2) / (kern_ms * 1e-3) / 1e9,
+            "call_GBps": (wbytes + act) / (call_ms * 1e-3) / 1e9}
+
+
+def _quantize_measure(q, syn, device, reps=5):
+    lin = syn.WORKLOADS[WORKLOAD].layers[0]
+    W = torch.randn(3, lin.N, lin.K, device=device)           # 3 x 64 MiB rotated
+    outs = [q.empty_nf4(lin.N, lin.K, device) for _ in range(3)]
+    for i in range(3):
+        q.qlora_quantize(W[i], out=outs[i], check_finite=False)
+    torch.cuda.synchronize()
+    b, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b.record()
+    for i in range(reps):
+        q.qlora_quantize(W[i % 3], out=outs[i % 3], check_finite=False)
+    e.record()
+    torch.cuda.synchronize()
+    ms = b.elapsed_time(e) / reps
+    nbytes = lin.N * lin.K * 4 + outs[0].nbytes
+    return {"kernel_us": ms * 1e3, "GBps": nbytes / (ms * 1e-3) / 1e9,
+            "bytes_per_call": nbytes}
+
+
+def run_gpu(args):
+    import bit_nf4_quantised_b200 as q
+    from bit_nf4_quantised_b200 import synthetic as syn
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    q.lib()
+    lin = syn.WORKLOADS[WORKLOAD].layers[0]
+    sets = []
+    for s in range(2):                      # two input sets, alternated
+        import dataclasses
+        l2 = dataclasses.replace(lin, seed=lin.seed + 1000 * rank + s)
+        _, w, g = _setup_layer(q, syn, l2, device)
+        sets.append((w, g))
+    bufs = _bufs(lin, device)
+    ws = q.workspace(lin.M, lin.N, lin.K, lin.r, device)
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+
+    def one(i, events=None):
+        w, g = sets[i % 2]
+        _step(q, lin, w, g, bufs, ws, events)
+        if world > 1:
+            torch.distributed.all_reduce(bufs["dA"])
+            torch.distributed.all_reduce(bufs["dB"])
+
+    for i in range(args.warmup):
+        one(i)
+    _barrier(world)
+    if q.device_error_word(ws) != 0:
+        raise RuntimeError("device error word set during warm-up")
+    clocks = Clocks(local)
+    clocks.start()
+    _barrier(world)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(K):
+        one(i, evs[i])
+    t1.record()
+    _barrier(world)
+    clk = clocks.stop()
+    ms = _max_over_ranks(t0.elapsed_time(t1), world) / K
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
+    dx_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / K
+
+    flops = lin.fwd_bwd_flops()
+    value = world * flops / (ms * 1e-3) / 1e12
+    peaks, peak_kind = _peaks()
+    M, N, Kd, r = lin.M, lin.N, lin.K, lin.r
+    f_fwd = 2 * M * N * Kd + 2 * M * r * N          # main product + LoRA tail in the kernel
+    f_dx = 2 * M * N * Kd + 2 * M * r * Kd
+    achieved = (f_fwd + f_dx) / ((fwd_ms + dx_ms) * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    sha = _source_sha()
+    traffic = None
+    if GEMM_TRAFFIC["source_sha"] == sha and GEMM_TRAFFIC["fwd_bytes"]:
+        traffic = (GEMM_TRAFFIC["fwd_bytes"] + GEMM_TRAFFIC["dx_bytes"]) / 2
+    out = {
+        "metric": "QLoRA linear fwd+bwd TFLOP/s (% bf16 peak); NF4 dequant-GEMV GB/s (% HBM)",
+        "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M, "N": N, "K": Kd, "r": r, "alpha": lin.alpha,
+                   "step": "forward (Y, T) + backward (dX, dA, dB)",
+                   "l2": "two input sets alternated, each ~140 MB > 126 MB L2",
+                   "parallelism": f"replicas{world}" if world > 1 else "single"},
+        "roofline": {"bound": "tensor", "kernel": "qlora_gemm_kernel (forward + dX launches)",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} bf16 burst",
+                     "traffic": traffic, "fwd_us": round(fwd_ms * 1e3, 2),
+                     "dx_us": round(dx_ms * 1e3, 2)},
+        "gpu_launches": LAUNCHES_PER_STEP * K,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1:
+        out["gemv"] = _gemv_measure(q, syn, device)
+        out["gemv"]["frac_hbm"] = round(out["gemv"]["kernel_GBps"] / peaks["hbm_gbs"], 4)
+        out["quantize"] = _quantize_measure(q, syn, device)
+        out["e2e"] = _e2e(q, syn, lin, device, max(3, K // 2))
+        out["cpu_baseline"] = _cpu_baseline(seconds=args.cpu_seconds)
+    else:
+        out["e2e"] = _e2e(q, syn, lin, device, max(3, K // 2), world=world)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out))
+
+
+def _e2e(q, syn, lin, device, steps, world=1):
+    """Same step through the public API with host buffers: pinned host X and
+    dY copied in, Y, dX, dA, dB copied out, all inside the timed region."""
+    d = syn.make_layer(lin)
+    w = q.qlora_quantize(torch.from_numpy(d["W"]).to(device))
+    host_in = {k: d[k].pin_memory() for k in ("X", "dY")}
+    g = {k: d[k].to(device) for k in ("X", "A", "B", "dY")}
+    bufs = _bufs(lin, device)
+    host_out = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in bufs.items()
+                if k != "T"}
+    ws = q.workspace(lin.M, lin.N, lin.K, lin.r, device)
+
+    def one():
+        g["X"].copy_(host_in["X"], non_blocking=True)
+        g["dY"].copy_(host_in["dY"], non_blocking=True)
+        _step(q, lin, w, g, bufs, ws)
+        for k, v in host_out.items():
+            v.copy_(bufs[k], non_blocking=True)
+
+    for _ in range(2):
+        one()
+    _barrier(world)
+    b, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b.record()
+    for _ in range(steps):
+        one()
+    e.record()
+    _barrier(world)
+    ms = _max_over_ranks(b.elapsed_time(e), world) / steps
+    h2d = sum(v.numel() * v.element_size() for v in host_in.values())
+    d2h = sum(v.numel() * v.element_size() for v in host_out.values())
+    return {"value": round(world * lin.fwd_bwd_flops() / (ms * 1e-3) / 1e12, 2),
+            "unit": "TFLOP/s", "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h}
+
+
+# --------------------------------------------------------------- CPU oracle
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+class _OracleLayer:
+    """The oracle's pass over a token sample of the benchmark layer."""
+
+    def __init__(self, sample_tokens: int):
+        from bit_nf4_quantised_b200 import synthetic as syn
+        from oracle import nf4_oracle as o
+        self.o, self.syn = o, syn
+        self.lin = syn.WORKLOADS[WORKLOAD].layers[0]
+        d = syn.make_layer(self.lin)
+        self.store = o.quantize(d["W"])                      # the stored weight (setup)
+        m = sample_tokens
+        self.X, self.A, self.B, self.dY = (syn.as_f64(d[k]) for k in ("X", "A", "B", "dY"))
+        self.X, self.dY = self.X[:m], self.dY[:m]
+        self.m = m
+        lin = self.lin
+        self.flops = 4 * m * lin.N * lin.K + 6 * m * lin.r * (lin.N + lin.K)
+
+    def step(self):
+        o, lin = self.o, self.lin
+        Wt = o.dequantize(*self.store, lin.N, lin.K).astype(np.float64)
+        o.linear_forward(self.X, Wt, self.A, self.B, lin.gamma)
+        o.linear_backward(self.dY, self.X, Wt, self.A, self.B, lin.gamma)
+
+
+def _cpu_baseline(seconds: float = 10.0, sample_tokens: int = 256):
+    layer = _OracleLayer(sample_tokens)
+    layer.step()                                               # warm
+    n, t = 0, 0.0
+    while t < seconds or n < 2:
+        t0 = time.perf_counter()
+        layer.step()
+        t += time.perf_counter() - t0
+        n += 1
+    return {"value": round(layer.flops * n / t / 1e12, 5), "unit": "TFLOP/s",
+            "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{sample_tokens} of {layer.lin.M} tokens per pass, W dequantised once "
+                      f"per pass, fwd+bwd in fp64 numpy; {n} passes, {t:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    layer = _OracleLayer(sample_tokens=128)
+    for _ in range(args.warmup):
+        layer.step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        layer.step()
+    dt = (time.perf_counter() - t0) / args.steps
+    value = layer.flops / dt / 1e12
+    lin = layer.lin
+    out = {
+        "impl": "reference",
+        "metric": "QLoRA linear fwd+bwd TFLOP/s (% bf16 peak); NF4 dequant-GEMV GB/s (% HBM)",
+        "value": round(value, 5), "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": lin.M, "N": lin.N, "K": lin.K, "r": lin.r,
+                   "alpha": lin.alpha, "step": "forward (Y, T) + backward (dX, dA, dB)"},
+        "cpu_baseline": {"value": round(value, 5), "unit": "TFLOP/s", "kind": "oracle",
+                         "cores": _blas_threads(),
+                         "sample": f"{layer.m} of {lin.M} tokens per step, W dequantised once "
+                                   "per step, fp64 numpy"},
+        "e2e": {"value": round(value, 5), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

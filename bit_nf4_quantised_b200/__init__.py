@@ -1,0 +1,23 @@
+"""B200-native frozen-NF4 linear layer with a bf16 LoRA adapter.
+
+The computation lives in libqlora_nf4.so (CUDA, sm_100a); this package is its
+ctypes binding (``_lib``), the in-tree build script (``build``) and the seeded
+synthetic workload generator (``synthetic``).
+"""
+from ._lib import (  # noqa: F401
+    EXPORTED,
+    NF4Tensor,
+    QloraError,
+    device_error_word,
+    empty_nf4,
+    lib,
+    nf4_build_codebook,
+    qlora_dequantize,
+    qlora_linear_backward,
+    qlora_linear_forward,
+    qlora_linear_workspace_size,
+    qlora_quantize,
+    qlora_quantized_sizes,
+    status_string,
+    workspace,
+)

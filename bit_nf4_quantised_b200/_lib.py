@@ -1,0 +1,274 @@
+"""ctypes binding of libqlora_nf4.so (include/qlora_nf4.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  PyTorch supplies device memory and the current stream.  If the
+shared library is missing the import fails loudly; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libqlora_nf4.so")
+
+QLORA_OK = 0
+QLORA_ERR_NULL = 1
+QLORA_ERR_SHAPE = 2
+QLORA_ERR_ALIGN = 3
+QLORA_ERR_UNSUPPORTED = 4
+QLORA_ERR_NONFINITE = 5
+QLORA_ERR_CUDA = 6
+QLORA_ERR_WORKSPACE = 7
+
+BLOCK = 64
+GROUP = 256
+MAX_RANK = 128
+GEMV_MAX_TOKENS = 16
+
+EXPORTED = (
+    "qlora_status_string",
+    "nf4_build_codebook",
+    "qlora_quantized_sizes",
+    "qlora_quantize",
+    "qlora_dequantize",
+    "qlora_linear_workspace_size",
+    "qlora_linear_forward",
+    "qlora_linear_backward",
+    "qlora_linear_forward_ex",
+    "qlora_linear_backward_ex",
+)
+
+
+class QloraError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class _Events(ctypes.Structure):
+    _fields_ = [("gemm_begin", ctypes.c_void_p), ("gemm_end", ctypes.c_void_p)]
+
+
+def _events(events):
+    """(begin, end) torch.cuda.Event pair (timing enabled) -> qlora_events*."""
+    if events is None:
+        return None
+    b, e = events
+    return ctypes.byref(_Events(b.cuda_event if b is not None else None,
+                                e.cuda_event if e is not None else None))
+
+
+class _Tensor(ctypes.Structure):
+    _fields_ = [
+        ("packed", ctypes.c_void_p),
+        ("scale_codes", ctypes.c_void_p),
+        ("meta_scale", ctypes.c_void_p),
+        ("rows", ctypes.c_int64),
+        ("cols", ctypes.c_int64),
+    ]
+
+
+_LIB = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library once; raises if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with `python -m bit_nf4_quantised_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i64, i32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+        sz = ctypes.POINTER(ctypes.c_size_t)
+        tp = ctypes.POINTER(_Tensor)
+        L.qlora_status_string.argtypes = [i32]
+        L.qlora_status_string.restype = ctypes.c_char_p
+        L.nf4_build_codebook.argtypes = [vp, vp]
+        L.qlora_quantized_sizes.argtypes = [i64, i64, sz, sz, sz]
+        L.qlora_quantize.argtypes = [vp, tp, vp, vp]
+        L.qlora_dequantize.argtypes = [tp, vp, vp]
+        L.qlora_linear_workspace_size.argtypes = [i64, i64, i64, i32, sz]
+        fwd = [vp, i64, tp, vp, vp, i32, f32, vp, vp, vp, ctypes.c_size_t, vp]
+        bwd = [vp, vp, i64, tp, vp, vp, i32, f32, vp, vp, vp, vp, i32, vp, ctypes.c_size_t, vp]
+        L.qlora_linear_forward.argtypes = fwd
+        L.qlora_linear_backward.argtypes = bwd
+        L.qlora_linear_forward_ex.argtypes = fwd + [ctypes.c_void_p]
+        L.qlora_linear_backward_ex.argtypes = bwd + [ctypes.c_void_p]
+        for name in EXPORTED[1:]:
+            getattr(L, name).restype = i32
+        _LIB = L
+    return _LIB
+
+
+def status_string(status: int) -> str:
+    return lib().qlora_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != QLORA_OK:
+        raise QloraError(status, where)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _need(t: torch.Tensor, dtype, name: str) -> None:
+    if t.dtype != dtype or not t.is_contiguous() or not t.is_cuda:
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+
+
+# --------------------------------------------------------------------------
+@dataclass
+class NF4Tensor:
+    """A stored NF4 weight (three device buffers) of logical shape rows x cols."""
+    packed: torch.Tensor        # uint8 [nblocks * 32]
+    scale_codes: torch.Tensor   # uint8 [nblocks]
+    meta_scale: torch.Tensor    # float32 [ngroups]
+    rows: int
+    cols: int
+
+    def c_struct(self) -> _Tensor:
+        return _Tensor(self.packed.data_ptr(), self.scale_codes.data_ptr(),
+                       self.meta_scale.data_ptr(), self.rows, self.cols)
+
+    @property
+    def nbytes(self) -> int:
+        return self.packed.numel() + self.scale_codes.numel() + 4 * self.meta_scale.numel()
+
+
+def nf4_build_codebook():
+    codes = (ctypes.c_float * 16)()
+    mids = (ctypes.c_float * 15)()
+    _check(lib().nf4_build_codebook(ctypes.addressof(codes), ctypes.addressof(mids)),
+           "nf4_build_codebook")
+    return list(codes), list(mids)
+
+
+def qlora_quantized_sizes(rows: int, cols: int):
+    p, c, m = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().qlora_quantized_sizes(rows, cols, ctypes.byref(p), ctypes.byref(c),
+                                       ctypes.byref(m)), "qlora_quantized_sizes")
+    return p.value, c.value, m.value
+
+
+def empty_nf4(rows: int, cols: int, device="cuda") -> NF4Tensor:
+    p, c, m = qlora_quantized_sizes(rows, cols)
+    return NF4Tensor(torch.empty(max(p, 16), dtype=torch.uint8, device=device)[:p],
+                     torch.empty(max(c, 1), dtype=torch.uint8, device=device)[:c],
+                     torch.empty(max(m // 4, 1), dtype=torch.float32, device=device)[: m // 4],
+                     rows, cols)
+
+
+def qlora_quantize(W: torch.Tensor, out: NF4Tensor | None = None, check_finite: bool = True,
+                   stream=None) -> NF4Tensor:
+    """Quantise a fp32 [rows, cols] CUDA tensor.  With check_finite the call
+    synchronises the stream and raises QloraError(QLORA_ERR_NONFINITE) if the
+    kernel saw a NaN or an infinity."""
+    _need(W, torch.float32, "W")
+    rows, cols = (W.shape[0], W.shape[1]) if W.dim() == 2 else (1, W.numel())
+    out = out if out is not None else empty_nf4(rows, cols, W.device)
+    flag = torch.zeros(1, dtype=torch.int32, device=W.device) if check_finite else None
+    st = out.c_struct()
+    _check(lib().qlora_quantize(W.data_ptr(), ctypes.byref(st), _ptr(flag), _stream(stream)),
+           "qlora_quantize")
+    if check_finite and int(flag.item()) != 0:
+        raise QloraError(QLORA_ERR_NONFINITE, "qlora_quantize")
+    return out
+
+
+def qlora_dequantize(w: NF4Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    out = out if out is not None else torch.empty(w.rows, w.cols, dtype=torch.bfloat16,
+                                                  device=w.packed.device)
+    _need(out, torch.bfloat16, "out")
+    st = w.c_struct()
+    _check(lib().qlora_dequantize(ctypes.byref(st), out.data_ptr(), _stream(stream)),
+           "qlora_dequantize")
+    return out
+
+
+def qlora_linear_workspace_size(M: int, N: int, K: int, r: int) -> int:
+    b = ctypes.c_size_t()
+    _check(lib().qlora_linear_workspace_size(M, N, K, r, ctypes.byref(b)),
+           "qlora_linear_workspace_size")
+    return b.value
+
+
+def workspace(M: int, N: int, K: int, r: int, device="cuda") -> torch.Tensor:
+    n = qlora_linear_workspace_size(M, N, K, r)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def qlora_linear_forward(X: torch.Tensor, w: NF4Tensor, A: torch.Tensor, B: torch.Tensor,
+                         scale: float, Y: torch.Tensor | None = None,
+                         T_save: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                         stream=None, events=None) -> torch.Tensor:
+    """Y = X W~^T + scale * (X A^T) B^T.  X [M,K] bf16, A [r,K], B [N,r].
+    events: optional (begin, end) torch.cuda.Event pair recorded around the
+    main weight kernel."""
+    _need(X, torch.bfloat16, "X")
+    _need(A, torch.bfloat16, "A")
+    _need(B, torch.bfloat16, "B")
+    M, K = X.shape
+    r = A.shape[0]
+    N = w.rows
+    Y = Y if Y is not None else torch.empty(M, N, dtype=torch.bfloat16, device=X.device)
+    _need(Y, torch.bfloat16, "Y")
+    if T_save is not None:
+        _need(T_save, torch.float32, "T_save")
+    ws = ws if ws is not None else workspace(M, N, K, r, X.device)
+    st = w.c_struct()
+    _check(lib().qlora_linear_forward_ex(X.data_ptr(), M, ctypes.byref(st), A.data_ptr(),
+                                         B.data_ptr(), r, float(scale), Y.data_ptr(),
+                                         _ptr(T_save), ws.data_ptr(), ws.numel(),
+                                         _stream(stream), _events(events)),
+           "qlora_linear_forward")
+    return Y
+
+
+def qlora_linear_backward(dY: torch.Tensor, X: torch.Tensor, w: NF4Tensor, A: torch.Tensor,
+                          B: torch.Tensor, scale: float, T_saved: torch.Tensor | None = None,
+                          dX: torch.Tensor | None = None, dA: torch.Tensor | None = None,
+                          dB: torch.Tensor | None = None, accumulate: bool = False,
+                          want_dX: bool = True, ws: torch.Tensor | None = None, stream=None,
+                          events=None):
+    """(dX, dA, dB) of the adapted layer; dX is None when want_dX is False."""
+    for t, n in ((dY, "dY"), (X, "X"), (A, "A"), (B, "B")):
+        _need(t, torch.bfloat16, n)
+    M, K = X.shape
+    r = A.shape[0]
+    N = w.rows
+    dev = X.device
+    if want_dX and dX is None:
+        dX = torch.empty(M, K, dtype=torch.bfloat16, device=dev)
+    dA = dA if dA is not None else torch.empty(r, K, dtype=torch.float32, device=dev)
+    dB = dB if dB is not None else torch.empty(N, r, dtype=torch.float32, device=dev)
+    if T_saved is not None:
+        _need(T_saved, torch.float32, "T_saved")
+    ws = ws if ws is not None else workspace(M, N, K, r, dev)
+    st = w.c_struct()
+    _check(lib().qlora_linear_backward_ex(dY.data_ptr(), X.data_ptr(), M, ctypes.byref(st),
+                                          A.data_ptr(), B.data_ptr(), r, float(scale),
+                                          _ptr(T_saved), _ptr(dX) if want_dX else None,
+                                          dA.data_ptr(), dB.data_ptr(), int(bool(accumulate)),
+                                          ws.data_ptr(), ws.numel(), _stream(stream),
+                                          _events(events)),
+           "qlora_linear_backward")
+    return (dX if want_dX else None), dA, dB
+
+
+def device_error_word(ws: torch.Tensor) -> int:
+    """The kernels' error word (first 4 bytes of the workspace); 0 = no error,
+    bit 0 = a bounded wait inside the GEMM expired."""
+    return int(ws[:4].view(torch.int32).item())

@@ -1,0 +1,105 @@
+// Internal launch interface between the host layer (qlora_api.cu) and the
+// kernels.  Not part of the public C ABI.
+#pragma once
+
+#include "common.cuh"
+
+namespace qnf4 {
+
+// ---------------------------------------------------------------- K1 / K6
+cudaError_t launch_quantize(const float* W, int64_t numel, uint8_t* packed, uint8_t* scale_codes,
+                            float* meta, int* nonfinite_flag, const Nf4Table& tab,
+                            cudaStream_t stream);
+
+cudaError_t launch_dequantize(const uint8_t* packed, const uint8_t* scale_codes, const float* meta,
+                              int64_t numel, uint16_t* out, const Nf4Table& tab, int num_sms,
+                              cudaStream_t stream);
+
+// ---------------------------------------------------------------- K2 / K3
+struct GemmArgs {
+    const uint8_t* scale_codes;
+    const float* meta;
+    uint16_t* D;          // output, row-major [M x d_cols]
+    int64_t M;            // tokens
+    int64_t Nw;           // rows of W (out features)
+    int64_t d_cols;       // Nw (forward) or Kw (input gradient)
+    int64_t nkb;          // NF4 blocks per row of W = Kw / 64
+    int main_steps;       // 64-wide contraction steps over W
+    int tail_steps;       // ceil(r / 64) LoRA steps
+    int r;
+    int m_tiles;
+    int* err;             // device error word
+    Nf4Table tab;
+};
+
+cudaError_t launch_gemm(bool trans, const CUtensorMap& act, const CUtensorMap& packed,
+                        const CUtensorMap& lora_a, const CUtensorMap& lora_b, const GemmArgs& args,
+                        cudaStream_t stream);
+int gemm_tile_m();
+int gemm_tile_n();
+
+// -------------------------------------------------------------- K4 (LoRA)
+// part[s][i][j] = sum over the s-th contraction slice of P(i,c) * Q(c,j), fp32.
+//   p_kmajor: P stored [I][C] (ld = ldp) else [C][I].
+//   q_kmajor: Q stored [J][C] (ld = ldq) else [C][J].
+// J <= 128 and J % 8 == 0; C % 8 == 0; leading dimensions % 8 == 0.
+struct SkinnyArgs {
+    const uint16_t* P;
+    const uint16_t* Q;
+    float* part;
+    int64_t I, J, C;
+    int64_t ldp, ldq;
+    int splits;           // contraction slices (grid.y)
+    int64_t c_per_split;  // multiple of 64
+};
+cudaError_t launch_skinny(bool p_kmajor, bool q_kmajor, const SkinnyArgs& a, cudaStream_t stream);
+
+// out = alpha * sum_s part[s]  (+ out if accumulate), optionally transposed,
+// and/or a bf16 copy scaled by beta into a zero-padded [I x ldb] buffer.
+struct FinalizeArgs {
+    const float* part;
+    int splits;
+    int64_t I, J;
+    float alpha;
+    float* out;           // nullable; [I x J], or [J x I] if transpose
+    int transpose;
+    int accumulate;
+    uint16_t* out_bf16;   // nullable; [I x ldb], columns >= J zeroed
+    int64_t ldb;
+    float beta;
+};
+cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t stream);
+
+// dst[R2 x C2] (bf16) = src[R1 x C1] zero-padded (R1 <= R2, C1 <= C2).
+cudaError_t launch_pad_copy(const uint16_t* src, int64_t R1, int64_t C1, uint16_t* dst, int64_t R2,
+                            int64_t C2, cudaStream_t stream);
+
+// --------------------------------------------------------------------- K5
+struct GemvArgs {
+    const uint8_t* packed;
+    const uint8_t* scale_codes;
+    const float* meta;
+    const uint16_t* X;    // [M x K] bf16, M <= 16
+    float* part;          // [splits][M][N] fp32
+    int64_t M, N, K;
+    int splits;
+    int64_t k_per_split;  // multiple of 64
+    Nf4Table tab;
+};
+cudaError_t launch_gemv(const GemvArgs& a, int* smem_bytes_out, cudaStream_t stream);
+int gemv_rows_per_cta();
+
+// Y[m][n] = bf16( sum_s part[s][m][n] + sum_j G[m][j] * B[n][j] )
+struct GemvFinalizeArgs {
+    const float* part;
+    int splits;
+    const uint16_t* G;    // gamma*T, bf16 [M x ldg]
+    int64_t ldg;
+    const uint16_t* B;    // [N x r]
+    int r;
+    uint16_t* Y;
+    int64_t M, N;
+};
+cudaError_t launch_gemv_finalize(const GemvFinalizeArgs& a, cudaStream_t stream);
+
+}  // namespace qnf4

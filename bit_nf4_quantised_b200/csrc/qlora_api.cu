@@ -1,0 +1,464 @@
+// Host layer of libqlora_nf4.so: the exported C ABI (include/qlora_nf4.h).
+// Argument validation, the workspace plan, TMA descriptors, the NF4 codebook
+// construction, and the launch sequence of each entry point.  No device
+// memory is allocated here; every buffer is the caller's.
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "kernels.cuh"
+
+using namespace qnf4;
+
+namespace {
+
+// ------------------------------------------------------------- codebook
+// Standard-normal CDF and its inverse by safeguarded Newton iteration on
+// erfc, in double precision.
+double norm_cdf(double x) { return 0.5 * std::erfc(-x / std::sqrt(2.0)); }
+
+double norm_quantile(double p) {
+    double lo = -40.0, hi = 40.0, x = 0.0;
+    const double inv_sqrt_2pi = 0.3989422804014327;
+    for (int it = 0; it < 200; ++it) {
+        const double f = norm_cdf(x) - p;
+        if (f < 0) lo = x; else hi = x;
+        const double dens = inv_sqrt_2pi * std::exp(-0.5 * x * x);
+        double xn = x - f / dens;
+        if (!(xn > lo && xn < hi)) xn = 0.5 * (lo + hi);
+        if (xn == x) break;
+        x = xn;
+    }
+    return x;
+}
+
+// "QLoRA, explained", "NormalFloat 4 (NF4)": averages of adjacent quantiles,
+// a 9-level positive half and an 8-level negative half sharing zero (the
+// offset delta averages the two halves' outermost probabilities), scaled to
+// [-1, 1].
+void build_table(float codes[16], float mids[15]) {
+    const double delta = 0.5 * ((1.0 - 1.0 / 30.0) + (1.0 - 1.0 / 32.0));
+    double v[16];
+    int n = 0;
+    for (int j = 6; j >= 0; --j) v[n++] = -norm_quantile(delta - j * (delta - 0.5) / 7.0);
+    v[n++] = 0.0;
+    for (int i = 7; i >= 0; --i) v[n++] = norm_quantile(delta - i * (delta - 0.5) / 8.0);
+    std::sort(v, v + 16);
+    const double top = norm_quantile(delta);
+    for (int i = 0; i < 16; ++i) codes[i] = static_cast<float>(v[i] / top);
+    codes[0] = -1.0f;      // exact by construction; pinned against rounding of v/top
+    codes[7] = 0.0f;
+    codes[15] = 1.0f;
+    for (int i = 0; i < 15; ++i)
+        mids[i] = static_cast<float>((static_cast<double>(codes[i]) + codes[i + 1]) / 2.0);
+}
+
+const Nf4Table& table() {
+    static Nf4Table t;
+    static std::once_flag once;
+    std::call_once(once, [] { build_table(t.code, t.mid); });
+    return t;
+}
+
+// ---------------------------------------------------------------- TMA
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                 CUtensorMapSwizzle swz) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------- validation
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_tensor(const qlora_nf4_tensor* w) {
+    if (!w || !w->packed || !w->scale_codes || !w->meta_scale) return QLORA_ERR_NULL;
+    if (w->rows < 0 || w->cols < 0) return QLORA_ERR_SHAPE;
+    if (w->cols > 0 && w->rows > INT64_MAX / w->cols) return QLORA_ERR_SHAPE;
+    if (!aligned(w->packed, 16) || !aligned(w->meta_scale, 4)) return QLORA_ERR_ALIGN;
+    return QLORA_OK;
+}
+
+int num_sms() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+// ------------------------------------------------------- workspace plan
+constexpr int64_t kAlign = 256;
+constexpr int64_t kTargetCtas = 296;     // two CTAs per SM of a 148-SM B200
+constexpr int64_t kGemvSlice = 2048;
+
+int64_t up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+struct Split {
+    int splits;
+    int64_t per;
+};
+
+// contraction slices for a skinny product with I long-side rows and C depth
+Split skinny_split(int64_t I, int64_t C) {
+    const int64_t chunks = std::max<int64_t>(1, cdiv(C, 64));
+    int64_t s = std::max<int64_t>(1, cdiv(kTargetCtas, std::max<int64_t>(1, cdiv(I, 64))));
+    s = std::min(s, chunks);
+    const int64_t per = cdiv(chunks, s) * 64;
+    return {static_cast<int>(cdiv(C, per)), per};
+}
+
+Split gemv_split(int64_t K) {
+    const int64_t per = std::min(K, kGemvSlice);
+    return {static_cast<int>(cdiv(K, per)), per};
+}
+
+struct Plan {
+    int64_t rp;          // rank padded to 64
+    int64_t off_err, off_part, off_gt, off_gu, off_bp, off_ap, total;
+};
+
+Plan make_plan(int64_t M, int64_t N, int64_t K, int r) {
+    Plan p;
+    p.rp = up(r, 64);
+    int64_t part = 0;
+    const Split sT = skinny_split(M, K), sU = skinny_split(M, N), sB = skinny_split(N, M),
+                sA = skinny_split(K, M);
+    part = std::max(part, int64_t(sT.splits) * M * r);
+    part = std::max(part, int64_t(sU.splits) * M * r);
+    part = std::max(part, int64_t(sB.splits) * N * r);
+    part = std::max(part, int64_t(sA.splits) * K * r);
+    if (M <= QLORA_GEMV_MAX_TOKENS) part = std::max(part, int64_t(gemv_split(K).splits) * M * N);
+    int64_t o = 0;
+    p.off_err = o;  o += kAlign;
+    p.off_part = o; o += up(part * 4, kAlign);
+    p.off_gt = o;   o += up(M * p.rp * 2, kAlign);
+    p.off_gu = o;   o += up(M * p.rp * 2, kAlign);
+    p.off_bp = o;   o += up(N * p.rp * 2, kAlign);
+    p.off_ap = o;   o += up(p.rp * K * 2, kAlign);
+    p.total = o;
+    return p;
+}
+
+int check_linear_shapes(int64_t M, int64_t N, int64_t K, int r) {
+    if (M < 0 || N < 0 || K < 0) return QLORA_ERR_SHAPE;
+    if (K < 64 || N < 8 || K % 64 != 0 || N % 8 != 0) return QLORA_ERR_UNSUPPORTED;
+    if (r < 8 || r > QLORA_MAX_RANK || r % 8 != 0) return QLORA_ERR_UNSUPPORTED;
+    if (M > (int64_t(1) << 31) - 1 || N > (int64_t(1) << 31) - 1 || K > (int64_t(1) << 31) - 1)
+        return QLORA_ERR_UNSUPPORTED;
+    return QLORA_OK;
+}
+
+cudaError_t record(const qlora_events* ev, bool begin, cudaStream_t s) {
+    if (!ev) return cudaSuccess;
+    void* e = begin ? ev->gemm_begin : ev->gemm_end;
+    return e ? cudaEventRecord(reinterpret_cast<cudaEvent_t>(e), s) : cudaSuccess;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
+
+#define QTRY(expr)                                   \
+    do {                                             \
+        cudaError_t _e = (expr);                     \
+        if (_e != cudaSuccess) return QLORA_ERR_CUDA; \
+    } while (0)
+
+template <class T>
+T* at(void* ws, int64_t off) {
+    return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+// T = X A^T -> (optional fp32 T_save, bf16 gamma*T padded to rp) ; uses part
+cudaError_t run_T(const uint16_t* X, const uint16_t* A, int64_t M, int64_t K, int r, float gamma,
+                  float* T_save, uint16_t* Gt, int64_t rp, float* part, cudaStream_t s) {
+    const Split sp = skinny_split(M, K);
+    SkinnyArgs a{X, A, part, M, r, K, K, K, sp.splits, sp.per};
+    cudaError_t e = launch_skinny(true, true, a, s);
+    if (e != cudaSuccess) return e;
+    FinalizeArgs f{part, sp.splits, M, r, 1.0f, T_save, 0, 0, Gt, rp, gamma};
+    return launch_finalize(f, s);
+}
+
+}  // namespace
+
+// ===================================================================== ABI
+extern "C" {
+
+const char* qlora_status_string(int status) {
+    switch (status) {
+        case QLORA_OK: return "ok";
+        case QLORA_ERR_NULL: return "null pointer";
+        case QLORA_ERR_SHAPE: return "bad shape";
+        case QLORA_ERR_ALIGN: return "misaligned pointer";
+        case QLORA_ERR_UNSUPPORTED: return "unsupported size";
+        case QLORA_ERR_NONFINITE: return "non-finite weight";
+        case QLORA_ERR_CUDA: return "CUDA error";
+        case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
+        default: return "unknown status";
+    }
+}
+
+int nf4_build_codebook(float codes[16], float midpoints[15]) {
+    if (!codes || !midpoints) return QLORA_ERR_NULL;
+    const Nf4Table& t = table();
+    std::memcpy(codes, t.code, sizeof(t.code));
+    std::memcpy(midpoints, t.mid, sizeof(t.mid));
+    return QLORA_OK;
+}
+
+int qlora_quantized_sizes(int64_t rows, int64_t cols, size_t* packed_bytes, size_t* codes_bytes,
+                          size_t* meta_bytes) {
+    if (!packed_bytes || !codes_bytes || !meta_bytes) return QLORA_ERR_NULL;
+    if (rows < 0 || cols < 0) return QLORA_ERR_SHAPE;
+    if (cols > 0 && rows > INT64_MAX / cols) return QLORA_ERR_SHAPE;
+    const int64_t numel = rows * cols;
+    const int64_t nblocks = cdiv(numel, QLORA_BLOCK);
+    const int64_t ngroups = cdiv(nblocks, QLORA_GROUP);
+    *packed_bytes = static_cast<size_t>(nblocks) * (QLORA_BLOCK / 2);
+    *codes_bytes = static_cast<size_t>(nblocks);
+    *meta_bytes = static_cast<size_t>(ngroups) * 4;
+    return QLORA_OK;
+}
+
+int qlora_quantize(const float* W, const qlora_nf4_tensor* out, int* d_nonfinite_flag,
+                   qlora_stream_t stream) {
+    if (!W) return QLORA_ERR_NULL;
+    int st = check_tensor(out);
+    if (st != QLORA_OK) return st;
+    if (!aligned(W, 16)) return QLORA_ERR_ALIGN;
+    const int64_t numel = out->rows * out->cols;
+    if (numel == 0) return QLORA_OK;
+    return cuda_status(launch_quantize(W, numel, out->packed, out->scale_codes, out->meta_scale,
+                                       d_nonfinite_flag, table(),
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int qlora_dequantize(const qlora_nf4_tensor* w, uint16_t* W_out, qlora_stream_t stream) {
+    if (!W_out) return QLORA_ERR_NULL;
+    int st = check_tensor(w);
+    if (st != QLORA_OK) return st;
+    if (!aligned(W_out, 16)) return QLORA_ERR_ALIGN;
+    const int64_t numel = w->rows * w->cols;
+    if (numel == 0) return QLORA_OK;
+    return cuda_status(launch_dequantize(w->packed, w->scale_codes, w->meta_scale, numel, W_out,
+                                         table(), num_sms(),
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int qlora_linear_workspace_size(int64_t M, int64_t N, int64_t K, int r, size_t* bytes) {
+    if (!bytes) return QLORA_ERR_NULL;
+    int st = check_linear_shapes(M, N, K, r);
+    if (st != QLORA_OK) return st;
+    *bytes = static_cast<size_t>(make_plan(M, N, K, r).total);
+    return QLORA_OK;
+}
+
+int qlora_linear_forward_ex(const uint16_t* X, int64_t M, const qlora_nf4_tensor* w,
+                            const uint16_t* A, const uint16_t* B, int r, float scale, uint16_t* Y,
+                            float* T_save, void* ws, size_t ws_bytes, qlora_stream_t stream,
+                            const qlora_events* ev) {
+    if (!X || !A || !B || !Y) return QLORA_ERR_NULL;
+    int st = check_tensor(w);
+    if (st != QLORA_OK) return st;
+    const int64_t N = w->rows, K = w->cols;
+    st = check_linear_shapes(M, N, K, r);
+    if (st != QLORA_OK) return st;
+    if (!aligned(X, 16) || !aligned(A, 16) || !aligned(B, 16) || !aligned(Y, 16) ||
+        (T_save && !aligned(T_save, 16)))
+        return QLORA_ERR_ALIGN;
+    const Plan p = make_plan(M, N, K, r);
+    if (!ws || ws_bytes < static_cast<size_t>(p.total)) return QLORA_ERR_WORKSPACE;
+    if (!aligned(ws, kAlign)) return QLORA_ERR_ALIGN;
+    if (M == 0) return QLORA_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int* err = at<int>(ws, p.off_err);
+    float* part = at<float>(ws, p.off_part);
+    uint16_t* Gt = at<uint16_t>(ws, p.off_gt);
+    QTRY(cudaMemsetAsync(err, 0, sizeof(int), s));
+    QTRY(run_T(X, A, M, K, r, scale, T_save, Gt, p.rp, part, s));
+
+    if (M <= QLORA_GEMV_MAX_TOKENS) {
+        const Split sp = gemv_split(K);
+        GemvArgs g{w->packed, w->scale_codes, w->meta_scale, X, part, M, N, K, sp.splits, sp.per,
+                   table()};
+        QTRY(record(ev, true, s));
+        QTRY(launch_gemv(g, nullptr, s));
+        QTRY(record(ev, false, s));
+        GemvFinalizeArgs f{part, sp.splits, Gt, p.rp, B, r, Y, M, N};
+        QTRY(launch_gemv_finalize(f, s));
+        return QLORA_OK;
+    }
+
+    uint16_t* Bp = at<uint16_t>(ws, p.off_bp);
+    QTRY(launch_pad_copy(B, N, r, Bp, N, p.rp, s));
+    CUtensorMap m_act, m_packed, m_la, m_lb;
+    bool ok = make_map_2d(&m_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 128,
+                          CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map_2d(&m_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->packed, K / 2, N, K / 2, 32,
+                          256, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+              make_map_2d(&m_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Gt, p.rp, M, p.rp * 2, 64, 128,
+                          CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map_2d(&m_lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Bp, p.rp, N, p.rp * 2, 64, 256,
+                          CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return QLORA_ERR_CUDA;
+    GemmArgs g{};
+    g.scale_codes = w->scale_codes;
+    g.meta = w->meta_scale;
+    g.D = Y;
+    g.M = M;
+    g.Nw = N;
+    g.d_cols = N;
+    g.nkb = K / 64;
+    g.main_steps = static_cast<int>(K / 64);
+    g.tail_steps = static_cast<int>(cdiv(r, 64));
+    g.r = r;
+    g.m_tiles = static_cast<int>(cdiv(M, gemm_tile_m()));
+    g.err = err;
+    g.tab = table();
+    QTRY(record(ev, true, s));
+    QTRY(launch_gemm(false, m_act, m_packed, m_la, m_lb, g, s));
+    QTRY(record(ev, false, s));
+    return QLORA_OK;
+}
+
+int qlora_linear_forward(const uint16_t* X, int64_t M, const qlora_nf4_tensor* w,
+                         const uint16_t* A, const uint16_t* B, int r, float scale, uint16_t* Y,
+                         float* T_save, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+    return qlora_linear_forward_ex(X, M, w, A, B, r, scale, Y, T_save, ws, ws_bytes, stream,
+                                   nullptr);
+}
+
+int qlora_linear_backward_ex(const uint16_t* dY, const uint16_t* X, int64_t M,
+                             const qlora_nf4_tensor* w, const uint16_t* A, const uint16_t* B,
+                             int r, float scale, const float* T_saved, uint16_t* dX, float* dA,
+                             float* dB, int accumulate, void* ws, size_t ws_bytes,
+                             qlora_stream_t stream, const qlora_events* ev) {
+    if (!dY || !X || !A || !B || !dA || !dB) return QLORA_ERR_NULL;
+    int st = check_tensor(w);
+    if (st != QLORA_OK) return st;
+    const int64_t N = w->rows, K = w->cols;
+    st = check_linear_shapes(M, N, K, r);
+    if (st != QLORA_OK) return st;
+    if (!aligned(dY, 16) || !aligned(X, 16) || !aligned(A, 16) || !aligned(B, 16) ||
+        !aligned(dA, 16) || !aligned(dB, 16) || (dX && !aligned(dX, 16)) ||
+        (T_saved && !aligned(T_saved, 16)))
+        return QLORA_ERR_ALIGN;
+    const Plan p = make_plan(M, N, K, r);
+    if (!ws || ws_bytes < static_cast<size_t>(p.total)) return QLORA_ERR_WORKSPACE;
+    if (!aligned(ws, kAlign)) return QLORA_ERR_ALIGN;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (M == 0) {
+        // empty batch: gradients are zero (or unchanged when accumulating)
+        if (!accumulate) {
+            QTRY(cudaMemsetAsync(dA, 0, size_t(r) * K * 4, s));
+            QTRY(cudaMemsetAsync(dB, 0, size_t(N) * r * 4, s));
+        }
+        return QLORA_OK;
+    }
+    int* err = at<int>(ws, p.off_err);
+    float* part = at<float>(ws, p.off_part);
+    uint16_t* Gt = at<uint16_t>(ws, p.off_gt);
+    uint16_t* Gu = at<uint16_t>(ws, p.off_gu);
+    QTRY(cudaMemsetAsync(err, 0, sizeof(int), s));
+
+    // gamma * T in bf16 (from the saved T or recomputed)
+    if (T_saved) {
+        FinalizeArgs f{T_saved, 1, M, r, 1.0f, nullptr, 0, 0, Gt, p.rp, scale};
+        QTRY(launch_finalize(f, s));
+    } else {
+        QTRY(run_T(X, A, M, K, r, scale, nullptr, Gt, p.rp, part, s));
+    }
+    // U = dY B  ->  gamma * U in bf16
+    {
+        const Split sp = skinny_split(M, N);
+        SkinnyArgs a{dY, B, part, M, r, N, N, r, sp.splits, sp.per};
+        QTRY(launch_skinny(true, false, a, s));
+        FinalizeArgs f{part, sp.splits, M, r, 1.0f, nullptr, 0, 0, Gu, p.rp, scale};
+        QTRY(launch_finalize(f, s));
+    }
+    // dB = dY^T (gamma T)
+    {
+        const Split sp = skinny_split(N, M);
+        SkinnyArgs a{dY, Gt, part, N, r, M, N, p.rp, sp.splits, sp.per};
+        QTRY(launch_skinny(false, false, a, s));
+        FinalizeArgs f{part, sp.splits, N, r, 1.0f, dB, 0, accumulate, nullptr, 0, 1.0f};
+        QTRY(launch_finalize(f, s));
+    }
+    // dX = dY W~ + (gamma U) A
+    if (dX) {
+        uint16_t* Ap = at<uint16_t>(ws, p.off_ap);
+        QTRY(launch_pad_copy(A, r, K, Ap, p.rp, K, s));
+        CUtensorMap m_act, m_packed, m_la, m_lb;
+        bool ok = make_map_2d(&m_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, 128,
+                              CU_TENSOR_MAP_SWIZZLE_128B) &&
+                  make_map_2d(&m_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->packed, K / 2, N, K / 2,
+                              128, 64, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                  make_map_2d(&m_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Gu, p.rp, M, p.rp * 2, 64,
+                              128, CU_TENSOR_MAP_SWIZZLE_128B) &&
+                  make_map_2d(&m_lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Ap, K, p.rp, K * 2, 64, 64,
+                              CU_TENSOR_MAP_SWIZZLE_128B);
+        if (!ok) return QLORA_ERR_CUDA;
+        GemmArgs g{};
+        g.scale_codes = w->scale_codes;
+        g.meta = w->meta_scale;
+        g.D = dX;
+        g.M = M;
+        g.Nw = N;
+        g.d_cols = K;
+        g.nkb = K / 64;
+        g.main_steps = static_cast<int>(cdiv(N, 64));
+        g.tail_steps = static_cast<int>(cdiv(r, 64));
+        g.r = r;
+        g.m_tiles = static_cast<int>(cdiv(M, gemm_tile_m()));
+        g.err = err;
+        g.tab = table();
+        QTRY(record(ev, true, s));
+        QTRY(launch_gemm(true, m_act, m_packed, m_la, m_lb, g, s));
+        QTRY(record(ev, false, s));
+    }
+    // dA^T = X^T (gamma U), written transposed into dA [r x K]
+    {
+        const Split sp = skinny_split(K, M);
+        SkinnyArgs a{X, Gu, part, K, r, M, K, p.rp, sp.splits, sp.per};
+        QTRY(launch_skinny(false, false, a, s));
+        FinalizeArgs f{part, sp.splits, K, r, 1.0f, dA, 1, accumulate, nullptr, 0, 1.0f};
+        QTRY(launch_finalize(f, s));
+    }
+    return QLORA_OK;
+}
+
+int qlora_linear_backward(const uint16_t* dY, const uint16_t* X, int64_t M,
+                          const qlora_nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r,
+                          float scale, const float* T_saved, uint16_t* dX, float* dA, float* dB,
+                          int accumulate, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+    return qlora_linear_backward_ex(dY, X, M, w, A, B, r, scale, T_saved, dX, dA, dB, accumulate,
+                                    ws, ws_bytes, stream, nullptr);
+}
+
+}  // extern "C"

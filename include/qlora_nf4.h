@@ -1,0 +1,244 @@
+/*
+ * qlora_nf4.h -- C ABI of libqlora_nf4.so: the frozen-NF4 linear layer with a
+ * bf16 LoRA adapter on one NVIDIA B200 (sm_100a).
+ *
+ * Method: "QLoRA, explained" (pofe.ai).  Storage follows its section "The
+ * math: what is stored and what is computed" (sub-sections "Blockwise absmax
+ * quantisation", "NormalFloat 4 (NF4)", "Double quantisation"); compute
+ * follows "The forward pass and gradients" and "The algorithm, step by step".
+ *
+ * Conventions for every entry point
+ *   - Every pointer argument named d_* or documented as "device" is device
+ *     memory owned by the caller; the library never allocates, frees or keeps
+ *     a pointer after the call returns.  Scratch space for the linear layer
+ *     is a caller-provided workspace whose size
+ *     qlora_linear_workspace_size() reports.
+ *   - bf16 tensors are passed as uint16_t* holding IEEE bfloat16 bit patterns
+ *     (the layout of __nv_bfloat16 and torch.bfloat16).
+ *   - All matrices are row-major and densely packed (row stride = columns).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All device
+ *     work is enqueued asynchronously on it; a call returns once its kernels
+ *     are launched.  Outputs are valid after the stream reaches that point.
+ *   - The return value is a qlora_status.  Argument errors are detected on
+ *     the host before anything is launched and leave every output untouched.
+ *     QLORA_ERR_CUDA reports a failed launch (cudaGetLastError()).
+ *   - The library holds no global state and no locks; calls on different
+ *     streams with disjoint outputs and workspaces may run concurrently.
+ */
+#ifndef QLORA_NF4_H
+#define QLORA_NF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define QLORA_API __attribute__((visibility("default")))
+#else
+#define QLORA_API
+#endif
+
+struct CUstream_st;                       /* == cudaStream_t's pointee */
+typedef struct CUstream_st* qlora_stream_t;
+
+typedef enum {
+    QLORA_OK = 0,
+    QLORA_ERR_NULL = 1,         /* a required pointer is NULL               */
+    QLORA_ERR_SHAPE = 2,        /* a size is negative or inconsistent       */
+    QLORA_ERR_ALIGN = 3,        /* a pointer is not 16-byte aligned         */
+    QLORA_ERR_UNSUPPORTED = 4,  /* a size outside what the kernels handle   */
+    QLORA_ERR_NONFINITE = 5,    /* non-finite weight seen by qlora_quantize */
+    QLORA_ERR_CUDA = 6,         /* a CUDA runtime call or launch failed     */
+    QLORA_ERR_WORKSPACE = 7     /* workspace pointer NULL or too small      */
+} qlora_status;
+
+/* Fixed format parameters ("Blockwise absmax quantisation": blocks of 64;
+ * "Double quantisation": one fp32 constant per 256 block scales). */
+#define QLORA_BLOCK 64
+#define QLORA_GROUP 256
+/* Largest LoRA rank the linear layer accepts; the rank must be a multiple of 8. */
+#define QLORA_MAX_RANK 128
+/* Token counts up to this go to the bandwidth-bound dequant-GEMV kernel. */
+#define QLORA_GEMV_MAX_TOKENS 16
+
+/*
+ * A stored NF4 tensor: a non-owning view of three device buffers.
+ *
+ * The logical tensor is W[rows][cols] (fp32 before quantisation), flattened
+ * in row-major order and cut into blocks of 64 consecutive elements
+ * (nblocks = ceil(rows*cols / 64)); blocks are grouped 256 at a time
+ * (ngroups = ceil(nblocks / 256)).
+ *   packed      : nblocks*32 bytes.  Byte j holds element 2j in its low
+ *                 nibble and element 2j+1 in its high nibble; each nibble is
+ *                 the index (0..15) of the element's nearest NF4 code.  The
+ *                 padding of a final partial block holds index 7, the code 0.
+ *   scale_codes : nblocks bytes.  The FP8 E4M3 (e4m3fn) code of block b's
+ *                 absmax c_b divided by its group's meta scale.
+ *   meta_scale  : ngroups fp32.  The group's largest c_b divided by 448.
+ * The dequantised weight is  w~ = bf16_rne( fp32( q[idx] * c~_b ) )  with
+ * c~_b = fp32( e4m3(scale_code_b) * meta_scale_g ).
+ */
+typedef struct {
+    uint8_t* packed;
+    uint8_t* scale_codes;
+    float* meta_scale;
+    int64_t rows;   /* N: output features of the linear layer */
+    int64_t cols;   /* K: input features                        */
+} qlora_nf4_tensor;
+
+/* Human-readable name of a qlora_status value (static string). */
+QLORA_API const char* qlora_status_string(int status);
+
+/*
+ * nf4_build_codebook -- the 16 NF4 codes and the 15 decision midpoints.
+ * "QLoRA, explained", "NormalFloat 4 (NF4)": codes at averages of adjacent
+ * standard-normal quantiles, halves of 8 and 9 levels sharing an exact zero,
+ * renormalised to [-1, 1].  Host only, deterministic, no CUDA call.
+ *   codes     (host, 16 floats, written): ascending; codes[0] = -1,
+ *             codes[7] = 0, codes[15] = 1.
+ *   midpoints (host, 15 floats, written): midpoints[i] is the exact average
+ *             of codes[i] and codes[i+1] rounded to nearest fp32.  An element
+ *             x maps to the number of midpoints strictly below it (a value
+ *             equal to a midpoint takes the lower code).
+ * Errors: QLORA_ERR_NULL if either pointer is NULL.
+ */
+QLORA_API int nf4_build_codebook(float codes[16], float midpoints[15]);
+
+/*
+ * qlora_quantized_sizes -- byte sizes of the three buffers of a stored
+ * rows x cols tensor (layout above).  Host only.
+ * Errors: QLORA_ERR_NULL (an output pointer NULL), QLORA_ERR_SHAPE (a
+ * negative size or rows*cols overflowing int64).
+ */
+QLORA_API int qlora_quantized_sizes(int64_t rows, int64_t cols, size_t* packed_bytes,
+                          size_t* codes_bytes, size_t* meta_bytes);
+
+/*
+ * qlora_quantize -- blockwise absmax NF4 quantisation plus double
+ * quantisation of the scales ("The algorithm, step by step": split into
+ * blocks of 64, absmax, nearest NF4 code of w / c_b, FP8 scales in groups of
+ * 256 with fp32 constants).
+ *   W     (device, fp32, rows*cols, read): the weight, row-major.
+ *   out   (host struct, read): rows, cols and the three device buffers to
+ *         write, sized by qlora_quantized_sizes.  All of them are written.
+ *   d_nonfinite_flag (device int, nullable): if given, the kernel stores a
+ *         non-zero value there when any element of W is NaN or +-Inf (it
+ *         never clears it; zero it first).  Outputs are then unspecified.
+ *         The host call cannot see device data, so it still returns
+ *         QLORA_OK; read the flag after synchronising the stream.
+ * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE, QLORA_ERR_ALIGN (W, packed not
+ * 16-byte aligned; meta_scale not 4-byte aligned), QLORA_ERR_CUDA.
+ */
+QLORA_API int qlora_quantize(const float* W, const qlora_nf4_tensor* out,
+                   int* d_nonfinite_flag, qlora_stream_t stream);
+
+/*
+ * qlora_dequantize -- dDQ of a whole stored tensor to bf16 ("The forward
+ * pass and gradients": dequantise the FP8 scales with the fp32 constants,
+ * then the NF4 indices with those scales, producing bf16 W~).
+ *   w     (host struct, read): the stored tensor.
+ *   W_out (device, bf16 bits, rows*cols, written): W~ row-major; bit-exact
+ *         to bf16_rne(fp32(q[idx] * c~_b)).
+ * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE, QLORA_ERR_ALIGN (W_out and packed
+ * 16-byte aligned), QLORA_ERR_CUDA.
+ */
+QLORA_API int qlora_dequantize(const qlora_nf4_tensor* w, uint16_t* W_out,
+                     qlora_stream_t stream);
+
+/*
+ * qlora_linear_workspace_size -- bytes of device workspace that
+ * qlora_linear_forward and qlora_linear_backward need for these sizes.
+ * M tokens, N = w.rows, K = w.cols, r the LoRA rank.  Host only.
+ * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE, QLORA_ERR_UNSUPPORTED (see the
+ * shape rules of qlora_linear_forward).
+ */
+QLORA_API int qlora_linear_workspace_size(int64_t M, int64_t N, int64_t K, int r,
+                                size_t* bytes);
+
+/*
+ * qlora_linear_forward -- Y = X W~^T + scale * (X A^T) B^T
+ * ("The forward pass and gradients"; "The algorithm, step by step", forward).
+ * W~ exists only tile by tile inside the kernels; it is never written out.
+ *   X      (device, bf16, M x K, read)
+ *   M      tokens, >= 0 (M = 0 launches nothing)
+ *   w      (host struct, read): the stored weight, rows = N, cols = K
+ *   A      (device, bf16, r x K, read): LoRA down-projection
+ *   B      (device, bf16, N x r, read): LoRA up-projection
+ *   r      LoRA rank: 8 <= r <= 128, r % 8 == 0
+ *   scale  gamma = alpha / r
+ *   Y      (device, bf16, M x N, written)
+ *   T_save (device, fp32, M x r, nullable, written): X A^T, for the backward
+ *   ws, ws_bytes (device workspace, >= qlora_linear_workspace_size bytes,
+ *          256-byte aligned); contents on entry are ignored.  After the
+ *          call its first 4 bytes hold the kernels' error word (0 = none;
+ *          bit 0 = a bounded wait inside the GEMM kernel expired, in which
+ *          case the outputs are unspecified).
+ *   M <= 16 runs the bandwidth-bound dequant-GEMV kernel, larger M the
+ *   tensor-core dequant-GEMM; both compute the same function.
+ * Shape rules: K % 64 == 0, N % 8 == 0, K >= 64, N >= 8.
+ * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE, QLORA_ERR_ALIGN (every tensor
+ * 16-byte aligned), QLORA_ERR_UNSUPPORTED, QLORA_ERR_WORKSPACE,
+ * QLORA_ERR_CUDA.
+ */
+QLORA_API int qlora_linear_forward(const uint16_t* X, int64_t M, const qlora_nf4_tensor* w,
+                         const uint16_t* A, const uint16_t* B, int r, float scale,
+                         uint16_t* Y, float* T_save, void* ws, size_t ws_bytes,
+                         qlora_stream_t stream);
+
+/*
+ * qlora_linear_backward -- gradients of the adapted layer with W~ frozen
+ * ("The forward pass and gradients": the input gradient dequantises the block
+ * a second time; the adapter gradients are LoRA's with W~ in place of W0; no
+ * gradient is formed for the stored NF4 weight).
+ *   dX = dY W~ + scale * (dY B) A          (bf16, M x K)
+ *   dA = scale * (dY B)^T X                (fp32, r x K)
+ *   dB = scale * dY^T (X A^T)              (fp32, N x r)
+ *   dY      (device, bf16, M x N, read)
+ *   X       (device, bf16, M x K, read)
+ *   T_saved (device, fp32, M x r, nullable): X A^T from the forward; NULL
+ *           recomputes it
+ *   dX      (device, bf16, M x K, nullable = not computed, written)
+ *   dA, dB  (device, fp32, written; accumulate != 0 adds to their contents)
+ *   other arguments as in qlora_linear_forward.
+ * Errors as qlora_linear_forward.
+ */
+QLORA_API int qlora_linear_backward(const uint16_t* dY, const uint16_t* X, int64_t M,
+                          const qlora_nf4_tensor* w, const uint16_t* A,
+                          const uint16_t* B, int r, float scale,
+                          const float* T_saved, uint16_t* dX, float* dA,
+                          float* dB, int accumulate, void* ws, size_t ws_bytes,
+                          qlora_stream_t stream);
+
+/*
+ * Profiling variants.  Identical to qlora_linear_forward / _backward, plus
+ * optional CUDA events (cudaEvent_t handles created by the caller, either may
+ * be NULL) that are recorded on `stream` immediately before and after the
+ * launch of the layer's main weight kernel: the tensor-core dequant-GEMM
+ * (forward Y, or dX in the backward), or the dequant-GEMV when M <= 16.  They
+ * let a caller time that kernel inside a running workload without a profiler.
+ * ev itself may be NULL.
+ */
+typedef struct {
+    void* gemm_begin;
+    void* gemm_end;
+} qlora_events;
+
+QLORA_API int qlora_linear_forward_ex(const uint16_t* X, int64_t M, const qlora_nf4_tensor* w,
+                                      const uint16_t* A, const uint16_t* B, int r, float scale,
+                                      uint16_t* Y, float* T_save, void* ws, size_t ws_bytes,
+                                      qlora_stream_t stream, const qlora_events* ev);
+
+QLORA_API int qlora_linear_backward_ex(const uint16_t* dY, const uint16_t* X, int64_t M,
+                                       const qlora_nf4_tensor* w, const uint16_t* A,
+                                       const uint16_t* B, int r, float scale,
+                                       const float* T_saved, uint16_t* dX, float* dA, float* dB,
+                                       int accumulate, void* ws, size_t ws_bytes,
+                                       qlora_stream_t stream, const qlora_events* ev);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QLORA_NF4_H */

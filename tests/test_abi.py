@@ -1,0 +1,113 @@
+"""CPU tests of the C-ABI library: it loads, exports every symbol the header
+declares, and its host-only entry points agree with the oracle.  No CUDA
+compute call is made here: the validation tests only reach paths that return
+before any launch."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import nf4_oracle as o
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qlora_nf4.h")
+
+
+@pytest.fixture(scope="module")
+def q():
+    import bit_nf4_quantised_b200 as pkg
+    pkg.lib()
+    return pkg
+
+
+def _declared():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"QLORA_API\s+[\w\s\*]+?\b(\w+)\s*\(", txt)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("nf4_build_codebook", "qlora_quantize", "qlora_dequantize",
+              "qlora_linear_forward", "qlora_linear_backward"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(q):
+    L = ctypes.CDLL(q._lib.LIB_PATH)
+    for n in _declared():
+        assert hasattr(L, n), n
+    assert set(_declared()) == set(q.EXPORTED)
+
+
+def test_host_codebook_bit_exact_with_oracle(q):
+    codes, mids = q.nf4_build_codebook()
+    oc, om = o.nf4_codebook()
+    assert np.array_equal(np.array(codes, np.float32).view(np.uint32), oc.view(np.uint32))
+    assert np.array_equal(np.array(mids, np.float32).view(np.uint32), om.view(np.uint32))
+
+
+@pytest.mark.parametrize("rows,cols", [(4096, 4096), (11008, 4096), (3, 100), (1, 1), (0, 5),
+                                       (28672, 8192), (7, 64 * 256 + 3)])
+def test_quantized_sizes_match_oracle(q, rows, cols):
+    assert q.qlora_quantized_sizes(rows, cols) == o.quantized_nbytes(rows * cols)
+
+
+def test_status_strings(q):
+    for s in range(8):
+        assert q.status_string(s)
+    assert "unknown" in q.status_string(99)
+
+
+def test_workspace_size_rules(q):
+    L = q.lib()
+    b = ctypes.c_size_t()
+    assert L.qlora_linear_workspace_size(64, 256, 512, 8, ctypes.byref(b)) == 0 and b.value > 0
+    assert L.qlora_linear_workspace_size(64, 256, 500, 8, ctypes.byref(b)) == q._lib.QLORA_ERR_UNSUPPORTED
+    assert L.qlora_linear_workspace_size(64, 250, 512, 8, ctypes.byref(b)) == q._lib.QLORA_ERR_UNSUPPORTED
+    assert L.qlora_linear_workspace_size(64, 256, 512, 12, ctypes.byref(b)) == q._lib.QLORA_ERR_UNSUPPORTED
+    assert L.qlora_linear_workspace_size(64, 256, 512, 136, ctypes.byref(b)) == q._lib.QLORA_ERR_UNSUPPORTED
+    assert L.qlora_linear_workspace_size(-1, 256, 512, 8, ctypes.byref(b)) == q._lib.QLORA_ERR_SHAPE
+    assert L.qlora_linear_workspace_size(64, 256, 512, 8, None) == q._lib.QLORA_ERR_NULL
+
+
+def test_argument_errors_return_before_any_launch(q):
+    """Bad arguments are rejected on the host (fake pointers never touched)."""
+    L = q.lib()
+    T = q._lib._Tensor
+    good = T(0x10000, 0x20000, 0x30000, 256, 512)
+    fake = 0x40000
+    ws_n = ctypes.c_size_t()
+    L.qlora_linear_workspace_size(64, 256, 512, 8, ctypes.byref(ws_n))
+    # null input
+    assert L.qlora_linear_forward(None, 64, ctypes.byref(good), fake, fake, 8, 2.0, fake, None,
+                                  fake, ws_n.value, None) == q._lib.QLORA_ERR_NULL
+    # misaligned X
+    assert L.qlora_linear_forward(fake + 2, 64, ctypes.byref(good), fake, fake, 8, 2.0, fake,
+                                  None, fake, ws_n.value, None) == q._lib.QLORA_ERR_ALIGN
+    # unsupported rank
+    assert L.qlora_linear_forward(fake, 64, ctypes.byref(good), fake, fake, 7, 2.0, fake, None,
+                                  fake, ws_n.value, None) == q._lib.QLORA_ERR_UNSUPPORTED
+    # workspace too small
+    assert L.qlora_linear_forward(fake, 64, ctypes.byref(good), fake, fake, 8, 2.0, fake, None,
+                                  fake, ws_n.value - 1, None) == q._lib.QLORA_ERR_WORKSPACE
+    # null tensor buffer
+    bad = T(0, 0x20000, 0x30000, 256, 512)
+    assert L.qlora_dequantize(ctypes.byref(bad), fake, None) == q._lib.QLORA_ERR_NULL
+    neg = T(0x10000, 0x20000, 0x30000, -1, 512)
+    assert L.qlora_quantize(fake, ctypes.byref(neg), None, None) == q._lib.QLORA_ERR_SHAPE
+    mis = T(0x10008, 0x20000, 0x30000, 256, 512)
+    assert L.qlora_quantize(fake, ctypes.byref(mis), None, None) == q._lib.QLORA_ERR_ALIGN
+    assert L.qlora_linear_backward(fake, fake, 64, ctypes.byref(good), fake, fake, 8, 2.0, None,
+                                   fake, None, fake, 0, fake, ws_n.value, None) == q._lib.QLORA_ERR_NULL
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    import bit_nf4_quantised_b200._lib as L
+    monkeypatch.setattr(L, "_LIB", None)
+    monkeypatch.setattr(L, "LIB_PATH", str(tmp_path / "nope.so"))
+    with pytest.raises(ImportError):
+        L.lib()

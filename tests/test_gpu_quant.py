@@ -1,0 +1,129 @@
+"""GPU parity of the storage kernels through the C-ABI: packed indices, FP8
+scale codes and meta scales bit-exact with the oracle, and the dequantised
+bf16 weight bit-exact."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import nf4_oracle as o
+from bit_nf4_quantised_b200 import synthetic as syn
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def q():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    import bit_nf4_quantised_b200 as pkg
+    pkg.lib()
+    return pkg
+
+
+def _gpu_store(q, W):
+    t = torch.from_numpy(np.ascontiguousarray(W, np.float32)).cuda()
+    if t.dim() == 1:
+        t = t.view(1, -1)
+    w = q.qlora_quantize(t)
+    torch.cuda.synchronize()
+    return w
+
+
+def _compare_store(q, W, numel=None):
+    w = _gpu_store(q, W)
+    packed, sc, meta = o.quantize(W)
+    gp = w.packed.cpu().numpy()
+    gs = w.scale_codes.cpu().numpy()
+    gm = w.meta_scale.cpu().numpy()
+    assert gp.shape == packed.shape and np.array_equal(gp, packed), \
+        f"packed differs at {np.flatnonzero(gp != packed)[:10]}"
+    assert np.array_equal(gs, sc), f"scale codes differ at {np.flatnonzero(gs != sc)[:10]}"
+    assert np.array_equal(gm.view(np.uint32), meta.view(np.uint32)), "meta scales differ"
+    # dequantised bf16, bit-exact
+    deq = q.qlora_dequantize(w)
+    torch.cuda.synchronize()
+    bits = deq.view(torch.int16).cpu().numpy().view(np.uint16).reshape(-1)
+    ref = o.dequantize_bits(packed, sc, meta, W.size)
+    assert np.array_equal(bits, ref), f"dequant differs at {np.flatnonzero(bits != ref)[:10]}"
+    return w
+
+
+def test_single_layer_weight(q):
+    lin = syn.WORKLOADS["single_256x512_m64_r8"].layers[0]
+    W = syn.make_weight(lin, np.random.default_rng(lin.seed))
+    _compare_store(q, W)
+
+
+@pytest.mark.parametrize("shape", [(3, 100), (1, 37), (1, 64), (2, 64 * 256 * 2 + 70),
+                                   (17, 1000), (64, 64 * 5)])
+def test_ragged_shapes(q, shape):
+    rng = np.random.default_rng(sum(shape))
+    W = rng.normal(0, 0.02, shape).astype(np.float32)
+    _compare_store(q, W)
+
+
+def test_edge_values(q):
+    """Zero blocks, an all-zero group, exact midpoint ties, tiny scale ratios
+    (subnormal FP8 codes) and sign patterns."""
+    codes, mids = o.nf4_codebook()
+    nblk = 256 * 3
+    W = np.random.default_rng(11).normal(0, 0.02, (nblk, 64)).astype(np.float32)
+    W[3] = 0.0                                       # zero block
+    W[256:512] = 0.0                                 # all-zero group
+    W[600, 0] = 1.0                                  # absmax 1: x = w exactly
+    W[600, 1:16] = mids                              # ties at every midpoint
+    W[600, 16:31] = np.nextafter(mids, np.float32(2))
+    W[600, 31:46] = np.nextafter(mids, np.float32(-2))
+    W[601] = np.float32(-0.5) * codes[np.arange(64) % 16]
+    W[700, 5] = 300.0                                # one huge block in the group
+    W[701:703] *= np.float32(0.1)                    # subnormal E4M3 scale codes
+    W[703:705] *= np.float32(1e-3)                   # scale codes that round to zero
+    W[705] = np.float32(1e-30)                       # near-underflow block
+    _compare_store(q, W.reshape(-1))
+
+
+def test_attn_projection_full(q):
+    lin = syn.WORKLOADS["llama7b_attn_proj_4096x4096_m4096_r16"].layers[0]
+    W = syn.make_weight(lin, np.random.default_rng(lin.seed))
+    _compare_store(q, W)
+
+
+def test_decode_weight_sampled_groups(q):
+    """28672 x 8192 weight quantised in full on the GPU; the oracle checks 24
+    sampled double-quantisation groups (whole groups, so its bytes are the
+    same as for the full tensor) plus the first and the last."""
+    lin = syn.WORKLOADS["decode_gemv_28672x8192_m1"].layers[0]
+    W = syn.make_weight(lin, np.random.default_rng(lin.seed))
+    w = _gpu_store(q, W)
+    deq = q.qlora_dequantize(w)
+    torch.cuda.synchronize()
+    flat = W.reshape(-1)
+    per_group = o.BLOCK * o.GROUP
+    ngroups = flat.size // per_group
+    rng = np.random.default_rng(5)
+    picks = sorted(set([0, ngroups - 1] + rng.integers(0, ngroups, 24).tolist()))
+    gp, gs, gm = w.packed, w.scale_codes, w.meta_scale
+    dbits = deq.view(-1).view(torch.int16)
+    for g in picks:
+        sub = flat[g * per_group:(g + 1) * per_group]
+        packed, sc, meta = o.quantize(sub)
+        assert np.array_equal(gp[g * per_group // 2:(g + 1) * per_group // 2].cpu().numpy(), packed)
+        assert np.array_equal(gs[g * o.GROUP:(g + 1) * o.GROUP].cpu().numpy(), sc)
+        assert gm[g].item() == float(meta[0])
+        ref = o.dequantize_bits(packed, sc, meta, sub.size)
+        got = dbits[g * per_group:(g + 1) * per_group].cpu().numpy().view(np.uint16)
+        assert np.array_equal(got, ref)
+
+
+def test_nonfinite_is_reported(q):
+    W = torch.ones(4, 128, device="cuda")
+    W[2, 5] = float("nan")
+    with pytest.raises(q.QloraError) as ei:
+        q.qlora_quantize(W)
+    assert ei.value.status == q._lib.QLORA_ERR_NONFINITE
+    W[2, 5] = float("inf")
+    with pytest.raises(q.QloraError):
+        q.qlora_quantize(W)
+    q.qlora_quantize(torch.ones(4, 128, device="cuda"))      # finite: no error
