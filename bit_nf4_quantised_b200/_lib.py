@@ -57,9 +57,15 @@ def _events(events):
     """(begin, end) torch.cuda.Event pair (timing enabled) -> qlora_events*."""
     if events is None:
         return None
-    b, e = events
-    return ctypes.byref(_Events(b.cuda_event if b is not None else None,
-                                e.cuda_event if e is not None else None))
+    handles = []
+    for ev in events:
+        if ev is None:
+            handles.append(None)
+            continue
+        if not ev.cuda_event:          # torch creates the CUDA event on first record
+            ev.record()
+        handles.append(ev.cuda_event)
+    return ctypes.byref(_Events(*handles))
 
 
 class _Tensor(ctypes.Structure):

@@ -72,7 +72,10 @@ gemv_kernel(GemvArgs a, int x_pitch_bytes) {
         const int m = q / vec_per_row, v = q % vec_per_row;
         uint4 val = make_uint4(0, 0, 0, 0);
         if (m < a.M) val = *reinterpret_cast<const uint4*>(a.X + m * a.K + k_beg + v * 8);
-        *reinterpret_cast<uint4*>(sx + m * x_pitch_bytes + v * 16) = val;
+        // rows are 8-byte aligned only (pitch = 8 mod 16): two 8-byte stores
+        uint2* dst = reinterpret_cast<uint2*>(sx + m * x_pitch_bytes + v * 16);
+        dst[0] = make_uint2(val.x, val.y);
+        dst[1] = make_uint2(val.z, val.w);
     }
     __syncthreads();
 

@@ -283,7 +283,8 @@ int qlora_linear_forward_ex(const uint16_t* X, int64_t M, const qlora_nf4_tensor
                             const uint16_t* A, const uint16_t* B, int r, float scale, uint16_t* Y,
                             float* T_save, void* ws, size_t ws_bytes, qlora_stream_t stream,
                             const qlora_events* ev) {
-    if (!X || !A || !B || !Y) return QLORA_ERR_NULL;
+    // an empty batch may come with NULL activation pointers
+    if (!A || !B || (M != 0 && (!X || !Y))) return QLORA_ERR_NULL;
     int st = check_tensor(w);
     if (st != QLORA_OK) return st;
     const int64_t N = w->rows, K = w->cols;
@@ -359,7 +360,7 @@ int qlora_linear_backward_ex(const uint16_t* dY, const uint16_t* X, int64_t M,
                              int r, float scale, const float* T_saved, uint16_t* dX, float* dA,
                              float* dB, int accumulate, void* ws, size_t ws_bytes,
                              qlora_stream_t stream, const qlora_events* ev) {
-    if (!dY || !X || !A || !B || !dA || !dB) return QLORA_ERR_NULL;
+    if (!A || !B || !dA || !dB || (M != 0 && (!dY || !X))) return QLORA_ERR_NULL;
     int st = check_tensor(w);
     if (st != QLORA_OK) return st;
     const int64_t N = w->rows, K = w->cols;

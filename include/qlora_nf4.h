@@ -163,7 +163,7 @@ QLORA_API int qlora_linear_workspace_size(int64_t M, int64_t N, int64_t K, int r
  * ("The forward pass and gradients"; "The algorithm, step by step", forward).
  * W~ exists only tile by tile inside the kernels; it is never written out.
  *   X      (device, bf16, M x K, read)
- *   M      tokens, >= 0 (M = 0 launches nothing)
+ *   M      tokens, >= 0 (M = 0 launches nothing; X and Y may then be NULL)
  *   w      (host struct, read): the stored weight, rows = N, cols = K
  *   A      (device, bf16, r x K, read): LoRA down-projection
  *   B      (device, bf16, N x r, read): LoRA up-projection
@@ -202,6 +202,8 @@ QLORA_API int qlora_linear_forward(const uint16_t* X, int64_t M, const qlora_nf4
  *           recomputes it
  *   dX      (device, bf16, M x K, nullable = not computed, written)
  *   dA, dB  (device, fp32, written; accumulate != 0 adds to their contents)
+ *   M = 0 writes zero gradients (or leaves them unchanged when accumulating);
+ *   dY and X may then be NULL.
  *   other arguments as in qlora_linear_forward.
  * Errors as qlora_linear_forward.
  */
