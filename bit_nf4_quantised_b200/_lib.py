@@ -40,6 +40,7 @@ EXPORTED = (
     "qlora_linear_backward",
     "qlora_linear_forward_ex",
     "qlora_linear_backward_ex",
+    "qlora_linear_forward_noalloc",
 )
 
 

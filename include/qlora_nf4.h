@@ -240,6 +240,30 @@ QLORA_API int qlora_linear_backward_ex(const uint16_t* dY, const uint16_t* X, in
                                        int accumulate, void* ws, size_t ws_bytes,
                                        qlora_stream_t stream, const qlora_events* ev);
 
+/*
+ * qlora_linear_forward_noalloc -- qlora_linear_forward for callers that cannot
+ * allocate device memory.  The paper has no counterpart to this entry point;
+ * it exists for callers such as plug-ins inside a host framework that owns
+ * every device allocation and exposes no allocator, or deployments that ban
+ * device allocation after start-up, which therefore cannot hand over the
+ * workspace qlora_linear_forward needs.
+ *   Same arguments and result as qlora_linear_forward, without ws/ws_bytes:
+ *   the scratch is a fixed 16 MiB device array inside this library, present
+ *   on every GPU that loads it until the process exits.  No cudaMalloc,
+ *   cudaFree or other allocating routine is called.
+ *   The first call on a device looks up that array's device address with
+ *   cudaGetSymbolAddress (the device must be current); make that first call
+ *   before any stream capture.  Every call on a device shares the one array:
+ *   calls that may overlap on the GPU (unordered streams) race on it.
+ * Errors: as qlora_linear_forward; QLORA_ERR_WORKSPACE when these sizes need
+ * more than the 16 MiB array (qlora_linear_workspace_size reports the need);
+ * QLORA_ERR_CUDA if the address lookup fails.
+ */
+QLORA_API int qlora_linear_forward_noalloc(const uint16_t* X, int64_t M,
+                                           const qlora_nf4_tensor* w, const uint16_t* A,
+                                           const uint16_t* B, int r, float scale, uint16_t* Y,
+                                           float* T_save, qlora_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
