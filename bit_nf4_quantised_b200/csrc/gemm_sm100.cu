@@ -1,5 +1,5 @@
 // K2/K3: fused NF4 dequant-GEMM on the 5th-generation tensor cores (tcgen05,
-// accumulators in TMEM), with the LoRA term folded into the same accumulator.
+// accumulators in TMEM), with the LoRA term folded into the same accumulators.
 //
 //   forward (kTrans = false):  Y  = X  W~^T + (gamma T) B^T        D = [M x N]
 //   input grad (kTrans = true): dX = dY W~  + (gamma U) A          D = [M x K]
@@ -8,51 +8,63 @@
 // block from the stored NF4 indices and double-quantised scales, exists only
 // transiently, and is produced a second time for the input gradient.
 //
-// Design (one CTA per 128 x 256 output tile, 320 threads, warp-specialised):
-//   warp 0      TMA producer: the activation tile (X or dY, 128 x 64 bf16,
-//               128-byte swizzle) and the packed-nibble tile of W for each
-//               64-wide contraction step, into a 3-stage shared-memory ring.
-//   warps 2..9  dequantisers: one thread per 64-element NF4 block per step.
-//               A thread builds its block's 16-entry table of
-//               bf16_rne(fp32(q[i] * c~)) once, then maps each nibble to its
-//               bf16 with byte permutes (no per-element multiply or memory
-//               lookup), and stores the row straight into the swizzled
-//               operand layout tcgen05 reads: K-major rows of W~ for the
-//               forward, MN-major rows (W~ untransposed) for dX, so the
-//               "transposed dequant" is only a different descriptor.
-//   warp 1      MMA issuer: 4 x tcgen05.mma (128 x 256 x 16) per step into a
-//               128 x 256 fp32 TMEM accumulator; tcgen05.commit frees the
-//               stage.  After the K loop, ceil(r/64) extra steps feed
+// Design: a cluster of two CTAs on two SMs computes a 512 x 256 output tile
+// with the pair MMA (tcgen05.mma.cta_group::2, 256 x 256 x 16): each CTA holds
+// 128 of every 256 tokens (A operand) and 128 of the 256 output columns
+// (B operand, its half of the W~ tile), and two accumulators of 128 lanes x
+// 256 fp32 columns fill its 512-column TMEM.  One dequantised W~ element thus
+// feeds 512 tokens, and each SM expands only half of the tile: this is what
+// keeps the dequantisation (integer/permute work on the CUDA cores) below the
+// tensor-core rate.
+//   warp 0      TMA producer: two 128 x 64 activation tiles (X or dY, 128-byte
+//               swizzle) per 64-wide contraction step, counted on the even
+//               CTA's barrier, and this CTA's packed-nibble tile (32- or
+//               64-byte swizzle, so the dequantisers read it conflict-free),
+//               counted locally; 4-stage ring.
+//   warps 2..9  dequantisers in two groups of four that take alternate steps:
+//               one thread per 64-element NF4 block of this CTA's B half.  A
+//               thread builds its block's 16-entry table of
+//               bf16_rne(fp32(q[i] * c~)) once, maps each nibble to its bf16
+//               with byte permutes, and stores the row straight into the
+//               swizzled operand layout tcgen05 reads: K-major rows of W~ for
+//               the forward, MN-major rows (W~ untransposed) for dX, so the
+//               "transposed dequant" is only a different descriptor.  Each
+//               warp then signals the even CTA's barrier.
+//   warp 1      TMEM allocation (both CTAs); on the even CTA the MMA issuer:
+//               8 pair MMAs per step, tcgen05.commit multicast to both CTAs
+//               frees the stage.  After the K loop ceil(r/64) extra steps feed
 //               (gamma T | gamma U) and (B | A) by TMA into the same ring and
-//               accumulator: the LoRA term costs no separate pass over Y.
+//               accumulators: the LoRA term costs no separate pass over Y.
 //   warps 2..9  then drain TMEM (tcgen05.ld), round to bf16 and store.
-// Every mbarrier wait is bounded (see common.cuh); on a timeout the kernel
-// records an error word, lets in-flight copies and MMAs land, frees TMEM and
-// returns.
+// Every mbarrier wait is bounded (common.cuh); on a timeout the kernel records
+// an error word, lets in-flight copies and MMAs land, frees TMEM and returns.
 #include "kernels.cuh"
 
 namespace qnf4 {
 
 namespace {
 
-constexpr int BM = 128;            // tokens per tile (MMA M)
-constexpr int BN = 256;            // output columns per tile (MMA N)
+constexpr int kTileM = 512;        // tokens per pair tile (2 accumulators x 256)
+constexpr int kTileN = 256;        // output columns per pair tile (MMA N)
+constexpr int kHalfN = kTileN / 2; // B rows held by each CTA
 constexpr int BK = 64;             // contraction per pipeline step (one NF4 block)
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kThreads = 320;
-constexpr int kDeqThreads = 256;
-constexpr int kSA = BM * BK * 2;   // 16 KiB activation tile
-constexpr int kSB = BN * BK * 2;   // 32 KiB W~ (or LoRA) tile
-constexpr int kSP = BN * BK / 2;   //  8 KiB packed nibbles
+constexpr int kGroupThreads = 128; // dequantisers per step group
+constexpr int kSA1 = 128 * BK * 2; // 16 KiB: one 128-row activation tile
+constexpr int kSA = 2 * kSA1;      // both accumulators' activation tiles
+constexpr int kSB = kHalfN * BK * 2;   // 16 KiB: this CTA's half of W~ (or LoRA)
+constexpr int kSP = kHalfN * BK / 2;   //  4 KiB: packed nibbles of that half
 constexpr int kStageBytes = kSA + kSB + kSP;
-constexpr int kTmemCols = 256;
+constexpr int kTmemCols = 512;
 static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
 
 struct __align__(8) Barriers {
-    uint64_t full_tma[kStages];
-    uint64_t full_deq[kStages];
-    uint64_t empty[kStages];
-    uint64_t acc_full;
+    uint64_t a_full[kStages];      // even CTA: both CTAs' TMA bytes of a stage
+    uint64_t pk_full[kStages];     // local: this CTA's packed tile
+    uint64_t deq_full[kStages];    // even CTA: 8 dequant warps of the pair
+    uint64_t empty[kStages];       // local: MMAs of the stage done
+    uint64_t acc_full;             // local: all MMAs done
     uint64_t drain;
     uint32_t tmem_slot;
     int abort_flag;
@@ -76,6 +88,8 @@ __device__ __forceinline__ void dequant_block_to_smem(const uint32_t (&w)[8], fl
         lo_plane[p] = prmt(t2[2 * p], t2[2 * p + 1], 0x6420u);
         hi_plane[p] = prmt(t2[2 * p], t2[2 * p + 1], 0x7531u);
     }
+    // chunk c lands at (c ^ swz) * 16 = row_addr ^ (c << 4) with swz folded in
+    const uint32_t base = row_addr | (swz << 4);
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
         const uint32_t v = w[c];
@@ -95,7 +109,7 @@ __device__ __forceinline__ void dequant_block_to_smem(const uint32_t (&w)[8], fl
             o[2 * h] = prmt(lo, hi, 0x5140u);
             o[2 * h + 1] = prmt(lo, hi, 0x7362u);
         }
-        const uint32_t dst = row_addr + ((static_cast<uint32_t>(c) ^ swz) << 4);
+        const uint32_t dst = base ^ (static_cast<uint32_t>(c) << 4);
         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(o[0]), "r"(o[1]),
                      "r"(o[2]), "r"(o[3])
                      : "memory");
@@ -116,16 +130,20 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
     volatile int* abort_flag = &bars->abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m_tile = blockIdx.x % a.m_tiles;
-    const int n_tile = blockIdx.x / a.m_tiles;
-    const int m0 = m_tile * BM;
-    const int n0 = n_tile * BN;          // first output column of this tile
+    const uint32_t rank = cluster_ctarank();          // 0 = even CTA (issues the MMAs)
+    const int pair = blockIdx.x >> 1;
+    const int m_tile = pair % a.m_tiles;
+    const int n_tile = pair / a.m_tiles;
+    const int m0 = m_tile * kTileM;
+    const int n0 = n_tile * kTileN;                   // first output column of the pair tile
+    const int nh0 = n0 + static_cast<int>(rank) * kHalfN;   // this CTA's B half
     const int total_steps = a.main_steps + a.tail_steps;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&bars->full_tma[s], 1);
-            mbar_init(&bars->full_deq[s], kDeqThreads / 32);
+            mbar_init(&bars->a_full[s], 1);
+            mbar_init(&bars->pk_full[s], 1);
+            mbar_init(&bars->deq_full[s], 2 * kGroupThreads / 32);
             mbar_init(&bars->empty[s], 1);
         }
         mbar_init(&bars->acc_full, 1);
@@ -138,10 +156,10 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
         prefetch_tensormap(&tm_lora_b);
     }
     if (warp == 1) {
-        tmem_alloc(&bars->tmem_slot, kTmemCols);
+        tmem_alloc_pair(&bars->tmem_slot, kTmemCols);
         tc_fence_before();
     }
-    __syncthreads();
+    cluster_sync();                                   // barrier inits visible pair-wide
     tc_fence_after();
     const uint32_t tmem_d = bars->tmem_slot;
 
@@ -157,44 +175,52 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
                 uint8_t* sA = smem + s * kStageBytes;
                 uint8_t* sB = sA + kSA;
                 uint8_t* sP = sB + kSB;
+                const uint32_t a_full0 = mapa_shared(smem_u32(&bars->a_full[s]), 0);
+                const int arow = m0 + static_cast<int>(rank) * 128;
                 if (step < a.main_steps) {
-                    mbar_arrive_expect_tx(&bars->full_tma[s], kSA + kSP);
-                    tma_load_2d(sA, &tm_act, step * BK, m0, &bars->full_tma[s]);
+                    if (rank == 0) mbar_arrive_expect_tx(&bars->a_full[s], 2 * kSA);
+                    tma_load_2d_pair(sA, &tm_act, step * BK, arow, a_full0);
+                    tma_load_2d_pair(sA + kSA1, &tm_act, step * BK, arow + 256, a_full0);
+                    mbar_arrive_expect_tx(&bars->pk_full[s], kSP);
                     if (!kTrans)
-                        tma_load_2d(sP, &tm_packed, step * (BK / 2), n0, &bars->full_tma[s]);
+                        tma_load_2d(sP, &tm_packed, step * (BK / 2), nh0, &bars->pk_full[s]);
                     else
-                        tma_load_2d(sP, &tm_packed, n0 / 2, step * BK, &bars->full_tma[s]);
+                        tma_load_2d(sP, &tm_packed, nh0 / 2, step * BK, &bars->pk_full[s]);
+                    armed[s] = static_cast<int>(ph);
                 } else {
                     const int j = step - a.main_steps;
-                    mbar_arrive_expect_tx(&bars->full_tma[s], kSA + kSB);
-                    tma_load_2d(sA, &tm_lora_a, j * BK, m0, &bars->full_tma[s]);
+                    if (rank == 0) mbar_arrive_expect_tx(&bars->a_full[s], 2 * (kSA + kSB));
+                    tma_load_2d_pair(sA, &tm_lora_a, j * BK, arow, a_full0);
+                    tma_load_2d_pair(sA + kSA1, &tm_lora_a, j * BK, arow + 256, a_full0);
                     if (!kTrans) {
-                        tma_load_2d(sB, &tm_lora_b, j * BK, n0, &bars->full_tma[s]);
+                        tma_load_2d_pair(sB, &tm_lora_b, j * BK, nh0, a_full0);
                     } else {
-#pragma unroll
-                        for (int c = 0; c < BN / 64; ++c)
-                            tma_load_2d(sB + c * (64 * 128), &tm_lora_b, n0 + 64 * c, j * BK,
-                                        &bars->full_tma[s]);
+                        tma_load_2d_pair(sB, &tm_lora_b, nh0, j * BK, a_full0);
+                        tma_load_2d_pair(sB + 64 * 128, &tm_lora_b, nh0 + 64, j * BK, a_full0);
                     }
                 }
-                armed[s] = static_cast<int>(ph);
             }
             if (*abort_flag) {
                 for (int s = 0; s < kStages; ++s)
-                    if (armed[s] >= 0) mbar_drain(&bars->full_tma[s], armed[s], a.err);
+                    if (armed[s] >= 0) mbar_drain(&bars->pk_full[s], armed[s], a.err);
+                // copies counted on the even CTA's barrier cannot be awaited
+                // here: give them time to land before the CTA exits
+                const unsigned long long t0 = globaltimer_ns();
+                while (globaltimer_ns() - t0 < 50000ull) {
+                }
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, false, kTrans);
+        if (rank == 0 && lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16_f32(256, kTileN, false, kTrans);
             bool ok = true;
             for (int step = 0; step < total_steps && ok; ++step) {
                 const int s = step % kStages;
                 const uint32_t ph = (step / kStages) & 1;
                 const bool main = step < a.main_steps;
-                ok = mbar_wait(&bars->full_tma[s], ph, abort_flag, a.err);
-                if (ok && main) ok = mbar_wait(&bars->full_deq[s], ph, abort_flag, a.err);
+                ok = mbar_wait_cluster(&bars->a_full[s], ph, abort_flag, a.err);
+                if (ok && main) ok = mbar_wait_cluster(&bars->deq_full[s], ph, abort_flag, a.err);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t a_base = smem_u32(smem + s * kStageBytes);
@@ -205,92 +231,106 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
                     nk = min(BK / 16, (rem + 15) / 16);
                 }
                 for (int kk = 0; kk < nk; ++kk) {
-                    const uint64_t adesc = smem_desc_sw128(a_base + kk * 32, 16, 1024);
                     const uint64_t bdesc =
                         kTrans ? smem_desc_sw128(b_base + kk * 2048, 64 * 128, 1024)
                                : smem_desc_sw128(b_base + kk * 32, 16, 1024);
-                    tc_mma_bf16(tmem_d, adesc, bdesc, idesc, (step | kk) != 0 ? 1u : 0u);
+#pragma unroll
+                    for (int acc = 0; acc < 2; ++acc) {
+                        const uint64_t adesc =
+                            smem_desc_sw128(a_base + acc * kSA1 + kk * 32, 16, 1024);
+                        tc_mma_bf16_pair(tmem_d + acc * kTileN, adesc, bdesc, idesc,
+                                         (step | kk) != 0 ? 1u : 0u);
+                    }
                 }
-                tc_commit(&bars->empty[s]);
+                tc_commit_pair(&bars->empty[s], 0x3);
             }
             if (ok) {
-                tc_commit(&bars->acc_full);
+                tc_commit_pair(&bars->acc_full, 0x3);
+                mbar_drain(&bars->acc_full, 0, a.err);       // MMAs done before teardown
             } else {
-                tc_commit(&bars->drain);           // let issued MMAs finish before exit
+                tc_commit_pair(&bars->drain, 0x1);
                 mbar_drain(&bars->drain, 0, a.err);
             }
         }
     } else {
         // ------------------------------------------------- dequantisers
-        const int t = threadIdx.x - 64;            // 0..255
-        const uint32_t swz = static_cast<uint32_t>(t & 7);
-        // fwd: row n0+t of W, block = step.   dX: row step*64+(t&63), block k0/64+(t>>6).
+        const int group = (warp - 2) >> 2;                      // takes steps group, group+2, ...
+        const int t = ((warp - 2) & 3) * 32 + lane;             // 0..127
         const int64_t nkb = a.nkb;
-        const int kb_fixed = (n0 >> 6) + (t >> 6);
-        auto code_index = [&](int step, int64_t& ci) -> bool {
-            if (!kTrans) {
-                const int64_t n = int64_t(n0) + t;
-                ci = n * nkb + step;
-                return n < a.Nw;
-            } else {
-                const int64_t n = int64_t(step) * BK + (t & 63);
-                ci = n * nkb + kb_fixed;
-                return n < a.Nw && kb_fixed < nkb;
-            }
-        };
-        auto load_scale = [&](int step, uint32_t& code, float& meta) {
-            int64_t ci;
+        // forward: row nh0+t of W, block = step.
+        // dX: row step*64 + (t & 63) of W, block nh0/64 + (t >> 6).
+        const int nr = t & 63, kbl = t >> 6;
+        const int64_t kb_fixed = (nh0 >> 6) + kbl;
+        auto scale_of = [&](int step, uint32_t& code, float& meta) {
             code = 0;
             meta = 0.f;
-            if (step < a.main_steps && code_index(step, ci)) {
-                code = __ldg(a.scale_codes + ci);
-                meta = __ldg(a.meta + (ci >> 8));
+            if (step >= a.main_steps) return;
+            int64_t n, ci;
+            if (!kTrans) {
+                n = int64_t(nh0) + t;
+                ci = n * nkb + step;
+                if (n >= a.Nw) return;
+            } else {
+                n = int64_t(step) * BK + nr;
+                ci = n * nkb + kb_fixed;
+                if (n >= a.Nw || kb_fixed >= nkb) return;
             }
+            code = __ldg(a.scale_codes + ci);
+            meta = __ldg(a.meta + (ci >> 8));
         };
         uint32_t code_cur, code_next;
         float meta_cur, meta_next;
-        load_scale(0, code_cur, meta_cur);
-        load_scale(1, code_next, meta_next);
-        const uint32_t prow_off = kTrans ? static_cast<uint32_t>((t & 63) * 128 + (t >> 6) * 32)
-                                         : static_cast<uint32_t>(t * 32);
-        const uint32_t brow_off =
-            kTrans ? static_cast<uint32_t>((t >> 6) * (64 * 128) + (t & 63) * 128)
-                   : static_cast<uint32_t>(t * 128);
-        for (int step = 0; step < a.main_steps; ++step) {
+        scale_of(group, code_cur, meta_cur);
+        scale_of(group + 2, code_next, meta_next);
+        uint32_t p_off0, p_off1, b_off, swz;
+        if (!kTrans) {
+            const uint32_t x = static_cast<uint32_t>((t >> 2) & 1);       // 32-byte swizzle
+            p_off0 = t * 32 + ((0u ^ x) << 4);
+            p_off1 = t * 32 + ((1u ^ x) << 4);
+            b_off = t * 128;
+            swz = t & 7;
+        } else {
+            const uint32_t x = static_cast<uint32_t>((nr >> 1) & 3);      // 64-byte swizzle
+            p_off0 = nr * 64 + (((2u * kbl) ^ x) << 4);
+            p_off1 = nr * 64 + (((2u * kbl + 1u) ^ x) << 4);
+            b_off = kbl * (64 * 128) + nr * 128;
+            swz = nr & 7;
+        }
+        for (int step = group; step < a.main_steps; step += 2) {
             const int s = step % kStages;
             const uint32_t ph = (step / kStages) & 1;
-            if (!mbar_wait(&bars->full_tma[s], ph, abort_flag, a.err)) break;
+            if (!mbar_wait(&bars->pk_full[s], ph, abort_flag, a.err)) break;
             const uint32_t sbase = smem_u32(smem + s * kStageBytes);
-            const uint32_t prow = sbase + kSA + kSB + prow_off;
+            const uint32_t pbase = sbase + kSA + kSB;
             uint32_t w[8];
             asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                          : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                         : "r"(prow));
+                         : "r"(pbase + p_off0));
             asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                          : "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
-                         : "r"(prow + 16));
+                         : "r"(pbase + p_off1));
             const float ct = __fmul_rn(e4m3_to_float(static_cast<uint8_t>(code_cur)), meta_cur);
-            dequant_block_to_smem(w, ct, a.tab, sbase + kSA + brow_off, swz);
+            dequant_block_to_smem(w, ct, a.tab, sbase + kSA + b_off, swz);
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->full_deq[s]);
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&bars->deq_full[s]), 0));
             code_cur = code_next;
             meta_cur = meta_next;
-            load_scale(step + 2, code_next, meta_next);
+            scale_of(step + 4, code_next, meta_next);
         }
 
         // -------------------------------------------------- epilogue
         if (mbar_wait(&bars->acc_full, 0, abort_flag, a.err)) {
             tc_fence_after();
             const int q = warp & 3;                 // TMEM lane quarter of this warp
-            const int half = (warp - 2) >> 2;       // which 128 columns
-            const int64_t m = int64_t(m0) + q * 32 + lane;
+            const int acc = group;                  // accumulator drained by this warp
+            const int64_t m = int64_t(m0) + acc * 256 + rank * 128 + q * 32 + lane;
             uint16_t* drow = a.D + m * a.d_cols;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                const int col = half * 128 + c * 32;
+            for (int c = 0; c < kTileN / 32; ++c) {
+                const int col = c * 32;
                 uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + col, r);
+                tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + acc * kTileN + col, r);
                 tc_wait_ld();
                 uint32_t p[16];
 #pragma unroll
@@ -310,11 +350,33 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
     }
 
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_d, kTmemCols);
+        tmem_dealloc_pair(tmem_d, kTmemCols);
     }
+}
+
+template <bool kTrans>
+cudaError_t launch_one(const CUtensorMap& act, const CUtensorMap& packed, const CUtensorMap& la,
+                       const CUtensorMap& lb, const GemmArgs& args, unsigned pairs,
+                       cudaStream_t stream) {
+    cudaError_t e = cudaFuncSetAttribute(qlora_gemm_kernel<kTrans>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * pairs);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, qlora_gemm_kernel<kTrans>, act, packed, la, lb, args);
 }
 
 }  // namespace
@@ -322,27 +384,23 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
 cudaError_t launch_gemm(bool trans, const CUtensorMap& act, const CUtensorMap& packed,
                         const CUtensorMap& lora_a, const CUtensorMap& lora_b, const GemmArgs& args,
                         cudaStream_t stream) {
-    const int64_t d_tiles = (args.d_cols + BN - 1) / BN;
-    const int64_t grid = int64_t(args.m_tiles) * d_tiles;
-    if (grid <= 0) return cudaSuccess;
-    if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    if (!trans) {
-        cudaError_t e = cudaFuncSetAttribute(qlora_gemm_kernel<false>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e != cudaSuccess) return e;
-        qlora_gemm_kernel<false><<<dim3(static_cast<unsigned>(grid)), kThreads, kSmemBytes, stream>>>(
-            act, packed, lora_a, lora_b, args);
-    } else {
-        cudaError_t e = cudaFuncSetAttribute(qlora_gemm_kernel<true>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e != cudaSuccess) return e;
-        qlora_gemm_kernel<true><<<dim3(static_cast<unsigned>(grid)), kThreads, kSmemBytes, stream>>>(
-            act, packed, lora_a, lora_b, args);
-    }
+    const int64_t n_tiles = (args.d_cols + kTileN - 1) / kTileN;
+    const int64_t pairs = int64_t(args.m_tiles) * n_tiles;
+    if (pairs <= 0) return cudaSuccess;
+    if (2 * pairs > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const cudaError_t e =
+        trans ? launch_one<true>(act, packed, lora_a, lora_b, args, unsigned(pairs), stream)
+              : launch_one<false>(act, packed, lora_a, lora_b, args, unsigned(pairs), stream);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
-int gemm_tile_m() { return BM; }
-int gemm_tile_n() { return BN; }
+int gemm_tile_m() { return kTileM; }
+int gemm_tile_n() { return kTileN; }
+// TMA boxes the host must encode for the packed-weight map of this kernel:
+// forward {32 bytes, 128 rows} with 32-byte swizzle; dX {64 bytes, 64 rows}
+// with 64-byte swizzle.  The LoRA B-operand box is 128 rows (forward) or
+// 64 x 64 (dX); activation boxes are {64, 128} with 128-byte swizzle.
+int gemm_half_n() { return kHalfN; }
 
 }  // namespace qnf4

@@ -35,8 +35,9 @@ struct GemmArgs {
 cudaError_t launch_gemm(bool trans, const CUtensorMap& act, const CUtensorMap& packed,
                         const CUtensorMap& lora_a, const CUtensorMap& lora_b, const GemmArgs& args,
                         cudaStream_t stream);
-int gemm_tile_m();
-int gemm_tile_n();
+int gemm_tile_m();   // tokens per output tile (a CTA pair)
+int gemm_tile_n();   // output columns per output tile
+int gemm_half_n();   // output columns whose W~ rows each CTA of the pair expands
 
 // -------------------------------------------------------------- K4 (LoRA)
 // part[s][i][j] = sum over the s-th contraction slice of P(i,c) * Q(c,j), fp32.

@@ -322,11 +322,11 @@ int qlora_linear_forward_ex(const uint16_t* X, int64_t M, const qlora_nf4_tensor
     bool ok = make_map_2d(&m_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 128,
                           CU_TENSOR_MAP_SWIZZLE_128B) &&
               make_map_2d(&m_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->packed, K / 2, N, K / 2, 32,
-                          256, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                          gemm_half_n(), CU_TENSOR_MAP_SWIZZLE_32B) &&
               make_map_2d(&m_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Gt, p.rp, M, p.rp * 2, 64, 128,
                           CU_TENSOR_MAP_SWIZZLE_128B) &&
-              make_map_2d(&m_lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Bp, p.rp, N, p.rp * 2, 64, 256,
-                          CU_TENSOR_MAP_SWIZZLE_128B);
+              make_map_2d(&m_lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Bp, p.rp, N, p.rp * 2, 64,
+                          gemm_half_n(), CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return QLORA_ERR_CUDA;
     GemmArgs g{};
     g.scale_codes = w->scale_codes;
@@ -419,7 +419,7 @@ int qlora_linear_backward_ex(const uint16_t* dY, const uint16_t* X, int64_t M,
         bool ok = make_map_2d(&m_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, 128,
                               CU_TENSOR_MAP_SWIZZLE_128B) &&
                   make_map_2d(&m_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->packed, K / 2, N, K / 2,
-                              128, 64, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                              gemm_half_n() / 2, 64, CU_TENSOR_MAP_SWIZZLE_64B) &&
                   make_map_2d(&m_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Gu, p.rp, M, p.rp * 2, 64,
                               128, CU_TENSOR_MAP_SWIZZLE_128B) &&
                   make_map_2d(&m_lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Ap, K, p.rp, K * 2, 64, 64,
