@@ -36,11 +36,10 @@ if ROOT not in sys.path:
 WORKLOAD = "llama7b_attn_proj_4096x4096_m4096_r16"
 GEMV_WORKLOAD = "decode_gemv_28672x8192_m1"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# Kernels the library launches per step (forward: LoRA T product, its
-# finalize, B padding, dequant-GEMM; backward: gamma*T conversion, U product
-# + finalize, dB product + finalize, A padding, dequant-GEMM dX, dA product +
-# finalize).  The memsets of the workspace error word are runtime memsets.
-LAUNCHES_PER_STEP = 4 + 9
+# Kernels the library launches per step (forward: LoRA T product with its
+# in-cluster reduction, dequant-GEMM; backward: U product (also converting
+# the saved T), dB product, dequant-GEMM dX, dA product).
+LAUNCHES_PER_STEP = 2 + 4
 # ncu DRAM traffic (read + write bytes) of one dequant-GEMM launch of this
 # workload, valid only for the source it was captured on.
 GEMM_TRAFFIC = {"source_sha": None, "fwd_bytes": None, "dx_bytes": None}

@@ -40,40 +40,37 @@ int gemm_tile_n();   // output columns per output tile
 int gemm_half_n();   // output columns whose W~ rows each CTA of the pair expands
 
 // -------------------------------------------------------------- K4 (LoRA)
-// part[s][i][j] = sum over the s-th contraction slice of P(i,c) * Q(c,j), fp32.
+// out = alpha * sum_c P(i,c) * Q(c,j) over i < I, j < J (J <= 128, J % 8 == 0),
+// the contraction split over `splits` CTAs of one cluster (<= 8) and reduced
+// in distributed shared memory by the first CTA, which also writes:
+//   out       fp32 [I x J] (or [J x I] if transpose), += when accumulate;
+//   out_bf16  bf16 of (alpha*sum*beta), [I x ldb], columns J..ldb-1 zero;
+//   cvt_dst   bf16 of cvt_src*cvt_scale for the same rows ([I x J] fp32 in,
+//             [I x ldb] out, zero padded) -- an optional side copy.
 //   p_kmajor: P stored [I][C] (ld = ldp) else [C][I].
 //   q_kmajor: Q stored [J][C] (ld = ldq) else [C][J].
-// J <= 128 and J % 8 == 0; C % 8 == 0; leading dimensions % 8 == 0.
+//   err_zero: if set, one thread stores 0 there (clears the call's error word).
+constexpr int kMaxSkinnySplits = 8;
 struct SkinnyArgs {
     const uint16_t* P;
     const uint16_t* Q;
-    float* part;
     int64_t I, J, C;
     int64_t ldp, ldq;
-    int splits;           // contraction slices (grid.y)
-    int64_t c_per_split;  // multiple of 64
-};
-cudaError_t launch_skinny(bool p_kmajor, bool q_kmajor, const SkinnyArgs& a, cudaStream_t stream);
-
-// out = alpha * sum_s part[s]  (+ out if accumulate), optionally transposed,
-// and/or a bf16 copy scaled by beta into a zero-padded [I x ldb] buffer.
-struct FinalizeArgs {
-    const float* part;
     int splits;
-    int64_t I, J;
+    int64_t c_per_split;  // multiple of 64
     float alpha;
-    float* out;           // nullable; [I x J], or [J x I] if transpose
+    float* out;
     int transpose;
     int accumulate;
-    uint16_t* out_bf16;   // nullable; [I x ldb], columns >= J zeroed
+    uint16_t* out_bf16;
     int64_t ldb;
     float beta;
+    const float* cvt_src;
+    uint16_t* cvt_dst;
+    float cvt_scale;
+    int* err_zero;
 };
-cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t stream);
-
-// dst[R2 x C2] (bf16) = src[R1 x C1] zero-padded (R1 <= R2, C1 <= C2).
-cudaError_t launch_pad_copy(const uint16_t* src, int64_t R1, int64_t C1, uint16_t* dst, int64_t R2,
-                            int64_t C2, cudaStream_t stream);
+cudaError_t launch_skinny(bool p_kmajor, bool q_kmajor, const SkinnyArgs& a, cudaStream_t stream);
 
 // --------------------------------------------------------------------- K5
 struct GemvArgs {

@@ -114,7 +114,6 @@ int num_sms() {
 
 // ------------------------------------------------------- workspace plan
 constexpr int64_t kAlign = 256;
-constexpr int64_t kTargetCtas = 296;     // two CTAs per SM of a 148-SM B200
 constexpr int64_t kGemvSlice = 2048;
 
 int64_t up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
@@ -125,13 +124,12 @@ struct Split {
     int64_t per;
 };
 
-// contraction slices for a skinny product with I long-side rows and C depth
-Split skinny_split(int64_t I, int64_t C) {
+// contraction slices of a LoRA side product: one cluster of up to 8 CTAs
+Split skinny_split(int64_t C) {
     const int64_t chunks = std::max<int64_t>(1, cdiv(C, 64));
-    int64_t s = std::max<int64_t>(1, cdiv(kTargetCtas, std::max<int64_t>(1, cdiv(I, 64))));
-    s = std::min(s, chunks);
+    const int64_t s = std::min<int64_t>(kMaxSkinnySplits, chunks);
     const int64_t per = cdiv(chunks, s) * 64;
-    return {static_cast<int>(cdiv(C, per)), per};
+    return {static_cast<int>(cdiv(std::max<int64_t>(C, 1), per)), per};
 }
 
 Split gemv_split(int64_t K) {
@@ -141,27 +139,19 @@ Split gemv_split(int64_t K) {
 
 struct Plan {
     int64_t rp;          // rank padded to 64
-    int64_t off_err, off_part, off_gt, off_gu, off_bp, off_ap, total;
+    int64_t off_err, off_part, off_gt, off_gu, total;
 };
 
 Plan make_plan(int64_t M, int64_t N, int64_t K, int r) {
     Plan p;
     p.rp = up(r, 64);
     int64_t part = 0;
-    const Split sT = skinny_split(M, K), sU = skinny_split(M, N), sB = skinny_split(N, M),
-                sA = skinny_split(K, M);
-    part = std::max(part, int64_t(sT.splits) * M * r);
-    part = std::max(part, int64_t(sU.splits) * M * r);
-    part = std::max(part, int64_t(sB.splits) * N * r);
-    part = std::max(part, int64_t(sA.splits) * K * r);
-    if (M <= QLORA_GEMV_MAX_TOKENS) part = std::max(part, int64_t(gemv_split(K).splits) * M * N);
+    if (M <= QLORA_GEMV_MAX_TOKENS) part = int64_t(gemv_split(K).splits) * M * N;
     int64_t o = 0;
     p.off_err = o;  o += kAlign;
     p.off_part = o; o += up(part * 4, kAlign);
     p.off_gt = o;   o += up(M * p.rp * 2, kAlign);
     p.off_gu = o;   o += up(M * p.rp * 2, kAlign);
-    p.off_bp = o;   o += up(N * p.rp * 2, kAlign);
-    p.off_ap = o;   o += up(p.rp * K * 2, kAlign);
     p.total = o;
     return p;
 }
@@ -194,15 +184,35 @@ T* at(void* ws, int64_t off) {
     return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
-// T = X A^T -> (optional fp32 T_save, bf16 gamma*T padded to rp) ; uses part
+SkinnyArgs skinny_args(const uint16_t* P, const uint16_t* Q, int64_t I, int64_t J, int64_t C,
+                       int64_t ldp, int64_t ldq) {
+    SkinnyArgs a{};
+    a.P = P;
+    a.Q = Q;
+    a.I = I;
+    a.J = J;
+    a.C = C;
+    a.ldp = ldp;
+    a.ldq = ldq;
+    const Split sp = skinny_split(C);
+    a.splits = sp.splits;
+    a.c_per_split = sp.per;
+    a.alpha = 1.0f;
+    a.beta = 1.0f;
+    a.cvt_scale = 1.0f;
+    return a;
+}
+
+// T = X A^T -> optional fp32 T_save and bf16 gamma*T padded to rp columns
 cudaError_t run_T(const uint16_t* X, const uint16_t* A, int64_t M, int64_t K, int r, float gamma,
-                  float* T_save, uint16_t* Gt, int64_t rp, float* part, cudaStream_t s) {
-    const Split sp = skinny_split(M, K);
-    SkinnyArgs a{X, A, part, M, r, K, K, K, sp.splits, sp.per};
-    cudaError_t e = launch_skinny(true, true, a, s);
-    if (e != cudaSuccess) return e;
-    FinalizeArgs f{part, sp.splits, M, r, 1.0f, T_save, 0, 0, Gt, rp, gamma};
-    return launch_finalize(f, s);
+                  float* T_save, uint16_t* Gt, int64_t rp, int* err_zero, cudaStream_t s) {
+    SkinnyArgs a = skinny_args(X, A, M, r, K, K, K);
+    a.out = T_save;
+    a.out_bf16 = Gt;
+    a.ldb = rp;
+    a.beta = gamma;
+    a.err_zero = err_zero;
+    return launch_skinny(true, true, a, s);
 }
 
 }  // namespace
@@ -301,8 +311,7 @@ int qlora_linear_forward_ex(const uint16_t* X, int64_t M, const qlora_nf4_tensor
     int* err = at<int>(ws, p.off_err);
     float* part = at<float>(ws, p.off_part);
     uint16_t* Gt = at<uint16_t>(ws, p.off_gt);
-    QTRY(cudaMemsetAsync(err, 0, sizeof(int), s));
-    QTRY(run_T(X, A, M, K, r, scale, T_save, Gt, p.rp, part, s));
+    QTRY(run_T(X, A, M, K, r, scale, T_save, Gt, p.rp, err, s));
 
     if (M <= QLORA_GEMV_MAX_TOKENS) {
         const Split sp = gemv_split(K);
@@ -316,8 +325,7 @@ int qlora_linear_forward_ex(const uint16_t* X, int64_t M, const qlora_nf4_tensor
         return QLORA_OK;
     }
 
-    uint16_t* Bp = at<uint16_t>(ws, p.off_bp);
-    QTRY(launch_pad_copy(B, N, r, Bp, N, p.rp, s));
+    // B [N x r] is read in place: the 64-wide TMA box zero-fills columns >= r
     CUtensorMap m_act, m_packed, m_la, m_lb;
     bool ok = make_map_2d(&m_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 128,
                           CU_TENSOR_MAP_SWIZZLE_128B) &&
@@ -325,7 +333,7 @@ int qlora_linear_forward_ex(const uint16_t* X, int64_t M, const qlora_nf4_tensor
                           gemm_half_n(), CU_TENSOR_MAP_SWIZZLE_32B) &&
               make_map_2d(&m_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Gt, p.rp, M, p.rp * 2, 64, 128,
                           CU_TENSOR_MAP_SWIZZLE_128B) &&
-              make_map_2d(&m_lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Bp, p.rp, N, p.rp * 2, 64,
+              make_map_2d(&m_lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, B, r, N, int64_t(r) * 2, 64,
                           gemm_half_n(), CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return QLORA_ERR_CUDA;
     GemmArgs g{};
@@ -383,38 +391,38 @@ int qlora_linear_backward_ex(const uint16_t* dY, const uint16_t* X, int64_t M,
         return QLORA_OK;
     }
     int* err = at<int>(ws, p.off_err);
-    float* part = at<float>(ws, p.off_part);
     uint16_t* Gt = at<uint16_t>(ws, p.off_gt);
     uint16_t* Gu = at<uint16_t>(ws, p.off_gu);
-    QTRY(cudaMemsetAsync(err, 0, sizeof(int), s));
+    int* err_first = err;                 // cleared by the first kernel of the call
 
-    // gamma * T in bf16 (from the saved T or recomputed)
-    if (T_saved) {
-        FinalizeArgs f{T_saved, 1, M, r, 1.0f, nullptr, 0, 0, Gt, p.rp, scale};
-        QTRY(launch_finalize(f, s));
-    } else {
-        QTRY(run_T(X, A, M, K, r, scale, nullptr, Gt, p.rp, part, s));
+    if (!T_saved) {                       // recompute gamma * T in bf16
+        QTRY(run_T(X, A, M, K, r, scale, nullptr, Gt, p.rp, err_first, s));
+        err_first = nullptr;
     }
-    // U = dY B  ->  gamma * U in bf16
+    // U = dY B -> gamma * U in bf16; converts a saved T to gamma * T on the side
     {
-        const Split sp = skinny_split(M, N);
-        SkinnyArgs a{dY, B, part, M, r, N, N, r, sp.splits, sp.per};
+        SkinnyArgs a = skinny_args(dY, B, M, r, N, N, r);
+        a.out_bf16 = Gu;
+        a.ldb = p.rp;
+        a.beta = scale;
+        if (T_saved) {
+            a.cvt_src = T_saved;
+            a.cvt_dst = Gt;
+            a.cvt_scale = scale;
+        }
+        a.err_zero = err_first;
         QTRY(launch_skinny(true, false, a, s));
-        FinalizeArgs f{part, sp.splits, M, r, 1.0f, nullptr, 0, 0, Gu, p.rp, scale};
-        QTRY(launch_finalize(f, s));
     }
     // dB = dY^T (gamma T)
     {
-        const Split sp = skinny_split(N, M);
-        SkinnyArgs a{dY, Gt, part, N, r, M, N, p.rp, sp.splits, sp.per};
+        SkinnyArgs a = skinny_args(dY, Gt, N, r, M, N, p.rp);
+        a.out = dB;
+        a.accumulate = accumulate;
         QTRY(launch_skinny(false, false, a, s));
-        FinalizeArgs f{part, sp.splits, N, r, 1.0f, dB, 0, accumulate, nullptr, 0, 1.0f};
-        QTRY(launch_finalize(f, s));
     }
     // dX = dY W~ + (gamma U) A
     if (dX) {
-        uint16_t* Ap = at<uint16_t>(ws, p.off_ap);
-        QTRY(launch_pad_copy(A, r, K, Ap, p.rp, K, s));
+        // A [r x K] is read in place: the 64-row TMA box zero-fills rows >= r
         CUtensorMap m_act, m_packed, m_la, m_lb;
         bool ok = make_map_2d(&m_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, 128,
                               CU_TENSOR_MAP_SWIZZLE_128B) &&
@@ -422,7 +430,7 @@ int qlora_linear_backward_ex(const uint16_t* dY, const uint16_t* X, int64_t M,
                               gemm_half_n() / 2, 64, CU_TENSOR_MAP_SWIZZLE_64B) &&
                   make_map_2d(&m_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Gu, p.rp, M, p.rp * 2, 64,
                               128, CU_TENSOR_MAP_SWIZZLE_128B) &&
-                  make_map_2d(&m_lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Ap, K, p.rp, K * 2, 64, 64,
+                  make_map_2d(&m_lb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, A, K, r, K * 2, 64, 64,
                               CU_TENSOR_MAP_SWIZZLE_128B);
         if (!ok) return QLORA_ERR_CUDA;
         GemmArgs g{};
@@ -445,11 +453,11 @@ int qlora_linear_backward_ex(const uint16_t* dY, const uint16_t* X, int64_t M,
     }
     // dA^T = X^T (gamma U), written transposed into dA [r x K]
     {
-        const Split sp = skinny_split(K, M);
-        SkinnyArgs a{X, Gu, part, K, r, M, K, p.rp, sp.splits, sp.per};
+        SkinnyArgs a = skinny_args(X, Gu, K, r, M, K, p.rp);
+        a.out = dA;
+        a.transpose = 1;
+        a.accumulate = accumulate;
         QTRY(launch_skinny(false, false, a, s));
-        FinalizeArgs f{part, sp.splits, K, r, 1.0f, dA, 1, accumulate, nullptr, 0, 1.0f};
-        QTRY(launch_finalize(f, s));
     }
     return QLORA_OK;
 }

@@ -2,15 +2,23 @@
 // ("QLoRA, explained", "The forward pass and gradients"):
 //   T = X A^T,  U = dY B,  dB = gamma dY^T T,  dA^T = X^T (gamma U).
 // All are one long contraction (over K, N or the M tokens) with one short
-// output side (r <= 128), so they are HBM-bound streams over X or dY.  One
-// kernel covers the four operand layouts: a CTA of 4 warps owns 64 rows of
-// the long output side and all r columns, streams its contraction slice
-// through a 2-stage cp.async ring, and feeds mma.sync m16n8k16 (bf16 in, fp32
+// output side (r <= 128): HBM-bound streams over X or dY.  One kernel covers
+// the four operand layouts.  A CTA of 4 warps owns 64 rows of the long output
+// side and all r columns of one contraction slice, streams the slice through
+// a 3-stage cp.async ring and feeds mma.sync m16n8k16 (bf16 in, fp32
 // accumulate) through ldmatrix (.trans where the stored layout is the
-// transpose).  Slices write fp32 partials; a finalize pass sums them, applies
-// gamma, and emits the fp32 result and/or the bf16 copy the tcgen05 kernels
-// consume.
+// transpose).  The slices of a row block form one thread-block cluster (up to
+// 8 CTAs): each parks its fp32 partial in shared memory, then every CTA sums
+// one slice of the rows over all partials through distributed shared memory
+// and writes the finished result -- scaled fp32 (optionally transposed or
+// accumulated) and/or the zero-padded bf16 copy the tensor-core kernels
+// consume.  No partial buffer in HBM, no separate reduction launch, and a
+// fixed summation order.
+#include <cooperative_groups.h>
+
 #include "kernels.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace qnf4 {
 
@@ -19,6 +27,7 @@ namespace {
 constexpr int kThreads = 128;
 constexpr int TI = 64;           // output rows per CTA
 constexpr int TC = 64;           // contraction per stage
+constexpr int kStages = 3;
 constexpr int kPitchK = TC * 2 + 16;   // bytes per 64-wide row (+16 against bank conflicts)
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
@@ -60,7 +69,8 @@ struct SkinnyTile {
     static constexpr int kQPitch = QK ? kPitchK : (JP * 2 + 16);
     static constexpr int kQBytes = QK ? JP * kPitchK : TC * kQPitch;
     static constexpr int kStage = kPBytes + kQBytes;
-    static constexpr int kSmem = 2 * kStage;
+    static constexpr int kRedBytes = TI * JP * 4;                       // fp32 partial tile
+    static constexpr int kSmem = (kStages * kStage > kRedBytes) ? kStages * kStage : kRedBytes;
 };
 
 template <bool PK, bool QK, int JT16>
@@ -68,20 +78,22 @@ __global__ void __launch_bounds__(kThreads)
 skinny_kernel(SkinnyArgs a) {
     using Tl = SkinnyTile<PK, QK, JT16>;
     extern __shared__ __align__(16) uint8_t smem[];
+    cg::cluster_group cluster = cg::this_cluster();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t i0 = int64_t(blockIdx.x) * TI;
-    const int64_t c_beg = int64_t(blockIdx.y) * a.c_per_split;
+    const int split = blockIdx.y;
+    const int64_t c_beg = int64_t(split) * a.c_per_split;
     const int64_t c_end = min(a.C, c_beg + a.c_per_split);
-    const int nchunks = static_cast<int>((c_end - c_beg + TC - 1) / TC);
+    const int nchunks = c_end > c_beg ? static_cast<int>((c_end - c_beg + TC - 1) / TC) : 0;
     const uint32_t sbase = smem_u32(smem);
+    if (a.err_zero != nullptr && blockIdx.x == 0 && split == 0 && tid == 0) *a.err_zero = 0;
 
     auto load_stage = [&](int chunk, int st) {
         const int64_t c0 = c_beg + int64_t(chunk) * TC;
         const uint32_t sp = sbase + st * Tl::kStage;
         const uint32_t sq = sp + Tl::kPBytes;
-        // P tile: 64 x 64 elements = 512 chunks of 16 B
 #pragma unroll
-        for (int q = tid; q < TI * 8; q += kThreads) {
+        for (int q = tid; q < TI * 8; q += kThreads) {          // P tile: 64 x 64
             const int row = q >> 3, ch = q & 7;
             const uint16_t* src;
             bool ok;
@@ -102,7 +114,7 @@ skinny_kernel(SkinnyArgs a) {
                 cp_async16(sq + row * Tl::kQPitch + ch * 16, ok ? src : a.Q, ok);
             }
         } else {
-            constexpr int cpr = Tl::JP / 8;            // chunks per row
+            constexpr int cpr = Tl::JP / 8;                        // chunks per row
             for (int q = tid; q < TC * cpr; q += kThreads) {
                 const int row = q / cpr, ch = q % cpr;
                 const bool ok = (c0 + row < c_end) && (ch * 8 < a.J);
@@ -120,13 +132,16 @@ skinny_kernel(SkinnyArgs a) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[j][t][e] = 0.f;
 
-    if (nchunks > 0) load_stage(0, 0);
-    cp_async_commit();
-    for (int chunk = 0; chunk < nchunks; ++chunk) {
-        const int st = chunk & 1;
-        if (chunk + 1 < nchunks) load_stage(chunk + 1, st ^ 1);
+#pragma unroll
+    for (int st = 0; st < kStages - 1; ++st) {
+        if (st < nchunks) load_stage(st, st);
         cp_async_commit();
-        cp_async_wait<1>();
+    }
+    for (int chunk = 0; chunk < nchunks; ++chunk) {
+        const int st = chunk % kStages;
+        if (chunk + kStages - 1 < nchunks) load_stage(chunk + kStages - 1, (chunk + kStages - 1) % kStages);
+        cp_async_commit();
+        cp_async_wait<kStages - 1>();
         __syncthreads();
         const uint32_t sp = sbase + st * Tl::kStage;
         const uint32_t sq = sp + Tl::kPBytes;
@@ -161,23 +176,89 @@ skinny_kernel(SkinnyArgs a) {
         }
         __syncthreads();
     }
+    cp_async_wait<0>();
+    __syncthreads();
 
-    // write the partial tile
-    float* part = a.part + int64_t(blockIdx.y) * a.I * a.J;
+    // park the partial tile [64][JP] in shared memory
+    float* red = reinterpret_cast<float*>(smem);
     const int g = lane >> 2, c = lane & 3;
 #pragma unroll
     for (int jt = 0; jt < JT16; ++jt)
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            const int64_t j = jt * 16 + t * 8 + 2 * c;
+        for (int t = 0; t < 2; ++t)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const int64_t i = i0 + warp * 16 + g + h * 8;
-                if (i < a.I && j < a.J)
-                    *reinterpret_cast<float2*>(part + i * a.J + j) =
-                        make_float2(acc[jt][t][2 * h], acc[jt][t][2 * h + 1]);
+                const int row = warp * 16 + g + h * 8;
+                const int col = jt * 16 + t * 8 + 2 * c;
+                *reinterpret_cast<float2*>(red + row * Tl::JP + col) =
+                    make_float2(acc[jt][t][2 * h], acc[jt][t][2 * h + 1]);
+            }
+    cluster.sync();
+
+    // Every CTA of the cluster finalises its own slice of the 64 rows, summing
+    // the partials of all slices (float4 loads, issued before any use).
+    const int nsplit = static_cast<int>(cluster.num_blocks());
+    const int rank = static_cast<int>(cluster.block_rank());
+    const int rows_per = (TI + nsplit - 1) / nsplit;
+    const int r0 = rank * rows_per, r1 = min(TI, r0 + rows_per);
+    constexpr int kC4 = Tl::JP / 4;
+    const float4* parts[kMaxSkinnySplits];
+#pragma unroll
+    for (int q = 0; q < kMaxSkinnySplits; ++q)
+        parts[q] = reinterpret_cast<const float4*>(cluster.map_shared_rank(red, q < nsplit ? q : 0));
+    for (int g4 = tid; g4 < (r1 - r0) * kC4; g4 += kThreads) {
+        const int li = r0 + g4 / kC4, c4 = g4 % kC4;
+        const int64_t i = i0 + li;
+        float4 v[kMaxSkinnySplits];
+#pragma unroll
+        for (int q = 0; q < kMaxSkinnySplits; ++q)
+            if (q < nsplit) v[q] = parts[q][li * kC4 + c4];
+        float sum[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int q = 0; q < kMaxSkinnySplits; ++q)
+            if (q < nsplit) {
+                sum[0] += v[q].x;
+                sum[1] += v[q].y;
+                sum[2] += v[q].z;
+                sum[3] += v[q].w;
+            }
+        if (i >= a.I) continue;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int j = c4 * 4 + e;
+            const float val = sum[e] * a.alpha;
+            if (j < a.J && a.out) {
+                float* o = a.transpose ? (a.out + int64_t(j) * a.I + i) : (a.out + i * a.J + j);
+                *o = a.accumulate ? (*o + val) : val;
+            }
+            if (a.out_bf16 && j < a.ldb) {
+                __nv_bfloat16 bv = __float2bfloat16_rn(j < a.J ? val * a.beta : 0.f);
+                a.out_bf16[i * a.ldb + j] = *reinterpret_cast<uint16_t*>(&bv);
             }
         }
+    }
+    if (a.out_bf16 && a.ldb > Tl::JP) {          // zero padding beyond the tile width
+        const int padw = static_cast<int>(a.ldb) - Tl::JP;
+        for (int e = tid; e < (r1 - r0) * padw; e += kThreads) {
+            const int64_t i = i0 + r0 + e / padw;
+            if (i < a.I) a.out_bf16[i * a.ldb + Tl::JP + e % padw] = 0;
+        }
+    }
+    // side job: bf16 copy of a fp32 [I x J] source for the same rows
+    if (a.cvt_src != nullptr) {
+        const int c4w = static_cast<int>(a.ldb) / 4;
+        for (int e = tid; e < (r1 - r0) * c4w; e += kThreads) {
+            const int64_t i = i0 + r0 + e / c4w;
+            const int j = (e % c4w) * 4;
+            if (i >= a.I) continue;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (j < a.J) v = *reinterpret_cast<const float4*>(a.cvt_src + i * a.J + j);
+            const uint32_t lo = pack_bf16x2(v.x * a.cvt_scale, v.y * a.cvt_scale);
+            const uint32_t hi = pack_bf16x2(v.z * a.cvt_scale, v.w * a.cvt_scale);
+            *reinterpret_cast<uint2*>(a.cvt_dst + i * a.ldb + j) = make_uint2(lo, hi);
+        }
+    }
+    cluster.sync();            // keep every partial alive until the sum is done
 }
 
 template <bool PK, bool QK, int JT16>
@@ -186,9 +267,19 @@ cudaError_t run_skinny(const SkinnyArgs& a, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(skinny_kernel<PK, QK, JT16>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Tl::kSmem);
     if (e != cudaSuccess) return e;
-    dim3 grid(static_cast<unsigned>((a.I + TI - 1) / TI), static_cast<unsigned>(a.splits));
-    skinny_kernel<PK, QK, JT16><<<grid, kThreads, Tl::kSmem, stream>>>(a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((a.I + TI - 1) / TI), static_cast<unsigned>(a.splits));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = Tl::kSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = static_cast<unsigned>(a.splits);
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, skinny_kernel<PK, QK, JT16>, a);
 }
 
 template <bool PK, bool QK>
@@ -206,69 +297,15 @@ cudaError_t dispatch_j(const SkinnyArgs& a, cudaStream_t stream) {
     }
 }
 
-__global__ void finalize_kernel(FinalizeArgs a) {
-    const int64_t total = a.I * (a.out_bf16 ? a.ldb : a.J);
-    const int64_t width = a.out_bf16 ? a.ldb : a.J;
-    for (int64_t idx = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; idx < total;
-         idx += int64_t(gridDim.x) * blockDim.x) {
-        const int64_t i = idx / width, j = idx % width;
-        if (j >= a.J) {                              // zero padding of the bf16 copy
-            a.out_bf16[i * a.ldb + j] = 0;
-            continue;
-        }
-        float s = 0.f;
-        for (int k = 0; k < a.splits; ++k) s += a.part[(int64_t(k) * a.I + i) * a.J + j];
-        s *= a.alpha;
-        if (a.out) {
-            float* o = a.transpose ? (a.out + j * a.I + i) : (a.out + i * a.J + j);
-            *o = a.accumulate ? (*o + s) : s;
-        }
-        if (a.out_bf16) {
-            __nv_bfloat16 b = __float2bfloat16_rn(s * a.beta);
-            a.out_bf16[i * a.ldb + j] = *reinterpret_cast<uint16_t*>(&b);
-        }
-    }
-}
-
-__global__ void pad_copy_kernel(const uint16_t* src, int64_t R1, int64_t C1, uint16_t* dst,
-                                int64_t R2, int64_t C2) {
-    const int64_t total = R2 * C2;
-    for (int64_t idx = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; idx < total;
-         idx += int64_t(gridDim.x) * blockDim.x) {
-        const int64_t r = idx / C2, c = idx % C2;
-        dst[idx] = (r < R1 && c < C1) ? src[r * C1 + c] : uint16_t(0);
-    }
-}
-
-unsigned grid_for(int64_t n, int threads) {
-    int64_t g = (n + threads - 1) / threads;
-    if (g > 4096) g = 4096;
-    if (g < 1) g = 1;
-    return static_cast<unsigned>(g);
-}
-
 }  // namespace
 
 cudaError_t launch_skinny(bool p_kmajor, bool q_kmajor, const SkinnyArgs& a, cudaStream_t stream) {
-    if (a.I <= 0 || a.J <= 0) return cudaSuccess;
+    if (a.I <= 0 || a.J <= 0 || a.splits < 1 || a.splits > kMaxSkinnySplits)
+        return a.I <= 0 ? cudaSuccess : cudaErrorInvalidValue;
     if (p_kmajor && q_kmajor) return dispatch_j<true, true>(a, stream);
     if (p_kmajor && !q_kmajor) return dispatch_j<true, false>(a, stream);
     if (!p_kmajor && !q_kmajor) return dispatch_j<false, false>(a, stream);
     return dispatch_j<false, true>(a, stream);
-}
-
-cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t stream) {
-    const int64_t total = a.I * (a.out_bf16 ? a.ldb : a.J);
-    if (total <= 0) return cudaSuccess;
-    finalize_kernel<<<grid_for(total, 256), 256, 0, stream>>>(a);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_pad_copy(const uint16_t* src, int64_t R1, int64_t C1, uint16_t* dst, int64_t R2,
-                            int64_t C2, cudaStream_t stream) {
-    if (R2 * C2 <= 0) return cudaSuccess;
-    pad_copy_kernel<<<grid_for(R2 * C2, 256), 256, 0, stream>>>(src, R1, C1, dst, R2, C2);
-    return cudaGetLastError();
 }
 
 }  // namespace qnf4
