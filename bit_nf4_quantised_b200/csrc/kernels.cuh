@@ -78,23 +78,30 @@ struct GemvArgs {
     const uint8_t* scale_codes;
     const float* meta;
     const uint16_t* X;    // [M x K] bf16, M <= 16
-    float* part;          // [splits][M][N] fp32
+    const uint16_t* A;    // [r x K] bf16 (LoRA down-projection)
+    int r;
+    float* part;          // [splits][M][N] fp32 partial products
+    float* Tpart;         // [splits][M][r] fp32 partial T = X A^T
+    int* counters;        // [splits] row-tile counters, zero on entry
     int64_t M, N, K;
     int splits;
-    int64_t k_per_split;  // multiple of 64
+    int64_t k_per_split;  // multiple of 256 (or K)
     Nf4Table tab;
 };
-cudaError_t launch_gemv(const GemvArgs& a, int* smem_bytes_out, cudaStream_t stream);
-int gemv_rows_per_cta();
+// Largest activation slice (bytes, 8 or 16 rows x slice x 2 + pitch padding)
+// the GEMV kernel can hold next to its lookup table.
+int gemv_max_activation_bytes();
+cudaError_t launch_gemv(const GemvArgs& a, int num_sms, cudaStream_t stream);
 
-// Y[m][n] = bf16( sum_s part[s][m][n] + sum_j G[m][j] * B[n][j] )
+// T = sum_s Tpart[s] (also to T_save); Y = bf16(sum_s part[s] + gamma T B^T)
 struct GemvFinalizeArgs {
     const float* part;
+    const float* Tpart;
     int splits;
-    const uint16_t* G;    // gamma*T, bf16 [M x ldg]
-    int64_t ldg;
     const uint16_t* B;    // [N x r]
     int r;
+    float gamma;
+    float* T_save;        // nullable
     uint16_t* Y;
     int64_t M, N;
 };

@@ -114,7 +114,8 @@ int num_sms() {
 
 // ------------------------------------------------------- workspace plan
 constexpr int64_t kAlign = 256;
-constexpr int64_t kGemvSlice = 2048;
+constexpr int64_t kControlBytes = 1024;     // error word + GEMV tile counters
+constexpr int64_t kMaxGemvSlices = 200;
 
 int64_t up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -132,24 +133,39 @@ Split skinny_split(int64_t C) {
     return {static_cast<int>(cdiv(std::max<int64_t>(C, 1), per)), per};
 }
 
-Split gemv_split(int64_t K) {
-    const int64_t per = std::min(K, kGemvSlice);
+// contraction slices of the GEMV: each slice's activations (8 or 16 rows)
+// must fit next to the kernel's lookup table; slices are multiples of 256
+Split gemv_split(int64_t M, int64_t K) {
+    const int64_t rows = M <= 8 ? 8 : 16;
+    const int64_t cap = ((gemv_max_activation_bytes() / rows - 8) / 2) / 256 * 256;
+    int64_t s = cdiv(K, cap);
+    int64_t per = up(cdiv(K, s), 256);
+    while (per > cap) {
+        ++s;
+        per = up(cdiv(K, s), 256);
+    }
+    if (per >= K) return {1, K};
     return {static_cast<int>(cdiv(K, per)), per};
 }
 
 struct Plan {
     int64_t rp;          // rank padded to 64
-    int64_t off_err, off_part, off_gt, off_gu, total;
+    int64_t off_err, off_part, off_tpart, off_gt, off_gu, total;
 };
 
 Plan make_plan(int64_t M, int64_t N, int64_t K, int r) {
     Plan p;
     p.rp = up(r, 64);
-    int64_t part = 0;
-    if (M <= QLORA_GEMV_MAX_TOKENS) part = int64_t(gemv_split(K).splits) * M * N;
+    int64_t part = 0, tpart = 0;
+    if (M <= QLORA_GEMV_MAX_TOKENS) {
+        const Split sp = gemv_split(M, K);
+        part = int64_t(sp.splits) * M * N;
+        tpart = int64_t(sp.splits) * M * r;
+    }
     int64_t o = 0;
-    p.off_err = o;  o += kAlign;
+    p.off_err = o;  o += kControlBytes;
     p.off_part = o; o += up(part * 4, kAlign);
+    p.off_tpart = o; o += up(tpart * 4, kAlign);
     p.off_gt = o;   o += up(M * p.rp * 2, kAlign);
     p.off_gu = o;   o += up(M * p.rp * 2, kAlign);
     p.total = o;
@@ -311,19 +327,38 @@ int qlora_linear_forward_ex(const uint16_t* X, int64_t M, const qlora_nf4_tensor
     int* err = at<int>(ws, p.off_err);
     float* part = at<float>(ws, p.off_part);
     uint16_t* Gt = at<uint16_t>(ws, p.off_gt);
-    QTRY(run_T(X, A, M, K, r, scale, T_save, Gt, p.rp, err, s));
-
     if (M <= QLORA_GEMV_MAX_TOKENS) {
-        const Split sp = gemv_split(K);
-        GemvArgs g{w->packed, w->scale_codes, w->meta_scale, X, part, M, N, K, sp.splits, sp.per,
-                   table()};
+        // decode path: T is computed inside the GEMV kernel; the control
+        // words (error word, tile counters) start at zero
+        const Split sp = gemv_split(M, K);
+        if (sp.splits > kMaxGemvSlices) return QLORA_ERR_UNSUPPORTED;
+        float* tpart = at<float>(ws, p.off_tpart);
+        int* counters = err + 4;
+        QTRY(cudaMemsetAsync(err, 0, size_t(4 + sp.splits) * sizeof(int), s));
+        GemvArgs g{};
+        g.packed = w->packed;
+        g.scale_codes = w->scale_codes;
+        g.meta = w->meta_scale;
+        g.X = X;
+        g.A = A;
+        g.r = r;
+        g.part = part;
+        g.Tpart = tpart;
+        g.counters = counters;
+        g.M = M;
+        g.N = N;
+        g.K = K;
+        g.splits = sp.splits;
+        g.k_per_split = sp.per;
+        g.tab = table();
         QTRY(record(ev, true, s));
-        QTRY(launch_gemv(g, nullptr, s));
+        QTRY(launch_gemv(g, num_sms(), s));
         QTRY(record(ev, false, s));
-        GemvFinalizeArgs f{part, sp.splits, Gt, p.rp, B, r, Y, M, N};
+        GemvFinalizeArgs f{part, tpart, sp.splits, B, r, scale, T_save, Y, M, N};
         QTRY(launch_gemv_finalize(f, s));
         return QLORA_OK;
     }
+    QTRY(run_T(X, A, M, K, r, scale, T_save, Gt, p.rp, err, s));
 
     // B [N x r] is read in place: the 64-wide TMA box zero-fills columns >= r
     CUtensorMap m_act, m_packed, m_la, m_lb;
