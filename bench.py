@@ -141,9 +141,17 @@ def _bufs(lin, device):
 def _max_over_ranks(x: float, world: int) -> float:
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def allreduce_adapter_grads(dA: torch.Tensor, dB: torch.Tensor) -> None:
+    """Data parallelism over tokens: each rank's adapter gradients are partial
+    sums over its shard; the exchange is one sum over ranks."""
+    torch.distributed.all_reduce(dA)
+    torch.distributed.all_reduce(dB)
 
 
 def _barrier(world):
@@ -233,8 +241,7 @@ def run_gpu(args):
         w, g = sets[i % 2]
         _step(q, lin, w, g, bufs, ws, events)
         if world > 1:
-            torch.distributed.all_reduce(bufs["dA"])
-            torch.distributed.all_reduce(bufs["dB"])
+            allreduce_adapter_grads(bufs["dA"], bufs["dB"])
 
     for i in range(args.warmup):
         one(i)

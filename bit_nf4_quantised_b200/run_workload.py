@@ -1,0 +1,46 @@
+"""Run a few calls of one synthetic workload through the library (for
+profilers such as ncu, which want a short process around the kernels).
+
+  python -m bit_nf4_quantised_b200.run_workload --workload NAME [--calls 2]
+         [--forward-only]
+
+NAME is a key of synthetic.WORKLOADS; for a multi-layer workload only its
+first layer runs.  Each call is one forward (and, unless --forward-only, one
+backward) of that layer on cuda:0.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from . import _lib as q
+from . import synthetic as syn
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="llama7b_attn_proj_4096x4096_m4096_r16")
+    ap.add_argument("--calls", type=int, default=2)
+    ap.add_argument("--forward-only", action="store_true")
+    args = ap.parse_args()
+    lin = syn.WORKLOADS[args.workload].layers[0]
+    d = syn.make_layer(lin, with_grad=not args.forward_only)
+    w = q.qlora_quantize(torch.from_numpy(d["W"]).cuda())
+    g = {k: v.cuda() for k, v in d.items() if isinstance(v, torch.Tensor)}
+    ws = q.workspace(lin.M, lin.N, lin.K, lin.r)
+    T = torch.empty(lin.M, lin.r, dtype=torch.float32, device="cuda")
+    for _ in range(args.calls):
+        q.qlora_linear_forward(g["X"], w, g["A"], g["B"], lin.gamma, T_save=T, ws=ws)
+        if not args.forward_only:
+            q.qlora_linear_backward(g["dY"], g["X"], w, g["A"], g["B"], lin.gamma, T_saved=T,
+                                    ws=ws)
+    torch.cuda.synchronize()
+    err = q.device_error_word(ws)
+    print(f"{args.workload}: {args.calls} call(s), device error word {err}")
+    if err:
+        raise SystemExit(1)
+
+
+if __name__ == "__main__":
+    main()
