@@ -82,7 +82,8 @@ struct GemvArgs {
     int r;
     float* part;          // [splits][M][N] fp32 partial products
     float* Tpart;         // [splits][M][r] fp32 partial T = X A^T
-    int* counters;        // [splits] row-tile counters, zero on entry
+    int* counters;        // [splits] work-unit counters, zero on entry
+    int* err;             // device error word
     int64_t M, N, K;
     int splits;
     int64_t k_per_split;  // multiple of 256 (or K)
@@ -91,7 +92,10 @@ struct GemvArgs {
 // Largest activation slice (bytes, 8 or 16 rows x slice x 2 + pitch padding)
 // the GEMV kernel can hold next to its lookup table.
 int gemv_max_activation_bytes();
-cudaError_t launch_gemv(const GemvArgs& a, int num_sms, cudaStream_t stream);
+// tm_packed: 3-D view of the packed weight {128 bytes, N rows, K/256 chunks},
+// strides {K/2, 128} bytes, box {128, 16, 8}, 128-byte swizzle.
+cudaError_t launch_gemv(const CUtensorMap& tm_packed, const GemvArgs& a, int num_sms,
+                        cudaStream_t stream);
 
 // T = sum_s Tpart[s] (also to T_save); Y = bf16(sum_s part[s] + gamma T B^T)
 struct GemvFinalizeArgs {

@@ -95,6 +95,20 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uin
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Packed weight seen as {128 bytes, N rows, K/256 chunks of 128 bytes}; box
+// {128, 16, 8} = 16 rows x 1024 contiguous bytes, 128-byte swizzle.
+bool make_map_3d_packed(CUtensorMap* map, const void* packed, int64_t N, int64_t K) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(K / 256)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K / 2), 128};
+    const cuuint32_t box[3] = {128, 16, 8};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(packed), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------- validation
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -133,20 +147,24 @@ Split skinny_split(int64_t C) {
     return {static_cast<int>(cdiv(std::max<int64_t>(C, 1), per)), per};
 }
 
-// contraction slices of the GEMV: each slice's activations (8 or 16 rows)
-// must fit next to the kernel's lookup table; slices are multiples of 256
-Split gemv_split(int64_t M, int64_t K) {
-    const int64_t rows = M <= 8 ? 8 : 16;
-    const int64_t cap = ((gemv_max_activation_bytes() / rows - 8) / 2) / 256 * 256;
-    int64_t s = cdiv(K, cap);
+// contraction slices of the GEMV: each slice's M activation rows must fit the
+// kernel's activation budget; slices are multiples of 256, and there are
+// enough of them that every SM pulls several 16-row work units.
+Split gemv_split(int64_t M, int64_t N, int64_t K) {
+    const int64_t m = std::max<int64_t>(M, 1);
+    const int64_t cap = std::max<int64_t>(256, ((gemv_max_activation_bytes() / m - 8) / 2) / 256 * 256);
+    const int64_t units = cdiv(N, 16);
+    int64_t s = std::max(cdiv(K, cap), cdiv(8 * 148, units));
+    s = std::min(s, std::max<int64_t>(1, K / 256));
     int64_t per = up(cdiv(K, s), 256);
-    while (per > cap) {
-        ++s;
-        per = up(cdiv(K, s), 256);
-    }
+    while (per > cap) per = up(cdiv(K, ++s), 256);
     if (per >= K) return {1, K};
     return {static_cast<int>(cdiv(K, per)), per};
 }
+
+// M <= 16 with K % 256 == 0 runs the bandwidth-bound GEMV (its 3-D weight view
+// takes 256-wide chunks); every other shape runs the tensor-core GEMM.
+bool use_gemv(int64_t M, int64_t K) { return M <= QLORA_GEMV_MAX_TOKENS && K % 256 == 0; }
 
 struct Plan {
     int64_t rp;          // rank padded to 64
@@ -157,8 +175,8 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r) {
     Plan p;
     p.rp = up(r, 64);
     int64_t part = 0, tpart = 0;
-    if (M <= QLORA_GEMV_MAX_TOKENS) {
-        const Split sp = gemv_split(M, K);
+    if (use_gemv(M, K)) {
+        const Split sp = gemv_split(M, N, K);
         part = int64_t(sp.splits) * M * N;
         tpart = int64_t(sp.splits) * M * r;
     }
@@ -327,10 +345,10 @@ int qlora_linear_forward_ex(const uint16_t* X, int64_t M, const qlora_nf4_tensor
     int* err = at<int>(ws, p.off_err);
     float* part = at<float>(ws, p.off_part);
     uint16_t* Gt = at<uint16_t>(ws, p.off_gt);
-    if (M <= QLORA_GEMV_MAX_TOKENS) {
+    if (use_gemv(M, K)) {
         // decode path: T is computed inside the GEMV kernel; the control
-        // words (error word, tile counters) start at zero
-        const Split sp = gemv_split(M, K);
+        // words (error word, work-unit counters) start at zero
+        const Split sp = gemv_split(M, N, K);
         if (sp.splits > kMaxGemvSlices) return QLORA_ERR_UNSUPPORTED;
         float* tpart = at<float>(ws, p.off_tpart);
         int* counters = err + 4;
@@ -350,9 +368,12 @@ int qlora_linear_forward_ex(const uint16_t* X, int64_t M, const qlora_nf4_tensor
         g.K = K;
         g.splits = sp.splits;
         g.k_per_split = sp.per;
+        g.err = err;
         g.tab = table();
+        CUtensorMap m_w;
+        if (!make_map_3d_packed(&m_w, w->packed, N, K)) return QLORA_ERR_CUDA;
         QTRY(record(ev, true, s));
-        QTRY(launch_gemv(g, num_sms(), s));
+        QTRY(launch_gemv(m_w, g, num_sms(), s));
         QTRY(record(ev, false, s));
         GemvFinalizeArgs f{part, tpart, sp.splits, B, r, scale, T_save, Y, M, N};
         QTRY(launch_gemv_finalize(f, s));

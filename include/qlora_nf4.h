@@ -61,7 +61,7 @@ typedef enum {
 #define QLORA_GROUP 256
 /* Largest LoRA rank the linear layer accepts; the rank must be a multiple of 8. */
 #define QLORA_MAX_RANK 128
-/* Token counts up to this go to the bandwidth-bound dequant-GEMV kernel. */
+/* Token counts up to this (with K % 256 == 0) go to the dequant-GEMV kernel. */
 #define QLORA_GEMV_MAX_TOKENS 16
 
 /*
@@ -176,8 +176,9 @@ QLORA_API int qlora_linear_workspace_size(int64_t M, int64_t N, int64_t K, int r
  *          call its first 4 bytes hold the kernels' error word (0 = none;
  *          bit 0 = a bounded wait inside the GEMM kernel expired, in which
  *          case the outputs are unspecified).
- *   M <= 16 runs the bandwidth-bound dequant-GEMV kernel, larger M the
- *   tensor-core dequant-GEMM; both compute the same function.
+ *   M <= 16 with K % 256 == 0 runs the bandwidth-bound dequant-GEMV kernel,
+ *   every other shape the tensor-core dequant-GEMM; both compute the same
+ *   function.
  * Shape rules: K % 64 == 0, N % 8 == 0, K >= 64, N >= 8.
  * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE, QLORA_ERR_ALIGN (every tensor
  * 16-byte aligned), QLORA_ERR_UNSUPPORTED, QLORA_ERR_WORKSPACE,
