@@ -248,11 +248,12 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
                     const float mt = (((p0.ci0 + i) >> 8) == (p0.ci0 >> 8)) ? p0.m_first : p0.m_last;
                     ct[i] = __fmul_rn(e4m3_to_float(uint8_t(cw[i >> 2] >> (8 * (i & 3)))), mt);
                 }
-                const uint32_t sdst = sp.scales + s * kScaleBytes + (row * kTileBlocks + bt0) * 4;
+                // scales are stored [block][row] so that the consumers' reads
+                // (8 rows of one block per warp) hit 8 consecutive words
+                const uint32_t sdst = sp.scales + s * kScaleBytes + (bt0 * kTileRows + row) * 4;
 #pragma unroll
-                for (int i = 0; i < 16; i += 4)
-                    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(sdst + i * 4),
-                                 "f"(ct[i]), "f"(ct[i + 1]), "f"(ct[i + 2]), "f"(ct[i + 3])
+                for (int i = 0; i < 16; ++i)
+                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(sdst + i * kTileRows * 4), "f"(ct[i])
                                  : "memory");
             }
             if (lane == 0) {
@@ -379,8 +380,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
             asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];"
                          : "=r"(wb0), "=r"(wb1)
                          : "r"(chunk + (g + 8) * 128 + ((unit16 ^ (g & 7)) << 4)));
-            const float cta = __uint_as_float(lds32(scl + (g * kTileBlocks + bt) * 4));
-            const float ctb = __uint_as_float(lds32(scl + ((g + 8) * kTileBlocks + bt) * 4));
+            const float cta = __uint_as_float(lds32(scl + (bt * kTileRows + g) * 4));
+            const float ctb = __uint_as_float(lds32(scl + (bt * kTileRows + g + 8) * 4));
             float blk[NT][4];
 #pragma unroll
             for (int t = 0; t < NT; ++t) blk[t][0] = blk[t][1] = blk[t][2] = blk[t][3] = 0.f;
