@@ -24,9 +24,9 @@
 //              block's MMAs accumulate into fresh registers, and the block
 //              partial is scaled by its c~ once.  At the end of a unit the 16
 //              warps' partials are summed through shared memory.
-// Each slice's first CTA also computes that slice's part of T = X A^T.  Slices
-// write fp32 partials; the finalize kernel sums them, adds gamma T B^T and
-// rounds Y to bf16.
+// The first few CTAs of each slice also compute a share of T = X A^T.  Slices
+// and T shares write fp32 partials; the finalize kernel sums them, adds
+// gamma T B^T and rounds Y to bf16.
 //
 // Deviation from the dequantise kernel, stated: the table holds bf16(q[i])
 // rather than bf16(q[i] * c~), so each weight enters as bf16(q) * c~ in fp32;
@@ -47,11 +47,28 @@ constexpr int kConsumerWarps = 16;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;   // + producer warp
 constexpr int kLutBytes = 256 * 256;                  // 256 rows of 256 bytes
 constexpr int kSmemBytes = 227 * 1024;
-constexpr int kStages = 4;
+constexpr int kMaxStages = 6;
 constexpr int kTileRows = 16;
 constexpr int kTileBlocks = 32;                       // NF4 blocks per tile and row
 constexpr int kTileBytes = kTileRows * kTileBlocks * 32;      // 16 KiB
-constexpr int kScaleBytes = kTileRows * kTileBlocks * 4;      // 2 KiB of c~ per tile
+// Raw scale data of a tile, copied next to it by the producer: the FP8 codes
+// [16 rows][kCodePitch bytes] (the pitch puts the 8 rows a consumer load
+// reads on distinct banks), then the meta scales [16 rows][2] fp32 of each
+// row's first and last block (a row's 32 blocks span at most two groups of
+// 256 scales).
+constexpr int kCodePitch = 36;
+constexpr int kMetaOffset = kTileRows * kCodePitch;
+constexpr int kScaleBytes = kMetaOffset + kTileRows * 8;
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, bool valid) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(valid ? 4 : 0)
+                 : "memory");
+}
+// Arrive on `bar` once this thread's earlier cp.async copies have landed (the
+// arrival counts against the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -68,10 +85,59 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
     return v;
 }
 
+// The main loop's shared-memory loads and MMAs are plain (not volatile) asm so
+// that the compiler may interleave them freely.  They are kept after the
+// stage's full-barrier wait by taking their addresses from opaque_zero(),
+// issued after the wait, and before the stage's release by feeding their
+// results to keep_before() ahead of the arrive.
+__device__ __forceinline__ uint32_t opaque_zero() {
+    uint32_t z;
+    asm volatile("mov.u32 %0, 0;" : "=r"(z)::"memory");
+    return z;
+}
+
+__device__ __forceinline__ void keep_before(float v) { asm volatile("" ::"f"(v)); }
+
+__device__ __forceinline__ uint32_t lds32_nv(uint32_t addr) {
+    uint32_t v;
+    asm("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t lds16_nv(uint32_t addr) {
+    uint16_t v;
+    asm("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ float2 lds64f_nv(uint32_t addr) {
+    float2 v;
+    asm("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
+    return v;
+}
+
+// c~ = fp32(e4m3 code * meta), exactly: the code's magnitude bits shifted into
+// an fp32 exponent/mantissa give its value times 2^-120 (subnormal codes
+// included); the first multiply restores the value exactly, the second rounds
+// the product once.
+__device__ __forceinline__ float decode_scale(uint32_t code, float meta) {
+    const uint32_t b = code & 0xFFu;
+    const float v = __uint_as_float(((b & 0x7Fu) << 20) | ((b & 0x80u) << 24)) * 0x1p120f;
+    return __fmul_rn(v, meta);
+}
+
+__device__ __forceinline__ void mma16816_nv(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                            uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // bf16 pair of byte k of w: lane_reg = table base + 4*lane, bits 8..15 clear.
 template <int k>
 __device__ __forceinline__ uint32_t lut_pair(uint32_t w, uint32_t lane_reg) {
-    return lds32(prmt(w, lane_reg, 0x7604u | (k << 4)));
+    return lds32_nv(prmt(w, lane_reg, 0x7604u | (k << 4)));
 }
 
 __device__ __forceinline__ void tma_load_3d(uint32_t smem_dst, const CUtensorMap* map, int32_t c0,
@@ -84,13 +150,16 @@ __device__ __forceinline__ void tma_load_3d(uint32_t smem_dst, const CUtensorMap
 }
 
 // Shared-memory plan: the table sits at the first 64 KiB boundary; everything
-// else is placed first-fit in the space before it, then after it.
+// else is placed first-fit in the space before it, then after it.  The host
+// evaluates the same plan to pick the stage count; the kernel re-checks it
+// against its real shared-memory base and reports a misfit.
 struct SmemPlan {
     uint32_t lut, ring, scales, units, red, x, bars;
     bool ok;
 };
 
-__device__ __forceinline__ SmemPlan plan_smem(uint32_t start, uint32_t x_bytes, uint32_t red_bytes) {
+__host__ __device__ inline SmemPlan plan_smem(uint32_t start, int stages, uint32_t x_bytes,
+                                              uint32_t red_bytes) {
     SmemPlan p;
     p.lut = (start + 0xFFFFu) & ~0xFFFFu;
     uint32_t lo = start;
@@ -112,16 +181,26 @@ __device__ __forceinline__ SmemPlan plan_smem(uint32_t start, uint32_t x_bytes, 
         p.ok = false;
         return start;
     };
-    p.ring = take(kStages * kTileBytes, 1024);
-    p.scales = take(kStages * kScaleBytes, 16);
+    p.ring = take(stages * kTileBytes, 1024);
+    p.scales = take(stages * kScaleBytes, 16);
     p.red = take(red_bytes, 16);
     p.x = take(x_bytes, 16);
-    p.units = take(kStages * 8, 8);
-    p.bars = take((2 * kStages + 4) * 8 + 8, 8);   // full, empty, rdone[2], rfree[2], flag
+    p.units = take(stages * 8, 8);
+    p.bars = take((2 * stages + 4) * 8 + 8, 8);   // full, empty, rdone[2], rfree[2], flag
     return p;
 }
 
-template <int NT>
+// Activation slab bytes (rows 16-byte aligned, pitch 16 mod 128 bytes) and
+// reduction-buffer bytes (two [warp][16 rows][M] fp32 buffers, which also
+// hold the [M][r] reduction of T) for M tokens over a kslab-wide slice.
+__host__ __device__ inline uint32_t gemv_x_bytes(int64_t M, int64_t kslab) {
+    return static_cast<uint32_t>(M * (kslab * 2 + 16));
+}
+__host__ __device__ inline uint32_t gemv_red_bytes(int64_t M) {
+    return static_cast<uint32_t>(2 * kConsumerWarps * kTileRows * M * 4);
+}
+
+template <int NT, int kStages>
 __global__ void __launch_bounds__(kThreads, 1)
 gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
@@ -133,11 +212,10 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
     const int kslab = static_cast<int>(k_end - k_beg);
     const int nblk = kslab / QLORA_BLOCK;
     const int tiles_per_unit = (nblk + kTileBlocks - 1) / kTileBlocks;
-    const uint32_t x_pitch = static_cast<uint32_t>(kslab * 2 + 8);
+    const uint32_t x_pitch = static_cast<uint32_t>(kslab * 2 + 16);   // as gemv_x_bytes
     const int xrows = static_cast<int>(a.M);
-    constexpr int kTok = 8 * NT;
-    constexpr uint32_t kRedHalf = kConsumerWarps * kTileRows * kTok * 4u;
-    const SmemPlan sp = plan_smem(start, xrows * x_pitch, 2u * kRedHalf);
+    const uint32_t red_half = gemv_red_bytes(a.M) / 2;
+    const SmemPlan sp = plan_smem(start, kStages, gemv_x_bytes(a.M, kslab), 2u * red_half);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + (sp.bars - start));
     uint64_t* empty = full + kStages;
     uint64_t* rdone = empty + kStages;          // [2] per reduction buffer: partials written
@@ -149,7 +227,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
         *abort_flag = sp.ok ? 0 : 1;
         if (!sp.ok) atomicOr(a.err, 2);
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], 1 + 32);           // producer lane 0 + the lanes' scale copies
             mbar_init(&empty[s], kConsumerWarps);
         }
         for (int p = 0; p < 2; ++p) {
@@ -159,21 +237,22 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
         fence_barrier_init();
         prefetch_tensormap(&tm_packed);
     }
-    // lookup table: byte -> (bf16 q[lo nibble], bf16 q[hi nibble]), per lane
-    for (int e = tid; e < 256 * 32; e += kThreads) {
-        const int b = e >> 5, l = e & 31;
+    // lookup table: byte -> (bf16 q[lo nibble], bf16 q[hi nibble]), one copy
+    // per lane, written four lanes' copies at a time
+    for (int e = tid; e < 256 * 8; e += kThreads) {
+        const int b = e >> 3, l4 = e & 7;
         const uint32_t v = pack_bf16x2(a.tab.code[b & 15], a.tab.code[b >> 4]);
-        asm volatile("st.shared.b32 [%0], %1;" ::"r"(sp.lut + b * 256 + l * 4), "r"(v) : "memory");
+        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(sp.lut + b * 256 + l4 * 16), "r"(v)
+                     : "memory");
     }
-    // activation slice, M rows (8-byte stores: the pitch is 8 mod 16 so that
-    // fragment loads spread over all banks)
+    // activation slice, M rows; the pitch is 16 mod 128 bytes so that the
+    // consumers' 16-byte fragment loads (8 lanes a phase) hit distinct banks
     const int vec_per_row = kslab / 8;
     for (int q = tid; q < xrows * vec_per_row; q += kThreads) {
         const int m = q / vec_per_row, v = q % vec_per_row;
         const uint4 val = *reinterpret_cast<const uint4*>(a.X + m * a.K + k_beg + v * 8);
-        const uint32_t dst = sp.x + m * x_pitch + v * 16;
-        asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(dst), "r"(val.x), "r"(val.y) : "memory");
-        asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(dst + 8), "r"(val.z), "r"(val.w)
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sp.x + m * x_pitch + v * 16),
+                     "r"(val.x), "r"(val.y), "r"(val.z), "r"(val.w)
                      : "memory");
     }
     __syncthreads();
@@ -186,106 +265,74 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
 
     if (warp == kConsumerWarps) {
         // -------------------------------------------------------- producer
-        // Work items are (unit, tile) in order; the scale codes and meta
-        // scales of the next two items are in flight while one is published,
-        // and the unit after the current one is already claimed.
-        const int row = lane >> 1;                  // this lane's (row, 16 blocks) of a tile
-        const int bt0 = (lane & 1) * 16;
-        const bool vec_codes = (nkb % 16) == 0 && (kb_beg % 16) == 0 &&
-                               (reinterpret_cast<uintptr_t>(a.scale_codes) & 15u) == 0;
-        struct Pref {
-            uint4 codes;
-            float m_first, m_last;
-            int64_t ci0;
-        };
+        // Per work item (unit, tile), once its stage is free: lane 0 starts
+        // the tile's TMA load; every lane copies a quarter row of FP8 scale
+        // codes (cp.async, zeros past the slice or the matrix) and one meta
+        // scale into the stage's scale area, and arrives on the stage's full
+        // barrier when its copies land.  Units are claimed one ahead.
+        const int row = lane >> 1, h = lane & 1;   // this lane's row and half of a tile
+        const int chunk0 = static_cast<int>(k_beg / 256);
+        // Claims run one unit ahead: lane 0 holds the result of an atomic
+        // issued a unit earlier, so no claim waits for its round trip.  Claims
+        // increase, so once the work passes the last unit the claim still
+        // outstanding lies past it too and no unit is left unprocessed.
+        int pend = 0;
+        if (lane == 0) pend = atomicAdd(a.counters + slice, 1);
         auto claim = [&]() -> int {
-            int u = 0;
-            if (lane == 0) u = atomicAdd(a.counters + slice, 1);
-            return __shfl_sync(0xffffffffu, u, 0);
+            const int u = __shfl_sync(0xffffffffu, pend, 0);
+            if (lane == 0) pend = atomicAdd(a.counters + slice, 1);
+            return u;
         };
-        auto fetch = [&](int unit, int tile) -> Pref {
-            Pref p;
-            p.codes = make_uint4(0, 0, 0, 0);
-            p.m_first = p.m_last = 0.f;
-            const int64_t n = int64_t(unit) * kTileRows + row;
-            const int bs0 = tile * kTileBlocks + bt0;
-            p.ci0 = n * nkb + kb_beg + bs0;
-            if (unit >= nunits || n >= a.N || bs0 >= nblk) return p;
-            const int cnt = min(16, nblk - bs0);
-            if (vec_codes && cnt == 16) {
-                p.codes = __ldg(reinterpret_cast<const uint4*>(a.scale_codes + p.ci0));
-            } else {
-                uint32_t w[4] = {0, 0, 0, 0};
-                for (int i = 0; i < cnt; ++i) w[i >> 2] |= uint32_t(__ldg(a.scale_codes + p.ci0 + i)) << (8 * (i & 3));
-                p.codes = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-            p.m_first = __ldg(a.meta + (p.ci0 >> 8));
-            p.m_last = __ldg(a.meta + ((p.ci0 + cnt - 1) >> 8));
-            return p;
-        };
-        uint32_t it = 0;
+        int u = claim(), t = 0;
+        bool ok = true;
         int armed[kStages];
         for (int s = 0; s < kStages; ++s) armed[s] = -1;
-        bool ok = true;
-        int cur_u = claim(), next_u = claim(), cur_t = 0;
-        // the item after (u, t): (u, t+1) or (next unit, 0)
-        int nx_u = tiles_per_unit > 1 ? cur_u : next_u, nx_t = tiles_per_unit > 1 ? 1 : 0;
-        Pref p0 = fetch(cur_u, cur_t);
-        Pref p1 = fetch(nx_u, nx_t);
-        for (;; ++it) {
-            const int s = it % kStages;
+        for (uint32_t it = 0;; ++it) {
+            const int s = static_cast<int>(it % kStages);
             const uint32_t ph = (it / kStages) & 1;
-            const bool done = cur_u >= nunits;
+            const bool done = u >= nunits;
             if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, a.err)) {
                 ok = false;
                 break;
             }
-            if (!done) {
-                const uint32_t cw[4] = {p0.codes.x, p0.codes.y, p0.codes.z, p0.codes.w};
-                float ct[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float mt = (((p0.ci0 + i) >> 8) == (p0.ci0 >> 8)) ? p0.m_first : p0.m_last;
-                    ct[i] = __fmul_rn(e4m3_to_float(uint8_t(cw[i >> 2] >> (8 * (i & 3)))), mt);
-                }
-                // scales are stored [block][row] so that the consumers' reads
-                // (8 rows of one block per warp) hit 8 consecutive words
-                const uint32_t sdst = sp.scales + s * kScaleBytes + (bt0 * kTileRows + row) * 4;
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(sdst + i * kTileRows * 4), "f"(ct[i])
-                                 : "memory");
-            }
             if (lane == 0) {
-                uslot[2 * s] = done ? -1 : cur_u;
-                uslot[2 * s + 1] = cur_t;
-            }
-            __syncwarp();
-            if (lane == 0) {
+                uslot[2 * s] = done ? -1 : u;
+                uslot[2 * s + 1] = t;
                 if (done) {
                     mbar_arrive(&full[s]);
                 } else {
                     mbar_arrive_expect_tx(&full[s], kTileBytes);
-                    tma_load_3d(sp.ring + s * kTileBytes, &tm_packed, 0, cur_u * kTileRows,
-                                static_cast<int>(k_beg / 256) + cur_t * (kTileBlocks / 4), &full[s]);
+                    tma_load_3d(sp.ring + s * kTileBytes, &tm_packed, 0, u * kTileRows,
+                                chunk0 + t * (kTileBlocks / 4), &full[s]);
                     armed[s] = static_cast<int>(ph);
                 }
             }
-            if (done) break;
-            // advance: the next item becomes current, fetch the one after it
-            cur_u = nx_u;
-            cur_t = nx_t;
-            p0 = p1;
-            if (cur_t == 0 && cur_u == next_u) next_u = claim();   // entered a new unit
-            if (cur_t + 1 < tiles_per_unit) {
-                nx_u = cur_u;
-                nx_t = cur_t + 1;
-            } else {
-                nx_u = next_u;
-                nx_t = 0;
+            if (!done) {
+                // K is a multiple of 256, so a group of 4 blocks is all inside
+                // or all outside the slice
+                const int64_t n = int64_t(u) * kTileRows + row;
+                const int bs_row = t * kTileBlocks;            // the row's first block
+                const int cnt_row = n < a.N ? max(0, min(kTileBlocks, nblk - bs_row)) : 0;
+                const int64_t ci_row = n * nkb + kb_beg + bs_row;
+                const uint32_t dst = sp.scales + s * kScaleBytes + row * kCodePitch + h * 16;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const int b0 = h * 16 + 4 * q4;
+                    const bool live = b0 < cnt_row;
+                    cp_async4(dst + 4 * q4, a.scale_codes + (live ? ci_row + b0 : 0), live);
+                }
+                const int64_t mi = h == 0 ? (ci_row >> 8) : ((ci_row + cnt_row - 1) >> 8);
+                cp_async4(sp.scales + s * kScaleBytes + kMetaOffset + (row * 2 + h) * 4,
+                          a.meta + (cnt_row > 0 ? mi : 0), cnt_row > 0);
             }
-            p1 = fetch(nx_u, nx_t);
+            cp_async_arrive(&full[s]);
+            if (done) break;
+            if (++t == tiles_per_unit) {
+                t = 0;
+                u = claim();
+            }
         }
+        asm volatile("cp.async.wait_all;" ::: "memory");
         if (!ok && lane == 0) {
             for (int s = 0; s < kStages; ++s)
                 if (armed[s] >= 0) mbar_drain(&full[s], armed[s], a.err);
@@ -294,17 +341,19 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
     }
 
     // ---------------------------------------------------------- consumers
-    if (blockIdx.x == 0) {
-        // this slice's part of T = X A^T, k-steps split over the 16 warps;
-        // reduced in the first reduction buffer, then published
+    if (blockIdx.x < a.t_ctas) {
+        // a share of this slice's T = X A^T: CTA x of the first t_ctas takes
+        // an equal run of the slice's 16-wide k-steps, spread over its warps;
+        // reduced in the first reduction buffer, then written as one partial
         constexpr int kMaxJT = QLORA_MAX_RANK / 8;
         float tacc[kMaxJT][4];
 #pragma unroll
         for (int j = 0; j < kMaxJT; ++j) tacc[j][0] = tacc[j][1] = tacc[j][2] = tacc[j][3] = 0.f;
         const int ksteps = kslab / 16;
-        const int per = (ksteps + kConsumerWarps - 1) / kConsumerWarps;
-        const int s0 = warp * per, s1 = min(ksteps, s0 + per);
-        for (int st = s0; st < s1; ++st) {
+        const int x = blockIdx.x;
+        const int s0 = static_cast<int>(int64_t(ksteps) * x / a.t_ctas);
+        const int s1 = static_cast<int>(int64_t(ksteps) * (x + 1) / a.t_ctas);
+        for (int st = s0 + warp; st < s1; st += kConsumerWarps) {
             const int kk = st * 16 + 2 * c;
             const uint32_t a0 = g < xrows ? lds32(sp.x + g * x_pitch + kk * 2) : 0u;
             const uint32_t a2 = g < xrows ? lds32(sp.x + g * x_pitch + (kk + 8) * 2) : 0u;
@@ -320,34 +369,41 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
                 }
             }
         }
-        // 16 rows x 128 columns of fp32 = 8 KiB, inside reduction buffer 0
+        // [M][r] fp32, inside the reduction buffers (M r <= 2048 M floats)
         const uint32_t tred = sp.red;
-        for (int e = lane; e < 16 * QLORA_MAX_RANK / kConsumerWarps; e += 32)
-            asm volatile("st.shared.b32 [%0], %1;" ::"r"(tred + (warp * 128 + e) * 4), "r"(0u)
-                         : "memory");
+        for (int e = warp * 32 + lane; e < a.M * a.r; e += kConsumerWarps * 32)
+            asm volatile("st.shared.b32 [%0], %1;" ::"r"(tred + e * 4), "r"(0u) : "memory");
         asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+        if (s0 + warp < s1) {
 #pragma unroll
-        for (int jt = 0; jt < kMaxJT; ++jt) {
-            if (jt * 8 < a.r) {
-                const int j = jt * 8 + 2 * c;
-                const uint32_t r0 = tred + (g * QLORA_MAX_RANK + j) * 4;
-                const uint32_t r1 = tred + ((g + 8) * QLORA_MAX_RANK + j) * 4;
-                asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(r0), "f"(tacc[jt][0]) : "memory");
-                asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(r0 + 4), "f"(tacc[jt][1]) : "memory");
-                asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(r1), "f"(tacc[jt][2]) : "memory");
-                asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(r1 + 4), "f"(tacc[jt][3]) : "memory");
+            for (int jt = 0; jt < kMaxJT; ++jt) {
+                if (jt * 8 < a.r) {
+                    const int j = jt * 8 + 2 * c;
+                    if (g < xrows) {
+                        const uint32_t r0 = tred + (g * a.r + j) * 4;
+                        asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(r0), "f"(tacc[jt][0]) : "memory");
+                        asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(r0 + 4), "f"(tacc[jt][1]) : "memory");
+                    }
+                    if (g + 8 < xrows) {
+                        const uint32_t r1 = tred + ((g + 8) * a.r + j) * 4;
+                        asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(r1), "f"(tacc[jt][2]) : "memory");
+                        asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(r1 + 4), "f"(tacc[jt][3]) : "memory");
+                    }
+                }
             }
         }
         asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
-        for (int e = warp * 32 + lane; e < a.M * a.r; e += kConsumerWarps * 32) {
-            const int m = e / a.r, j = e % a.r;
-            a.Tpart[(int64_t(slice) * a.M + m) * a.r + j] =
-                __uint_as_float(lds32(tred + (m * QLORA_MAX_RANK + j) * 4));
-        }
+        float* tp = a.Tpart + (int64_t(slice) * a.t_ctas + x) * a.M * a.r;
+        for (int e = warp * 32 + lane; e < a.M * a.r; e += kConsumerWarps * 32)
+            tp[e] = __uint_as_float(lds32(tred + e * 4));
         asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
     }
 
-    // main loop: 2 blocks of every tile, all 16 rows
+    // main loop: 2 blocks of every tile, all 16 rows.  MMA row g (and g + 8)
+    // holds tile row rg (and rg + 8), rg = 2 (g mod 4) + g / 4: the half-warp
+    // that a 64-bit shared load serves then reads rows 0, 2, 4, 6 (or 1, 3,
+    // 5, 7), whose swizzled 16-byte units cover all 32 banks.
+    const int rg = 2 * (g & 3) + (g >> 2);
     float acc[NT][4];
 #pragma unroll
     for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
@@ -361,65 +417,110 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
         const int unit = uslot[2 * s];
         const int tile = uslot[2 * s + 1];
         if (unit < 0) break;                                  // no more work
-        const uint32_t ring = sp.ring + s * kTileBytes;
-        const uint32_t scl = sp.scales + s * kScaleBytes;
+        const uint32_t z = opaque_zero();
+        const uint32_t ring = sp.ring + s * kTileBytes + z;
+        const uint32_t scl = sp.scales + s * kScaleBytes + z;
+        // operands of both blocks first, then the lookups and MMAs
+        uint32_t wa[2][2], wb[2][2], xk[2];
+        float ct[2][2];
+        // this warp's two blocks of rows rg and rg + 8: FP8 codes (16 bits
+        // per row) and the rows' meta scales; a row's blocks before `split`
+        // belong to its first block's group of 256 scales
+        const uint32_t cra = lds16_nv(scl + rg * kCodePitch + 2 * warp);
+        const uint32_t crb = lds16_nv(scl + (rg + 8) * kCodePitch + 2 * warp);
+        const float2 mra = lds64f_nv(scl + kMetaOffset + rg * 8);
+        const float2 mrb = lds64f_nv(scl + kMetaOffset + (rg + 8) * 8);
+        // (the low 8 bits of the row's first scale index; 32-bit wrap-around
+        // keeps them exact)
+        const uint32_t ci_lo = static_cast<uint32_t>(unit) * kTileRows * static_cast<uint32_t>(nkb) +
+                               static_cast<uint32_t>(kb_beg + tile * kTileBlocks);
+        const int split_a = 256 - static_cast<int>((ci_lo + rg * static_cast<uint32_t>(nkb)) & 255u);
+        const int split_b = 256 - static_cast<int>((ci_lo + (rg + 8) * static_cast<uint32_t>(nkb)) & 255u);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             const int bt = 2 * warp + j;                      // block within the tile
             const int bs = tile * kTileBlocks + bt;           // block within the slice
-            if (bs >= nblk) break;
+            // Blocks past the slice carry c~ = 0 and finite table values;
+            // their activations are taken as zero so they add nothing.
+            const bool valid = bs < nblk;
             // tile layout [chunk of 4 blocks][row][128 bytes], 16-byte units
-            // swizzled by (row & 7); lane (g, c) reads 8 bytes of rows g, g+8
+            // swizzled by (row & 7); lane (g, c) reads 8 bytes of rows rg, rg+8
             const int within = (bt & 3) * 32 + c * 8;
             const uint32_t unit16 = static_cast<uint32_t>(within >> 4);
-            const uint32_t chunk = ring + (bt >> 2) * (kTileRows * 128) + (within & 15);
-            uint32_t wa0, wa1, wb0, wb1;
-            asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];"
-                         : "=r"(wa0), "=r"(wa1)
-                         : "r"(chunk + g * 128 + ((unit16 ^ (g & 7)) << 4)));
-            asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];"
-                         : "=r"(wb0), "=r"(wb1)
-                         : "r"(chunk + (g + 8) * 128 + ((unit16 ^ (g & 7)) << 4)));
-            const float cta = __uint_as_float(lds32(scl + (bt * kTileRows + g) * 4));
-            const float ctb = __uint_as_float(lds32(scl + (bt * kTileRows + g + 8) * 4));
-            float blk[NT][4];
+            const uint32_t chunk = ring + (bt >> 2) * (kTileRows * 128) + (within & 15) +
+                                   ((unit16 ^ static_cast<uint32_t>(rg & 7)) << 4);
+            asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(wa[j][0]), "=r"(wa[j][1]) : "r"(chunk + rg * 128));
+            asm("ld.shared.v2.b32 {%0, %1}, [%2];"
+                : "=r"(wb[j][0]), "=r"(wb[j][1])
+                : "r"(chunk + (rg + 8) * 128));
+            ct[j][0] = decode_scale(cra >> (8 * j), bt < split_a ? mra.x : mra.y);
+            ct[j][1] = decode_scale(crb >> (8 * j), bt < split_b ? mrb.x : mrb.y);
+            xk[j] = valid ? sp.x + z + static_cast<uint32_t>((bs * 64 + c * 16) * 2) : 0u;
+        }
+        float blk[2][NT][4];
 #pragma unroll
-            for (int t = 0; t < NT; ++t) blk[t][0] = blk[t][1] = blk[t][2] = blk[t][3] = 0.f;
-            const uint32_t xk = sp.x + static_cast<uint32_t>((bs * 64 + c * 16) * 2);
+        for (int j = 0; j < 2; ++j)
 #pragma unroll
-            for (int st = 0; st < 4; ++st) {
-                const uint32_t wa = st < 2 ? wa0 : wa1;
-                const uint32_t wb = st < 2 ? wb0 : wb1;
-                uint32_t a0, a1, a2, a3;
-                if (st & 1) {
-                    a0 = lut_pair<2>(wa, lane_reg);
-                    a2 = lut_pair<3>(wa, lane_reg);
-                    a1 = lut_pair<2>(wb, lane_reg);
-                    a3 = lut_pair<3>(wb, lane_reg);
-                } else {
-                    a0 = lut_pair<0>(wa, lane_reg);
-                    a2 = lut_pair<1>(wa, lane_reg);
-                    a1 = lut_pair<0>(wb, lane_reg);
-                    a3 = lut_pair<1>(wb, lane_reg);
-                }
+            for (int t = 0; t < NT; ++t) blk[j][t][0] = blk[j][t][1] = blk[j][t][2] = blk[j][t][3] = 0.f;
+        // one token tile: the two blocks' steps interleave; two token tiles:
+        // block after block, which keeps fewer activation registers live
+        uint32_t xb[2][NT][8];
+#pragma unroll
+        for (int o = 0; o < 8; ++o) {
+            const int st = NT == 1 ? (o >> 1) : (o & 3);
+            const int j = NT == 1 ? (o & 1) : (o >> 2);
+            if (st == 0) {
+                // activations of lane c's 16 contraction positions, two
+                // 16-byte loads (zero for a block past the slice)
 #pragma unroll
                 for (int t = 0; t < NT; ++t) {
                     const int tok = g + 8 * t;
-                    uint32_t b0 = 0, b1 = 0;
-                    if (tok < xrows)
-                        asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];"
-                                     : "=r"(b0), "=r"(b1)
-                                     : "r"(xk + tok * x_pitch + st * 8));
-                    mma16816(blk[t], a0, a1, a2, a3, b0, b1);
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) xb[j][t][h] = 0u;
+                    if (xk[j] != 0u && tok < xrows) {
+                        const uint32_t xa = xk[j] + tok * x_pitch;
+                        asm("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                            : "=r"(xb[j][t][0]), "=r"(xb[j][t][1]), "=r"(xb[j][t][2]), "=r"(xb[j][t][3])
+                            : "r"(xa));
+                        asm("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                            : "=r"(xb[j][t][4]), "=r"(xb[j][t][5]), "=r"(xb[j][t][6]), "=r"(xb[j][t][7])
+                            : "r"(xa + 16));
+                    }
                 }
             }
+            const uint32_t wA = wa[j][st >> 1];
+            const uint32_t wB = wb[j][st >> 1];
+            uint32_t a0, a1, a2, a3;
+            if (st & 1) {
+                a0 = lut_pair<2>(wA, lane_reg);
+                a2 = lut_pair<3>(wA, lane_reg);
+                a1 = lut_pair<2>(wB, lane_reg);
+                a3 = lut_pair<3>(wB, lane_reg);
+            } else {
+                a0 = lut_pair<0>(wA, lane_reg);
+                a2 = lut_pair<1>(wA, lane_reg);
+                a1 = lut_pair<0>(wB, lane_reg);
+                a3 = lut_pair<1>(wB, lane_reg);
+            }
+#pragma unroll
+            for (int t = 0; t < NT; ++t)
+                mma16816_nv(blk[j][t], a0, a1, a2, a3, xb[j][t][2 * st], xb[j][t][2 * st + 1]);
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
-                acc[t][0] = fmaf(cta, blk[t][0], acc[t][0]);
-                acc[t][1] = fmaf(cta, blk[t][1], acc[t][1]);
-                acc[t][2] = fmaf(ctb, blk[t][2], acc[t][2]);
-                acc[t][3] = fmaf(ctb, blk[t][3], acc[t][3]);
+                acc[t][0] = fmaf(ct[j][0], blk[j][t][0], acc[t][0]);
+                acc[t][1] = fmaf(ct[j][0], blk[j][t][1], acc[t][1]);
+                acc[t][2] = fmaf(ct[j][1], blk[j][t][2], acc[t][2]);
+                acc[t][3] = fmaf(ct[j][1], blk[j][t][3], acc[t][3]);
             }
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            keep_before(acc[t][0]);
+            keep_before(acc[t][1]);
+            keep_before(acc[t][2]);
+            keep_before(acc[t][3]);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
@@ -429,33 +530,40 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
             // reused every second unit; rfree[p] says its last sum was read.
             const int p = units_done & 1;
             const uint32_t use = units_done >> 1;
-            const uint32_t red = sp.red + p * kRedHalf;
+            const uint32_t red = sp.red + p * red_half;
             bool ok = true;
             if (use > 0) ok = mbar_wait(&rfree[p], (use - 1) & 1, abort_flag, a.err);
             if (!ok) break;
+            // buffer layout [warp][16 rows][M]; only existing tokens are kept
+            const uint32_t base = red + static_cast<uint32_t>(warp * kTileRows * xrows) * 4;
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
                 const int tok = 8 * t + 2 * c;
-                const uint32_t base = red + (warp * kTileRows) * kTok * 4;
-                asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(base + (g * kTok + tok) * 4),
-                             "f"(acc[t][0]), "f"(acc[t][1]) : "memory");
-                asm volatile("st.shared.v2.f32 [%0], {%1, %2};"
-                             ::"r"(base + ((g + 8) * kTok + tok) * 4), "f"(acc[t][2]), "f"(acc[t][3])
-                             : "memory");
+                const uint32_t ra = base + (rg * xrows + tok) * 4;
+                const uint32_t rb = base + ((rg + 8) * xrows + tok) * 4;
+                if (tok < xrows) {
+                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(ra), "f"(acc[t][0]) : "memory");
+                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(rb), "f"(acc[t][2]) : "memory");
+                }
+                if (tok + 1 < xrows) {
+                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(ra + 4), "f"(acc[t][1]) : "memory");
+                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(rb + 4), "f"(acc[t][3]) : "memory");
+                }
                 acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&rdone[p]);
             if (warp == unit % kConsumerWarps) {
                 if (!mbar_wait(&rdone[p], use & 1, abort_flag, a.err)) break;
-                for (int e = lane; e < kTileRows * kTok; e += 32) {
-                    const int row = e / kTok, tok = e % kTok;
+                // rows x M sums of 16 partials, in a fixed order
+                for (int e = lane; e < kTileRows * xrows; e += 32) {
                     float sum = 0.f;
 #pragma unroll 4
                     for (int w = 0; w < kConsumerWarps; ++w)
-                        sum += __uint_as_float(lds32(red + ((w * kTileRows + row) * kTok + tok) * 4));
+                        sum += __uint_as_float(lds32(red + (w * kTileRows * xrows + e) * 4));
+                    const int row = e / xrows, tok = e % xrows;
                     const int64_t n = int64_t(unit) * kTileRows + row;
-                    if (tok < a.M && n < a.N) part[int64_t(tok) * a.N + n] = sum;
+                    if (n < a.N) part[int64_t(tok) * a.N + n] = sum;
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&rfree[p]);
@@ -465,16 +573,39 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
     }
 }
 
-// One thread per output column n: T = sum of the slices' parts (staged in
+// One thread per output column n: T = sum of the T partials (staged in
 // shared memory), Y[m][n] = bf16( sum_s part[s][m][n] + gamma * T[m] . B[n] ).
 __global__ void __launch_bounds__(256)
 gemv_finalize_kernel(GemvFinalizeArgs a) {
     __shared__ float st[16 * QLORA_MAX_RANK];
-    for (int e = threadIdx.x; e < a.M * a.r; e += blockDim.x) {
-        float t = 0.f;
-        for (int s = 0; s < a.splits; ++s) t += a.Tpart[int64_t(s) * a.M * a.r + e];
-        st[e] = t;
-        if (blockIdx.x == 0 && a.T_save) a.T_save[e] = t;
+    __shared__ float tsum[256];
+    // T: with E = M r <= 256 values, the 256 threads form 256 / E groups that
+    // sum interleaved subsets of the partials, then the groups' sums are added
+    // in group order; with more values each thread sums whole columns.  The
+    // order is fixed either way.
+    const int E = static_cast<int>(a.M) * a.r;
+    if (E <= 256) {
+        const int groups = 256 / E;
+        const int e = threadIdx.x % E, gi = threadIdx.x / E;
+        if (gi < groups) {
+            float t = 0.f;
+            for (int s = gi; s < a.t_parts; s += groups) t += a.Tpart[int64_t(s) * E + e];
+            tsum[threadIdx.x] = t;
+        }
+        __syncthreads();
+        if (threadIdx.x < E) {
+            float t = 0.f;
+            for (int g2 = 0; g2 < groups; ++g2) t += tsum[g2 * E + threadIdx.x];
+            st[threadIdx.x] = t;
+            if (blockIdx.x == 0 && a.T_save) a.T_save[threadIdx.x] = t;
+        }
+    } else {
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            float t = 0.f;
+            for (int s = 0; s < a.t_parts; ++s) t += a.Tpart[int64_t(s) * E + e];
+            st[e] = t;
+            if (blockIdx.x == 0 && a.T_save) a.T_save[e] = t;
+        }
     }
     __syncthreads();
     const int64_t n = blockIdx.x * int64_t(blockDim.x) + threadIdx.x;
@@ -520,21 +651,36 @@ int gemv_max_activation_bytes() {
     return 32 * 1024;
 }
 
+int gemv_stages(int64_t M, int64_t kslab) {
+    // dynamic shared memory starts after the 1 KiB the driver reserves; the
+    // plan must also hold for a base 1 KiB either side of that
+    for (int st = kMaxStages; st >= 4; st -= 2) {
+        bool ok = true;
+        for (uint32_t start : {0u, 1024u, 2048u})
+            ok = ok && plan_smem(start, st, gemv_x_bytes(M, kslab), gemv_red_bytes(M)).ok;
+        if (ok) return st;
+    }
+    return 0;
+}
+
+template <int NT, int ST>
+static cudaError_t launch_one(dim3 grid, const CUtensorMap& tm, const GemvArgs& a, cudaStream_t stream) {
+    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<NT, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemBytes);
+    if (e != cudaSuccess) return e;
+    gemv_kernel<NT, ST><<<grid, kThreads, kSmemBytes, stream>>>(tm, a);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_gemv(const CUtensorMap& tm_packed, const GemvArgs& a, int num_sms,
                         cudaStream_t stream) {
     const unsigned per_slice = static_cast<unsigned>(std::max(1, num_sms / std::max(1, a.splits)));
     dim3 grid(per_slice, static_cast<unsigned>(a.splits));
-    cudaError_t e;
-    if (a.M > 8) {
-        e = cudaFuncSetAttribute(gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e != cudaSuccess) return e;
-        gemv_kernel<2><<<grid, kThreads, kSmemBytes, stream>>>(tm_packed, a);
-    } else {
-        e = cudaFuncSetAttribute(gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-        if (e != cudaSuccess) return e;
-        gemv_kernel<1><<<grid, kThreads, kSmemBytes, stream>>>(tm_packed, a);
-    }
-    return cudaGetLastError();
+    const int st = gemv_stages(a.M, std::min<int64_t>(a.K, a.k_per_split));
+    if (st == 0) return cudaErrorInvalidConfiguration;
+    if (a.M > 8) return st == 6 ? launch_one<2, 6>(grid, tm_packed, a, stream)
+                                : launch_one<2, 4>(grid, tm_packed, a, stream);
+    return st == 6 ? launch_one<1, 6>(grid, tm_packed, a, stream) : launch_one<1, 4>(grid, tm_packed, a, stream);
 }
 
 cudaError_t launch_gemv_finalize(const GemvFinalizeArgs& a, cudaStream_t stream) {

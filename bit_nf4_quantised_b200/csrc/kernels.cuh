@@ -81,12 +81,13 @@ struct GemvArgs {
     const uint16_t* A;    // [r x K] bf16 (LoRA down-projection)
     int r;
     float* part;          // [splits][M][N] fp32 partial products
-    float* Tpart;         // [splits][M][r] fp32 partial T = X A^T
+    float* Tpart;         // [splits][t_ctas][M][r] fp32 partial T = X A^T
     int* counters;        // [splits] work-unit counters, zero on entry
     int* err;             // device error word
     int64_t M, N, K;
     int splits;
     int64_t k_per_split;  // multiple of 256 (or K)
+    int t_ctas;           // CTAs of each slice that compute a share of T
     Nf4Table tab;
 };
 // Largest activation slice (bytes, 8 or 16 rows x slice x 2 + pitch padding)
@@ -97,11 +98,13 @@ int gemv_max_activation_bytes();
 cudaError_t launch_gemv(const CUtensorMap& tm_packed, const GemvArgs& a, int num_sms,
                         cudaStream_t stream);
 
-// T = sum_s Tpart[s] (also to T_save); Y = bf16(sum_s part[s] + gamma T B^T)
+// T = sum of the t_parts partials (also to T_save);
+// Y = bf16(sum_s part[s] + gamma T B^T)
 struct GemvFinalizeArgs {
     const float* part;
     const float* Tpart;
-    int splits;
+    int splits;           // partial outputs
+    int t_parts;          // partial T
     const uint16_t* B;    // [N x r]
     int r;
     float gamma;

@@ -116,7 +116,8 @@ int check_tensor(const qlora_nf4_tensor* w) {
     if (!w || !w->packed || !w->scale_codes || !w->meta_scale) return QLORA_ERR_NULL;
     if (w->rows < 0 || w->cols < 0) return QLORA_ERR_SHAPE;
     if (w->cols > 0 && w->rows > INT64_MAX / w->cols) return QLORA_ERR_SHAPE;
-    if (!aligned(w->packed, 16) || !aligned(w->meta_scale, 4)) return QLORA_ERR_ALIGN;
+    if (!aligned(w->packed, 16) || !aligned(w->scale_codes, 4) || !aligned(w->meta_scale, 4))
+        return QLORA_ERR_ALIGN;
     return QLORA_OK;
 }
 
@@ -152,7 +153,7 @@ Split skinny_split(int64_t C) {
 // enough of them that every SM pulls several 16-row work units.
 Split gemv_split(int64_t M, int64_t N, int64_t K) {
     const int64_t m = std::max<int64_t>(M, 1);
-    const int64_t cap = std::max<int64_t>(256, ((gemv_max_activation_bytes() / m - 8) / 2) / 256 * 256);
+    const int64_t cap = std::max<int64_t>(256, ((gemv_max_activation_bytes() / m - 16) / 2) / 256 * 256);
     const int64_t units = cdiv(N, 16);
     int64_t s = std::max(cdiv(K, cap), cdiv(8 * 148, units));
     s = std::min(s, std::max<int64_t>(1, K / 256));
@@ -166,6 +167,21 @@ Split gemv_split(int64_t M, int64_t N, int64_t K) {
 // takes 256-wide chunks); every other shape runs the tensor-core GEMM.
 bool use_gemv(int64_t M, int64_t K) { return M <= QLORA_GEMV_MAX_TOKENS && K % 256 == 0; }
 
+// T = X A^T is spread thinly over the CTAs of each slice, so that each share
+// is a k-step or two that overlaps the first weight tile's latency; every CTA
+// of the share writes one fp32 partial, which the finalize sums.  The shares
+// stop growing once the finalize would read more than kGemvTReadCap partial
+// values per CTA, and never exceed kGemvTParts partials in all.
+constexpr int kGemvTParts = 256;
+constexpr int64_t kGemvTReadCap = 8192;
+int gemv_t_ctas(int splits, int sms, int64_t M, int r) {
+    const int sp = std::max(1, splits);
+    const int per_slice = std::max(1, sms / sp);
+    const int64_t by_read = kGemvTReadCap / std::max<int64_t>(1, M * r * sp);
+    const int64_t by_total = kGemvTParts / sp;
+    return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>({per_slice, by_read, by_total})));
+}
+
 struct Plan {
     int64_t rp;          // rank padded to 64
     int64_t off_err, off_part, off_tpart, off_gt, off_gu, total;
@@ -178,7 +194,7 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r) {
     if (use_gemv(M, K)) {
         const Split sp = gemv_split(M, N, K);
         part = int64_t(sp.splits) * M * N;
-        tpart = int64_t(sp.splits) * M * r;
+        tpart = int64_t(std::max(sp.splits, kGemvTParts)) * M * r;
     }
     int64_t o = 0;
     p.off_err = o;  o += kControlBytes;
@@ -368,6 +384,7 @@ int qlora_linear_forward_ex(const uint16_t* X, int64_t M, const qlora_nf4_tensor
         g.K = K;
         g.splits = sp.splits;
         g.k_per_split = sp.per;
+        g.t_ctas = gemv_t_ctas(sp.splits, num_sms(), M, r);
         g.err = err;
         g.tab = table();
         CUtensorMap m_w;
@@ -375,7 +392,7 @@ int qlora_linear_forward_ex(const uint16_t* X, int64_t M, const qlora_nf4_tensor
         QTRY(record(ev, true, s));
         QTRY(launch_gemv(m_w, g, num_sms(), s));
         QTRY(record(ev, false, s));
-        GemvFinalizeArgs f{part, tpart, sp.splits, B, r, scale, T_save, Y, M, N};
+        GemvFinalizeArgs f{part, tpart, sp.splits, sp.splits * g.t_ctas, B, r, scale, T_save, Y, M, N};
         QTRY(launch_gemv_finalize(f, s));
         return QLORA_OK;
     }

@@ -130,7 +130,7 @@ QLORA_API int qlora_quantized_sizes(int64_t rows, int64_t cols, size_t* packed_b
  *         The host call cannot see device data, so it still returns
  *         QLORA_OK; read the flag after synchronising the stream.
  * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE, QLORA_ERR_ALIGN (W, packed not
- * 16-byte aligned; meta_scale not 4-byte aligned), QLORA_ERR_CUDA.
+ * 16-byte aligned; scale_codes, meta_scale not 4-byte aligned), QLORA_ERR_CUDA.
  */
 QLORA_API int qlora_quantize(const float* W, const qlora_nf4_tensor* out,
                    int* d_nonfinite_flag, qlora_stream_t stream);
@@ -143,7 +143,7 @@ QLORA_API int qlora_quantize(const float* W, const qlora_nf4_tensor* out,
  *   W_out (device, bf16 bits, rows*cols, written): W~ row-major; bit-exact
  *         to bf16_rne(fp32(q[idx] * c~_b)).
  * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE, QLORA_ERR_ALIGN (W_out and packed
- * 16-byte aligned), QLORA_ERR_CUDA.
+ * 16-byte aligned; scale_codes, meta_scale 4-byte aligned), QLORA_ERR_CUDA.
  */
 QLORA_API int qlora_dequantize(const qlora_nf4_tensor* w, uint16_t* W_out,
                      qlora_stream_t stream);
@@ -181,7 +181,7 @@ QLORA_API int qlora_linear_workspace_size(int64_t M, int64_t N, int64_t K, int r
  *   function.
  * Shape rules: K % 64 == 0, N % 8 == 0, K >= 64, N >= 8.
  * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE, QLORA_ERR_ALIGN (every tensor
- * 16-byte aligned), QLORA_ERR_UNSUPPORTED, QLORA_ERR_WORKSPACE,
+ * 16-byte aligned, except scale_codes and meta_scale: 4-byte), QLORA_ERR_UNSUPPORTED, QLORA_ERR_WORKSPACE,
  * QLORA_ERR_CUDA.
  */
 QLORA_API int qlora_linear_forward(const uint16_t* X, int64_t M, const qlora_nf4_tensor* w,

@@ -71,6 +71,9 @@ CASES = [
     (8, 264, 192, 8),
     (9, 256, 4096, 64),
     (16, 1024, 2048, 128),
+    (4, 512, 4352, 16),      # 17 contraction chunks of 256: many one-chunk slices
+    (2, 4104, 2304, 8),      # ragged last row tile, half-filled last weight tile
+    (12, 40, 768, 24),
 ]
 
 
