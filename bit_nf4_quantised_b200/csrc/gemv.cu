@@ -48,17 +48,17 @@ constexpr int kThreads = (kConsumerWarps + 1) * 32;   // + producer warp
 constexpr int kLutBytes = 256 * 256;                  // 256 rows of 256 bytes
 constexpr int kSmemBytes = 227 * 1024;
 constexpr int kMaxStages = 6;
-constexpr int kTileRows = 16;
-constexpr int kTileBlocks = 32;                       // NF4 blocks per tile and row
-constexpr int kTileBytes = kTileRows * kTileBlocks * 32;      // 16 KiB
+// A weight tile is 16 KiB: R rows x D chunks of 256 contraction positions
+// (128 packed bytes), R D = 128, D in {1, 2, 4, 8} chosen per launch so that
+// a contraction slice is a whole number of tiles.  A work unit is R rows x the
+// whole slice.
+constexpr int kTileBytes = 16384;
 // Raw scale data of a tile, copied next to it by the producer: the FP8 codes
-// [16 rows][kCodePitch bytes] (the pitch puts the 8 rows a consumer load
-// reads on distinct banks), then the meta scales [16 rows][2] fp32 of each
-// row's first and last block (a row's 32 blocks span at most two groups of
-// 256 scales).
-constexpr int kCodePitch = 36;
-constexpr int kMetaOffset = kTileRows * kCodePitch;
-constexpr int kScaleBytes = kMetaOffset + kTileRows * 8;
+// [R rows][4 D + 4 bytes] (the pitch puts the 8 rows a consumer load reads on
+// distinct banks), then the meta scales [R rows][2] fp32 of each row's first
+// and last block (a row's blocks in a tile span at most two groups of 256
+// scales).  At most 512 + 12 R <= 2048 bytes.
+constexpr int kScaleBytes = 2048;
 
 __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, bool valid) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(valid ? 4 : 0)
@@ -197,10 +197,10 @@ __host__ __device__ inline uint32_t gemv_x_bytes(int64_t M, int64_t kslab) {
     return static_cast<uint32_t>(M * (kslab * 2 + 16));
 }
 __host__ __device__ inline uint32_t gemv_red_bytes(int64_t M) {
-    return static_cast<uint32_t>(2 * kConsumerWarps * kTileRows * M * 4);
+    return static_cast<uint32_t>(2 * kConsumerWarps * 16 * M * 4);
 }
 
-template <int NT, int kStages>
+template <int NT, int kStages, int D>
 __global__ void __launch_bounds__(kThreads, 1)
 gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
@@ -211,7 +211,12 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
     const int64_t k_end = min(a.K, k_beg + a.k_per_split);
     const int kslab = static_cast<int>(k_end - k_beg);
     const int nblk = kslab / QLORA_BLOCK;
-    const int tiles_per_unit = (nblk + kTileBlocks - 1) / kTileBlocks;
+    // D: 256-wide chunks per tile (= a.tile_chunks)
+    constexpr int R = 128 / D;                   // rows per tile and unit
+    constexpr int bpr = 4 * D;                   // blocks per tile row
+    constexpr int code_pitch = bpr + 4;
+    constexpr int meta_off = R * code_pitch;     // a multiple of 16
+    const int tiles_per_unit = (nblk + bpr - 1) / bpr;
     const uint32_t x_pitch = static_cast<uint32_t>(kslab * 2 + 16);   // as gemv_x_bytes
     const int xrows = static_cast<int>(a.M);
     const uint32_t red_half = gemv_red_bytes(a.M) / 2;
@@ -232,7 +237,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
         }
         for (int p = 0; p < 2; ++p) {
             mbar_init(&rdone[p], kConsumerWarps);
-            mbar_init(&rfree[p], 1);
+            mbar_init(&rfree[p], min(kConsumerWarps, xrows));
         }
         fence_barrier_init();
         prefetch_tensormap(&tm_packed);
@@ -260,17 +265,17 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
 
     const int64_t nkb = a.K / QLORA_BLOCK;
     const int kb_beg = static_cast<int>(k_beg / QLORA_BLOCK);
-    const int64_t nunits = (a.N + kTileRows - 1) / kTileRows;
+    const int64_t nunits = (a.N + R - 1) / R;
     const int g = lane >> 2, c = lane & 3;
 
     if (warp == kConsumerWarps) {
         // -------------------------------------------------------- producer
         // Per work item (unit, tile), once its stage is free: lane 0 starts
-        // the tile's TMA load; every lane copies a quarter row of FP8 scale
-        // codes (cp.async, zeros past the slice or the matrix) and one meta
-        // scale into the stage's scale area, and arrives on the stage's full
-        // barrier when its copies land.  Units are claimed one ahead.
-        const int row = lane >> 1, h = lane & 1;   // this lane's row and half of a tile
+        // the tile's TMA load; the lanes copy the tile's FP8 scale codes (four
+        // 4-byte groups each, cp.async, zeros past the slice or the matrix)
+        // and each row's two meta scales into the stage's scale area, and
+        // arrive on the stage's full barrier when their copies land.  Units
+        // are claimed one ahead.
         const int chunk0 = static_cast<int>(k_beg / 256);
         // Claims run one unit ahead: lane 0 holds the result of an atomic
         // issued a unit earlier, so no claim waits for its round trip.  Claims
@@ -302,28 +307,33 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
                     mbar_arrive(&full[s]);
                 } else {
                     mbar_arrive_expect_tx(&full[s], kTileBytes);
-                    tma_load_3d(sp.ring + s * kTileBytes, &tm_packed, 0, u * kTileRows,
-                                chunk0 + t * (kTileBlocks / 4), &full[s]);
+                    tma_load_3d(sp.ring + s * kTileBytes, &tm_packed, 0, u * R, chunk0 + t * D, &full[s]);
                     armed[s] = static_cast<int>(ph);
                 }
             }
             if (!done) {
                 // K is a multiple of 256, so a group of 4 blocks is all inside
                 // or all outside the slice
-                const int64_t n = int64_t(u) * kTileRows + row;
-                const int bs_row = t * kTileBlocks;            // the row's first block
-                const int cnt_row = n < a.N ? max(0, min(kTileBlocks, nblk - bs_row)) : 0;
-                const int64_t ci_row = n * nkb + kb_beg + bs_row;
-                const uint32_t dst = sp.scales + s * kScaleBytes + row * kCodePitch + h * 16;
+                const uint32_t area = sp.scales + s * kScaleBytes;
+                const int bs_row = t * bpr;                    // each row's first block
+                const int cnt_full = max(0, min(bpr, nblk - bs_row));
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
-                    const int b0 = h * 16 + 4 * q4;
-                    const bool live = b0 < cnt_row;
-                    cp_async4(dst + 4 * q4, a.scale_codes + (live ? ci_row + b0 : 0), live);
+                    const int gi = lane + 32 * q4;             // 128 groups: R rows x D
+                    const int row = gi / D, grp = gi % D;
+                    const int64_t n = int64_t(u) * R + row;
+                    const bool live = n < a.N && 4 * grp < cnt_full;
+                    cp_async4(area + row * code_pitch + 4 * grp,
+                              a.scale_codes + (live ? n * nkb + kb_beg + bs_row + 4 * grp : 0), live);
                 }
-                const int64_t mi = h == 0 ? (ci_row >> 8) : ((ci_row + cnt_row - 1) >> 8);
-                cp_async4(sp.scales + s * kScaleBytes + kMetaOffset + (row * 2 + h) * 4,
-                          a.meta + (cnt_row > 0 ? mi : 0), cnt_row > 0);
+#pragma unroll
+                for (int mi = lane; mi < 2 * R; mi += 32) {
+                    const int row = mi >> 1, last = mi & 1;
+                    const int64_t n = int64_t(u) * R + row;
+                    const bool live = n < a.N && cnt_full > 0;
+                    const int64_t ci = n * nkb + kb_beg + bs_row + (last ? cnt_full - 1 : 0);
+                    cp_async4(area + meta_off + mi * 4, a.meta + (live ? (ci >> 8) : 0), live);
+                }
             }
             cp_async_arrive(&full[s]);
             if (done) break;
@@ -404,6 +414,10 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
     // that a 64-bit shared load serves then reads rows 0, 2, 4, 6 (or 1, 3,
     // 5, 7), whose swizzled 16-byte units cover all 32 banks.
     const int rg = 2 * (g & 3) + (g >> 2);
+    // this warp's pairs 2 warp, 2 warp + 1 of (block, 16-row group): blocks
+    // btw, btw + 1 of rows ra = 16 rq + rg and rb = ra + 8 of every tile
+    const int rq = (2 * warp) / bpr, btw = (2 * warp) % bpr;
+    const int ra = rq * 16 + rg, rb = ra + 8;
     float acc[NT][4];
 #pragma unroll
     for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
@@ -426,33 +440,32 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
         // this warp's two blocks of rows rg and rg + 8: FP8 codes (16 bits
         // per row) and the rows' meta scales; a row's blocks before `split`
         // belong to its first block's group of 256 scales
-        const uint32_t cra = lds16_nv(scl + rg * kCodePitch + 2 * warp);
-        const uint32_t crb = lds16_nv(scl + (rg + 8) * kCodePitch + 2 * warp);
-        const float2 mra = lds64f_nv(scl + kMetaOffset + rg * 8);
-        const float2 mrb = lds64f_nv(scl + kMetaOffset + (rg + 8) * 8);
+        const uint32_t cra = lds16_nv(scl + ra * code_pitch + btw);
+        const uint32_t crb = lds16_nv(scl + rb * code_pitch + btw);
+        const float2 mra = lds64f_nv(scl + meta_off + ra * 8);
+        const float2 mrb = lds64f_nv(scl + meta_off + rb * 8);
         // (the low 8 bits of the row's first scale index; 32-bit wrap-around
         // keeps them exact)
-        const uint32_t ci_lo = static_cast<uint32_t>(unit) * kTileRows * static_cast<uint32_t>(nkb) +
-                               static_cast<uint32_t>(kb_beg + tile * kTileBlocks);
-        const int split_a = 256 - static_cast<int>((ci_lo + rg * static_cast<uint32_t>(nkb)) & 255u);
-        const int split_b = 256 - static_cast<int>((ci_lo + (rg + 8) * static_cast<uint32_t>(nkb)) & 255u);
+        const uint32_t ci_lo = static_cast<uint32_t>(unit) * static_cast<uint32_t>(R) * static_cast<uint32_t>(nkb) +
+                               static_cast<uint32_t>(kb_beg + tile * bpr);
+        const int split_a = 256 - static_cast<int>((ci_lo + ra * static_cast<uint32_t>(nkb)) & 255u);
+        const int split_b = 256 - static_cast<int>((ci_lo + rb * static_cast<uint32_t>(nkb)) & 255u);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
-            const int bt = 2 * warp + j;                      // block within the tile
-            const int bs = tile * kTileBlocks + bt;           // block within the slice
+            const int bt = btw + j;                           // block within the tile row
+            const int bs = tile * bpr + bt;                   // block within the slice
             // Blocks past the slice carry c~ = 0 and finite table values;
             // their activations are taken as zero so they add nothing.
             const bool valid = bs < nblk;
-            // tile layout [chunk of 4 blocks][row][128 bytes], 16-byte units
-            // swizzled by (row & 7); lane (g, c) reads 8 bytes of rows rg, rg+8
+            // tile layout [chunk of 4 blocks][R rows][128 bytes], 16-byte
+            // units swizzled by (row & 7); lane (g, c) reads 8 bytes of rows
+            // ra and rb (both = rg mod 8)
             const int within = (bt & 3) * 32 + c * 8;
             const uint32_t unit16 = static_cast<uint32_t>(within >> 4);
-            const uint32_t chunk = ring + (bt >> 2) * (kTileRows * 128) + (within & 15) +
+            const uint32_t chunk = ring + (bt >> 2) * (R * 128) + (within & 15) +
                                    ((unit16 ^ static_cast<uint32_t>(rg & 7)) << 4);
-            asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(wa[j][0]), "=r"(wa[j][1]) : "r"(chunk + rg * 128));
-            asm("ld.shared.v2.b32 {%0, %1}, [%2];"
-                : "=r"(wb[j][0]), "=r"(wb[j][1])
-                : "r"(chunk + (rg + 8) * 128));
+            asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(wa[j][0]), "=r"(wa[j][1]) : "r"(chunk + ra * 128));
+            asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(wb[j][0]), "=r"(wb[j][1]) : "r"(chunk + rb * 128));
             ct[j][0] = decode_scale(cra >> (8 * j), bt < split_a ? mra.x : mra.y);
             ct[j][1] = decode_scale(crb >> (8 * j), bt < split_b ? mrb.x : mrb.y);
             xk[j] = valid ? sp.x + z + static_cast<uint32_t>((bs * 64 + c * 16) * 2) : 0u;
@@ -526,43 +539,47 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
         if (lane == 0) mbar_arrive(&empty[s]);
         ++it;
         if (tile == tiles_per_unit - 1) {
-            // the unit is complete: sum the 16 warps' partials.  Buffer p is
-            // reused every second unit; rfree[p] says its last sum was read.
+            // The unit is complete.  Each warp writes its 16 rows x M
+            // partials; then min(M, 16) warps, a different run of warps for
+            // each unit, share the 256 M additions (each output adds the
+            // partials of the bpr / 2 warps of its row group, in warp order).
+            // Buffer p is reused every second unit; rfree[p] says the summing
+            // warps have read its last contents.
             const int p = units_done & 1;
             const uint32_t use = units_done >> 1;
             const uint32_t red = sp.red + p * red_half;
-            bool ok = true;
-            if (use > 0) ok = mbar_wait(&rfree[p], (use - 1) & 1, abort_flag, a.err);
-            if (!ok) break;
+            if (use > 0 && !mbar_wait(&rfree[p], (use - 1) & 1, abort_flag, a.err)) break;
             // buffer layout [warp][16 rows][M]; only existing tokens are kept
-            const uint32_t base = red + static_cast<uint32_t>(warp * kTileRows * xrows) * 4;
+            const uint32_t base = red + static_cast<uint32_t>(warp * 16 * xrows) * 4;
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
                 const int tok = 8 * t + 2 * c;
-                const uint32_t ra = base + (rg * xrows + tok) * 4;
-                const uint32_t rb = base + ((rg + 8) * xrows + tok) * 4;
+                const uint32_t r0 = base + (rg * xrows + tok) * 4;
+                const uint32_t r1 = base + ((rg + 8) * xrows + tok) * 4;
                 if (tok < xrows) {
-                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(ra), "f"(acc[t][0]) : "memory");
-                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(rb), "f"(acc[t][2]) : "memory");
+                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(r0), "f"(acc[t][0]) : "memory");
+                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(r1), "f"(acc[t][2]) : "memory");
                 }
                 if (tok + 1 < xrows) {
-                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(ra + 4), "f"(acc[t][1]) : "memory");
-                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(rb + 4), "f"(acc[t][3]) : "memory");
+                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(r0 + 4), "f"(acc[t][1]) : "memory");
+                    asm volatile("st.shared.f32 [%0], %1;" ::"r"(r1 + 4), "f"(acc[t][3]) : "memory");
                 }
                 acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&rdone[p]);
-            if (warp == unit % kConsumerWarps) {
+            const int nsum = min(kConsumerWarps, xrows);
+            const int idx = (warp - unit * nsum) & (kConsumerWarps - 1);
+            if (idx < nsum) {
                 if (!mbar_wait(&rdone[p], use & 1, abort_flag, a.err)) break;
-                // rows x M sums of 16 partials, in a fixed order
-                for (int e = lane; e < kTileRows * xrows; e += 32) {
-                    float sum = 0.f;
-#pragma unroll 4
-                    for (int w = 0; w < kConsumerWarps; ++w)
-                        sum += __uint_as_float(lds32(red + (w * kTileRows * xrows + e) * 4));
+                const int wpg = bpr / 2;                      // warps per row group
+                for (int e = idx * 32 + lane; e < R * xrows; e += nsum * 32) {
                     const int row = e / xrows, tok = e % xrows;
-                    const int64_t n = int64_t(unit) * kTileRows + row;
+                    const int w0 = (row >> 4) * wpg, r16 = row & 15;
+                    float sum = 0.f;
+                    for (int w = w0; w < w0 + wpg; ++w)
+                        sum += __uint_as_float(lds32(red + ((w * 16 + r16) * xrows + tok) * 4));
+                    const int64_t n = int64_t(unit) * R + row;
                     if (n < a.N) part[int64_t(tok) * a.N + n] = sum;
                 }
                 __syncwarp();
@@ -643,14 +660,6 @@ gemv_finalize_kernel(GemvFinalizeArgs a) {
 
 }  // namespace
 
-int gemv_max_activation_bytes() {
-    // The table's 64 KiB alignment leaves the rest of shared memory in two
-    // pieces whose sizes depend on where dynamic shared memory starts; 32 KiB
-    // of activations fit next to the ring, scales and reduction buffers in
-    // every split (the kernel re-checks its plan and reports a misfit).
-    return 32 * 1024;
-}
-
 int gemv_stages(int64_t M, int64_t kslab) {
     // dynamic shared memory starts after the 1 KiB the driver reserves; the
     // plan must also hold for a base 1 KiB either side of that
@@ -663,13 +672,24 @@ int gemv_stages(int64_t M, int64_t kslab) {
     return 0;
 }
 
-template <int NT, int ST>
+template <int NT, int ST, int D>
 static cudaError_t launch_one(dim3 grid, const CUtensorMap& tm, const GemvArgs& a, cudaStream_t stream) {
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<NT, ST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<NT, ST, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kSmemBytes);
     if (e != cudaSuccess) return e;
-    gemv_kernel<NT, ST><<<grid, kThreads, kSmemBytes, stream>>>(tm, a);
+    gemv_kernel<NT, ST, D><<<grid, kThreads, kSmemBytes, stream>>>(tm, a);
     return cudaGetLastError();
+}
+
+template <int NT, int ST>
+static cudaError_t launch_depth(dim3 grid, const CUtensorMap& tm, const GemvArgs& a, cudaStream_t stream) {
+    switch (a.tile_chunks) {
+        case 1: return launch_one<NT, ST, 1>(grid, tm, a, stream);
+        case 2: return launch_one<NT, ST, 2>(grid, tm, a, stream);
+        case 4: return launch_one<NT, ST, 4>(grid, tm, a, stream);
+        case 8: return launch_one<NT, ST, 8>(grid, tm, a, stream);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 cudaError_t launch_gemv(const CUtensorMap& tm_packed, const GemvArgs& a, int num_sms,
@@ -678,9 +698,9 @@ cudaError_t launch_gemv(const CUtensorMap& tm_packed, const GemvArgs& a, int num
     dim3 grid(per_slice, static_cast<unsigned>(a.splits));
     const int st = gemv_stages(a.M, std::min<int64_t>(a.K, a.k_per_split));
     if (st == 0) return cudaErrorInvalidConfiguration;
-    if (a.M > 8) return st == 6 ? launch_one<2, 6>(grid, tm_packed, a, stream)
-                                : launch_one<2, 4>(grid, tm_packed, a, stream);
-    return st == 6 ? launch_one<1, 6>(grid, tm_packed, a, stream) : launch_one<1, 4>(grid, tm_packed, a, stream);
+    if (a.M > 8) return st == 6 ? launch_depth<2, 6>(grid, tm_packed, a, stream)
+                                : launch_depth<2, 4>(grid, tm_packed, a, stream);
+    return st == 6 ? launch_depth<1, 6>(grid, tm_packed, a, stream) : launch_depth<1, 4>(grid, tm_packed, a, stream);
 }
 
 cudaError_t launch_gemv_finalize(const GemvFinalizeArgs& a, cudaStream_t stream) {

@@ -87,14 +87,16 @@ struct GemvArgs {
     int64_t M, N, K;
     int splits;
     int64_t k_per_split;  // multiple of 256 (or K)
+    int tile_chunks;      // D: 256-wide chunks per weight tile (1, 2, 4, 8); tiles are 128 / D rows
     int t_ctas;           // CTAs of each slice that compute a share of T
     Nf4Table tab;
 };
-// Largest activation slice (bytes, 8 or 16 rows x slice x 2 + pitch padding)
-// the GEMV kernel can hold next to its lookup table.
-int gemv_max_activation_bytes();
+// Pipeline stages the GEMV kernel runs with for M tokens over a kslab-wide
+// contraction slice (0: its activations do not fit in shared memory).
+int gemv_stages(int64_t M, int64_t kslab);
 // tm_packed: 3-D view of the packed weight {128 bytes, N rows, K/256 chunks},
-// strides {K/2, 128} bytes, box {128, 16, 8}, 128-byte swizzle.
+// strides {K/2, 128} bytes, box {128, 128 / D rows, D chunks}, 128-byte
+// swizzle, D = a.tile_chunks.
 cudaError_t launch_gemv(const CUtensorMap& tm_packed, const GemvArgs& a, int num_sms,
                         cudaStream_t stream);
 

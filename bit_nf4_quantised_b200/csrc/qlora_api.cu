@@ -97,12 +97,12 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uin
 
 // Packed weight seen as {128 bytes, N rows, K/256 chunks of 128 bytes}; box
 // {128, 16, 8} = 16 rows x 1024 contiguous bytes, 128-byte swizzle.
-bool make_map_3d_packed(CUtensorMap* map, const void* packed, int64_t N, int64_t K) {
+bool make_map_3d_packed(CUtensorMap* map, const void* packed, int64_t N, int64_t K, int chunks) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(K / 256)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K / 2), 128};
-    const cuuint32_t box[3] = {128, 16, 8};
+    const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(128 / chunks), static_cast<cuuint32_t>(chunks)};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(packed), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -137,7 +137,8 @@ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 struct Split {
     int splits;
-    int64_t per;
+    int64_t per;     // contraction slice width (the last slice may be shorter)
+    int chunks;      // weight tile depth D in 256-wide chunks
 };
 
 // contraction slices of a LoRA side product: one cluster of up to 8 CTAs
@@ -145,22 +146,52 @@ Split skinny_split(int64_t C) {
     const int64_t chunks = std::max<int64_t>(1, cdiv(C, 64));
     const int64_t s = std::min<int64_t>(kMaxSkinnySplits, chunks);
     const int64_t per = cdiv(chunks, s) * 64;
-    return {static_cast<int>(cdiv(std::max<int64_t>(C, 1), per)), per};
+    return {static_cast<int>(cdiv(std::max<int64_t>(C, 1), per)), per, 0};
 }
 
-// contraction slices of the GEMV: each slice's M activation rows must fit the
-// kernel's activation budget; slices are multiples of 256, and there are
-// enough of them that every SM pulls several 16-row work units.
+// Contraction slices for the GEMV: as wide as the activations allow in shared
+// memory, but at least enough slices for ~8 16-row units per SM.  Tiles are D
+// chunks deep with D dividing the slice width (so no tile reads a neighbour's
+// columns) -- except with a single slice, where a tile past K is zero-filled.
 Split gemv_split(int64_t M, int64_t N, int64_t K) {
-    const int64_t m = std::max<int64_t>(M, 1);
-    const int64_t cap = std::max<int64_t>(256, ((gemv_max_activation_bytes() / m - 16) / 2) / 256 * 256);
+    int64_t cap = 256;
+    for (int64_t c = std::min<int64_t>(K, 32768) / 256 * 256; c >= 256; c -= 256)
+        if (gemv_stages(M, c) > 0) {
+            cap = c;
+            break;
+        }
     const int64_t units = cdiv(N, 16);
     int64_t s = std::max(cdiv(K, cap), cdiv(8 * 148, units));
     s = std::min(s, std::max<int64_t>(1, K / 256));
     int64_t per = up(cdiv(K, s), 256);
     while (per > cap) per = up(cdiv(K, ++s), 256);
-    if (per >= K) return {1, K};
-    return {static_cast<int>(cdiv(K, per)), per};
+    Split r;
+    if (per >= K) {
+        r.splits = 1;
+        r.per = K;
+    } else {
+        r.splits = static_cast<int>(cdiv(K, per));
+        r.per = per;
+    }
+    // prefer deeper tiles: widen the slice to a multiple of 2048 (or 1024,
+    // 512) when that keeps the slice count and fits the activation budget
+    if (r.splits > 1) {
+        for (int64_t q : {2048, 1024, 512}) {
+            const int64_t wide = up(r.per, q);
+            if (wide <= cap && cdiv(K, wide) == r.splits) {
+                r.per = wide;
+                break;
+            }
+        }
+    }
+    const int64_t chunks = r.per / 256;
+    if (r.splits == 1 && chunks >= 8) {
+        r.chunks = 8;
+    } else {
+        r.chunks = 1;
+        while (r.chunks < 8 && chunks % (2 * r.chunks) == 0) r.chunks *= 2;
+    }
+    return r;
 }
 
 // M <= 16 with K % 256 == 0 runs the bandwidth-bound GEMV (its 3-D weight view
@@ -384,11 +415,12 @@ int qlora_linear_forward_ex(const uint16_t* X, int64_t M, const qlora_nf4_tensor
         g.K = K;
         g.splits = sp.splits;
         g.k_per_split = sp.per;
+        g.tile_chunks = sp.chunks;
         g.t_ctas = gemv_t_ctas(sp.splits, num_sms(), M, r);
         g.err = err;
         g.tab = table();
         CUtensorMap m_w;
-        if (!make_map_3d_packed(&m_w, w->packed, N, K)) return QLORA_ERR_CUDA;
+        if (!make_map_3d_packed(&m_w, w->packed, N, K, sp.chunks)) return QLORA_ERR_CUDA;
         QTRY(record(ev, true, s));
         QTRY(launch_gemv(m_w, g, num_sms(), s));
         QTRY(record(ev, false, s));
