@@ -116,14 +116,16 @@ __device__ __forceinline__ float2 lds64f_nv(uint32_t addr) {
     return v;
 }
 
-// c~ = fp32(e4m3 code * meta), exactly: the code's magnitude bits shifted into
-// an fp32 exponent/mantissa give its value times 2^-120 (subnormal codes
-// included); the first multiply restores the value exactly, the second rounds
-// the product once.
-__device__ __forceinline__ float decode_scale(uint32_t code, float meta) {
-    const uint32_t b = code & 0xFFu;
-    const float v = __uint_as_float(((b & 0x7Fu) << 20) | ((b & 0x80u) << 24)) * 0x1p120f;
-    return __fmul_rn(v, meta);
+// Two FP8 E4M3 codes (low byte first) to their exact fp32 values: E4M3 is a
+// subset of f16, and f16 widens exactly to fp32.
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t codes16) {
+    uint32_t h2;
+    asm("{ .reg .b16 c; cvt.u16.u32 c, %1; cvt.rn.f16x2.e4m3x2 %0, c; }" : "=r"(h2) : "r"(codes16));
+    float2 v;
+    asm("{ .reg .b16 lo, hi; mov.b32 {lo, hi}, %2; cvt.f32.f16 %0, lo; cvt.f32.f16 %1, hi; }"
+        : "=f"(v.x), "=f"(v.y)
+        : "r"(h2));
+    return v;
 }
 
 __device__ __forceinline__ void mma16816_nv(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -355,49 +357,51 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
         // a share of this slice's T = X A^T: CTA x of the first t_ctas takes
         // an equal run of the slice's 16-wide k-steps, spread over its warps;
         // reduced in the first reduction buffer, then written as one partial
-        constexpr int kMaxJT = QLORA_MAX_RANK / 8;
-        float tacc[kMaxJT][4];
-#pragma unroll
-        for (int j = 0; j < kMaxJT; ++j) tacc[j][0] = tacc[j][1] = tacc[j][2] = tacc[j][3] = 0.f;
         const int ksteps = kslab / 16;
         const int x = blockIdx.x;
         const int s0 = static_cast<int>(int64_t(ksteps) * x / a.t_ctas);
         const int s1 = static_cast<int>(int64_t(ksteps) * (x + 1) / a.t_ctas);
-        for (int st = s0 + warp; st < s1; st += kConsumerWarps) {
-            const int kk = st * 16 + 2 * c;
-            const uint32_t a0 = g < xrows ? lds32(sp.x + g * x_pitch + kk * 2) : 0u;
-            const uint32_t a2 = g < xrows ? lds32(sp.x + g * x_pitch + (kk + 8) * 2) : 0u;
-            const uint32_t a1 = g + 8 < xrows ? lds32(sp.x + (g + 8) * x_pitch + kk * 2) : 0u;
-            const uint32_t a3 = g + 8 < xrows ? lds32(sp.x + (g + 8) * x_pitch + (kk + 8) * 2) : 0u;
-#pragma unroll
-            for (int jt = 0; jt < kMaxJT; ++jt) {
-                if (jt * 8 < a.r) {
-                    const uint16_t* ap = a.A + int64_t(jt * 8 + g) * a.K + k_beg + kk;
-                    const uint32_t b0 = __ldg(reinterpret_cast<const uint32_t*>(ap));
-                    const uint32_t b1 = __ldg(reinterpret_cast<const uint32_t*>(ap + 8));
-                    mma16816(tacc[jt], a0, a1, a2, a3, b0, b1);
-                }
-            }
-        }
         // [M][r] fp32, inside the reduction buffers (M r <= 2048 M floats)
         const uint32_t tred = sp.red;
         for (int e = warp * 32 + lane; e < a.M * a.r; e += kConsumerWarps * 32)
             asm volatile("st.shared.b32 [%0], %1;" ::"r"(tred + e * 4), "r"(0u) : "memory");
         asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
-        if (s0 + warp < s1) {
+        // four 8-column tiles of T at a time keep the accumulators small
+        for (int jg = 0; jg * 8 < a.r; jg += 4) {
+            float tacc[4][4];
 #pragma unroll
-            for (int jt = 0; jt < kMaxJT; ++jt) {
-                if (jt * 8 < a.r) {
-                    const int j = jt * 8 + 2 * c;
-                    if (g < xrows) {
-                        const uint32_t r0 = tred + (g * a.r + j) * 4;
-                        asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(r0), "f"(tacc[jt][0]) : "memory");
-                        asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(r0 + 4), "f"(tacc[jt][1]) : "memory");
+            for (int j = 0; j < 4; ++j) tacc[j][0] = tacc[j][1] = tacc[j][2] = tacc[j][3] = 0.f;
+            for (int st = s0 + warp; st < s1; st += kConsumerWarps) {
+                const int kk = st * 16 + 2 * c;
+                const uint32_t a0 = g < xrows ? lds32(sp.x + g * x_pitch + kk * 2) : 0u;
+                const uint32_t a2 = g < xrows ? lds32(sp.x + g * x_pitch + (kk + 8) * 2) : 0u;
+                const uint32_t a1 = g + 8 < xrows ? lds32(sp.x + (g + 8) * x_pitch + kk * 2) : 0u;
+                const uint32_t a3 = g + 8 < xrows ? lds32(sp.x + (g + 8) * x_pitch + (kk + 8) * 2) : 0u;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if ((jg + j) * 8 < a.r) {
+                        const uint16_t* ap = a.A + int64_t((jg + j) * 8 + g) * a.K + k_beg + kk;
+                        const uint32_t b0 = __ldg(reinterpret_cast<const uint32_t*>(ap));
+                        const uint32_t b1 = __ldg(reinterpret_cast<const uint32_t*>(ap + 8));
+                        mma16816(tacc[j], a0, a1, a2, a3, b0, b1);
                     }
-                    if (g + 8 < xrows) {
-                        const uint32_t r1 = tred + ((g + 8) * a.r + j) * 4;
-                        asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(r1), "f"(tacc[jt][2]) : "memory");
-                        asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(r1 + 4), "f"(tacc[jt][3]) : "memory");
+                }
+            }
+            if (s0 + warp < s1) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if ((jg + j) * 8 < a.r) {
+                        const int col = (jg + j) * 8 + 2 * c;
+                        if (g < xrows) {
+                            const uint32_t r0 = tred + (g * a.r + col) * 4;
+                            asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(r0), "f"(tacc[j][0]) : "memory");
+                            asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(r0 + 4), "f"(tacc[j][1]) : "memory");
+                        }
+                        if (g + 8 < xrows) {
+                            const uint32_t r1 = tred + ((g + 8) * a.r + col) * 4;
+                            asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(r1), "f"(tacc[j][2]) : "memory");
+                            asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(r1 + 4), "f"(tacc[j][3]) : "memory");
+                        }
                     }
                 }
             }
@@ -428,8 +432,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
         const int s = it % kStages;
         const uint32_t ph = (it / kStages) & 1;
         if (!mbar_wait(&full[s], ph, abort_flag, a.err)) break;
-        const int unit = uslot[2 * s];
-        const int tile = uslot[2 * s + 1];
+        int unit, tile;
+        asm volatile("ld.shared.v2.s32 {%0, %1}, [%2];" : "=r"(unit), "=r"(tile) : "r"(sp.units + s * 8) : "memory");
         if (unit < 0) break;                                  // no more work
         const uint32_t z = opaque_zero();
         const uint32_t ring = sp.ring + s * kTileBytes + z;
@@ -444,6 +448,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
         const uint32_t crb = lds16_nv(scl + rb * code_pitch + btw);
         const float2 mra = lds64f_nv(scl + meta_off + ra * 8);
         const float2 mrb = lds64f_nv(scl + meta_off + rb * 8);
+        const float2 va = e4m3x2_to_float2(cra), vb = e4m3x2_to_float2(crb);
         // (the low 8 bits of the row's first scale index; 32-bit wrap-around
         // keeps them exact)
         const uint32_t ci_lo = static_cast<uint32_t>(unit) * static_cast<uint32_t>(R) * static_cast<uint32_t>(nkb) +
@@ -466,8 +471,9 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
                                    ((unit16 ^ static_cast<uint32_t>(rg & 7)) << 4);
             asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(wa[j][0]), "=r"(wa[j][1]) : "r"(chunk + ra * 128));
             asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(wb[j][0]), "=r"(wb[j][1]) : "r"(chunk + rb * 128));
-            ct[j][0] = decode_scale(cra >> (8 * j), bt < split_a ? mra.x : mra.y);
-            ct[j][1] = decode_scale(crb >> (8 * j), bt < split_b ? mrb.x : mrb.y);
+            // c~ = fp32(e4m3 code * meta scale), one rounding
+            ct[j][0] = __fmul_rn(j == 0 ? va.x : va.y, bt < split_a ? mra.x : mra.y);
+            ct[j][1] = __fmul_rn(j == 0 ? vb.x : vb.y, bt < split_b ? mrb.x : mrb.y);
             xk[j] = valid ? sp.x + z + static_cast<uint32_t>((bs * 64 + c * 16) * 2) : 0u;
         }
         float blk[2][NT][4];
@@ -518,16 +524,17 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
 #pragma unroll
             for (int t = 0; t < NT; ++t)
                 mma16816_nv(blk[j][t], a0, a1, a2, a3, xb[j][t][2 * st], xb[j][t][2 * st + 1]);
-        }
+            if (st == 3) {
+                // the block is done: scale its sums into the accumulators
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                acc[t][0] = fmaf(ct[j][0], blk[j][t][0], acc[t][0]);
-                acc[t][1] = fmaf(ct[j][0], blk[j][t][1], acc[t][1]);
-                acc[t][2] = fmaf(ct[j][1], blk[j][t][2], acc[t][2]);
-                acc[t][3] = fmaf(ct[j][1], blk[j][t][3], acc[t][3]);
+                for (int t = 0; t < NT; ++t) {
+                    acc[t][0] = fmaf(ct[j][0], blk[j][t][0], acc[t][0]);
+                    acc[t][1] = fmaf(ct[j][0], blk[j][t][1], acc[t][1]);
+                    acc[t][2] = fmaf(ct[j][1], blk[j][t][2], acc[t][2]);
+                    acc[t][3] = fmaf(ct[j][1], blk[j][t][3], acc[t][3]);
+                }
             }
+        }
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
             keep_before(acc[t][0]);
