@@ -326,6 +326,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // Exact E4M3 (e4m3fn) -> fp32: every E4M3 value is representable in fp16.
+// Programmatic dependent launch.  launch_dependents lets the next kernel in
+// the stream (launched with programmatic stream serialisation) start once
+// every CTA of this grid has executed it or exited; grid_dependency_wait
+// blocks until the preceding grid has completed and its writes are visible
+// (it returns at once when the kernel was launched without the attribute).
+__device__ __forceinline__ void launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ float e4m3_to_float(uint8_t code) {
     __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(code), __NV_E4M3);
     return __half2float(__half(h));

@@ -189,6 +189,10 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
                     armed[s] = static_cast<int>(ph);
                 } else {
                     const int j = step - a.main_steps;
+                    // (gamma T | gamma U) comes from the preceding kernel: with
+                    // a programmatic launch, wait for it here, not before the
+                    // main loop
+                    if (j == 0) grid_dependency_wait();
                     if (rank == 0) mbar_arrive_expect_tx(&bars->a_full[s], 2 * (kSA + kSB));
                     tma_load_2d_pair(sA, &tm_lora_a, j * BK, arow, a_full0);
                     tma_load_2d_pair(sA + kSA1, &tm_lora_a, j * BK, arow + 256, a_full0);
@@ -359,7 +363,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
 
 template <bool kTrans>
 cudaError_t launch_one(const CUtensorMap& act, const CUtensorMap& packed, const CUtensorMap& la,
-                       const CUtensorMap& lb, const GemmArgs& args, unsigned pairs,
+                       const CUtensorMap& lb, const GemmArgs& args, unsigned pairs, bool after_lora,
                        cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(qlora_gemm_kernel<kTrans>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
@@ -369,13 +373,15 @@ cudaError_t launch_one(const CUtensorMap& act, const CUtensorMap& packed, const 
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = after_lora ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, qlora_gemm_kernel<kTrans>, act, packed, la, lb, args);
 }
 
@@ -383,14 +389,14 @@ cudaError_t launch_one(const CUtensorMap& act, const CUtensorMap& packed, const 
 
 cudaError_t launch_gemm(bool trans, const CUtensorMap& act, const CUtensorMap& packed,
                         const CUtensorMap& lora_a, const CUtensorMap& lora_b, const GemmArgs& args,
-                        cudaStream_t stream) {
+                        bool after_lora, cudaStream_t stream) {
     const int64_t n_tiles = (args.d_cols + kTileN - 1) / kTileN;
     const int64_t pairs = int64_t(args.m_tiles) * n_tiles;
     if (pairs <= 0) return cudaSuccess;
     if (2 * pairs > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     const cudaError_t e =
-        trans ? launch_one<true>(act, packed, lora_a, lora_b, args, unsigned(pairs), stream)
-              : launch_one<false>(act, packed, lora_a, lora_b, args, unsigned(pairs), stream);
+        trans ? launch_one<true>(act, packed, lora_a, lora_b, args, unsigned(pairs), after_lora, stream)
+              : launch_one<false>(act, packed, lora_a, lora_b, args, unsigned(pairs), after_lora, stream);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -209,6 +209,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t start = smem_u32(smem);
     const int slice = blockIdx.y;
+    launch_dependents();                         // the finalize waits for this grid
     const int64_t k_beg = int64_t(slice) * a.k_per_split;
     const int64_t k_end = min(a.K, k_beg + a.k_per_split);
     const int kslab = static_cast<int>(k_end - k_beg);
@@ -603,6 +604,8 @@ __global__ void __launch_bounds__(256)
 gemv_finalize_kernel(GemvFinalizeArgs a) {
     __shared__ float st[16 * QLORA_MAX_RANK];
     __shared__ float tsum[256];
+    // launched as the GEMV's programmatic dependent: all inputs come from it
+    grid_dependency_wait();
     // T: with E = M r <= 256 values, the 256 threads form 256 / E groups that
     // sum interleaved subsets of the partials, then the groups' sums are added
     // in group order; with more values each thread sums whole columns.  The
@@ -712,8 +715,17 @@ cudaError_t launch_gemv(const CUtensorMap& tm_packed, const GemvArgs& a, int num
 
 cudaError_t launch_gemv_finalize(const GemvFinalizeArgs& a, cudaStream_t stream) {
     if (a.M <= 0 || a.N <= 0) return cudaSuccess;
-    const unsigned grid = static_cast<unsigned>((a.N + 255) / 256);
-    gemv_finalize_kernel<<<grid, 256, 0, stream>>>(a);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((a.N + 255) / 256));
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, gemv_finalize_kernel, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -32,9 +32,12 @@ struct GemmArgs {
     Nf4Table tab;
 };
 
+// after_lora: the kernel directly before it in `stream` is the LoRA kernel
+// that writes (gamma T | gamma U); the GEMM is then launched as its
+// programmatic dependent and waits for it only before the LoRA steps.
 cudaError_t launch_gemm(bool trans, const CUtensorMap& act, const CUtensorMap& packed,
                         const CUtensorMap& lora_a, const CUtensorMap& lora_b, const GemmArgs& args,
-                        cudaStream_t stream);
+                        bool after_lora, cudaStream_t stream);
 int gemm_tile_m();   // tokens per output tile (a CTA pair)
 int gemm_tile_n();   // output columns per output tile
 int gemm_half_n();   // output columns whose W~ rows each CTA of the pair expands

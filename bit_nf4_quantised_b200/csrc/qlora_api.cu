@@ -121,6 +121,37 @@ int check_tensor(const qlora_nf4_tensor* w) {
     return QLORA_OK;
 }
 
+// Per device: a high-priority stream for the input-gradient GEMM, so that
+// the backward's LoRA side products (dB, dA) run beside it on the caller's
+// stream and fill the SMs its last wave of tiles leaves idle, and the two
+// events of that fork and join.  The mutex keeps concurrent callers from
+// interleaving their use of the events.
+struct SideStream {
+    std::mutex mu;
+    cudaStream_t hp = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    bool ready = false;
+};
+
+SideStream* side_stream() {
+    constexpr int kMaxDevices = 64;
+    static SideStream devs[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    SideStream& d = devs[dev];
+    std::lock_guard<std::mutex> lock(d.mu);
+    if (!d.ready) {
+        int least = 0, greatest = 0;
+        if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return nullptr;
+        if (cudaStreamCreateWithPriority(&d.hp, cudaStreamNonBlocking, greatest) != cudaSuccess ||
+            cudaEventCreateWithFlags(&d.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&d.join, cudaEventDisableTiming) != cudaSuccess)
+            return nullptr;
+        d.ready = true;
+    }
+    return &d;
+}
+
 int num_sms() {
     int dev = 0, n = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -455,8 +486,9 @@ int qlora_linear_forward_ex(const uint16_t* X, int64_t M, const qlora_nf4_tensor
     g.m_tiles = static_cast<int>(cdiv(M, gemm_tile_m()));
     g.err = err;
     g.tab = table();
+    // an event record between the two kernels would serialise them fully
     QTRY(record(ev, true, s));
-    QTRY(launch_gemm(false, m_act, m_packed, m_la, m_lb, g, s));
+    QTRY(launch_gemm(false, m_act, m_packed, m_la, m_lb, g, ev == nullptr, s));
     QTRY(record(ev, false, s));
     return QLORA_OK;
 }
@@ -518,14 +550,13 @@ int qlora_linear_backward_ex(const uint16_t* dY, const uint16_t* X, int64_t M,
         a.err_zero = err_first;
         QTRY(launch_skinny(true, false, a, s));
     }
-    // dB = dY^T (gamma T)
-    {
-        SkinnyArgs a = skinny_args(dY, Gt, N, r, M, N, p.rp);
-        a.out = dB;
-        a.accumulate = accumulate;
-        QTRY(launch_skinny(false, false, a, s));
-    }
-    // dX = dY W~ + (gamma U) A
+    // dX = dY W~ + (gamma U) A on the high-priority side stream, forked after
+    // U; dB = dY^T (gamma T) and dA^T = X^T (gamma U) follow U on the caller's
+    // stream and run beside the GEMM; the caller's stream then joins it.
+    SideStream* side = dX ? side_stream() : nullptr;
+    if (dX && !side) return QLORA_ERR_CUDA;
+    std::unique_lock<std::mutex> lock;
+    if (side) lock = std::unique_lock<std::mutex>(side->mu);
     if (dX) {
         // A [r x K] is read in place: the 64-row TMA box zero-fills rows >= r
         CUtensorMap m_act, m_packed, m_la, m_lb;
@@ -552,11 +583,19 @@ int qlora_linear_backward_ex(const uint16_t* dY, const uint16_t* X, int64_t M,
         g.m_tiles = static_cast<int>(cdiv(M, gemm_tile_m()));
         g.err = err;
         g.tab = table();
-        QTRY(record(ev, true, s));
-        QTRY(launch_gemm(true, m_act, m_packed, m_la, m_lb, g, s));
-        QTRY(record(ev, false, s));
+        QTRY(cudaEventRecord(side->fork, s));
+        QTRY(cudaStreamWaitEvent(side->hp, side->fork, 0));
+        QTRY(record(ev, true, side->hp));
+        QTRY(launch_gemm(true, m_act, m_packed, m_la, m_lb, g, false, side->hp));
+        QTRY(record(ev, false, side->hp));
+        QTRY(cudaEventRecord(side->join, side->hp));
     }
-    // dA^T = X^T (gamma U), written transposed into dA [r x K]
+    {
+        SkinnyArgs a = skinny_args(dY, Gt, N, r, M, N, p.rp);
+        a.out = dB;
+        a.accumulate = accumulate;
+        QTRY(launch_skinny(false, false, a, s));
+    }
     {
         SkinnyArgs a = skinny_args(X, Gu, K, r, M, K, p.rp);
         a.out = dA;
@@ -564,6 +603,7 @@ int qlora_linear_backward_ex(const uint16_t* dY, const uint16_t* X, int64_t M,
         a.accumulate = accumulate;
         QTRY(launch_skinny(false, false, a, s));
     }
+    if (dX) QTRY(cudaStreamWaitEvent(s, side->join, 0));
     return QLORA_OK;
 }
 

@@ -78,6 +78,9 @@ __global__ void __launch_bounds__(kThreads)
 skinny_kernel(SkinnyArgs a) {
     using Tl = SkinnyTile<PK, QK, JT16>;
     extern __shared__ __align__(16) uint8_t smem[];
+    // a dependent tensor-core GEMM may start streaming its weight tiles now;
+    // it waits for this grid only before it reads this kernel's output
+    launch_dependents();
     cg::cluster_group cluster = cg::this_cluster();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t i0 = int64_t(blockIdx.x) * TI;

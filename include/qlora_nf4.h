@@ -22,7 +22,10 @@
  *   - The return value is a qlora_status.  Argument errors are detected on
  *     the host before anything is launched and leave every output untouched.
  *     QLORA_ERR_CUDA reports a failed launch (cudaGetLastError()).
- *   - The library holds no global state and no locks; calls on different
+ *   - Global state is limited to, per device: the internal high-priority
+ *     stream and two events that qlora_linear_backward forks its input-
+ *     gradient GEMM onto (created on first use, guarded by a lock), and the
+ *     scratch array of qlora_linear_forward_noalloc.  Calls on different
  *     streams with disjoint outputs and workspaces may run concurrently.
  */
 #ifndef QLORA_NF4_H
@@ -206,6 +209,12 @@ QLORA_API int qlora_linear_forward(const uint16_t* X, int64_t M, const qlora_nf4
  *   M = 0 writes zero gradients (or leaves them unchanged when accumulating);
  *   dY and X may then be NULL.
  *   other arguments as in qlora_linear_forward.
+ * Streams: when dX is computed, its tensor-core GEMM runs on an internal
+ * high-priority stream forked from `stream` (after the kernel producing
+ * dY B) and joined back into `stream` before the call returns, so that the
+ * adapter-gradient kernels on `stream` fill the SMs the GEMM leaves idle.
+ * Ordering against other work on `stream` is as if everything ran on it; the
+ * fork and join are plain event waits, valid under stream capture.
  * Errors as qlora_linear_forward.
  */
 QLORA_API int qlora_linear_backward(const uint16_t* dY, const uint16_t* X, int64_t M,
@@ -218,8 +227,9 @@ QLORA_API int qlora_linear_backward(const uint16_t* dY, const uint16_t* X, int64
 /*
  * Profiling variants.  Identical to qlora_linear_forward / _backward, plus
  * optional CUDA events (cudaEvent_t handles created by the caller, either may
- * be NULL) that are recorded on `stream` immediately before and after the
- * launch of the layer's main weight kernel: the tensor-core dequant-GEMM
+ * be NULL) that are recorded immediately before and after the launch of the
+ * layer's main weight kernel, on the stream it runs on (`stream`, or the
+ * internal stream for dX in the backward): the tensor-core dequant-GEMM
  * (forward Y, or dX in the backward), or the dequant-GEMV when M <= 16.  They
  * let a caller time that kernel inside a running workload without a profiler.
  * ev itself may be NULL.
