@@ -213,6 +213,111 @@ def _quantize_measure(q, syn, device, reps=5):
             "bytes_per_call": nbytes}
 
 
+def _gemv_sweep(q, syn, device, reps=10):
+    """The decode sweep: 28672 x 8192 and 8192 x 28672 weights with 1, 4 and
+    16 tokens.  Per shape the GEMV kernel's CUDA-event time (weights rotated
+    over 3 stored copies, 363 MB > 2x L2) and its algorithmic bytes (stored
+    weight + activations) per second."""
+    out = []
+    for (N, K) in ((28672, 8192), (8192, 28672)):
+        lin0 = syn.WORKLOADS[f"decode_gemv_{N}x{K}_m1"].layers[0]
+        W0 = syn.make_weight(lin0, np.random.default_rng(lin0.seed))
+        Wd = torch.from_numpy(W0).to(device)
+        copies = [q.qlora_quantize(Wd) for _ in range(3)]
+        del Wd, W0
+        for M in (1, 4, 16):
+            lin = syn.WORKLOADS[f"decode_gemv_{N}x{K}_m{M}"].layers[0]
+            d = syn.make_layer(lin, with_grad=False)
+            X, A, B = (d[k].to(device) for k in ("X", "A", "B"))
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device=device)
+            ws = q.workspace(M, N, K, lin.r, device)
+            for i in range(3):
+                q.qlora_linear_forward(X, copies[i % 3], A, B, lin.gamma, Y=Y, ws=ws)
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(reps)]
+            torch.cuda.synchronize()
+            for i in range(reps):
+                q.qlora_linear_forward(X, copies[i % 3], A, B, lin.gamma, Y=Y, ws=ws,
+                                       events=evs[i])
+            torch.cuda.synchronize()
+            us = sum(b.elapsed_time(e) for b, e in evs) / reps * 1e3
+            nbytes = copies[0].nbytes + M * K * 2
+            out.append({"workload": f"decode_gemv_{N}x{K}_m{M}", "kernel_us": round(us, 2),
+                        "GBps": round(nbytes / (us * 1e-6) / 1e9, 1)})
+        del copies
+    return out
+
+
+def _decoder_measure(q, syn, device, steps=2):
+    """The 32-layer decoder (224 linears, 4096 tokens, r = 16): one-time
+    quantise throughput over all 224 weights, then layer-by-layer forward of
+    every linear followed by the backward of every linear, timed with CUDA
+    events.  Weights and activations are drawn on the GPU from a seeded
+    generator (N(0, 0.02^2) weights, N(0, 1) activations): the timing does not
+    depend on the values, and drawing 6.5e9 weights on the host would take
+    minutes.  The seven linears of a layer (q, k, v, o, gate, up, down) each
+    have their own source weight and activations, shared across layers, so
+    consecutive calls never find their inputs in L2."""
+    lins = syn.WORKLOADS["llama7b_decoder_32layers_m4096_r16"].layers
+    gen = torch.Generator(device=device)
+    gen.manual_seed(5)
+    kinds = {l.name.split(".")[1]: (l.N, l.K) for l in lins}
+    kind = lambda l: l.name.split(".")[1]
+    src = {k: torch.randn(n, kk, device=device, generator=gen) * 0.02 for k, (n, kk) in kinds.items()}
+    ws = [q.empty_nf4(l.N, l.K, device) for l in lins]
+    for l, w in zip(lins[:7], ws[:7]):
+        q.qlora_quantize(src[kind(l)], out=w, check_finite=False)
+    torch.cuda.synchronize()
+    b, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b.record()
+    for l, w in zip(lins, ws):
+        q.qlora_quantize(src[kind(l)], out=w, check_finite=False)
+    e.record()
+    torch.cuda.synchronize()
+    q_ms = b.elapsed_time(e)
+    params = sum(l.N * l.K for l in lins)
+    q_bytes = params * 4 + sum(w.nbytes for w in ws)
+    del src
+    M, r = lins[0].M, lins[0].r
+    act = {}
+    for k, (N, K) in kinds.items():
+        act[k] = {
+            "X": torch.randn(M, K, device=device, generator=gen).bfloat16(),
+            "dY": torch.randn(M, N, device=device, generator=gen).bfloat16(),
+            "A": (torch.randn(r, K, device=device, generator=gen) / K ** 0.5).bfloat16(),
+            "B": (torch.randn(N, r, device=device, generator=gen) * 0.01).bfloat16(),
+            "Y": torch.empty(M, N, dtype=torch.bfloat16, device=device),
+            "dX": torch.empty(M, K, dtype=torch.bfloat16, device=device),
+            "dA": torch.empty(r, K, dtype=torch.float32, device=device),
+            "dB": torch.empty(N, r, dtype=torch.float32, device=device)}
+    Ts = [torch.empty(M, r, dtype=torch.float32, device=device) for _ in lins]
+    wsp = q.workspace(M, max(n for n, _ in kinds.values()), max(kk for _, kk in kinds.values()), r,
+                      device)
+
+    def step():
+        for l, w, T in zip(lins, ws, Ts):
+            a = act[kind(l)]
+            q.qlora_linear_forward(a["X"], w, a["A"], a["B"], l.gamma, Y=a["Y"], T_save=T, ws=wsp)
+        for l, w, T in zip(reversed(lins), reversed(ws), reversed(Ts)):
+            a = act[kind(l)]
+            q.qlora_linear_backward(a["dY"], a["X"], w, a["A"], a["B"], l.gamma, T_saved=T,
+                                    dX=a["dX"], dA=a["dA"], dB=a["dB"], ws=wsp)
+
+    step()
+    torch.cuda.synchronize()
+    b.record()
+    for _ in range(steps):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    ms = b.elapsed_time(e) / steps
+    flops = sum(l.fwd_bwd_flops() for l in lins)
+    return {"workload": "llama7b_decoder_32layers_m4096_r16", "linears": len(lins),
+            "fwd_bwd_ms": round(ms, 3), "fwd_bwd_TFLOPs": round(flops / (ms * 1e-3) / 1e12, 2),
+            "quantize_ms": round(q_ms, 3), "quantize_params": params,
+            "quantize_GBps": round(q_bytes / (q_ms * 1e-3) / 1e9, 1)}
+
+
 def run_gpu(args):
     import bit_nf4_quantised_b200 as q
     from bit_nf4_quantised_b200 import synthetic as syn
@@ -307,6 +412,11 @@ def run_gpu(args):
         out["gemv"] = _gemv_measure(q, syn, device)
         out["gemv"]["frac_hbm"] = round(out["gemv"]["kernel_GBps"] / peaks["hbm_gbs"], 4)
         out["quantize"] = _quantize_measure(q, syn, device)
+        out["gemv_sweep"] = _gemv_sweep(q, syn, device)
+        for row in out["gemv_sweep"]:
+            row["frac_hbm"] = round(row["GBps"] / peaks["hbm_gbs"], 4)
+        out["decoder"] = _decoder_measure(q, syn, device)
+        out["decoder"]["frac_bf16"] = round(out["decoder"]["fwd_bwd_TFLOPs"] / peak, 4)
         out["e2e"] = _e2e(q, syn, lin, device, max(3, K // 2))
         out["cpu_baseline"] = _cpu_baseline(seconds=args.cpu_seconds)
     else:

@@ -132,8 +132,8 @@ def test_attn_projection_full_size(q):
     assert_close("dB", dB, lin.gamma * dY.T @ (X @ A.T))
 
 
-@pytest.mark.parametrize("name", ["decode_gemv_28672x8192_m1", "decode_gemv_28672x8192_m16",
-                                  "decode_gemv_8192x28672_m4"])
+@pytest.mark.parametrize("name", [f"decode_gemv_{nk}_m{m}" for nk in ("28672x8192", "8192x28672")
+                                  for m in (1, 4, 16)])
 def test_decode_full_size_sampled_columns(q, name):
     lin = syn.WORKLOADS[name].layers[0]
     d = syn.make_layer(lin, with_grad=False)
