@@ -24,7 +24,9 @@ struct Nf4Table {
 
 // Device error bits written to the workspace error word.
 enum : int {
-    kErrWaitTimeout = 1,
+    kErrWaitTimeout = 1,      // a bounded wait expired
+    kErrSmemPlan = 2,         // the GEMV's shared-memory plan did not fit
+    kErrBadSchedule = 4,      // a GEMM tile schedule broke the width rules
 };
 
 // Spin limit for any mbarrier wait: 2 s of %globaltimer.  A healthy wait in

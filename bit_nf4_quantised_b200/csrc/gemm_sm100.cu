@@ -49,8 +49,9 @@ constexpr int kTileN = 256;        // output columns per pair tile (MMA N)
 constexpr int kHalfN = kTileN / 2; // B rows held by each CTA
 constexpr int BK = 64;             // contraction per pipeline step (one NF4 block)
 constexpr int kStages = 4;
-constexpr int kThreads = 320;
-constexpr int kGroupThreads = 128; // dequantisers per step group
+constexpr int kGroups = 4;          // dequantiser groups, taking steps in turn
+constexpr int kGroupThreads = 128;  // dequantisers per group: one per B row
+constexpr int kThreads = 64 + kGroups * kGroupThreads;
 constexpr int kSA1 = 128 * BK * 2; // 16 KiB: one 128-row activation tile
 constexpr int kSA = 2 * kSA1;      // both accumulators' activation tiles
 constexpr int kSB = kHalfN * BK * 2;   // 16 KiB: this CTA's half of W~ (or LoRA)
@@ -64,7 +65,8 @@ struct __align__(8) Barriers {
     uint64_t pk_full[kStages];     // local: this CTA's packed tile
     uint64_t deq_full[kStages];    // even CTA: 8 dequant warps of the pair
     uint64_t empty[kStages];       // local: MMAs of the stage done
-    uint64_t acc_full;             // local: all MMAs done
+    uint64_t acc_full;             // local: all MMAs of a tile done
+    uint64_t acc_empty;            // even CTA: 16 epilogue warps of the pair drained TMEM
     uint64_t drain;
     uint32_t tmem_slot;
     int abort_flag;
@@ -116,6 +118,35 @@ __device__ __forceinline__ void dequant_block_to_smem(const uint32_t (&w)[8], fl
     }
 }
 
+// The tiles of one CTA pair: its run [pair * col_budget, + col_budget) of the
+// output taken as m_tiles x cols_lin in row-major order, cut at 512-token row
+// boundaries and every 256 columns.
+struct TileIter {
+    int64_t pos, end, cols;
+    __device__ TileIter(const GemmArgs& a, int pair)
+        : pos(int64_t(pair) * a.col_budget),
+          end(min(int64_t(pair + 1) * a.col_budget, int64_t(a.m_tiles) * a.cols_lin)),
+          cols(a.cols_lin) {}
+    // Widths are multiples of the host's granule (32, or 128 for dX so that
+    // each CTA's half is whole NF4 blocks and its TMA x coordinates stay
+    // 16-byte aligned); a schedule that breaks this ends the walk with an
+    // error instead of issuing a misaligned copy.
+    __device__ bool next(int& m0, int& n0, int& w, bool trans, int* err) {
+        if (pos >= end) return false;
+        const int64_t c = pos % cols;
+        w = static_cast<int>(min(int64_t(kTileN), min(cols - c, end - pos)));
+        if ((w & (trans ? 127 : 31)) != 0 || (c & (trans ? 127 : 31)) != 0) {
+            atomicOr(err, kErrBadSchedule);
+            pos = end;
+            return false;
+        }
+        m0 = static_cast<int>(pos / cols) * kTileM;
+        n0 = static_cast<int>(c);
+        pos += w;
+        return true;
+    }
+};
+
 template <bool kTrans>
 __global__ void __launch_bounds__(kThreads, 1)
 qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M x Kc] bf16
@@ -132,11 +163,6 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();          // 0 = even CTA (issues the MMAs)
     const int pair = blockIdx.x >> 1;
-    const int m_tile = pair % a.m_tiles;
-    const int n_tile = pair / a.m_tiles;
-    const int m0 = m_tile * kTileM;
-    const int n0 = n_tile * kTileN;                   // first output column of the pair tile
-    const int nh0 = n0 + static_cast<int>(rank) * kHalfN;   // this CTA's B half
     const int total_steps = a.main_steps + a.tail_steps;
 
     if (threadIdx.x == 0) {
@@ -147,6 +173,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
             mbar_init(&bars->empty[s], 1);
         }
         mbar_init(&bars->acc_full, 1);
+        mbar_init(&bars->acc_empty, 2 * (kThreads / 32 - 2));
         mbar_init(&bars->drain, 1);
         bars->abort_flag = 0;
         fence_barrier_init();
@@ -168,39 +195,54 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
         if (lane == 0) {
             int armed[kStages];
             for (int s = 0; s < kStages; ++s) armed[s] = -1;
-            for (int step = 0; step < total_steps; ++step) {
-                const int s = step % kStages;
-                const uint32_t ph = (step / kStages) & 1;
-                if (!mbar_wait(&bars->empty[s], ph ^ 1, abort_flag, a.err)) break;
-                uint8_t* sA = smem + s * kStageBytes;
-                uint8_t* sB = sA + kSA;
-                uint8_t* sP = sB + kSB;
-                const uint32_t a_full0 = mapa_shared(smem_u32(&bars->a_full[s]), 0);
+            TileIter tiles(a, pair);
+            int m0, n0, w;
+            uint32_t gstep = 0;                       // steps over all of this pair's tiles
+            bool ok = true;
+            while (ok && tiles.next(m0, n0, w, kTrans, a.err)) {
+                const int nh0 = n0 + static_cast<int>(rank) * (w / 2);   // this CTA's B half
                 const int arow = m0 + static_cast<int>(rank) * 128;
-                if (step < a.main_steps) {
-                    if (rank == 0) mbar_arrive_expect_tx(&bars->a_full[s], 2 * kSA);
-                    tma_load_2d_pair(sA, &tm_act, step * BK, arow, a_full0);
-                    tma_load_2d_pair(sA + kSA1, &tm_act, step * BK, arow + 256, a_full0);
-                    mbar_arrive_expect_tx(&bars->pk_full[s], kSP);
-                    if (!kTrans)
-                        tma_load_2d(sP, &tm_packed, step * (BK / 2), nh0, &bars->pk_full[s]);
-                    else
-                        tma_load_2d(sP, &tm_packed, nh0 / 2, step * BK, &bars->pk_full[s]);
-                    armed[s] = static_cast<int>(ph);
-                } else {
-                    const int j = step - a.main_steps;
-                    // (gamma T | gamma U) comes from the preceding kernel: with
-                    // a programmatic launch, wait for it here, not before the
-                    // main loop
-                    if (j == 0) grid_dependency_wait();
-                    if (rank == 0) mbar_arrive_expect_tx(&bars->a_full[s], 2 * (kSA + kSB));
-                    tma_load_2d_pair(sA, &tm_lora_a, j * BK, arow, a_full0);
-                    tma_load_2d_pair(sA + kSA1, &tm_lora_a, j * BK, arow + 256, a_full0);
-                    if (!kTrans) {
-                        tma_load_2d_pair(sB, &tm_lora_b, j * BK, nh0, a_full0);
+                for (int step = 0; step < total_steps; ++step, ++gstep) {
+                    const int s = gstep % kStages;
+                    const uint32_t ph = (gstep / kStages) & 1;
+                    if (!mbar_wait(&bars->empty[s], ph ^ 1, abort_flag, a.err)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sA = smem + s * kStageBytes;
+                    uint8_t* sB = sA + kSA;
+                    uint8_t* sP = sB + kSB;
+                    const uint32_t a_full0 = mapa_shared(smem_u32(&bars->a_full[s]), 0);
+                    if (step < a.main_steps) {
+                        if (rank == 0) mbar_arrive_expect_tx(&bars->a_full[s], 2 * kSA);
+                        tma_load_2d_pair(sA, &tm_act, step * BK, arow, a_full0);
+                        tma_load_2d_pair(sA + kSA1, &tm_act, step * BK, arow + 256, a_full0);
+                        mbar_arrive_expect_tx(&bars->pk_full[s], kSP);
+                        if (!kTrans)
+                            tma_load_2d(sP, &tm_packed, step * (BK / 2), nh0, &bars->pk_full[s]);
+                        else
+                            tma_load_2d(sP, &tm_packed, nh0 / 2, step * BK, &bars->pk_full[s]);
+                        armed[s] = static_cast<int>(ph);
                     } else {
-                        tma_load_2d_pair(sB, &tm_lora_b, nh0, j * BK, a_full0);
-                        tma_load_2d_pair(sB + 64 * 128, &tm_lora_b, nh0 + 64, j * BK, a_full0);
+                        const int j = step - a.main_steps;
+                        // nothing to expand: the stage's packed-tile barrier
+                        // still takes one phase per step, so that every
+                        // stage's barriers stay in step over the tiles
+                        mbar_arrive(&bars->pk_full[s]);
+                        armed[s] = static_cast<int>(ph);
+                        // (gamma T | gamma U) comes from the preceding kernel:
+                        // with a programmatic launch, wait for it here, not
+                        // before the main loop
+                        if (j == 0) grid_dependency_wait();
+                        if (rank == 0) mbar_arrive_expect_tx(&bars->a_full[s], 2 * (kSA + kSB));
+                        tma_load_2d_pair(sA, &tm_lora_a, j * BK, arow, a_full0);
+                        tma_load_2d_pair(sA + kSA1, &tm_lora_a, j * BK, arow + 256, a_full0);
+                        if (!kTrans) {
+                            tma_load_2d_pair(sB, &tm_lora_b, j * BK, nh0, a_full0);
+                        } else {
+                            tma_load_2d_pair(sB, &tm_lora_b, nh0, j * BK, a_full0);
+                            tma_load_2d_pair(sB + 64 * 128, &tm_lora_b, nh0 + 64, j * BK, a_full0);
+                        }
                     }
                 }
             }
@@ -217,40 +259,56 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA
         if (rank == 0 && lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16_f32(256, kTileN, false, kTrans);
+            TileIter tiles(a, pair);
+            int m0, n0, w;
+            uint32_t gstep = 0;
+            int tile = 0;
             bool ok = true;
-            for (int step = 0; step < total_steps && ok; ++step) {
-                const int s = step % kStages;
-                const uint32_t ph = (step / kStages) & 1;
-                const bool main = step < a.main_steps;
-                ok = mbar_wait_cluster(&bars->a_full[s], ph, abort_flag, a.err);
-                if (ok && main) ok = mbar_wait_cluster(&bars->deq_full[s], ph, abort_flag, a.err);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t a_base = smem_u32(smem + s * kStageBytes);
-                const uint32_t b_base = a_base + kSA;
-                int nk = BK / 16;
-                if (!main) {
-                    const int rem = a.r - (step - a.main_steps) * BK;
-                    nk = min(BK / 16, (rem + 15) / 16);
+            while (ok && tiles.next(m0, n0, w, kTrans, a.err)) {
+                // the accumulators are free once both CTAs' epilogues of the
+                // previous tile have read them
+                if (tile > 0) {
+                    ok = mbar_wait_cluster(&bars->acc_empty, (tile - 1) & 1, abort_flag, a.err);
+                    if (!ok) break;
+                    tc_fence_after();
                 }
-                for (int kk = 0; kk < nk; ++kk) {
-                    const uint64_t bdesc =
-                        kTrans ? smem_desc_sw128(b_base + kk * 2048, 64 * 128, 1024)
-                               : smem_desc_sw128(b_base + kk * 32, 16, 1024);
-#pragma unroll
-                    for (int acc = 0; acc < 2; ++acc) {
-                        const uint64_t adesc =
-                            smem_desc_sw128(a_base + acc * kSA1 + kk * 32, 16, 1024);
-                        tc_mma_bf16_pair(tmem_d + acc * kTileN, adesc, bdesc, idesc,
-                                         (step | kk) != 0 ? 1u : 0u);
+                const uint32_t idesc = idesc_bf16_f32(256, w, false, kTrans);
+                for (int step = 0; step < total_steps; ++step, ++gstep) {
+                    const int s = gstep % kStages;
+                    const uint32_t ph = (gstep / kStages) & 1;
+                    const bool main = step < a.main_steps;
+                    ok = mbar_wait_cluster(&bars->a_full[s], ph, abort_flag, a.err);
+                    // (deq_full takes a phase on LoRA steps too, with no expansion)
+                    if (ok) ok = mbar_wait_cluster(&bars->deq_full[s], ph, abort_flag, a.err);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(smem + s * kStageBytes);
+                    const uint32_t b_base = a_base + kSA;
+                    int nk = BK / 16;
+                    if (!main) {
+                        const int rem = a.r - (step - a.main_steps) * BK;
+                        nk = min(BK / 16, (rem + 15) / 16);
                     }
+                    for (int kk = 0; kk < nk; ++kk) {
+                        const uint64_t bdesc =
+                            kTrans ? smem_desc_sw128(b_base + kk * 2048, 64 * 128, 1024)
+                                   : smem_desc_sw128(b_base + kk * 32, 16, 1024);
+#pragma unroll
+                        for (int acc = 0; acc < 2; ++acc) {
+                            const uint64_t adesc =
+                                smem_desc_sw128(a_base + acc * kSA1 + kk * 32, 16, 1024);
+                            tc_mma_bf16_pair(tmem_d + acc * kTileN, adesc, bdesc, idesc,
+                                             (step | kk) != 0 ? 1u : 0u);
+                        }
+                    }
+                    tc_commit_pair(&bars->empty[s], 0x3);
                 }
-                tc_commit_pair(&bars->empty[s], 0x3);
+                if (!ok) break;
+                tc_commit_pair(&bars->acc_full, 0x3);
+                ++tile;
             }
             if (ok) {
-                tc_commit_pair(&bars->acc_full, 0x3);
-                mbar_drain(&bars->acc_full, 0, a.err);       // MMAs done before teardown
+                if (tile > 0) mbar_drain(&bars->acc_full, (tile - 1) & 1, a.err);   // MMAs done before teardown
             } else {
                 tc_commit_pair(&bars->drain, 0x1);
                 mbar_drain(&bars->drain, 0, a.err);
@@ -258,34 +316,13 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
         }
     } else {
         // ------------------------------------------------- dequantisers
-        const int group = (warp - 2) >> 2;                      // takes steps group, group+2, ...
+        const int group = (warp - 2) >> 2;                      // takes steps group, group+kGroups, ...
         const int t = ((warp - 2) & 3) * 32 + lane;             // 0..127
         const int64_t nkb = a.nkb;
         // forward: row nh0+t of W, block = step.
         // dX: row step*64 + (t & 63) of W, block nh0/64 + (t >> 6).
+        // Threads past a narrower tile's half expand rows the MMA ignores.
         const int nr = t & 63, kbl = t >> 6;
-        const int64_t kb_fixed = (nh0 >> 6) + kbl;
-        auto scale_of = [&](int step, uint32_t& code, float& meta) {
-            code = 0;
-            meta = 0.f;
-            if (step >= a.main_steps) return;
-            int64_t n, ci;
-            if (!kTrans) {
-                n = int64_t(nh0) + t;
-                ci = n * nkb + step;
-                if (n >= a.Nw) return;
-            } else {
-                n = int64_t(step) * BK + nr;
-                ci = n * nkb + kb_fixed;
-                if (n >= a.Nw || kb_fixed >= nkb) return;
-            }
-            code = __ldg(a.scale_codes + ci);
-            meta = __ldg(a.meta + (ci >> 8));
-        };
-        uint32_t code_cur, code_next;
-        float meta_cur, meta_next;
-        scale_of(group, code_cur, meta_cur);
-        scale_of(group + 2, code_next, meta_next);
         uint32_t p_off0, p_off1, b_off, swz;
         if (!kTrans) {
             const uint32_t x = static_cast<uint32_t>((t >> 2) & 1);       // 32-byte swizzle
@@ -300,38 +337,80 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
             b_off = kbl * (64 * 128) + nr * 128;
             swz = nr & 7;
         }
-        for (int step = group; step < a.main_steps; step += 2) {
-            const int s = step % kStages;
-            const uint32_t ph = (step / kStages) & 1;
-            if (!mbar_wait(&bars->pk_full[s], ph, abort_flag, a.err)) break;
-            const uint32_t sbase = smem_u32(smem + s * kStageBytes);
-            const uint32_t pbase = sbase + kSA + kSB;
-            uint32_t w[8];
-            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                         : "r"(pbase + p_off0));
-            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
-                         : "r"(pbase + p_off1));
-            const float ct = __fmul_rn(e4m3_to_float(static_cast<uint8_t>(code_cur)), meta_cur);
-            dequant_block_to_smem(w, ct, a.tab, sbase + kSA + b_off, swz);
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&bars->deq_full[s]), 0));
-            code_cur = code_next;
-            meta_cur = meta_next;
-            scale_of(step + 4, code_next, meta_next);
-        }
+        const int q = warp & 3;                     // TMEM lane quarter of this warp
+        const int acc = group & 1;                  // accumulator drained by this warp
+        const int cpart = group >> 1;               // and its share of the 32-column chunks
+        TileIter tiles(a, pair);
+        int m0, n0, w;
+        uint32_t gbase = 0;                         // pair-wide index of the tile's first step
+        int tile = 0;
+        bool ok = true;
+        while (ok && tiles.next(m0, n0, w, kTrans, a.err)) {
+            const int nh0 = n0 + static_cast<int>(rank) * (w / 2);
+            const int64_t kb_fixed = (nh0 >> 6) + kbl;
+            auto scale_of = [&](int step, uint32_t& code, float& meta) {
+                code = 0;
+                meta = 0.f;
+                if (step >= a.main_steps) return;
+                int64_t n, ci;
+                if (!kTrans) {
+                    n = int64_t(nh0) + t;
+                    ci = n * nkb + step;
+                    if (n >= a.Nw) return;
+                } else {
+                    n = int64_t(step) * BK + nr;
+                    ci = n * nkb + kb_fixed;
+                    if (n >= a.Nw || kb_fixed >= nkb) return;
+                }
+                code = __ldg(a.scale_codes + ci);
+                meta = __ldg(a.meta + (ci >> 8));
+            };
+            uint32_t code_cur, code_next;
+            float meta_cur, meta_next;
+            scale_of(group, code_cur, meta_cur);
+            scale_of(group + kGroups, code_next, meta_next);
+            // main steps are expanded; on the LoRA steps the group only passes
+            // the stage's barriers on, keeping their phases in step
+            for (int step = group; step < total_steps; step += kGroups) {
+                const uint32_t gs = gbase + static_cast<uint32_t>(step);
+                const int s = gs % kStages;
+                const uint32_t ph = (gs / kStages) & 1;
+                if (!mbar_wait(&bars->pk_full[s], ph, abort_flag, a.err)) {
+                    ok = false;
+                    break;
+                }
+                if (step >= a.main_steps) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&bars->deq_full[s]), 0));
+                    continue;
+                }
+                const uint32_t sbase = smem_u32(smem + s * kStageBytes);
+                const uint32_t pbase = sbase + kSA + kSB;
+                uint32_t wv[8];
+                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(wv[0]), "=r"(wv[1]), "=r"(wv[2]), "=r"(wv[3])
+                             : "r"(pbase + p_off0));
+                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(wv[4]), "=r"(wv[5]), "=r"(wv[6]), "=r"(wv[7])
+                             : "r"(pbase + p_off1));
+                const float ct = __fmul_rn(e4m3_to_float(static_cast<uint8_t>(code_cur)), meta_cur);
+                dequant_block_to_smem(wv, ct, a.tab, sbase + kSA + b_off, swz);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&bars->deq_full[s]), 0));
+                code_cur = code_next;
+                meta_cur = meta_next;
+                scale_of(step + 2 * kGroups, code_next, meta_next);
+            }
+            if (!ok) break;
 
-        // -------------------------------------------------- epilogue
-        if (mbar_wait(&bars->acc_full, 0, abort_flag, a.err)) {
+            // ---------------------------------------------- epilogue
+            if (!mbar_wait(&bars->acc_full, tile & 1, abort_flag, a.err)) break;
             tc_fence_after();
-            const int q = warp & 3;                 // TMEM lane quarter of this warp
-            const int acc = group;                  // accumulator drained by this warp
             const int64_t m = int64_t(m0) + acc * 256 + rank * 128 + q * 32 + lane;
             uint16_t* drow = a.D + m * a.d_cols;
 #pragma unroll 1
-            for (int c = 0; c < kTileN / 32; ++c) {
+            for (int c = cpart; c < w / 32; c += kGroups / 2) {
                 const int col = c * 32;
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + acc * kTileN + col, r);
@@ -350,6 +429,13 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
                     }
                 }
             }
+            // this warp's reads of the accumulator are done: the next tile's
+            // MMAs may overwrite it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&bars->acc_empty), 0));
+            gbase += static_cast<uint32_t>(total_steps);
+            ++tile;
         }
     }
 
@@ -390,9 +476,9 @@ cudaError_t launch_one(const CUtensorMap& act, const CUtensorMap& packed, const 
 cudaError_t launch_gemm(bool trans, const CUtensorMap& act, const CUtensorMap& packed,
                         const CUtensorMap& lora_a, const CUtensorMap& lora_b, const GemmArgs& args,
                         bool after_lora, cudaStream_t stream) {
-    const int64_t n_tiles = (args.d_cols + kTileN - 1) / kTileN;
-    const int64_t pairs = int64_t(args.m_tiles) * n_tiles;
-    if (pairs <= 0) return cudaSuccess;
+    const int64_t total = int64_t(args.m_tiles) * args.cols_lin;
+    if (total <= 0 || args.col_budget <= 0) return cudaSuccess;
+    const int64_t pairs = (total + args.col_budget - 1) / args.col_budget;
     if (2 * pairs > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     const cudaError_t e =
         trans ? launch_one<true>(act, packed, lora_a, lora_b, args, unsigned(pairs), after_lora, stream)
@@ -408,5 +494,6 @@ int gemm_tile_n() { return kTileN; }
 // with 64-byte swizzle.  The LoRA B-operand box is 128 rows (forward) or
 // 64 x 64 (dX); activation boxes are {64, 128} with 128-byte swizzle.
 int gemm_half_n() { return kHalfN; }
+int gemm_col_granule(bool trans) { return trans ? 128 : 32; }
 
 }  // namespace qnf4

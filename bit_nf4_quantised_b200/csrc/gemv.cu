@@ -233,7 +233,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
 
     if (tid == 0) {
         *abort_flag = sp.ok ? 0 : 1;
-        if (!sp.ok) atomicOr(a.err, 2);
+        if (!sp.ok) atomicOr(a.err, kErrSmemPlan);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1 + 32);           // producer lane 0 + the lanes' scale copies
             mbar_init(&empty[s], kConsumerWarps);

@@ -28,6 +28,12 @@ struct GemmArgs {
     int tail_steps;       // ceil(r / 64) LoRA steps
     int r;
     int m_tiles;
+    // Tile schedule: the output, taken as m_tiles rows of cols_lin columns
+    // (d_cols rounded up) in one linear order, is dealt to the CTA pairs in
+    // runs of col_budget columns; a pair walks its run as tiles at most 256
+    // columns wide, each ending at a 512-token row boundary or its run's end.
+    int64_t cols_lin;
+    int64_t col_budget;
     int* err;             // device error word
     Nf4Table tab;
 };
@@ -39,8 +45,11 @@ cudaError_t launch_gemm(bool trans, const CUtensorMap& act, const CUtensorMap& p
                         const CUtensorMap& lora_a, const CUtensorMap& lora_b, const GemmArgs& args,
                         bool after_lora, cudaStream_t stream);
 int gemm_tile_m();   // tokens per output tile (a CTA pair)
-int gemm_tile_n();   // output columns per output tile
-int gemm_half_n();   // output columns whose W~ rows each CTA of the pair expands
+int gemm_tile_n();   // largest output tile width
+int gemm_half_n();   // W~ rows each CTA of the pair expands for the widest tile
+// Output-tile width granularity: a multiple of 32 columns for the forward
+// (one TMEM load), of 128 for dX (each CTA's half holds whole NF4 blocks).
+int gemm_col_granule(bool trans);
 
 // -------------------------------------------------------------- K4 (LoRA)
 // out = alpha * sum_c P(i,c) * Q(c,j) over i < I, j < J (J <= 128, J % 8 == 0),

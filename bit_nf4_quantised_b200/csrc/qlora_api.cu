@@ -277,6 +277,23 @@ int check_linear_shapes(int64_t M, int64_t N, int64_t K, int r) {
     return QLORA_OK;
 }
 
+// Tile schedule of the dequant-GEMM.  With one wave of 512 x 256 tiles, one
+// tile per CTA pair.  With more, the pairs are persistent and take equal runs
+// of whole 256-wide tiles (the same makespan as waves, and each pair's TMA
+// loads of its next tile overlap the epilogue of its current one).  Narrower
+// tiles are not used: they were measured slower per column than full ones
+// (each step's dequantisation does not shrink with the tile width).
+void gemm_schedule(GemmArgs& g, bool trans) {
+    (void)trans;
+    const int64_t tn = gemm_tile_n();
+    const int64_t pairs = std::max(1, num_sms() / 2);
+    const int64_t n_tiles = cdiv(g.d_cols, tn);
+    const int64_t tiles = int64_t(g.m_tiles) * n_tiles;
+    g.cols_lin = n_tiles * tn;
+    g.col_budget = tn;
+    if (tiles > pairs) g.col_budget = cdiv(tiles, pairs) * tn;
+}
+
 cudaError_t record(const qlora_events* ev, bool begin, cudaStream_t s) {
     if (!ev) return cudaSuccess;
     void* e = begin ? ev->gemm_begin : ev->gemm_end;
@@ -484,6 +501,7 @@ int qlora_linear_forward_ex(const uint16_t* X, int64_t M, const qlora_nf4_tensor
     g.tail_steps = static_cast<int>(cdiv(r, 64));
     g.r = r;
     g.m_tiles = static_cast<int>(cdiv(M, gemm_tile_m()));
+    gemm_schedule(g, false);
     g.err = err;
     g.tab = table();
     // an event record between the two kernels would serialise them fully
@@ -581,6 +599,7 @@ int qlora_linear_backward_ex(const uint16_t* dY, const uint16_t* X, int64_t M,
         g.tail_steps = static_cast<int>(cdiv(r, 64));
         g.r = r;
         g.m_tiles = static_cast<int>(cdiv(M, gemm_tile_m()));
+        gemm_schedule(g, true);
         g.err = err;
         g.tab = table();
         QTRY(cudaEventRecord(side->fork, s));

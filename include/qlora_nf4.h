@@ -177,15 +177,17 @@ QLORA_API int qlora_linear_workspace_size(int64_t M, int64_t N, int64_t K, int r
  *   ws, ws_bytes (device workspace, >= qlora_linear_workspace_size bytes,
  *          256-byte aligned); contents on entry are ignored.  After the
  *          call its first 4 bytes hold the kernels' error word (0 = none;
- *          bit 0 = a bounded wait inside the GEMM kernel expired, in which
- *          case the outputs are unspecified).
+ *          bit 0 = a bounded wait inside a kernel expired; bit 1 = the
+ *          GEMV's shared-memory plan did not fit; bit 2 = a GEMM tile
+ *          schedule broke its width rules; with any bit set the outputs
+ *          are unspecified).
  *   M <= 16 with K % 256 == 0 runs the bandwidth-bound dequant-GEMV kernel,
  *   every other shape the tensor-core dequant-GEMM; both compute the same
  *   function.
  * Shape rules: K % 64 == 0, N % 8 == 0, K >= 64, N >= 8.
  * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE, QLORA_ERR_ALIGN (every tensor
- * 16-byte aligned, except scale_codes and meta_scale: 4-byte), QLORA_ERR_UNSUPPORTED, QLORA_ERR_WORKSPACE,
- * QLORA_ERR_CUDA.
+ * 16-byte aligned, except scale_codes and meta_scale: 4-byte),
+ * QLORA_ERR_UNSUPPORTED, QLORA_ERR_WORKSPACE, QLORA_ERR_CUDA.
  */
 QLORA_API int qlora_linear_forward(const uint16_t* X, int64_t M, const qlora_nf4_tensor* w,
                          const uint16_t* A, const uint16_t* B, int r, float scale,

@@ -64,6 +64,7 @@ CASES = [
     (129, 256, 256, 64),
     (256, 512, 1024, 128),   # two LoRA tail steps
     (17, 136, 128, 8),       # one token above the GEMV threshold
+    (4608, 2200, 2304, 16),  # two waves: per-pair column runs (forward 288, dX 384 wide)
     #                         GEMV path (M <= 16)
     (1, 1000, 2048, 16),
     (4, 512, 4160, 16),      # ragged last contraction slice
