@@ -164,6 +164,11 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
     const uint32_t rank = cluster_ctarank();          // 0 = even CTA (issues the MMAs)
     const int pair = blockIdx.x >> 1;
     const int total_steps = a.main_steps + a.tail_steps;
+    // The whole grid is resident at once (one wave, or persistent pairs), so
+    // kernels launched as its programmatic dependents (the backward's LoRA
+    // products, which do not read this kernel's output) may start now and
+    // fill the SMs it leaves idle.
+    launch_dependents();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {

@@ -81,6 +81,10 @@ struct SkinnyArgs {
     uint16_t* cvt_dst;
     float cvt_scale;
     int* err_zero;
+    int trigger_dependents;   // let the next kernel (a programmatic dependent) start at once
+    int programmatic;         // launch as the previous kernel's programmatic dependent; the
+                              // kernel never waits for that grid, so its inputs must come
+                              // from earlier work
 };
 cudaError_t launch_skinny(bool p_kmajor, bool q_kmajor, const SkinnyArgs& a, cudaStream_t stream);
 

@@ -121,37 +121,6 @@ int check_tensor(const qlora_nf4_tensor* w) {
     return QLORA_OK;
 }
 
-// Per device: a high-priority stream for the input-gradient GEMM, so that
-// the backward's LoRA side products (dB, dA) run beside it on the caller's
-// stream and fill the SMs its last wave of tiles leaves idle, and the two
-// events of that fork and join.  The mutex keeps concurrent callers from
-// interleaving their use of the events.
-struct SideStream {
-    std::mutex mu;
-    cudaStream_t hp = nullptr;
-    cudaEvent_t fork = nullptr, join = nullptr;
-    bool ready = false;
-};
-
-SideStream* side_stream() {
-    constexpr int kMaxDevices = 64;
-    static SideStream devs[kMaxDevices];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    SideStream& d = devs[dev];
-    std::lock_guard<std::mutex> lock(d.mu);
-    if (!d.ready) {
-        int least = 0, greatest = 0;
-        if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return nullptr;
-        if (cudaStreamCreateWithPriority(&d.hp, cudaStreamNonBlocking, greatest) != cudaSuccess ||
-            cudaEventCreateWithFlags(&d.fork, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&d.join, cudaEventDisableTiming) != cudaSuccess)
-            return nullptr;
-        d.ready = true;
-    }
-    return &d;
-}
-
 int num_sms() {
     int dev = 0, n = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -332,15 +301,18 @@ SkinnyArgs skinny_args(const uint16_t* P, const uint16_t* Q, int64_t I, int64_t 
     return a;
 }
 
-// T = X A^T -> optional fp32 T_save and bf16 gamma*T padded to rp columns
+// T = X A^T -> optional fp32 T_save and bf16 gamma*T padded to rp columns.
+// trigger: a GEMM launched next as its programmatic dependent may start at once.
 cudaError_t run_T(const uint16_t* X, const uint16_t* A, int64_t M, int64_t K, int r, float gamma,
-                  float* T_save, uint16_t* Gt, int64_t rp, int* err_zero, cudaStream_t s) {
+                  float* T_save, uint16_t* Gt, int64_t rp, int* err_zero, bool trigger,
+                  cudaStream_t s) {
     SkinnyArgs a = skinny_args(X, A, M, r, K, K, K);
     a.out = T_save;
     a.out_bf16 = Gt;
     a.ldb = rp;
     a.beta = gamma;
     a.err_zero = err_zero;
+    a.trigger_dependents = trigger ? 1 : 0;
     return launch_skinny(true, true, a, s);
 }
 
@@ -476,7 +448,7 @@ int qlora_linear_forward_ex(const uint16_t* X, int64_t M, const qlora_nf4_tensor
         QTRY(launch_gemv_finalize(f, s));
         return QLORA_OK;
     }
-    QTRY(run_T(X, A, M, K, r, scale, T_save, Gt, p.rp, err, s));
+    QTRY(run_T(X, A, M, K, r, scale, T_save, Gt, p.rp, err, true, s));
 
     // B [N x r] is read in place: the 64-wide TMA box zero-fills columns >= r
     CUtensorMap m_act, m_packed, m_la, m_lb;
@@ -551,7 +523,7 @@ int qlora_linear_backward_ex(const uint16_t* dY, const uint16_t* X, int64_t M,
     int* err_first = err;                 // cleared by the first kernel of the call
 
     if (!T_saved) {                       // recompute gamma * T in bf16
-        QTRY(run_T(X, A, M, K, r, scale, nullptr, Gt, p.rp, err_first, s));
+        QTRY(run_T(X, A, M, K, r, scale, nullptr, Gt, p.rp, err_first, false, s));
         err_first = nullptr;
     }
     // U = dY B -> gamma * U in bf16; converts a saved T to gamma * T on the side
@@ -568,13 +540,13 @@ int qlora_linear_backward_ex(const uint16_t* dY, const uint16_t* X, int64_t M,
         a.err_zero = err_first;
         QTRY(launch_skinny(true, false, a, s));
     }
-    // dX = dY W~ + (gamma U) A on the high-priority side stream, forked after
-    // U; dB = dY^T (gamma T) and dA^T = X^T (gamma U) follow U on the caller's
-    // stream and run beside the GEMM; the caller's stream then joins it.
-    SideStream* side = dX ? side_stream() : nullptr;
-    if (dX && !side) return QLORA_ERR_CUDA;
-    std::unique_lock<std::mutex> lock;
-    if (side) lock = std::unique_lock<std::mutex>(side->mu);
+    // dX = dY W~ + (gamma U) A, launched as U's programmatic dependent (U does
+    // not signal early, so the GEMM starts as U completes; it waits for U
+    // again only before its LoRA steps).  dB = dY^T (gamma T) and
+    // dA^T = X^T (gamma U) follow as the GEMM's programmatic dependents: the
+    // GEMM signals on entry and they never wait for it (they read only U's
+    // outputs, dY and X), so they run beside it on the SMs it leaves idle.
+    // Profiling events between the kernels make the launches ordinary.
     if (dX) {
         // A [r x K] is read in place: the 64-row TMA box zero-fills rows >= r
         CUtensorMap m_act, m_packed, m_la, m_lb;
@@ -602,17 +574,16 @@ int qlora_linear_backward_ex(const uint16_t* dY, const uint16_t* X, int64_t M,
         gemm_schedule(g, true);
         g.err = err;
         g.tab = table();
-        QTRY(cudaEventRecord(side->fork, s));
-        QTRY(cudaStreamWaitEvent(side->hp, side->fork, 0));
-        QTRY(record(ev, true, side->hp));
-        QTRY(launch_gemm(true, m_act, m_packed, m_la, m_lb, g, false, side->hp));
-        QTRY(record(ev, false, side->hp));
-        QTRY(cudaEventRecord(side->join, side->hp));
+        QTRY(record(ev, true, s));
+        QTRY(launch_gemm(true, m_act, m_packed, m_la, m_lb, g, ev == nullptr, s));
+        QTRY(record(ev, false, s));
     }
     {
         SkinnyArgs a = skinny_args(dY, Gt, N, r, M, N, p.rp);
         a.out = dB;
         a.accumulate = accumulate;
+        a.programmatic = 1;
+        a.trigger_dependents = 1;      // dA need not wait for dB either
         QTRY(launch_skinny(false, false, a, s));
     }
     {
@@ -620,9 +591,9 @@ int qlora_linear_backward_ex(const uint16_t* dY, const uint16_t* X, int64_t M,
         a.out = dA;
         a.transpose = 1;
         a.accumulate = accumulate;
+        a.programmatic = 1;
         QTRY(launch_skinny(false, false, a, s));
     }
-    if (dX) QTRY(cudaStreamWaitEvent(s, side->join, 0));
     return QLORA_OK;
 }
 

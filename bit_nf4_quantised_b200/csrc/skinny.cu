@@ -80,7 +80,7 @@ skinny_kernel(SkinnyArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
     // a dependent tensor-core GEMM may start streaming its weight tiles now;
     // it waits for this grid only before it reads this kernel's output
-    launch_dependents();
+    if (a.trigger_dependents) launch_dependents();
     cg::cluster_group cluster = cg::this_cluster();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t i0 = int64_t(blockIdx.x) * TI;
@@ -275,13 +275,15 @@ cudaError_t run_skinny(const SkinnyArgs& a, cudaStream_t stream) {
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = Tl::kSmem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 1;
     attr[0].val.clusterDim.y = static_cast<unsigned>(a.splits);
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = a.programmatic ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, skinny_kernel<PK, QK, JT16>, a);
 }
 

@@ -22,11 +22,14 @@
  *   - The return value is a qlora_status.  Argument errors are detected on
  *     the host before anything is launched and leave every output untouched.
  *     QLORA_ERR_CUDA reports a failed launch (cudaGetLastError()).
- *   - Global state is limited to, per device: the internal high-priority
- *     stream and two events that qlora_linear_backward forks its input-
- *     gradient GEMM onto (created on first use, guarded by a lock), and the
- *     scratch array of qlora_linear_forward_noalloc.  Calls on different
- *     streams with disjoint outputs and workspaces may run concurrently.
+ *   - The only global state is the scratch array of
+ *     qlora_linear_forward_noalloc.  Calls on different streams with
+ *     disjoint outputs and workspaces may run concurrently.
+ *   - Within a call, some kernels are launched as programmatic dependents of
+ *     the kernel before them (they may start before it finishes and wait for
+ *     it, if at all, only where they read its output).  The call's first
+ *     kernel is an ordinary launch, so everything earlier on `stream` is
+ *     complete before any of the call's kernels starts.
  */
 #ifndef QLORA_NF4_H
 #define QLORA_NF4_H
@@ -211,12 +214,9 @@ QLORA_API int qlora_linear_forward(const uint16_t* X, int64_t M, const qlora_nf4
  *   M = 0 writes zero gradients (or leaves them unchanged when accumulating);
  *   dY and X may then be NULL.
  *   other arguments as in qlora_linear_forward.
- * Streams: when dX is computed, its tensor-core GEMM runs on an internal
- * high-priority stream forked from `stream` (after the kernel producing
- * dY B) and joined back into `stream` before the call returns, so that the
- * adapter-gradient kernels on `stream` fill the SMs the GEMM leaves idle.
- * Ordering against other work on `stream` is as if everything ran on it; the
- * fork and join are plain event waits, valid under stream capture.
+ * The adapter-gradient kernels (dA, dB) are launched as programmatic
+ * dependents of the dX GEMM and run beside it on the SMs it leaves idle;
+ * they read only dY, X and the first kernel's output.
  * Errors as qlora_linear_forward.
  */
 QLORA_API int qlora_linear_backward(const uint16_t* dY, const uint16_t* X, int64_t M,
@@ -229,9 +229,10 @@ QLORA_API int qlora_linear_backward(const uint16_t* dY, const uint16_t* X, int64
 /*
  * Profiling variants.  Identical to qlora_linear_forward / _backward, plus
  * optional CUDA events (cudaEvent_t handles created by the caller, either may
- * be NULL) that are recorded immediately before and after the launch of the
- * layer's main weight kernel, on the stream it runs on (`stream`, or the
- * internal stream for dX in the backward): the tensor-core dequant-GEMM
+ * be NULL) that are recorded on `stream` immediately before and after the
+ * launch of the layer's main weight kernel (an event between two kernels
+ * makes the second an ordinary launch, so with events the kernels no longer
+ * overlap): the tensor-core dequant-GEMM
  * (forward Y, or dX in the backward), or the dequant-GEMV when M <= 16.  They
  * let a caller time that kernel inside a running workload without a profiler.
  * ev itself may be NULL.
