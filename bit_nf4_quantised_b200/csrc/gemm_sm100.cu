@@ -72,8 +72,13 @@ struct __align__(8) Barriers {
     int abort_flag;
 };
 
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align slack*/ + 256 /*barriers*/;
-static_assert(sizeof(Barriers) <= 256, "barrier block");
+// Epilogue staging: 1 KiB per epilogue warp (32 rows x 16 bf16 columns),
+// written out by TMA tensor stores.
+constexpr int kStageOut = 1024;
+constexpr int kOutBytes = kGroups * 4 * kStageOut;
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align slack*/ + 1024 /*barriers*/ + kOutBytes;
+static_assert(sizeof(Barriers) <= 1024, "barrier block");
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 // 64 nibbles (8 words) of one NF4 block -> 64 bf16, stored as 8 16-byte chunks
 // of a 128-byte swizzled row.  Table entries are bf16_rne(fp32(q[i] * ct)).
@@ -153,6 +158,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
                   const __grid_constant__ CUtensorMap tm_packed, // packed W  [N x K/2] u8
                   const __grid_constant__ CUtensorMap tm_lora_a, // gamma T|U [M x rp] bf16
                   const __grid_constant__ CUtensorMap tm_lora_b, // B [N x rp] | A [rp x K]
+                  const __grid_constant__ CUtensorMap tm_out,    // D [M x d_cols] bf16, box {16, 32}
                   GemmArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -186,6 +192,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
         prefetch_tensormap(&tm_packed);
         prefetch_tensormap(&tm_lora_a);
         prefetch_tensormap(&tm_lora_b);
+        prefetch_tensormap(&tm_out);
     }
     if (warp == 1) {
         tmem_alloc_pair(&bars->tmem_slot, kTmemCols);
@@ -345,6 +352,8 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
         const int q = warp & 3;                     // TMEM lane quarter of this warp
         const int acc = group & 1;                  // accumulator drained by this warp
         const int cpart = group >> 1;               // and its share of the 32-column chunks
+        const uint32_t out_stage = smem_u32(smem + kStages * kStageBytes + 1024) +
+                                   static_cast<uint32_t>((warp - 2) * kStageOut);
         TileIter tiles(a, pair);
         int m0, n0, w;
         uint32_t gbase = 0;                         // pair-wide index of the tile's first step
@@ -412,25 +421,37 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
             // ---------------------------------------------- epilogue
             if (!mbar_wait(&bars->acc_full, tile & 1, abort_flag, a.err)) break;
             tc_fence_after();
-            const int64_t m = int64_t(m0) + acc * 256 + rank * 128 + q * 32 + lane;
-            uint16_t* drow = a.D + m * a.d_cols;
+            // Each 32-column TMEM chunk leaves as two 32-row x 16-column bf16
+            // boxes staged in this warp's 1 KiB and written by a TMA tensor
+            // store (full 32-byte sectors; rows past M, columns past d_cols
+            // are not written).
+            const int row0 = m0 + acc * 256 + static_cast<int>(rank) * 128 + q * 32;
 #pragma unroll 1
             for (int c = cpart; c < w / 32; c += kGroups / 2) {
                 const int col = c * 32;
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + acc * kTileN + col, r);
                 tc_wait_ld();
-                uint32_t p[16];
 #pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    p[j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-                if (m < a.M) {
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t p[8];
 #pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        const int64_t gc = int64_t(n0) + col + g * 8;
-                        if (gc < a.d_cols)
-                            *reinterpret_cast<uint4*>(drow + gc) =
-                                make_uint4(p[4 * g], p[4 * g + 1], p[4 * g + 2], p[4 * g + 3]);
+                    for (int j = 0; j < 8; ++j)
+                        p[j] = pack_bf16x2(__uint_as_float(r[16 * h + 2 * j]), __uint_as_float(r[16 * h + 2 * j + 1]));
+                    if (lane == 0) bulk_wait_read_all();    // the previous box has left the buffer
+                    __syncwarp();
+                    const uint32_t dst = out_stage + lane * 32;
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(p[0]), "r"(p[1]),
+                                 "r"(p[2]), "r"(p[3])
+                                 : "memory");
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16), "r"(p[4]),
+                                 "r"(p[5]), "r"(p[6]), "r"(p[7])
+                                 : "memory");
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tm_out, n0 + col + 16 * h, row0, out_stage);
+                        bulk_commit();
                     }
                 }
             }
@@ -442,6 +463,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
             gbase += static_cast<uint32_t>(total_steps);
             ++tile;
         }
+        if (lane == 0) bulk_wait_all();             // this warp's output stores have landed
     }
 
     tc_fence_before();
@@ -454,8 +476,8 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
 
 template <bool kTrans>
 cudaError_t launch_one(const CUtensorMap& act, const CUtensorMap& packed, const CUtensorMap& la,
-                       const CUtensorMap& lb, const GemmArgs& args, unsigned pairs, bool after_lora,
-                       cudaStream_t stream) {
+                       const CUtensorMap& lb, const CUtensorMap& out, const GemmArgs& args,
+                       unsigned pairs, bool after_lora, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(qlora_gemm_kernel<kTrans>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
@@ -473,21 +495,21 @@ cudaError_t launch_one(const CUtensorMap& act, const CUtensorMap& packed, const 
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = after_lora ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, qlora_gemm_kernel<kTrans>, act, packed, la, lb, args);
+    return cudaLaunchKernelEx(&cfg, qlora_gemm_kernel<kTrans>, act, packed, la, lb, out, args);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm(bool trans, const CUtensorMap& act, const CUtensorMap& packed,
-                        const CUtensorMap& lora_a, const CUtensorMap& lora_b, const GemmArgs& args,
-                        bool after_lora, cudaStream_t stream) {
+                        const CUtensorMap& lora_a, const CUtensorMap& lora_b, const CUtensorMap& out,
+                        const GemmArgs& args, bool after_lora, cudaStream_t stream) {
     const int64_t total = int64_t(args.m_tiles) * args.cols_lin;
     if (total <= 0 || args.col_budget <= 0) return cudaSuccess;
     const int64_t pairs = (total + args.col_budget - 1) / args.col_budget;
     if (2 * pairs > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     const cudaError_t e =
-        trans ? launch_one<true>(act, packed, lora_a, lora_b, args, unsigned(pairs), after_lora, stream)
-              : launch_one<false>(act, packed, lora_a, lora_b, args, unsigned(pairs), after_lora, stream);
+        trans ? launch_one<true>(act, packed, lora_a, lora_b, out, args, unsigned(pairs), after_lora, stream)
+              : launch_one<false>(act, packed, lora_a, lora_b, out, args, unsigned(pairs), after_lora, stream);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

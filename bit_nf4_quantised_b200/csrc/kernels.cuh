@@ -41,9 +41,10 @@ struct GemmArgs {
 // after_lora: the kernel directly before it in `stream` is the LoRA kernel
 // that writes (gamma T | gamma U); the GEMM is then launched as its
 // programmatic dependent and waits for it only before the LoRA steps.
+// out: 2-D map of D [M x d_cols] bf16, box {16 columns, 32 rows}, no swizzle.
 cudaError_t launch_gemm(bool trans, const CUtensorMap& act, const CUtensorMap& packed,
-                        const CUtensorMap& lora_a, const CUtensorMap& lora_b, const GemmArgs& args,
-                        bool after_lora, cudaStream_t stream);
+                        const CUtensorMap& lora_a, const CUtensorMap& lora_b, const CUtensorMap& out,
+                        const GemmArgs& args, bool after_lora, cudaStream_t stream);
 int gemm_tile_m();   // tokens per output tile (a CTA pair)
 int gemm_tile_n();   // largest output tile width
 int gemm_half_n();   // W~ rows each CTA of the pair expands for the widest tile

@@ -451,8 +451,10 @@ int qlora_linear_forward_ex(const uint16_t* X, int64_t M, const qlora_nf4_tensor
     QTRY(run_T(X, A, M, K, r, scale, T_save, Gt, p.rp, err, true, s));
 
     // B [N x r] is read in place: the 64-wide TMA box zero-fills columns >= r
-    CUtensorMap m_act, m_packed, m_la, m_lb;
-    bool ok = make_map_2d(&m_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 128,
+    CUtensorMap m_act, m_packed, m_la, m_lb, m_out;
+    bool ok = make_map_2d(&m_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, N * 2, 16, 32,
+                          CU_TENSOR_MAP_SWIZZLE_NONE) &&
+              make_map_2d(&m_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, 64, 128,
                           CU_TENSOR_MAP_SWIZZLE_128B) &&
               make_map_2d(&m_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->packed, K / 2, N, K / 2, 32,
                           gemm_half_n(), CU_TENSOR_MAP_SWIZZLE_32B) &&
@@ -478,7 +480,7 @@ int qlora_linear_forward_ex(const uint16_t* X, int64_t M, const qlora_nf4_tensor
     g.tab = table();
     // an event record between the two kernels would serialise them fully
     QTRY(record(ev, true, s));
-    QTRY(launch_gemm(false, m_act, m_packed, m_la, m_lb, g, ev == nullptr, s));
+    QTRY(launch_gemm(false, m_act, m_packed, m_la, m_lb, m_out, g, ev == nullptr, s));
     QTRY(record(ev, false, s));
     return QLORA_OK;
 }
@@ -549,8 +551,10 @@ int qlora_linear_backward_ex(const uint16_t* dY, const uint16_t* X, int64_t M,
     // Profiling events between the kernels make the launches ordinary.
     if (dX) {
         // A [r x K] is read in place: the 64-row TMA box zero-fills rows >= r
-        CUtensorMap m_act, m_packed, m_la, m_lb;
-        bool ok = make_map_2d(&m_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, 128,
+        CUtensorMap m_act, m_packed, m_la, m_lb, m_out;
+        bool ok = make_map_2d(&m_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dX, K, M, K * 2, 16, 32,
+                              CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                  make_map_2d(&m_act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, N, M, N * 2, 64, 128,
                               CU_TENSOR_MAP_SWIZZLE_128B) &&
                   make_map_2d(&m_packed, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->packed, K / 2, N, K / 2,
                               gemm_half_n() / 2, 64, CU_TENSOR_MAP_SWIZZLE_64B) &&
@@ -575,7 +579,7 @@ int qlora_linear_backward_ex(const uint16_t* dY, const uint16_t* X, int64_t M,
         g.err = err;
         g.tab = table();
         QTRY(record(ev, true, s));
-        QTRY(launch_gemm(true, m_act, m_packed, m_la, m_lb, g, ev == nullptr, s));
+        QTRY(launch_gemm(true, m_act, m_packed, m_la, m_lb, m_out, g, ev == nullptr, s));
         QTRY(record(ev, false, s));
     }
     {
