@@ -72,10 +72,12 @@ struct __align__(8) Barriers {
     int abort_flag;
 };
 
-// Epilogue staging: 1 KiB per epilogue warp (32 rows x 16 bf16 columns),
-// written out by TMA tensor stores.
-constexpr int kStageOut = 1024;
-constexpr int kOutBytes = kGroups * 4 * kStageOut;
+// Epilogue: the last two dequantiser groups (8 warps) drain the
+// accumulators; each stages its output in two alternating 1 KiB buffers of
+// 32 rows x 16 bf16 columns written out by TMA tensor stores.
+constexpr int kEpiWarps = 8;
+constexpr int kStageOut = 2048;
+constexpr int kOutBytes = kEpiWarps * kStageOut;
 constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align slack*/ + 1024 /*barriers*/ + kOutBytes;
 static_assert(sizeof(Barriers) <= 1024, "barrier block");
 static_assert(kSmemBytes <= 232448, "shared memory per CTA");
@@ -184,7 +186,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
             mbar_init(&bars->empty[s], 1);
         }
         mbar_init(&bars->acc_full, 1);
-        mbar_init(&bars->acc_empty, 2 * (kThreads / 32 - 2));
+        mbar_init(&bars->acc_empty, 2 * kEpiWarps);
         mbar_init(&bars->drain, 1);
         bars->abort_flag = 0;
         fence_barrier_init();
@@ -350,10 +352,13 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
             swz = nr & 7;
         }
         const int q = warp & 3;                     // TMEM lane quarter of this warp
-        const int acc = group & 1;                  // accumulator drained by this warp
-        const int cpart = group >> 1;               // and its share of the 32-column chunks
+        // groups kGroups-2 and kGroups-1 drain accumulators 0 and 1; the first
+        // groups go straight on to the next tile's first steps
+        const bool epi = group >= kGroups - 2;
+        const int acc = group - (kGroups - 2);
         const uint32_t out_stage = smem_u32(smem + kStages * kStageBytes + 1024) +
-                                   static_cast<uint32_t>((warp - 2) * kStageOut);
+                                   static_cast<uint32_t>((epi ? warp - 2 - 4 * (kGroups - 2) : 0) * kStageOut);
+        uint32_t nbox = 0;                          // boxes this warp has staged (buffer = nbox & 1)
         TileIter tiles(a, pair);
         int m0, n0, w;
         uint32_t gbase = 0;                         // pair-wide index of the tile's first step
@@ -418,48 +423,60 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
             }
             if (!ok) break;
 
-            // ---------------------------------------------- epilogue
+            // Every group waits for the tile's MMAs to finish: then every phase
+            // of every stage barrier of this tile is complete.  A stage's
+            // owning group changes at a tile boundary (a tile's step count
+            // need not be a multiple of kGroups), and a parity wait is only
+            // sound when the waiter is at most one phase ahead of the last
+            // completed phase, so no group may start the next tile earlier.
             if (!mbar_wait(&bars->acc_full, tile & 1, abort_flag, a.err)) break;
-            tc_fence_after();
-            // Each 32-column TMEM chunk leaves as two 32-row x 16-column bf16
-            // boxes staged in this warp's 1 KiB and written by a TMA tensor
-            // store (full 32-byte sectors; rows past M, columns past d_cols
-            // are not written).
-            const int row0 = m0 + acc * 256 + static_cast<int>(rank) * 128 + q * 32;
+
+            // ---------------------------------------------- epilogue
+            if (epi) {
+                tc_fence_after();
+                // Each 32-column TMEM chunk leaves as two 32-row x 16-column
+                // bf16 boxes, staged alternately in this warp's two buffers
+                // and written by TMA tensor stores (full 32-byte sectors; rows
+                // past M, columns past d_cols are not written), so that one
+                // box's copy-out overlaps the next box's staging.
+                const int row0 = m0 + acc * 256 + static_cast<int>(rank) * 128 + q * 32;
 #pragma unroll 1
-            for (int c = cpart; c < w / 32; c += kGroups / 2) {
-                const int col = c * 32;
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + acc * kTileN + col, r);
-                tc_wait_ld();
+                for (int c = 0; c < w / 32; ++c) {
+                    const int col = c * 32;
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(tmem_d + (static_cast<uint32_t>(q * 32) << 16) + acc * kTileN + col, r);
+                    tc_wait_ld();
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t p[8];
+                    for (int h = 0; h < 2; ++h, ++nbox) {
+                        const uint32_t buf = out_stage + (nbox & 1) * 1024;
+                        uint32_t p[8];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        p[j] = pack_bf16x2(__uint_as_float(r[16 * h + 2 * j]), __uint_as_float(r[16 * h + 2 * j + 1]));
-                    if (lane == 0) bulk_wait_read_all();    // the previous box has left the buffer
-                    __syncwarp();
-                    const uint32_t dst = out_stage + lane * 32;
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(p[0]), "r"(p[1]),
-                                 "r"(p[2]), "r"(p[3])
-                                 : "memory");
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16), "r"(p[4]),
-                                 "r"(p[5]), "r"(p[6]), "r"(p[7])
-                                 : "memory");
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&tm_out, n0 + col + 16 * h, row0, out_stage);
-                        bulk_commit();
+                        for (int j = 0; j < 8; ++j)
+                            p[j] = pack_bf16x2(__uint_as_float(r[16 * h + 2 * j]),
+                                               __uint_as_float(r[16 * h + 2 * j + 1]));
+                        if (lane == 0) bulk_wait_read_all_but_one();   // this buffer's last box has left
+                        __syncwarp();
+                        const uint32_t dst = buf + lane * 32;
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(p[0]),
+                                     "r"(p[1]), "r"(p[2]), "r"(p[3])
+                                     : "memory");
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16), "r"(p[4]),
+                                     "r"(p[5]), "r"(p[6]), "r"(p[7])
+                                     : "memory");
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tm_out, n0 + col + 16 * h, row0, buf);
+                            bulk_commit();
+                        }
                     }
                 }
+                // this warp's reads of the accumulator are done: the next
+                // tile's MMAs may overwrite it
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&bars->acc_empty), 0));
             }
-            // this warp's reads of the accumulator are done: the next tile's
-            // MMAs may overwrite it
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&bars->acc_empty), 0));
             gbase += static_cast<uint32_t>(total_steps);
             ++tile;
         }
