@@ -42,8 +42,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 LAUNCHES_PER_STEP = 2 + 4
 # ncu DRAM traffic (read + write bytes) of one dequant-GEMM launch of this
 # workload, valid only for the source it was captured on.
-GEMM_TRAFFIC = {"source_sha": "62e1eb3c30c6563c", "fwd_bytes": (42.977536 + 2.707712) * 1e6,
-                "dx_bytes": (43.006720 + 2.944256) * 1e6}
+GEMM_TRAFFIC = {"source_sha": "4c197ac7a6e2f9bb", "fwd_bytes": (44.354816 + 7.093248) * 1e6,
+                "dx_bytes": (44.429568 + 7.148032) * 1e6}
 
 
 def _peaks():
