@@ -62,55 +62,80 @@ def _source_sha():
 
 
 class Clocks:
-    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons, read through NVML (read-only queries)
+    every 2 ms by a host thread with host timestamps.  mark() brackets the
+    timed region; stop() summarises the samples inside it (falling back to
+    all samples, and saying so, when the region was shorter than a few
+    sampling periods).  nvidia-smi reads the same counters."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
 
     def __init__(self, index: int):
         self.index = index
-        self.proc = None
-        self.path = None
+        self.samples = []          # (host time, sm MHz, reasons bitmask)
+        self.window = None
+        self._stop = False
+        self._thread = None
+        self.error = None
 
     def start(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except OSError:
-            self.proc = None
-        time.sleep(0.3)
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report it instead of clocks
+            self.error = f"NVML unavailable: {type(e).__name__}"
+            return
+
+        def run():
+            nv = self._nvml
+            while not self._stop:
+                try:
+                    mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                    self.samples.append((time.perf_counter(), mhz, rs))
+                except Exception:
+                    pass
+                time.sleep(0.002)
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
+
+    def mark(self, t0: float, t1: float):
+        self.window = (t0, t1)
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
+        if self.error or self._thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.error or "not started"]}
+        self._stop = True
+        self._thread.join(timeout=5)
+        sel = self.samples
+        scope = "timed region"
+        if self.window is not None:
+            inside = [x for x in self.samples if self.window[0] <= x[0] <= self.window[1]]
+            if len(inside) >= 3:
+                sel = inside
+            else:
+                scope = "whole measurement (timed region shorter than the sampling period)"
+        reasons = set()
+        for _, _, rs in sel:
+            for name, const in self.REASONS:
+                bit = getattr(self._nvml, const, 0)
+                if bit and (rs & bit):
+                    reasons.add(name)
         try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for ln in f:
-                p = [x.strip() for x in ln.split(",")]
-                if len(p) < 9:
-                    continue
-                try:
-                    sm.append(float(p[1]))
-                    smax.append(float(p[2]))
-                except ValueError:
-                    continue
-                for nm, v in zip(names, p[5:9]):
-                    if v.lower() == "active":
-                        reasons.add(nm)
-        os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+            self._nvml.nvmlShutdown()
+        except Exception:
+            pass
+        return {"sm_mhz": statistics.median([m for _, m, _ in sel]) if sel else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons), "samples": len(sel),
+                "scope": scope}
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -359,11 +384,13 @@ def run_gpu(args):
     _barrier(world)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    h0 = time.perf_counter()
     t0.record()
     for i in range(K):
         one(i)
     t1.record()
     _barrier(world)
+    clocks.mark(h0, time.perf_counter())
     # The GEMM kernels' own durations come from the same K steps run again
     # right after, with CUDA events recorded around the two GEMM launches on
     # the streams they run on.  They are not recorded inside the timed steps:
