@@ -400,3 +400,41 @@ def linear_backward(dY, X, Wt, A, B, gamma):
     dA = gamma * (U.T @ X)
     dB = gamma * (dY.T @ (X @ A.T))
     return dX, dA, dB, U
+
+
+# ---------------------------------------------------------------------------
+# Merge for export.  "QLoRA, explained", "The forward pass and gradients": the
+# fine-tuned model is W~ + gamma B A (the adapter on the quantised base); the
+# same page's "Failure modes" ("Quality loss at merge time") names
+# dequantising W~ to bf16, adding the adapter and keeping the result in bf16
+# as the merge that preserves it.  "QLoRA" (finetunellm.com), "What it costs
+# you": a 4-bit deployment then quantises the merged bf16 weight again
+# (quantize() applied to its values).  Reading: the sum is exact (fp64 here)
+# and rounded to bf16 once, to nearest with ties to even.
+# ---------------------------------------------------------------------------
+BF16_MIN_SUBNORMAL_EXP = -133          # 2**-133, the smallest positive bf16
+
+
+def bf16_rne_f64(x: np.ndarray) -> np.ndarray:
+    """bf16 bits of fp64 values rounded to nearest, ties to even, directly
+    from fp64 (no intermediate fp32 rounding).  bf16 keeps 8 significant
+    bits, so the spacing at x = m 2^e (0.5 <= |m| < 1) is 2^(e-8), never finer
+    than the smallest subnormal; values that round to 2^128 or beyond become
+    infinities."""
+    x = np.asarray(x, dtype=np.float64)
+    _, e = np.frexp(x)
+    step = np.maximum(e - 8, BF16_MIN_SUBNORMAL_EXP)
+    with np.errstate(invalid="ignore", over="ignore"):
+        y = np.ldexp(np.rint(np.ldexp(x, -step)), step)     # rint: ties to even
+        y = np.where(np.abs(y) >= 2.0 ** 128, np.copysign(np.inf, x), y)
+        bits = (y.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    return np.where(np.isnan(x), np.uint16(0x7FC0), bits)
+
+
+def merge(packed, scale_codes, meta, rows: int, cols: int, A, B, gamma):
+    """-> (exact [rows, cols] fp64 value of W~ + gamma B A, its bf16 bits).
+    gamma is taken at fp32, the precision the library receives it in."""
+    Wt = dequantize(packed, scale_codes, meta, rows, cols).astype(np.float64)
+    g = float(np.float32(gamma))
+    exact = Wt + g * (np.asarray(B, np.float64) @ np.asarray(A, np.float64))
+    return exact, bf16_rne_f64(exact)

@@ -400,3 +400,134 @@ def test_no_lora_reduces_to_plain_product():
     assert np.allclose(Y, np.einsum("mk,nk->mn", X, W))
     dX, dA, dB, _ = o.linear_backward(dY, X, W, A, np.zeros_like(B), g)
     assert np.allclose(dX, np.einsum("mn,nk->mk", dY, W)) and np.allclose(dA, 0)
+
+
+# --------------------------------------------------------------------------
+# Merge for export
+# --------------------------------------------------------------------------
+def _all_finite_bf16():
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    with np.errstate(invalid="ignore"):
+        vals = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    keep = np.isfinite(vals)
+    return bits[keep], vals[keep]
+
+
+def _brute_bf16(x, bits, vals):
+    """Nearest finite bf16 by exhaustive search, ties to the even bit pattern;
+    beyond the overflow threshold (halfway past the largest finite value) an
+    infinity."""
+    out = np.empty(x.size, np.uint16)
+    pos = np.unique(vals[vals > 0])
+    top = float(pos[-1])
+    thresh = top + (top - float(pos[-2])) / 2
+    for i, xi in enumerate(x):
+        if abs(xi) >= thresh:
+            out[i] = 0x7F80 if xi > 0 else 0xFF80
+            continue
+        d = np.abs(vals - xi)
+        cand = np.flatnonzero(d == d.min())
+        # +0 and -0 are both at distance |x| from a tiny x: keep the sign of x
+        cand = [c for c in cand if vals[c] != 0 or np.signbit(vals[c]) == np.signbit(xi)] or list(cand)
+        even = [c for c in cand if (bits[c] & 1) == 0]
+        out[i] = bits[(even or cand)[0]]
+    return out
+
+
+def test_bf16_rne_f64_against_exhaustive_search():
+    bits, vals = _all_finite_bf16()
+    rng = np.random.default_rng(21)
+    pos = np.unique(vals[vals > 0])
+    lo = pos[rng.integers(0, pos.size - 1, 300)]
+    hi = np.array([pos[np.searchsorted(pos, v) + 1] for v in lo])
+    ties = (lo + hi) / 2                                     # exact in fp64
+    x = np.concatenate([
+        rng.standard_normal(400) * np.exp(rng.uniform(-60, 60, 400)),
+        ties, -ties, np.nextafter(ties, 0), np.nextafter(ties, np.inf),
+        [0.0, -0.0, 2.0 ** -133, 2.0 ** -134, 1.5 * 2.0 ** -134, 3 * 2.0 ** -135,
+         3.3e38, 3.39e38, 3.4e38, -3.4e38, 1e39],
+    ])
+    assert np.array_equal(o.bf16_rne_f64(x), _brute_bf16(x, bits, vals))
+
+
+def test_bf16_rne_f64_matches_torch_on_fp32_values():
+    """Where the input is already an fp32 value there is no double rounding,
+    so torch's fp32 -> bf16 cast (round to nearest even) must agree."""
+    rng = np.random.default_rng(22)
+    x = (rng.standard_normal(20000) * np.exp(rng.uniform(-40, 40, 20000))).astype(np.float32)
+    t = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(o.bf16_rne_f64(x.astype(np.float64)), t)
+
+
+def test_bf16_rne_f64_rounds_once():
+    """1 + 2^-8 + 2^-30 lies just above the tie between 1 and 1 + 2^-7: rounded
+    once it goes up; through fp32 first (which lands on the tie) it would go
+    to the even neighbour 1."""
+    x = 1.0 + 2.0 ** -8 + 2.0 ** -30
+    assert o.bf16_rne_f64(np.array([x]))[0] == 0x3F81
+    assert torch.tensor([x], dtype=torch.float64).float().to(torch.bfloat16).view(torch.int16).item() == 0x3F80
+
+
+def _merge_case(seed, N, K, r, gamma=0.5):
+    rng = np.random.default_rng(seed)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    A = o.round_to_bf16((rng.standard_normal((r, K)) * 0.05).astype(np.float32)).astype(np.float64)
+    B = o.round_to_bf16((rng.standard_normal((N, r)) * 0.05).astype(np.float32)).astype(np.float64)
+    return o.quantize(W), A, B, gamma
+
+
+def test_merge_is_the_model_the_layer_computes():
+    """The exact merged weight reproduces the layer: X W_m^T is the oracle's
+    forward Y, and dY W_m its input gradient (the page writes dX as
+    dY (W~ + gamma B A))."""
+    N, K, r = 24, 128, 8
+    (p, s, m), A, B, g = _merge_case(31, N, K, r)
+    exact, _ = o.merge(p, s, m, N, K, A, B, g)
+    Wt = o.dequantize(p, s, m, N, K)
+    rng = np.random.default_rng(32)
+    X, dY = rng.standard_normal((5, K)), rng.standard_normal((5, N))
+    Y, _ = o.linear_forward(X, Wt, A, B, g)
+    dX, *_ = o.linear_backward(dY, X, Wt, A, B, g)
+    assert np.allclose(X @ exact.T, Y, rtol=1e-12, atol=1e-12)
+    assert np.allclose(dY @ exact, dX, rtol=1e-12, atol=1e-12)
+
+
+def test_merge_elementwise_loop():
+    N, K, r = 4, 64, 8
+    (p, s, m), A, B, g = _merge_case(33, N, K, r, gamma=1.25)
+    exact, bits = o.merge(p, s, m, N, K, A, B, g)
+    Wt = o.dequantize(p, s, m, N, K)
+    for n in range(N):
+        for k in range(0, K, 7):
+            v = float(Wt[n, k]) + 1.25 * sum(float(B[n, j]) * float(A[j, k]) for j in range(r))
+            assert exact[n, k] == pytest.approx(v, rel=1e-14, abs=1e-18)
+    assert np.array_equal(bits, o.bf16_rne_f64(exact))
+
+
+@pytest.mark.parametrize("zero", ["B", "gamma"])
+def test_merge_without_adapter_is_the_dequantised_base(zero):
+    N, K, r = 16, 256, 16
+    (p, s, m), A, B, g = _merge_case(34, N, K, r)
+    if zero == "B":
+        B = np.zeros_like(B)
+    else:
+        g = 0.0
+    _, bits = o.merge(p, s, m, N, K, A, B, g)
+    ref = o.dequantize_bits(p, s, m, N * K).reshape(N, K)
+    unsign0 = lambda b: np.where(b == 0x8000, 0, b)       # -0 + 0 is +0
+    assert np.array_equal(unsign0(bits), unsign0(ref))
+
+
+def test_requantising_the_unmerged_base_keeps_every_index():
+    """quantize(W~) keeps each index of a block whose scale is non-zero: the
+    block's largest |w~| is bf16(c~), and w~ / bf16(c~) stays within 2^-8 of
+    its code, far inside the half-gap to the next code."""
+    N, K = 32, 1024
+    (p, s, m), _, _, _ = _merge_case(35, N, K, 8)
+    Wt = o.dequantize(p, s, m, N, K).astype(np.float32)
+    p2, _, _ = o.quantize(Wt)
+    idx = o.unpack_nibbles(p, N * K).reshape(-1, o.BLOCK)
+    idx2 = o.unpack_nibbles(p2, N * K).reshape(-1, o.BLOCK)
+    live = s != 0
+    assert live.mean() > 0.99
+    assert np.array_equal(idx[live], idx2[live])
