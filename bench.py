@@ -337,10 +337,74 @@ def _decoder_measure(q, syn, device, steps=2):
     torch.cuda.synchronize()
     ms = b.elapsed_time(e) / steps
     flops = sum(l.fwd_bwd_flops() for l in lins)
-    return {"workload": "llama7b_decoder_32layers_m4096_r16", "linears": len(lins),
-            "fwd_bwd_ms": round(ms, 3), "fwd_bwd_TFLOPs": round(flops / (ms * 1e-3) / 1e12, 2),
-            "quantize_ms": round(q_ms, 3), "quantize_params": params,
-            "quantize_GBps": round(q_bytes / (q_ms * 1e-3) / 1e9, 1)}
+    out = {"workload": "llama7b_decoder_32layers_m4096_r16", "linears": len(lins),
+           "fwd_bwd_ms": round(ms, 3), "fwd_bwd_TFLOPs": round(flops / (ms * 1e-3) / 1e12, 2),
+           "quantize_ms": round(q_ms, 3), "quantize_params": params,
+           "quantize_GBps": round(q_bytes / (q_ms * 1e-3) / 1e9, 1)}
+    del Ts, wsp
+    for a in act.values():
+        for k in ("X", "dY", "Y", "dX", "dA", "dB"):
+            del a[k]
+    out["export"] = _export_measure(q, lins, ws, act, kind, device)
+    return out
+
+
+def _export_measure(q, lins, ws, act, kind, device, reps=3):
+    """Export of the whole fine-tuned decoder: every one of the 224 stored
+    weights merged with its adapter into its own slice of one bf16 buffer
+    (13 GB, far beyond L2), timed with CUDA events over the 224 launches;
+    then the same buffer re-quantised to NF4, and, for comparison, the plain
+    dequantisation of every weight.  GB/s are algorithmic bytes: the stored
+    weight read, the adapter read and the bf16 weight written (merge), the
+    bf16 read and the stored weight written (re-quantise)."""
+    params = sum(l.N * l.K for l in lins)
+    buf = torch.empty(params, dtype=torch.bfloat16, device=device)
+    views, o = [], 0
+    for l in lins:
+        views.append(buf[o:o + l.N * l.K].view(l.N, l.K))
+        o += l.N * l.K
+    re_ws = [q.empty_nf4(l.N, l.K, device) for l in lins]
+    stored = sum(w.nbytes for w in ws)
+    adapter = sum((l.r * l.K + l.N * l.r) * 2 for l in lins)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        b, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b.record()
+        for _ in range(reps):
+            fn()
+        e.record()
+        torch.cuda.synchronize()
+        return b.elapsed_time(e) / reps
+
+    def merge_all():
+        for l, w, v in zip(lins, ws, views):
+            a = act[kind(l)]
+            q.qlora_merge(w, a["A"], a["B"], l.gamma, out=v)
+
+    def requant_all():
+        for w, v in zip(re_ws, views):
+            q.qlora_quantize_bf16(v, out=w, check_finite=False)
+
+    def dequant_all():
+        for w, v in zip(ws, views):
+            q.qlora_dequantize(w, out=v)
+
+    m_ms = timed(merge_all)
+    r_ms = timed(requant_all)
+    d_ms = timed(dequant_all)
+    m_bytes = stored + adapter + params * 2
+    r_bytes = params * 2 + sum(w.nbytes for w in re_ws)
+    d_bytes = stored + params * 2
+    del buf, views, re_ws
+    return {"linears": len(lins), "params": params,
+            "merge_ms": round(m_ms, 3), "merge_GBps": round(m_bytes / (m_ms * 1e-3) / 1e9, 1),
+            "merge_bytes": m_bytes,
+            "requantize_ms": round(r_ms, 3),
+            "requantize_GBps": round(r_bytes / (r_ms * 1e-3) / 1e9, 1),
+            "dequantize_ms": round(d_ms, 3),
+            "dequantize_GBps": round(d_bytes / (d_ms * 1e-3) / 1e9, 1)}
 
 
 def run_gpu(args):
@@ -444,6 +508,9 @@ def run_gpu(args):
             row["frac_hbm"] = round(row["GBps"] / peaks["hbm_gbs"], 4)
         out["decoder"] = _decoder_measure(q, syn, device)
         out["decoder"]["frac_bf16"] = round(out["decoder"]["fwd_bwd_TFLOPs"] / peak, 4)
+        ex = out["decoder"]["export"]
+        for k in ("merge", "requantize", "dequantize"):
+            ex[f"{k}_frac_hbm"] = round(ex[f"{k}_GBps"] / peaks["hbm_gbs"], 4)
         out["e2e"] = _e2e(q, syn, lin, device, max(3, K // 2))
         out["cpu_baseline"] = _cpu_baseline(seconds=args.cpu_seconds)
     else:

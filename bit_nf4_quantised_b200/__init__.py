@@ -16,7 +16,9 @@ from ._lib import (  # noqa: F401
     qlora_linear_backward,
     qlora_linear_forward,
     qlora_linear_workspace_size,
+    qlora_merge,
     qlora_quantize,
+    qlora_quantize_bf16,
     qlora_quantized_sizes,
     status_string,
     workspace,

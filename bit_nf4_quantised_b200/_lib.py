@@ -41,6 +41,8 @@ EXPORTED = (
     "qlora_linear_forward_ex",
     "qlora_linear_backward_ex",
     "qlora_linear_forward_noalloc",
+    "qlora_merge",
+    "qlora_quantize_bf16",
 )
 
 
@@ -99,6 +101,8 @@ def lib() -> ctypes.CDLL:
         L.qlora_quantized_sizes.argtypes = [i64, i64, sz, sz, sz]
         L.qlora_quantize.argtypes = [vp, tp, vp, vp]
         L.qlora_dequantize.argtypes = [tp, vp, vp]
+        L.qlora_quantize_bf16.argtypes = [vp, tp, vp, vp]
+        L.qlora_merge.argtypes = [tp, vp, vp, i32, f32, vp, vp]
         L.qlora_linear_workspace_size.argtypes = [i64, i64, i64, i32, sz]
         fwd = [vp, i64, tp, vp, vp, i32, f32, vp, vp, vp, ctypes.c_size_t, vp]
         bwd = [vp, vp, i64, tp, vp, vp, i32, f32, vp, vp, vp, vp, i32, vp, ctypes.c_size_t, vp]
@@ -202,6 +206,37 @@ def qlora_dequantize(w: NF4Tensor, out: torch.Tensor | None = None, stream=None)
     st = w.c_struct()
     _check(lib().qlora_dequantize(ctypes.byref(st), out.data_ptr(), _stream(stream)),
            "qlora_dequantize")
+    return out
+
+
+def qlora_quantize_bf16(W: torch.Tensor, out: NF4Tensor | None = None, check_finite: bool = True,
+                        stream=None) -> NF4Tensor:
+    """qlora_quantize of a bf16 [rows, cols] CUDA tensor (values widened
+    exactly to fp32): the re-quantisation of a merged weight."""
+    _need(W, torch.bfloat16, "W")
+    rows, cols = (W.shape[0], W.shape[1]) if W.dim() == 2 else (1, W.numel())
+    out = out if out is not None else empty_nf4(rows, cols, W.device)
+    flag = torch.zeros(1, dtype=torch.int32, device=W.device) if check_finite else None
+    st = out.c_struct()
+    _check(lib().qlora_quantize_bf16(W.data_ptr(), ctypes.byref(st), _ptr(flag), _stream(stream)),
+           "qlora_quantize_bf16")
+    if check_finite and int(flag.item()) != 0:
+        raise QloraError(QLORA_ERR_NONFINITE, "qlora_quantize_bf16")
+    return out
+
+
+def qlora_merge(w: NF4Tensor, A: torch.Tensor, B: torch.Tensor, scale: float,
+                out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """bf16 [rows, cols] merged weight W~ + scale * B A.  A [r, cols], B [rows, r]."""
+    _need(A, torch.bfloat16, "A")
+    _need(B, torch.bfloat16, "B")
+    r = A.shape[0]
+    out = out if out is not None else torch.empty(w.rows, w.cols, dtype=torch.bfloat16,
+                                                  device=w.packed.device)
+    _need(out, torch.bfloat16, "out")
+    st = w.c_struct()
+    _check(lib().qlora_merge(ctypes.byref(st), A.data_ptr(), B.data_ptr(), r, float(scale),
+                             out.data_ptr(), _stream(stream)), "qlora_merge")
     return out
 
 

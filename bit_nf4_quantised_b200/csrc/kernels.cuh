@@ -15,6 +15,28 @@ cudaError_t launch_dequantize(const uint8_t* packed, const uint8_t* scale_codes,
                               int64_t numel, uint16_t* out, const Nf4Table& tab, int num_sms,
                               cudaStream_t stream);
 
+// K1 on a bf16 weight (the re-quantisation of a merged export).
+cudaError_t launch_quantize_bf16(const uint16_t* W, int64_t numel, uint8_t* packed,
+                                 uint8_t* scale_codes, float* meta, int* nonfinite_flag,
+                                 const Nf4Table& tab, cudaStream_t stream);
+
+// ---------------------------------------------------------------- K7 merge
+struct MergeArgs {
+    const uint32_t* packed;      // N*K/8 words of packed indices
+    const uint8_t* scale_codes;
+    const float* meta;
+    const uint16_t* A;           // bf16 [r, K]
+    const uint16_t* B;           // bf16 [N, r]
+    uint16_t* out;               // bf16 [N, K]
+    int64_t N, K;                // K % 64 == 0
+    int r;                       // 8 <= r <= 128, r % 8 == 0
+    int rp;                      // r rounded up to 16 (set by launch_merge)
+    float gamma;
+    int64_t tiles;               // warp tiles of 16 x 64 (set by launch_merge)
+};
+int merge_smem_bytes(int r);
+cudaError_t launch_merge(const MergeArgs& a, const Nf4Table& tab, int num_sms, cudaStream_t stream);
+
 // ---------------------------------------------------------------- K2 / K3
 struct GemmArgs {
     const uint8_t* scale_codes;

@@ -1,0 +1,199 @@
+// K7: merge for export, W_m = bf16_rne( W~ + gamma * B A ).
+//
+// "QLoRA, explained", "The forward pass and gradients": the model that was
+// fine-tuned is W~ + gamma B A (the quantised base plus the adapter), not
+// W0 + gamma B A.  The same page's "Failure modes", "Quality loss at merge
+// time", gives dequantising W~ to bf16 and adding the adapter as the merge
+// that keeps that model; "QLoRA" (finetunellm.com), "What it costs you", adds
+// that a 4-bit deployment re-quantises the merged bf16 weight (qlora_quantize_bf16).
+// W~ is rebuilt exactly as K6 does (c~ = fp32(e4m3 * c2), w~ = bf16_rne(fp32(q *
+// c~))); the sum is formed in fp32 and rounded to bf16 once.
+//
+// HBM-bound: 0.516 B read and 2 B written per weight; A [r x K] and B [N x r]
+// stay in L2.  The rank-r product B A is a contraction of depth r <= 128, done
+// on the warp-level tensor cores (mma.sync m16n8k16, bf16 in, fp32
+// accumulate): at r = 16 that is 16 MMAs per 1024 weights, a few per cent of
+// the issue slots, so the kernel's time is set by its stores.
+//
+// Work unit: one warp tile of 16 rows x 64 columns (one NF4 block per row).
+// Units are ordered strip by strip (all row tiles of columns [c0, c0+64)
+// before the next strip) and cut into equal contiguous runs, one per warp of
+// a grid sized to the SMs' resident capacity.  Each warp keeps its strip's
+// slice of A in its own shared-memory slab, reloaded only when its run
+// crosses into the next strip, so no CTA-wide barrier is needed.
+//
+// Column ownership.  The MMA's output fragment gives lane (g, t) two adjacent
+// columns of each 8-wide n-tile.  The 8 n-tiles are mapped to the strip's
+// columns so that lane t of a quad owns columns 32i + 8t + (0..7) for i = 0, 1:
+// each quad then writes 64 contiguous bytes per store (full 32-byte sectors)
+// and reads its packed indices as one 32-bit word per row and i.  Logical
+// column n (0..7) of n-tile nt is physical column
+//     32 (nt / 4) + 8 (n / 2) + 2 (nt % 4) + (n % 2),
+// and the slab stores A's columns in that logical order so that ldmatrix.trans
+// yields the B-operand fragments directly.
+#include "kernels.cuh"
+
+namespace qnf4 {
+
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kStrip = 64;                 // columns per warp tile
+constexpr int kTileRows = 16;              // rows per warp tile (the MMA's M)
+constexpr int kSlabPitch = kStrip + 8;     // bf16 per slab row: 144 B, conflict-free ldmatrix
+
+__host__ __device__ constexpr int slab_bytes(int rp) { return rp * kSlabPitch * 2; }
+
+__global__ void __launch_bounds__(kThreads)
+merge_kernel(MergeArgs a, Nf4Table tab) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    float* scode = reinterpret_cast<float*>(smem);                       // 16 codes
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint16_t* slab = reinterpret_cast<uint16_t*>(smem + 64 + warp * slab_bytes(a.rp));
+    if (threadIdx.x == 0) {            // constant indices: no local copy of the table
+#pragma unroll
+        for (int q = 0; q < 16; ++q) scode[q] = tab.code[q];
+    }
+    __syncthreads();
+
+    const int g = lane >> 2, tq = lane & 3;
+    const int64_t row_tiles = (a.N + kTileRows - 1) / kTileRows;
+    const int64_t total_warps = int64_t(gridDim.x) * kWarps;
+    const int64_t gw = int64_t(blockIdx.x) * kWarps + warp;
+    const int64_t t_begin = a.tiles * gw / total_warps;
+    const int64_t t_end = a.tiles * (gw + 1) / total_warps;
+    const int64_t K = a.K;
+    const int64_t kwords = K / 8;              // 32-bit words of packed indices per row
+    const int64_t kblocks = K / kStrip;        // NF4 blocks per row
+
+    // The slab position lane l fills: A's physical columns 2l, 2l+1 are
+    // logical columns p0, p0 + 1 of the strip (see the column map above).
+    const int pc = 2 * lane;
+    const int p0 = 8 * (4 * (pc >> 5) + ((pc & 7) >> 1)) + 2 * ((pc & 31) >> 3);
+
+    // ldmatrix.x4.trans addressing: matrix m = lane / 8 covers slab rows
+    // (m & 1) * 8 + (lane & 7) of the k-step, n-tile (m >> 1) of the pair.
+    const int lm_row = ((lane >> 3) & 1) * 8 + (lane & 7);
+    const int lm_col = (lane >> 4) * 8;
+    const uint32_t slab_s = smem_u32(slab);
+
+    int64_t cur_strip = -1;
+    for (int64_t t = t_begin; t < t_end; ++t) {
+        const int64_t strip = t / row_tiles;
+        const int64_t n0 = (t - strip * row_tiles) * kTileRows;
+        const int64_t c0 = strip * kStrip;
+
+        // Issue this tile's weight loads first; they are the DRAM traffic.
+        uint32_t pw[2][2] = {{0u, 0u}, {0u, 0u}};
+        uint8_t sc[2] = {0, 0};
+        float mt[2] = {0.f, 0.f};
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+            const int64_t R = n0 + g + 8 * s;
+            if (R < a.N) {
+                const uint32_t* prow = a.packed + R * kwords + c0 / 8 + tq;
+                pw[s][0] = __ldcs(prow);
+                pw[s][1] = __ldcs(prow + 4);
+                const int64_t b = R * kblocks + strip;
+                sc[s] = a.scale_codes[b];
+                mt[s] = a.meta[b >> 8];
+            }
+        }
+
+        if (strip != cur_strip) {
+            __syncwarp();
+            for (int k = 0; k < a.rp; ++k) {
+                uint32_t v = 0u;
+                if (k < a.r) v = *reinterpret_cast<const uint32_t*>(a.A + int64_t(k) * K + c0 + pc);
+                *reinterpret_cast<uint32_t*>(slab + k * kSlabPitch + p0) = v;
+            }
+            __syncwarp();
+            cur_strip = strip;
+        }
+
+        // acc[nt][.] = (B A)[rows g, g+8][logical columns 2t, 2t+1 of n-tile nt]
+        float acc[8][4];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+
+        const int64_t R0 = n0 + g, R1 = n0 + g + 8;
+        for (int k0 = 0; k0 < a.rp; k0 += 16) {
+            uint32_t af[4];
+            const int ka = k0 + 2 * tq, kb = k0 + 8 + 2 * tq;
+            af[0] = (R0 < a.N && ka < a.r)
+                        ? *reinterpret_cast<const uint32_t*>(a.B + R0 * a.r + ka) : 0u;
+            af[1] = (R1 < a.N && ka < a.r)
+                        ? *reinterpret_cast<const uint32_t*>(a.B + R1 * a.r + ka) : 0u;
+            af[2] = (R0 < a.N && kb < a.r)
+                        ? *reinterpret_cast<const uint32_t*>(a.B + R0 * a.r + kb) : 0u;
+            af[3] = (R1 < a.N && kb < a.r)
+                        ? *reinterpret_cast<const uint32_t*>(a.B + R1 * a.r + kb) : 0u;
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(slab_s + 2u * uint32_t((k0 + lm_row) * kSlabPitch + np * 16 + lm_col),
+                          b0, b1, b2, b3);
+                mma_bf16_16816(acc[2 * np], af[0], af[1], af[2], af[3], b0, b1);
+                mma_bf16_16816(acc[2 * np + 1], af[0], af[1], af[2], af[3], b2, b3);
+            }
+        }
+
+        // Epilogue: W~ from the packed word, plus gamma * (B A), rounded once.
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+            const int64_t R = n0 + g + 8 * s;
+            const float ct = __fmul_rn(e4m3_to_float(sc[s]), mt[s]);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const uint32_t v = pw[s][i];
+                uint32_t o[4];
+#pragma unroll
+                for (int jp = 0; jp < 4; ++jp) {
+                    // physical columns 32i + 8t + 2jp, +1 <- n-tile 4i + jp, logical 2t, 2t+1
+                    const uint32_t wb = pack_bf16x2(__fmul_rn(scode[(v >> (8 * jp)) & 15u], ct),
+                                                    __fmul_rn(scode[(v >> (8 * jp + 4)) & 15u], ct));
+                    const float wlo = __uint_as_float(wb << 16);
+                    const float whi = __uint_as_float(wb & 0xffff0000u);
+                    o[jp] = pack_bf16x2(__fmaf_rn(a.gamma, acc[4 * i + jp][2 * s], wlo),
+                                        __fmaf_rn(a.gamma, acc[4 * i + jp][2 * s + 1], whi));
+                }
+                if (R < a.N)
+                    __stcs(reinterpret_cast<uint4*>(a.out + R * K + c0 + 32 * i + 8 * tq),
+                           make_uint4(o[0], o[1], o[2], o[3]));
+            }
+        }
+    }
+}
+
+}  // namespace
+
+int merge_smem_bytes(int r) {
+    const int rp = (r + 15) / 16 * 16;
+    return 64 + kWarps * slab_bytes(rp);
+}
+
+cudaError_t launch_merge(const MergeArgs& args, const Nf4Table& tab, int num_sms,
+                         cudaStream_t stream) {
+    MergeArgs a = args;
+    a.rp = (a.r + 15) / 16 * 16;
+    a.tiles = (a.K / kStrip) * ((a.N + kTileRows - 1) / kTileRows);
+    if (a.tiles == 0) return cudaSuccess;
+    const int smem = merge_smem_bytes(a.r);
+    cudaError_t e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, merge_kernel, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+    int64_t grid = int64_t(num_sms) * per_sm;
+    const int64_t need = (a.tiles + kWarps - 1) / kWarps;     // at least one tile per warp
+    if (grid > need) grid = need;
+    merge_kernel<<<dim3(static_cast<unsigned>(grid)), kThreads, smem, stream>>>(a, tab);
+    return cudaGetLastError();
+}
+
+}  // namespace qnf4

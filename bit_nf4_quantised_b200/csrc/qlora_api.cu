@@ -382,6 +382,43 @@ int qlora_dequantize(const qlora_nf4_tensor* w, uint16_t* W_out, qlora_stream_t 
                                          reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int qlora_quantize_bf16(const uint16_t* W, const qlora_nf4_tensor* out, int* d_nonfinite_flag,
+                        qlora_stream_t stream) {
+    if (!W) return QLORA_ERR_NULL;
+    int st = check_tensor(out);
+    if (st != QLORA_OK) return st;
+    if (!aligned(W, 16)) return QLORA_ERR_ALIGN;
+    const int64_t numel = out->rows * out->cols;
+    if (numel == 0) return QLORA_OK;
+    return cuda_status(launch_quantize_bf16(W, numel, out->packed, out->scale_codes,
+                                            out->meta_scale, d_nonfinite_flag, table(),
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int qlora_merge(const qlora_nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r,
+                float scale, uint16_t* W_out, qlora_stream_t stream) {
+    int st = check_tensor(w);
+    if (st != QLORA_OK) return st;
+    const int64_t N = w->rows, K = w->cols;
+    if (K % QLORA_BLOCK != 0) return QLORA_ERR_UNSUPPORTED;
+    if (r < 8 || r > QLORA_MAX_RANK || r % 8 != 0) return QLORA_ERR_UNSUPPORTED;
+    if (N == 0 || K == 0) return QLORA_OK;              // A, B, W_out may then be NULL
+    if (!A || !B || !W_out) return QLORA_ERR_NULL;
+    if (!aligned(A, 16) || !aligned(B, 16) || !aligned(W_out, 16)) return QLORA_ERR_ALIGN;
+    MergeArgs a{};
+    a.packed = reinterpret_cast<const uint32_t*>(w->packed);
+    a.scale_codes = w->scale_codes;
+    a.meta = w->meta_scale;
+    a.A = A;
+    a.B = B;
+    a.out = W_out;
+    a.N = N;
+    a.K = K;
+    a.r = r;
+    a.gamma = scale;
+    return cuda_status(launch_merge(a, table(), num_sms(), reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int qlora_linear_workspace_size(int64_t M, int64_t N, int64_t K, int r, size_t* bytes) {
     if (!bytes) return QLORA_ERR_NULL;
     int st = check_linear_shapes(M, N, K, r);

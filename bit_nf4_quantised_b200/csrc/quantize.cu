@@ -16,6 +16,9 @@
 // search over the midpoints in shared memory, and writes its four nibbles as
 // one 16-bit store, so a warp writes 64 contiguous bytes.  The block scales
 // stay in shared memory for the group-level FP8 pass at the end.
+//
+// The same kernel also takes a bf16 weight (a merged export being
+// re-quantised): each lane then loads 8 bytes, widened exactly to fp32.
 #include "kernels.cuh"
 
 namespace qnf4 {
@@ -35,9 +38,24 @@ __device__ __forceinline__ uint32_t nearest_code(float x, const float* smid) {
     return i;
 }
 
-template <bool kFull>
+// Four consecutive weights as fp32: fp32 input directly, bf16 input widened
+// exactly (a bf16 value is the top half of its fp32).
+__device__ __forceinline__ float4 load4(const float* W, int64_t e0) {
+    return __ldcs(reinterpret_cast<const float4*>(W + e0));
+}
+__device__ __forceinline__ float4 load4(const uint16_t* W, int64_t e0) {
+    const uint2 u = __ldcs(reinterpret_cast<const uint2*>(W + e0));
+    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                       __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+}
+__device__ __forceinline__ float load1(const float* W, int64_t e) { return W[e]; }
+__device__ __forceinline__ float load1(const uint16_t* W, int64_t e) {
+    return __uint_as_float(uint32_t(W[e]) << 16);
+}
+
+template <bool kFull, typename Tin>
 __global__ void __launch_bounds__(kThreads)
-quantize_kernel(const float* __restrict__ W, int64_t numel, int64_t nblocks,
+quantize_kernel(const Tin* __restrict__ W, int64_t numel, int64_t nblocks,
                 uint8_t* __restrict__ packed, uint8_t* __restrict__ scale_codes,
                 float* __restrict__ meta, int* __restrict__ nonfinite_flag, Nf4Table tab) {
     __shared__ float smid[16];
@@ -61,12 +79,12 @@ quantize_kernel(const float* __restrict__ W, int64_t numel, int64_t nblocks,
         const int64_t e0 = gbase + int64_t(blk) * QLORA_BLOCK + sub * 4;
         float4 v;
         if (kFull) {
-            v = __ldcs(reinterpret_cast<const float4*>(W + e0));
+            v = load4(W, e0);
         } else {
-            v.x = (e0 + 0 < numel) ? W[e0 + 0] : 0.f;
-            v.y = (e0 + 1 < numel) ? W[e0 + 1] : 0.f;
-            v.z = (e0 + 2 < numel) ? W[e0 + 2] : 0.f;
-            v.w = (e0 + 3 < numel) ? W[e0 + 3] : 0.f;
+            v.x = (e0 + 0 < numel) ? load1(W, e0 + 0) : 0.f;
+            v.y = (e0 + 1 < numel) ? load1(W, e0 + 1) : 0.f;
+            v.z = (e0 + 2 < numel) ? load1(W, e0 + 2) : 0.f;
+            v.w = (e0 + 3 < numel) ? load1(W, e0 + 3) : 0.f;
         }
         bad |= !(isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w));
         float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
@@ -111,26 +129,39 @@ quantize_kernel(const float* __restrict__ W, int64_t numel, int64_t nblocks,
     if (tid == 0) meta[group] = c2;
 }
 
-}  // namespace
-
-cudaError_t launch_quantize(const float* W, int64_t numel, uint8_t* packed, uint8_t* scale_codes,
-                            float* meta, int* nonfinite_flag, const Nf4Table& tab,
-                            cudaStream_t stream) {
+template <typename Tin>
+cudaError_t quantize_any(const Tin* W, int64_t numel, uint8_t* packed, uint8_t* scale_codes,
+                         float* meta, int* nonfinite_flag, const Nf4Table& tab,
+                         cudaStream_t stream) {
     const int64_t nblocks = (numel + QLORA_BLOCK - 1) / QLORA_BLOCK;
     const int64_t ngroups = (nblocks + QLORA_GROUP - 1) / QLORA_GROUP;
     const int64_t full = numel / kGroupElems;                  // groups with no tail
     if (full > 0) {
-        quantize_kernel<true><<<dim3(static_cast<unsigned>(full)), kThreads, 0, stream>>>(
+        quantize_kernel<true, Tin><<<dim3(static_cast<unsigned>(full)), kThreads, 0, stream>>>(
             W, numel, nblocks, packed, scale_codes, meta, nonfinite_flag, tab);
     }
     if (ngroups > full) {
         // the single trailing group, offset so blockIdx.x is its group index
         const int64_t off = full * kGroupElems;
-        quantize_kernel<false><<<1, kThreads, 0, stream>>>(
+        quantize_kernel<false, Tin><<<1, kThreads, 0, stream>>>(
             W + off, numel - off, nblocks - full * QLORA_GROUP, packed + full * (kGroupElems / 2),
             scale_codes + full * QLORA_GROUP, meta + full, nonfinite_flag, tab);
     }
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const float* W, int64_t numel, uint8_t* packed, uint8_t* scale_codes,
+                            float* meta, int* nonfinite_flag, const Nf4Table& tab,
+                            cudaStream_t stream) {
+    return quantize_any(W, numel, packed, scale_codes, meta, nonfinite_flag, tab, stream);
+}
+
+cudaError_t launch_quantize_bf16(const uint16_t* W, int64_t numel, uint8_t* packed,
+                                 uint8_t* scale_codes, float* meta, int* nonfinite_flag,
+                                 const Nf4Table& tab, cudaStream_t stream) {
+    return quantize_any(W, numel, packed, scale_codes, meta, nonfinite_flag, tab, stream);
 }
 
 }  // namespace qnf4

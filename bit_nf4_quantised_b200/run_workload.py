@@ -2,11 +2,12 @@
 profilers such as ncu, which want a short process around the kernels).
 
   python -m bit_nf4_quantised_b200.run_workload --workload NAME [--calls 2]
-         [--forward-only]
+         [--forward-only | --merge]
 
 NAME is a key of synthetic.WORKLOADS; for a multi-layer workload only its
 first layer runs.  Each call is one forward (and, unless --forward-only, one
-backward) of that layer on cuda:0.
+backward) of that layer on cuda:0; with --merge, one merge of the layer's
+weight and adapter into a bf16 weight instead.
 """
 from __future__ import annotations
 
@@ -23,11 +24,19 @@ def main() -> None:
     ap.add_argument("--workload", default="llama7b_attn_proj_4096x4096_m4096_r16")
     ap.add_argument("--calls", type=int, default=2)
     ap.add_argument("--forward-only", action="store_true")
+    ap.add_argument("--merge", action="store_true")
     args = ap.parse_args()
     lin = syn.WORKLOADS[args.workload].layers[0]
-    d = syn.make_layer(lin, with_grad=not args.forward_only)
+    d = syn.make_layer(lin, with_grad=not (args.forward_only or args.merge))
     w = q.qlora_quantize(torch.from_numpy(d["W"]).cuda())
     g = {k: v.cuda() for k, v in d.items() if isinstance(v, torch.Tensor)}
+    if args.merge:
+        out = torch.empty(lin.N, lin.K, dtype=torch.bfloat16, device="cuda")
+        for _ in range(args.calls):
+            q.qlora_merge(w, g["A"], g["B"], lin.gamma, out=out)
+        torch.cuda.synchronize()
+        print(f"{args.workload}: {args.calls} merge call(s)")
+        return
     ws = q.workspace(lin.M, lin.N, lin.K, lin.r)
     T = torch.empty(lin.M, lin.r, dtype=torch.float32, device="cuda")
     for _ in range(args.calls):

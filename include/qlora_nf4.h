@@ -155,6 +155,46 @@ QLORA_API int qlora_dequantize(const qlora_nf4_tensor* w, uint16_t* W_out,
                      qlora_stream_t stream);
 
 /*
+ * qlora_merge -- the fine-tuned weight for bf16 export,
+ *     W_out = bf16_rne( W~ + scale * B A ).
+ * "QLoRA, explained", "The forward pass and gradients": the model that was
+ * trained is W~ + gamma B A, the quantised base plus the adapter; the same
+ * page's "Failure modes" ("Quality loss at merge time") gives dequantising W~
+ * to bf16 and adding the adapter as the merge that keeps it.  W~ is rebuilt
+ * bit for bit as qlora_dequantize does; the sum is formed in fp32 (B A
+ * accumulated in fp32 from the exact bf16 products, then one fused
+ * multiply-add with W~) and rounded to bf16 once.
+ *   w     (host struct, read): the stored weight, rows = N, cols = K
+ *   A     (device, bf16, r x K, read): LoRA down-projection
+ *   B     (device, bf16, N x r, read): LoRA up-projection
+ *   r     LoRA rank: 8 <= r <= 128, r % 8 == 0
+ *   scale gamma = alpha / r
+ *   W_out (device, bf16 bits, N x K, written, row-major); must not overlap
+ *         the inputs.  Each element is within one bf16 rounding of the exact
+ *         value, plus fp32 accumulation error (at most (2r+4) 2^-24 of
+ *         |w~| + |gamma| sum_j |B_nj A_jk|).
+ * N = 0 or K = 0 launches nothing; A, B and W_out may then be NULL.
+ * Shape rules: K % 64 == 0 (every NF4 block lies inside one row); any N.
+ * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE, QLORA_ERR_UNSUPPORTED (K or r),
+ * QLORA_ERR_ALIGN (A, B, W_out and packed 16-byte aligned; scale_codes,
+ * meta_scale 4-byte), QLORA_ERR_CUDA.
+ */
+QLORA_API int qlora_merge(const qlora_nf4_tensor* w, const uint16_t* A, const uint16_t* B,
+                          int r, float scale, uint16_t* W_out, qlora_stream_t stream);
+
+/*
+ * qlora_quantize_bf16 -- qlora_quantize of a bf16 weight (each value widened
+ * exactly to fp32 first), the re-quantisation of a merged weight for a 4-bit
+ * deployment ("QLoRA" (finetunellm.com), "What it costs you": merging into
+ * 4-bit weights means merging in bf16 and quantising again, a second
+ * rounding).  Same result as qlora_quantize given the fp32 values of W.
+ *   W (device, bf16 bits, rows*cols, read); other arguments as qlora_quantize.
+ * Errors: as qlora_quantize (W 16-byte aligned).
+ */
+QLORA_API int qlora_quantize_bf16(const uint16_t* W, const qlora_nf4_tensor* out,
+                                  int* d_nonfinite_flag, qlora_stream_t stream);
+
+/*
  * qlora_linear_workspace_size -- bytes of device workspace that
  * qlora_linear_forward and qlora_linear_backward need for these sizes.
  * M tokens, N = w.rows, K = w.cols, r the LoRA rank.  Host only.

@@ -105,6 +105,33 @@ def test_argument_errors_return_before_any_launch(q):
                                    fake, None, fake, 0, fake, ws_n.value, None) == q._lib.QLORA_ERR_NULL
 
 
+def test_merge_and_bf16_quantize_argument_errors(q):
+    """qlora_merge / qlora_quantize_bf16 reject bad arguments on the host; an
+    empty weight returns before any launch."""
+    L = q.lib()
+    T = q._lib._Tensor
+    fake = 0x40000
+    good = T(0x10000, 0x20000, 0x30000, 256, 512)
+    E = q._lib
+    assert L.qlora_merge(ctypes.byref(good), None, fake, 16, 2.0, fake, None) == E.QLORA_ERR_NULL
+    assert L.qlora_merge(ctypes.byref(good), fake, fake, 16, 2.0, None, None) == E.QLORA_ERR_NULL
+    assert L.qlora_merge(None, fake, fake, 16, 2.0, fake, None) == E.QLORA_ERR_NULL
+    for r in (0, 4, 12, 136):
+        assert L.qlora_merge(ctypes.byref(good), fake, fake, r, 2.0, fake, None) == E.QLORA_ERR_UNSUPPORTED
+    odd_k = T(0x10000, 0x20000, 0x30000, 256, 500)
+    assert L.qlora_merge(ctypes.byref(odd_k), fake, fake, 16, 2.0, fake, None) == E.QLORA_ERR_UNSUPPORTED
+    assert L.qlora_merge(ctypes.byref(good), fake + 8, fake, 16, 2.0, fake, None) == E.QLORA_ERR_ALIGN
+    assert L.qlora_merge(ctypes.byref(good), fake, fake, 16, 2.0, fake + 2, None) == E.QLORA_ERR_ALIGN
+    neg = T(0x10000, 0x20000, 0x30000, -1, 512)
+    assert L.qlora_merge(ctypes.byref(neg), fake, fake, 16, 2.0, fake, None) == E.QLORA_ERR_SHAPE
+    empty = T(0x10000, 0x20000, 0x30000, 0, 512)
+    assert L.qlora_merge(ctypes.byref(empty), fake, fake, 16, 2.0, fake, None) == E.QLORA_OK
+    assert L.qlora_quantize_bf16(None, ctypes.byref(good), None, None) == E.QLORA_ERR_NULL
+    assert L.qlora_quantize_bf16(fake + 8, ctypes.byref(good), None, None) == E.QLORA_ERR_ALIGN
+    assert L.qlora_quantize_bf16(fake, ctypes.byref(neg), None, None) == E.QLORA_ERR_SHAPE
+    assert L.qlora_quantize_bf16(fake, ctypes.byref(empty), None, None) == E.QLORA_OK
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     import bit_nf4_quantised_b200._lib as L
     monkeypatch.setattr(L, "_LIB", None)
