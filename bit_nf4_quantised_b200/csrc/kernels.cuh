@@ -32,7 +32,7 @@ struct MergeArgs {
     int r;                       // 8 <= r <= 128, r % 8 == 0
     int rp;                      // r rounded up to 16 (set by launch_merge)
     float gamma;
-    int64_t tiles;               // warp tiles of 16 x 64 (set by launch_merge)
+    int64_t tiles;               // CTA units of 16 rows x 512 columns (set by launch_merge)
 };
 int merge_smem_bytes(int r);
 cudaError_t launch_merge(const MergeArgs& a, const Nf4Table& tab, int num_sms, cudaStream_t stream);

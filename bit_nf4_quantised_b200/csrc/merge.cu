@@ -15,12 +15,17 @@
 // accumulate): at r = 16 that is 16 MMAs per 1024 weights, a few per cent of
 // the issue slots, so the kernel's time is set by its stores.
 //
-// Work unit: one warp tile of 16 rows x 64 columns (one NF4 block per row).
-// Units are ordered strip by strip (all row tiles of columns [c0, c0+64)
-// before the next strip) and cut into equal contiguous runs, one per warp of
-// a grid sized to the SMs' resident capacity.  Each warp keeps its strip's
-// slice of A in its own shared-memory slab, reloaded only when its run
-// crosses into the next strip, so no CTA-wide barrier is needed.
+// Work unit: one CTA tile of 16 rows x 512 columns, each of the 8 warps
+// owning one 64-column strip (one NF4 block per row).  Units are ordered by
+// column block (all row tiles of columns [c0, c0+512) before the next block)
+// and cut into equal contiguous runs, one per CTA of a grid sized to the SMs'
+// resident capacity.  Each warp keeps its strip's slice of A in its own
+// shared-memory slab, reloaded only when its CTA's run enters the next column
+// block, so no CTA-wide barrier is needed.  The 8 warps of a CTA read the same
+// 16 rows of B and the same scale-code sectors at about the same time, so
+// those reads are served by L1 once per CTA rather than once per warp.  The
+// next unit's packed words, scale codes and group scales are loaded before
+// the current unit is computed.
 //
 // Column ownership.  The MMA's output fragment gives lane (g, t) two adjacent
 // columns of each 8-wide n-tile.  The 8 n-tiles are mapped to the strip's
@@ -39,11 +44,19 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kStrip = 64;                 // columns per warp tile
-constexpr int kTileRows = 16;              // rows per warp tile (the MMA's M)
+constexpr int kStrip = 64;                 // columns per warp (one NF4 block per row)
+constexpr int kTileRows = 16;              // rows per unit (the MMA's M)
 constexpr int kSlabPitch = kStrip + 8;     // bf16 per slab row: 144 B, conflict-free ldmatrix
 
 __host__ __device__ constexpr int slab_bytes(int rp) { return rp * kSlabPitch * 2; }
+
+// One lane's weight inputs for a unit: the packed words of its columns in
+// rows g and g+8, their blocks' FP8 scale codes and group scales.
+struct WeightRegs {
+    uint32_t w[2][2];
+    uint32_t sc[2];
+    float mt[2];
+};
 
 __global__ void __launch_bounds__(kThreads)
 merge_kernel(MergeArgs a, Nf4Table tab) {
@@ -58,14 +71,13 @@ merge_kernel(MergeArgs a, Nf4Table tab) {
     __syncthreads();
 
     const int g = lane >> 2, tq = lane & 3;
-    const int64_t row_tiles = (a.N + kTileRows - 1) / kTileRows;
-    const int64_t total_warps = int64_t(gridDim.x) * kWarps;
-    const int64_t gw = int64_t(blockIdx.x) * kWarps + warp;
-    const int64_t t_begin = a.tiles * gw / total_warps;
-    const int64_t t_end = a.tiles * (gw + 1) / total_warps;
-    const int64_t K = a.K;
-    const int64_t kwords = K / 8;              // 32-bit words of packed indices per row
-    const int64_t kblocks = K / kStrip;        // NF4 blocks per row
+    // N and K are below 2^31 (checked on the host); products of a row and K
+    // are formed in 64 bits.
+    const int N = static_cast<int>(a.N), K = static_cast<int>(a.K);
+    const int row_tiles = (N + kTileRows - 1) / kTileRows;
+    const int kblocks = K / kStrip;            // NF4 blocks (strips) per row
+    const int64_t u_begin = a.tiles * blockIdx.x / gridDim.x;
+    const int64_t u_end = a.tiles * (blockIdx.x + 1) / gridDim.x;
 
     // The slab position lane l fills: A's physical columns 2l, 2l+1 are
     // logical columns p0, p0 + 1 of the strip (see the column map above).
@@ -78,93 +90,125 @@ merge_kernel(MergeArgs a, Nf4Table tab) {
     const int lm_col = (lane >> 4) * 8;
     const uint32_t slab_s = smem_u32(slab);
 
-    int64_t cur_strip = -1;
-    for (int64_t t = t_begin; t < t_end; ++t) {
-        const int64_t strip = t / row_tiles;
-        const int64_t n0 = (t - strip * row_tiles) * kTileRows;
-        const int64_t c0 = strip * kStrip;
+    // Packed words: the quad loads its row's 32 bytes as four 8-byte pieces
+    // (one sector, one request); lane t then needs words t and t + 4, held by
+    // lanes t/2 and 2 + t/2 of its quad.
+    const int qbase = lane & ~3;
+    const int src_a = qbase + (tq >> 1), src_b = qbase + 2 + (tq >> 1);
 
-        // Issue this tile's weight loads first; they are the DRAM traffic.
-        uint32_t pw[2][2] = {{0u, 0u}, {0u, 0u}};
-        uint8_t sc[2] = {0, 0};
-        float mt[2] = {0.f, 0.f};
+    // Unit (column block cb, row tile rt); units advance row tile first.
+    auto load_unit = [&](int cb, int rt, WeightRegs& wr) {
+        const int strip = cb * kWarps + warp;
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
-            const int64_t R = n0 + g + 8 * s;
-            if (R < a.N) {
-                const uint32_t* prow = a.packed + R * kwords + c0 / 8 + tq;
-                pw[s][0] = __ldcs(prow);
-                pw[s][1] = __ldcs(prow + 4);
-                const int64_t b = R * kblocks + strip;
-                sc[s] = a.scale_codes[b];
-                mt[s] = a.meta[b >> 8];
+            const int R = rt * kTileRows + g + 8 * s;
+            uint2 v = make_uint2(0u, 0u);
+            wr.sc[s] = 0u;
+            wr.mt[s] = 0.f;
+            if (R < N && strip < kblocks) {
+                const uint64_t e0 = uint64_t(R) * uint64_t(K) + uint64_t(strip) * kStrip;
+                v = __ldcs(reinterpret_cast<const uint2*>(a.packed + (e0 >> 3)) + tq);
+                const uint64_t b = e0 >> 6;                     // flat block index
+                wr.sc[s] = a.scale_codes[b];
+                wr.mt[s] = a.meta[b >> 8];
             }
+            wr.w[s][0] = v.x;       // exchanged below, after the loads have been issued
+            wr.w[s][1] = v.y;
         }
-
-        if (strip != cur_strip) {
-            __syncwarp();
-            for (int k = 0; k < a.rp; ++k) {
-                uint32_t v = 0u;
-                if (k < a.r) v = *reinterpret_cast<const uint32_t*>(a.A + int64_t(k) * K + c0 + pc);
-                *reinterpret_cast<uint32_t*>(slab + k * kSlabPitch + p0) = v;
-            }
-            __syncwarp();
-            cur_strip = strip;
-        }
-
-        // acc[nt][.] = (B A)[rows g, g+8][logical columns 2t, 2t+1 of n-tile nt]
-        float acc[8][4];
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
-
-        const int64_t R0 = n0 + g, R1 = n0 + g + 8;
-        for (int k0 = 0; k0 < a.rp; k0 += 16) {
-            uint32_t af[4];
-            const int ka = k0 + 2 * tq, kb = k0 + 8 + 2 * tq;
-            af[0] = (R0 < a.N && ka < a.r)
-                        ? *reinterpret_cast<const uint32_t*>(a.B + R0 * a.r + ka) : 0u;
-            af[1] = (R1 < a.N && ka < a.r)
-                        ? *reinterpret_cast<const uint32_t*>(a.B + R1 * a.r + ka) : 0u;
-            af[2] = (R0 < a.N && kb < a.r)
-                        ? *reinterpret_cast<const uint32_t*>(a.B + R0 * a.r + kb) : 0u;
-            af[3] = (R1 < a.N && kb < a.r)
-                        ? *reinterpret_cast<const uint32_t*>(a.B + R1 * a.r + kb) : 0u;
-#pragma unroll
-            for (int np = 0; np < 4; ++np) {
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4_t(slab_s + 2u * uint32_t((k0 + lm_row) * kSlabPitch + np * 16 + lm_col),
-                          b0, b1, b2, b3);
-                mma_bf16_16816(acc[2 * np], af[0], af[1], af[2], af[3], b0, b1);
-                mma_bf16_16816(acc[2 * np + 1], af[0], af[1], af[2], af[3], b2, b3);
-            }
-        }
-
-        // Epilogue: W~ from the packed word, plus gamma * (B A), rounded once.
+    };
+    auto exchange = [&](WeightRegs& wr) {
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
-            const int64_t R = n0 + g + 8 * s;
-            const float ct = __fmul_rn(e4m3_to_float(sc[s]), mt[s]);
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const uint32_t v = pw[s][i];
-                uint32_t o[4];
-#pragma unroll
-                for (int jp = 0; jp < 4; ++jp) {
-                    // physical columns 32i + 8t + 2jp, +1 <- n-tile 4i + jp, logical 2t, 2t+1
-                    const uint32_t wb = pack_bf16x2(__fmul_rn(scode[(v >> (8 * jp)) & 15u], ct),
-                                                    __fmul_rn(scode[(v >> (8 * jp + 4)) & 15u], ct));
-                    const float wlo = __uint_as_float(wb << 16);
-                    const float whi = __uint_as_float(wb & 0xffff0000u);
-                    o[jp] = pack_bf16x2(__fmaf_rn(a.gamma, acc[4 * i + jp][2 * s], wlo),
-                                        __fmaf_rn(a.gamma, acc[4 * i + jp][2 * s + 1], whi));
+            const uint32_t ax = __shfl_sync(0xffffffffu, wr.w[s][0], src_a);
+            const uint32_t ay = __shfl_sync(0xffffffffu, wr.w[s][1], src_a);
+            const uint32_t bx = __shfl_sync(0xffffffffu, wr.w[s][0], src_b);
+            const uint32_t by = __shfl_sync(0xffffffffu, wr.w[s][1], src_b);
+            wr.w[s][0] = (tq & 1) ? ay : ax;
+            wr.w[s][1] = (tq & 1) ? by : bx;
+        }
+    };
+
+    int cb = static_cast<int>(u_begin / row_tiles);
+    int rt = static_cast<int>(u_begin - int64_t(cb) * row_tiles);
+    int ncb = cb, nrt = rt + 1;
+    if (nrt == row_tiles) { nrt = 0; ++ncb; }
+    WeightRegs cur, nxt;
+    if (u_begin < u_end) load_unit(cb, rt, cur);
+    int cur_cb = -1;
+    for (int64_t u = u_begin; u < u_end; ++u) {
+        if (u + 1 < u_end) load_unit(ncb, nrt, nxt);
+        exchange(cur);
+        const int strip = cb * kWarps + warp;
+        if (strip < kblocks) {
+            const int c0 = strip * kStrip;
+            if (cb != cur_cb) {
+                __syncwarp();
+                for (int k = 0; k < a.rp; ++k) {
+                    uint32_t v = 0u;
+                    if (k < a.r) v = *reinterpret_cast<const uint32_t*>(a.A + int64_t(k) * K + c0 + pc);
+                    *reinterpret_cast<uint32_t*>(slab + k * kSlabPitch + p0) = v;
                 }
-                if (R < a.N)
-                    __stcs(reinterpret_cast<uint4*>(a.out + R * K + c0 + 32 * i + 8 * tq),
-                           make_uint4(o[0], o[1], o[2], o[3]));
+                __syncwarp();
+                cur_cb = cb;
+            }
+            const int n0 = rt * kTileRows;
+
+            // acc[nt][.] = (B A)[rows g, g+8][logical columns 2t, 2t+1 of n-tile nt]
+            float acc[8][4];
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+
+            const int R0 = n0 + g, R1 = n0 + g + 8;
+            for (int k0 = 0; k0 < a.rp; k0 += 16) {
+                uint32_t af[4];
+                const int ka = k0 + 2 * tq, kb = k0 + 8 + 2 * tq;
+                const uint16_t* b0p = a.B + int64_t(R0) * a.r;
+                const uint16_t* b1p = a.B + int64_t(R1) * a.r;
+                af[0] = (R0 < N && ka < a.r) ? *reinterpret_cast<const uint32_t*>(b0p + ka) : 0u;
+                af[1] = (R1 < N && ka < a.r) ? *reinterpret_cast<const uint32_t*>(b1p + ka) : 0u;
+                af[2] = (R0 < N && kb < a.r) ? *reinterpret_cast<const uint32_t*>(b0p + kb) : 0u;
+                af[3] = (R1 < N && kb < a.r) ? *reinterpret_cast<const uint32_t*>(b1p + kb) : 0u;
+#pragma unroll
+                for (int np = 0; np < 4; ++np) {
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_t(slab_s + 2u * uint32_t((k0 + lm_row) * kSlabPitch + np * 16 + lm_col),
+                              b0, b1, b2, b3);
+                    mma_bf16_16816(acc[2 * np], af[0], af[1], af[2], af[3], b0, b1);
+                    mma_bf16_16816(acc[2 * np + 1], af[0], af[1], af[2], af[3], b2, b3);
+                }
+            }
+
+            // Epilogue: W~ from the packed word, plus gamma * (B A), rounded once.
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+                const int R = n0 + g + 8 * s;
+                uint16_t* orow = a.out + int64_t(R) * K + c0 + 8 * tq;
+                const float ct = __fmul_rn(e4m3_to_float(static_cast<uint8_t>(cur.sc[s])), cur.mt[s]);
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const uint32_t v = cur.w[s][i];
+                    uint32_t o[4];
+#pragma unroll
+                    for (int jp = 0; jp < 4; ++jp) {
+                        // physical columns 32i + 8t + 2jp, +1 <- n-tile 4i + jp, logical 2t, 2t+1
+                        const uint32_t wb = pack_bf16x2(__fmul_rn(scode[(v >> (8 * jp)) & 15u], ct),
+                                                        __fmul_rn(scode[(v >> (8 * jp + 4)) & 15u], ct));
+                        const float wlo = __uint_as_float(wb << 16);
+                        const float whi = __uint_as_float(wb & 0xffff0000u);
+                        o[jp] = pack_bf16x2(__fmaf_rn(a.gamma, acc[4 * i + jp][2 * s], wlo),
+                                            __fmaf_rn(a.gamma, acc[4 * i + jp][2 * s + 1], whi));
+                    }
+                    if (R < N)
+                        __stcs(reinterpret_cast<uint4*>(orow + 32 * i), make_uint4(o[0], o[1], o[2], o[3]));
+                }
             }
         }
+        cur = nxt;
+        cb = ncb;
+        rt = nrt;
+        if (++nrt == row_tiles) { nrt = 0; ++ncb; }
     }
 }
 
@@ -179,7 +223,8 @@ cudaError_t launch_merge(const MergeArgs& args, const Nf4Table& tab, int num_sms
                          cudaStream_t stream) {
     MergeArgs a = args;
     a.rp = (a.r + 15) / 16 * 16;
-    a.tiles = (a.K / kStrip) * ((a.N + kTileRows - 1) / kTileRows);
+    const int64_t col_blocks = (a.K / kStrip + kWarps - 1) / kWarps;
+    a.tiles = col_blocks * ((a.N + kTileRows - 1) / kTileRows);      // CTA units
     if (a.tiles == 0) return cudaSuccess;
     const int smem = merge_smem_bytes(a.r);
     cudaError_t e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -190,8 +235,7 @@ cudaError_t launch_merge(const MergeArgs& args, const Nf4Table& tab, int num_sms
     if (e != cudaSuccess) return e;
     if (per_sm < 1) per_sm = 1;
     int64_t grid = int64_t(num_sms) * per_sm;
-    const int64_t need = (a.tiles + kWarps - 1) / kWarps;     // at least one tile per warp
-    if (grid > need) grid = need;
+    if (grid > a.tiles) grid = a.tiles;                           // at least one unit per CTA
     merge_kernel<<<dim3(static_cast<unsigned>(grid)), kThreads, smem, stream>>>(a, tab);
     return cudaGetLastError();
 }

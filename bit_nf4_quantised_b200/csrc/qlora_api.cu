@@ -397,12 +397,15 @@ int qlora_quantize_bf16(const uint16_t* W, const qlora_nf4_tensor* out, int* d_n
 
 int qlora_merge(const qlora_nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r,
                 float scale, uint16_t* W_out, qlora_stream_t stream) {
-    int st = check_tensor(w);
-    if (st != QLORA_OK) return st;
+    if (!w) return QLORA_ERR_NULL;
     const int64_t N = w->rows, K = w->cols;
+    if (N < 0 || K < 0 || (K > 0 && N > INT64_MAX / K)) return QLORA_ERR_SHAPE;
     if (K % QLORA_BLOCK != 0) return QLORA_ERR_UNSUPPORTED;
     if (r < 8 || r > QLORA_MAX_RANK || r % 8 != 0) return QLORA_ERR_UNSUPPORTED;
-    if (N == 0 || K == 0) return QLORA_OK;              // A, B, W_out may then be NULL
+    if (N > (int64_t(1) << 31) - 1 || K > (int64_t(1) << 31) - 1) return QLORA_ERR_UNSUPPORTED;
+    if (N == 0 || K == 0) return QLORA_OK;              // nothing read or written
+    int st = check_tensor(w);
+    if (st != QLORA_OK) return st;
     if (!A || !B || !W_out) return QLORA_ERR_NULL;
     if (!aligned(A, 16) || !aligned(B, 16) || !aligned(W_out, 16)) return QLORA_ERR_ALIGN;
     MergeArgs a{};

@@ -173,8 +173,10 @@ QLORA_API int qlora_dequantize(const qlora_nf4_tensor* w, uint16_t* W_out,
  *         the inputs.  Each element is within one bf16 rounding of the exact
  *         value, plus fp32 accumulation error (at most (2r+4) 2^-24 of
  *         |w~| + |gamma| sum_j |B_nj A_jk|).
- * N = 0 or K = 0 launches nothing; A, B and W_out may then be NULL.
- * Shape rules: K % 64 == 0 (every NF4 block lies inside one row); any N.
+ * N = 0 or K = 0 launches nothing; every buffer (the stored tensor's, A, B,
+ * W_out) may then be NULL.
+ * Shape rules: K % 64 == 0 (every NF4 block lies inside one row); N and K
+ * below 2^31.
  * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE, QLORA_ERR_UNSUPPORTED (K or r),
  * QLORA_ERR_ALIGN (A, B, W_out and packed 16-byte aligned; scale_codes,
  * meta_scale 4-byte), QLORA_ERR_CUDA.
