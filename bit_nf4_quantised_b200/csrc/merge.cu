@@ -50,6 +50,17 @@ constexpr int kSlabPitch = kStrip + 8;     // bf16 per slab row: 144 B, conflict
 
 __host__ __device__ constexpr int slab_bytes(int rp) { return rp * kSlabPitch * 2; }
 
+// Shared memory: the 16 codes; the pair table; the warps' slabs.  The pair
+// table holds, for every byte value e of the packed indices, the codes of its
+// two nibbles (q[e & 15], q[e >> 4]) as a float pair, one copy per lane:
+// entry e of lane l at e * 256 + l * 8, so a warp's lookups never share a
+// bank beyond the two wavefronts an 8-byte load takes, and one byte permute
+// (the byte into bits 8-15) plus the lane's base address forms the address.
+constexpr int kCodesOff = 0;
+constexpr int kPairOff = 256;
+constexpr int kPairBytes = 256 * 32 * 8;                         // 64 KiB
+constexpr int kSlabOff = kPairOff + kPairBytes;
+
 // One lane's weight inputs for a unit: the packed words of its columns in
 // rows g and g+8, their blocks' FP8 scale codes and group scales.
 struct WeightRegs {
@@ -61,14 +72,24 @@ struct WeightRegs {
 __global__ void __launch_bounds__(kThreads)
 merge_kernel(MergeArgs a, Nf4Table tab) {
     extern __shared__ __align__(16) uint8_t smem[];
-    float* scode = reinterpret_cast<float*>(smem);                       // 16 codes
+    float* scode = reinterpret_cast<float*>(smem + kCodesOff);            // 16 codes
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint16_t* slab = reinterpret_cast<uint16_t*>(smem + 64 + warp * slab_bytes(a.rp));
+    uint16_t* slab = reinterpret_cast<uint16_t*>(smem + kSlabOff + warp * slab_bytes(a.rp));
     if (threadIdx.x == 0) {            // constant indices: no local copy of the table
 #pragma unroll
         for (int q = 0; q < 16; ++q) scode[q] = tab.code[q];
     }
     __syncthreads();
+    // Pair table: thread t writes 16-byte chunks t, t + 256, ...; chunk c holds
+    // entry c / 16 for lanes 2 (c % 16) and 2 (c % 16) + 1 (consecutive
+    // threads write consecutive chunks: no bank conflicts).
+    for (int c = threadIdx.x; c < kPairBytes / 16; c += kThreads) {
+        const int e = c >> 4;
+        const float lo = scode[e & 15], hi = scode[e >> 4];
+        *reinterpret_cast<float4*>(smem + kPairOff + c * 16) = make_float4(lo, hi, lo, hi);
+    }
+    __syncthreads();
+    const uint8_t* pair_lane = smem + kPairOff + lane * 8;
 
     const int g = lane >> 2, tq = lane & 3;
     // N and K are below 2^31 (checked on the host); products of a row and K
@@ -193,8 +214,9 @@ merge_kernel(MergeArgs a, Nf4Table tab) {
 #pragma unroll
                     for (int jp = 0; jp < 4; ++jp) {
                         // physical columns 32i + 8t + 2jp, +1 <- n-tile 4i + jp, logical 2t, 2t+1
-                        const uint32_t wb = pack_bf16x2(__fmul_rn(scode[(v >> (8 * jp)) & 15u], ct),
-                                                        __fmul_rn(scode[(v >> (8 * jp + 4)) & 15u], ct));
+                        const float2 qp = *reinterpret_cast<const float2*>(
+                            pair_lane + prmt(v, 0u, 0x4404u | (uint32_t(jp) << 4)));
+                        const uint32_t wb = pack_bf16x2(__fmul_rn(qp.x, ct), __fmul_rn(qp.y, ct));
                         const float wlo = __uint_as_float(wb << 16);
                         const float whi = __uint_as_float(wb & 0xffff0000u);
                         o[jp] = pack_bf16x2(__fmaf_rn(a.gamma, acc[4 * i + jp][2 * s], wlo),
@@ -216,7 +238,7 @@ merge_kernel(MergeArgs a, Nf4Table tab) {
 
 int merge_smem_bytes(int r) {
     const int rp = (r + 15) / 16 * 16;
-    return 64 + kWarps * slab_bytes(rp);
+    return kSlabOff + kWarps * slab_bytes(rp);
 }
 
 cudaError_t launch_merge(const MergeArgs& args, const Nf4Table& tab, int num_sms,
