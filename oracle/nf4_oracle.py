@@ -438,3 +438,60 @@ def merge(packed, scale_codes, meta, rows: int, cols: int, A, B, gamma):
     g = float(np.float32(gamma))
     exact = Wt + g * (np.asarray(B, np.float64) @ np.asarray(A, np.float64))
     return exact, bf16_rne_f64(exact)
+
+
+# ---------------------------------------------------------------------------
+# Format variants.  "QLoRA, explained", "A toy run: how much does NF4 lose
+# ...": the same blockwise absmax scheme with other 4-bit codebooks (E2M1
+# FP4, a symmetric 15-level INT4 grid) and other blocksizes (16 to 4096), and
+# "Double quantisation" as an option (without it every block keeps its fp32
+# absmax).  The steps are those of quantize() with the codebook, blocksize
+# and scale storage as parameters; the nearest code is again the number of
+# midpoints strictly below x (midpoints = exact averages of adjacent fp32
+# codes rounded to fp32), a zero block and the padding of a final partial
+# block take the index nearest to 0.
+# ---------------------------------------------------------------------------
+SCALES_FP32 = "fp32"
+SCALES_E4M3 = "e4m3"
+
+
+def midpoints_of(codes: np.ndarray) -> np.ndarray:
+    c64 = np.asarray(codes, dtype=np.float32).astype(np.float64)
+    return ((c64[:-1] + c64[1:]) / 2.0).astype(np.float32)
+
+
+def quantize_fmt(W: np.ndarray, codes: np.ndarray, block: int, scales: str):
+    """W (flattened, fp32) -> (packed, scales, meta).  scales 'fp32': one fp32
+    absmax per block and meta None; 'e4m3': FP8 codes and fp32 constants per
+    256 blocks, as quantize()."""
+    w = np.asarray(W, dtype=np.float32).reshape(-1)
+    if not np.all(np.isfinite(w)):
+        raise NonFiniteWeight("weights must be finite")
+    mids = midpoints_of(codes)
+    absmax = block_absmax(w, block)
+    idx = nearest_code_index(normalise_blocks(w, absmax, block), mids)
+    packed = pack_nibbles(idx)
+    if scales == SCALES_FP32:
+        return packed, absmax.astype(np.float32), None
+    sc, meta = double_quantize(absmax)
+    return packed, sc, meta
+
+
+def dequantize_fmt_bits(packed, scale_data, meta, numel: int, codes: np.ndarray, block: int,
+                        scales: str) -> np.ndarray:
+    """bf16 bits of w~ = bf16_rne(fp32(q[idx] * c~_b)), c~_b the fp32 absmax
+    ('fp32') or fp32(e4m3 * c2) ('e4m3')."""
+    c = (np.asarray(scale_data, dtype=np.float32) if scales == SCALES_FP32
+         else dequantize_scales(scale_data, meta))
+    nblocks = c.size
+    idx = unpack_nibbles(packed, nblocks * block).reshape(nblocks, block)
+    prod = (np.asarray(codes, dtype=np.float32)[idx] * c.reshape(nblocks, 1)).astype(np.float32)
+    return bf16_bits(prod).reshape(-1)[:numel]
+
+
+def format_nbytes(numel: int, block: int, scales: str) -> tuple[int, int, int]:
+    """(packed, scale, meta) byte counts of a stored tensor in a variant format."""
+    nblocks = -(-numel // block)
+    if scales == SCALES_FP32:
+        return nblocks * block // 2, 4 * nblocks, 0
+    return nblocks * block // 2, nblocks, 4 * (-(-nblocks // GROUP))

@@ -531,3 +531,63 @@ def test_requantising_the_unmerged_base_keeps_every_index():
     live = s != 0
     assert live.mean() > 0.99
     assert np.array_equal(idx[live], idx2[live])
+
+
+# --------------------------------------------------------------------------
+# Format variants (codebooks, blocksizes, scale storage)
+# --------------------------------------------------------------------------
+def test_quantize_fmt_nf4_b64_e4m3_is_quantize():
+    rng = np.random.default_rng(41)
+    W = (rng.standard_normal(64 * 256 * 3 + 100) * 0.02).astype(np.float32)
+    codes, _ = o.nf4_codebook()
+    p, s, m = o.quantize_fmt(W, codes, 64, o.SCALES_E4M3)
+    p0, s0, m0 = o.quantize(W)
+    assert np.array_equal(p, p0) and np.array_equal(s, s0)
+    assert np.array_equal(m.view(np.uint32), m0.view(np.uint32))
+    assert np.array_equal(o.dequantize_fmt_bits(p, s, m, W.size, codes, 64, o.SCALES_E4M3),
+                          o.dequantize_bits(p0, s0, m0, W.size))
+
+
+@pytest.mark.parametrize("cb", ["nf4", "fp4", "int4"])
+@pytest.mark.parametrize("block", [16, 64, 256, 4096])
+def test_fp32_scale_variant_matches_brute_force_toy(cb, block):
+    """With fp32 scales the variant reconstructs, before its bf16 rounding,
+    the brute-force toy of "A toy run ..." (argmin over the codebook)."""
+    codes = {"nf4": o.nf4_codebook()[0], "fp4": o.fp4_e2m1_codebook(),
+             "int4": o.int4_codebook()}[cb]
+    rng = np.random.default_rng(42)
+    w = (rng.standard_normal(4096 * 3 + 48) * 0.02).astype(np.float32)
+    p, s, _ = o.quantize_fmt(w, codes, block, o.SCALES_FP32)
+    idx = o.unpack_nibbles(p, s.size * block).reshape(s.size, block)
+    rec = (codes[idx] * s.reshape(-1, 1)).astype(np.float32).reshape(-1)[:w.size]
+    toy = o.single_quant_roundtrip(w, codes, block)
+    assert np.array_equal(rec, toy)
+    bits = o.dequantize_fmt_bits(p, s, None, w.size, codes, block, o.SCALES_FP32)
+    assert np.array_equal(bits, o.bf16_bits(rec))
+
+
+def test_variant_toy_statistics_through_bf16():
+    """M1-M3 of "A toy run ..." through the variant quantiser and its bf16
+    dequantisation: the bf16 rounding adds at most 2^-18 / 3 of relative
+    mean-square error (0.00013 points), so the printed tolerances widen by
+    0.0002 points."""
+    t = _golden_table("toy_statistics.txt")
+    rng = np.random.default_rng(0)
+    w = rng.normal(0, 0.02, 2 ** 20).astype(np.float32)
+    books = {"nf4": o.nf4_codebook()[0], "fp4": o.fp4_e2m1_codebook(), "int4": o.int4_codebook()}
+    cases = {"gauss_nf4_b64": ("nf4", 64), "gauss_fp4_b64": ("fp4", 64),
+             "gauss_int4_b64": ("int4", 64), "gauss_nf4_b16": ("nf4", 16),
+             "gauss_nf4_b4096": ("nf4", 4096)}
+    for key, (cb, block) in cases.items():
+        p, s, _ = o.quantize_fmt(w, books[cb], block, o.SCALES_FP32)
+        rec = o.bf16_bits_to_float(o.dequantize_fmt_bits(p, s, None, w.size, books[cb], block,
+                                                         o.SCALES_FP32)).astype(np.float64)
+        rel = 100 * np.mean((rec - w) ** 2) / np.mean(w.astype(np.float64) ** 2)
+        ref, tol = t[key]
+        assert abs(rel - ref) <= tol + 2e-4, (key, rel, ref)
+
+
+def test_format_nbytes():
+    assert o.format_nbytes(4096 * 4096, 64, o.SCALES_E4M3) == o.quantized_nbytes(4096 * 4096)
+    assert o.format_nbytes(100, 16, o.SCALES_FP32) == (56, 28, 0)
+    assert o.format_nbytes(2 ** 20, 4096, o.SCALES_E4M3) == (2 ** 19, 256, 4)
