@@ -238,6 +238,49 @@ def _quantize_measure(q, syn, device, reps=5):
             "bytes_per_call": nbytes}
 
 
+def _format_measure(q, device, reps=10):
+    """Format variants on a 28672 x 8192 weight (235 M weights, 940 MB fp32):
+    quantise and bf16 dequantise throughput for NF4 / FP4 at blocksize 64 with
+    FP8 scales, NF4 at 16 with fp32 scales and NF4 at 4096.  GB/s of
+    algorithmic bytes (fp32 read + stored written; stored read + bf16 written).
+    The codebooks are built here from their definitions: NF4 from the library,
+    E2M1 FP4 as {0, 0.5, 1, 1.5, 2, 3, 4, 6}/6 with sign."""
+    nf4, _ = q.nf4_build_codebook()
+    mags = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    fp4 = sorted(set([-m / 6.0 for m in mags] + [m / 6.0 for m in mags]))
+    n = 28672 * 8192
+    W = torch.randn(n, device=device) * 0.02
+    out = torch.empty(n, dtype=torch.bfloat16, device=device)
+    rows = []
+    for name, codes, block, sc in (("nf4_b64_e4m3", nf4, 64, q.QLORA_SCALES_E4M3),
+                                   ("fp4_b64_e4m3", fp4, 64, q.QLORA_SCALES_E4M3),
+                                   ("nf4_b16_fp32", nf4, 16, q.QLORA_SCALES_FP32),
+                                   ("nf4_b4096_e4m3", nf4, 4096, q.QLORA_SCALES_E4M3)):
+        f = q.Format(tuple(codes), block, sc)
+        p, s, m = q.qlora_quantize_fmt(W, f, check_finite=False)
+        stored = p.numel() + s.numel() * s.element_size() + (m.numel() * 4 if m is not None else 0)
+
+        def timed(fn):
+            fn()
+            torch.cuda.synchronize()
+            b, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            b.record()
+            for _ in range(reps):
+                fn()
+            e.record()
+            torch.cuda.synchronize()
+            return b.elapsed_time(e) / reps * 1e3
+
+        qu = timed(lambda: q.qlora_quantize_fmt(W, f, check_finite=False))
+        du = timed(lambda: q.qlora_dequantize_fmt(p, s, m, n, f, out=out))
+        rows.append({"format": name, "quantize_us": round(qu, 1),
+                     "quantize_GBps": round((n * 4 + stored) / qu / 1e3, 1),
+                     "dequantize_us": round(du, 1),
+                     "dequantize_GBps": round((n * 2 + stored) / du / 1e3, 1)})
+    del W, out
+    return rows
+
+
 def _gemv_sweep(q, syn, device, reps=10):
     """The decode sweep: 28672 x 8192 and 8192 x 28672 weights with 1, 4 and
     16 tokens.  Per shape the GEMV kernel's CUDA-event time (weights rotated
@@ -511,6 +554,12 @@ def run_gpu(args):
         ex = out["decoder"]["export"]
         for k in ("merge", "requantize", "dequantize"):
             ex[f"{k}_frac_hbm"] = round(ex[f"{k}_GBps"] / peaks["hbm_gbs"], 4)
+        try:
+            out["formats"] = _format_measure(q, device)
+            for row in out["formats"]:
+                row["dequantize_frac_hbm"] = round(row["dequantize_GBps"] / peaks["hbm_gbs"], 4)
+        except Exception as exc:           # an extra measurement never sinks the bench line
+            out["formats"] = {"error": f"{type(exc).__name__}: {exc}"}
         out["e2e"] = _e2e(q, syn, lin, device, max(3, K // 2))
         out["cpu_baseline"] = _cpu_baseline(seconds=args.cpu_seconds)
     else:

@@ -6,6 +6,9 @@ synthetic workload generator (``synthetic``).
 """
 from ._lib import (  # noqa: F401
     EXPORTED,
+    QLORA_SCALES_E4M3,
+    QLORA_SCALES_FP32,
+    Format,
     NF4Tensor,
     QloraError,
     device_error_word,
@@ -13,12 +16,15 @@ from ._lib import (  # noqa: F401
     lib,
     nf4_build_codebook,
     qlora_dequantize,
+    qlora_dequantize_fmt,
+    qlora_format_sizes,
     qlora_linear_backward,
     qlora_linear_forward,
     qlora_linear_workspace_size,
     qlora_merge,
     qlora_quantize,
     qlora_quantize_bf16,
+    qlora_quantize_fmt,
     qlora_quantized_sizes,
     status_string,
     workspace,

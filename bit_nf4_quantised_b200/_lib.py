@@ -43,7 +43,13 @@ EXPORTED = (
     "qlora_linear_forward_noalloc",
     "qlora_merge",
     "qlora_quantize_bf16",
+    "qlora_format_sizes",
+    "qlora_quantize_fmt",
+    "qlora_dequantize_fmt",
 )
+
+QLORA_SCALES_FP32 = 0
+QLORA_SCALES_E4M3 = 1
 
 
 class QloraError(RuntimeError):
@@ -81,6 +87,15 @@ class _Tensor(ctypes.Structure):
     ]
 
 
+class _Format(ctypes.Structure):
+    _fields_ = [
+        ("block", ctypes.c_int32),
+        ("ncodes", ctypes.c_int32),
+        ("codes", ctypes.c_float * 16),
+        ("scales", ctypes.c_int32),
+    ]
+
+
 _LIB = None
 
 
@@ -103,6 +118,10 @@ def lib() -> ctypes.CDLL:
         L.qlora_dequantize.argtypes = [tp, vp, vp]
         L.qlora_quantize_bf16.argtypes = [vp, tp, vp, vp]
         L.qlora_merge.argtypes = [tp, vp, vp, i32, f32, vp, vp]
+        fp = ctypes.POINTER(_Format)
+        L.qlora_format_sizes.argtypes = [i64, fp, sz, sz, sz]
+        L.qlora_quantize_fmt.argtypes = [vp, i64, fp, vp, vp, vp, vp, vp]
+        L.qlora_dequantize_fmt.argtypes = [vp, vp, vp, i64, fp, vp, vp]
         L.qlora_linear_workspace_size.argtypes = [i64, i64, i64, i32, sz]
         fwd = [vp, i64, tp, vp, vp, i32, f32, vp, vp, vp, ctypes.c_size_t, vp]
         bwd = [vp, vp, i64, tp, vp, vp, i32, f32, vp, vp, vp, vp, i32, vp, ctypes.c_size_t, vp]
@@ -237,6 +256,66 @@ def qlora_merge(w: NF4Tensor, A: torch.Tensor, B: torch.Tensor, scale: float,
     st = w.c_struct()
     _check(lib().qlora_merge(ctypes.byref(st), A.data_ptr(), B.data_ptr(), r, float(scale),
                              out.data_ptr(), _stream(stream)), "qlora_merge")
+    return out
+
+
+@dataclass
+class Format:
+    """A quantisation format: codebook (ascending, up to 16 codes), blocksize
+    (power of two, 16..4096) and scale storage (QLORA_SCALES_FP32 or _E4M3)."""
+    codes: tuple
+    block: int = BLOCK
+    scales: int = QLORA_SCALES_E4M3
+
+    def c_struct(self) -> _Format:
+        f = _Format()
+        f.block = int(self.block)
+        f.ncodes = len(self.codes)
+        for i, c in enumerate(self.codes):
+            f.codes[i] = float(c)
+        f.scales = int(self.scales)
+        return f
+
+
+def qlora_format_sizes(numel: int, fmt: Format):
+    p, c, m = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    f = fmt.c_struct()
+    _check(lib().qlora_format_sizes(numel, ctypes.byref(f), ctypes.byref(p), ctypes.byref(c),
+                                    ctypes.byref(m)), "qlora_format_sizes")
+    return p.value, c.value, m.value
+
+
+def qlora_quantize_fmt(W: torch.Tensor, fmt: Format, check_finite: bool = True, stream=None):
+    """(packed u8, scales (fp32 or u8), meta fp32 or None) of a contiguous fp32
+    CUDA tensor in format fmt."""
+    _need(W, torch.float32, "W")
+    n = W.numel()
+    pb, sb, mb = qlora_format_sizes(n, fmt)
+    dev = W.device
+    packed = torch.empty(max(pb, 16), dtype=torch.uint8, device=dev)[:pb]
+    if fmt.scales == QLORA_SCALES_FP32:
+        scales = torch.empty(max(sb // 4, 1), dtype=torch.float32, device=dev)[: sb // 4]
+        meta = None
+    else:
+        scales = torch.empty(max(sb, 4), dtype=torch.uint8, device=dev)[:sb]
+        meta = torch.empty(max(mb // 4, 1), dtype=torch.float32, device=dev)[: mb // 4]
+    flag = torch.zeros(1, dtype=torch.int32, device=dev) if check_finite else None
+    f = fmt.c_struct()
+    _check(lib().qlora_quantize_fmt(W.data_ptr(), n, ctypes.byref(f), _ptr(packed), _ptr(scales),
+                                    _ptr(meta), _ptr(flag), _stream(stream)), "qlora_quantize_fmt")
+    if check_finite and int(flag.item()) != 0:
+        raise QloraError(QLORA_ERR_NONFINITE, "qlora_quantize_fmt")
+    return packed, scales, meta
+
+
+def qlora_dequantize_fmt(packed: torch.Tensor, scales: torch.Tensor, meta, numel: int,
+                         fmt: Format, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    out = out if out is not None else torch.empty(numel, dtype=torch.bfloat16, device=packed.device)
+    _need(out, torch.bfloat16, "out")
+    f = fmt.c_struct()
+    _check(lib().qlora_dequantize_fmt(_ptr(packed), _ptr(scales), _ptr(meta), numel,
+                                      ctypes.byref(f), out.data_ptr(), _stream(stream)),
+           "qlora_dequantize_fmt")
     return out
 
 

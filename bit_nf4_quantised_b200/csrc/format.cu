@@ -1,0 +1,209 @@
+// K1 / K6 format variants: blockwise absmax quantisation with any codebook of
+// up to 16 codes, blocksizes 16 to 4096, and the block scales kept as fp32 or
+// double-quantised to FP8 E4M3 with one fp32 constant per 256 blocks.
+//
+// "QLoRA, explained", "A toy run: how much does NF4 lose ...": the same scheme
+// with the E2M1 FP4 and symmetric INT4 codebooks and blocksizes 16 and 4096
+// next to NF4 at 64; "Double quantisation" is the optional second level.
+// The steps are those of K1/K6: c_b = max |w| over the block, the index of
+// the nearest code of fp32(w / c_b) as the number of midpoints strictly below
+// it (a zero block and the padding of a final partial block take the index
+// nearest to 0), two indices per byte with the even element in the low
+// nibble; w~ = bf16_rne(fp32(q[idx] * c~_b)) with c~_b the fp32 absmax or
+// fp32(e4m3 * c2).
+//
+// Quantise: one CTA per group of 256 blocks.  A block is covered by
+// min(32, B/4) lanes that each load 16-byte pieces; the lanes reduce the
+// absmax with shuffles and then re-read their pieces (from L1/L2) to write the
+// indices, four per 16-bit store.  The group's scales stay in shared memory
+// for the FP8 pass, as in K1.  Dequantise: as K6, one packed word (8 weights)
+// per thread and one 16-byte store; the block index is a shift.
+#include "kernels.cuh"
+
+namespace qnf4 {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ uint32_t nearest_code(float x, const float* smid) {
+    // number of midpoints strictly below x; unused midpoints are +inf
+    uint32_t i = 0;
+    i += (x > smid[i + 7]) ? 8u : 0u;
+    i += (x > smid[i + 3]) ? 4u : 0u;
+    i += (x > smid[i + 1]) ? 2u : 0u;
+    i += (x > smid[i + 0]) ? 1u : 0u;
+    return i;
+}
+
+template <bool kFull>
+__global__ void __launch_bounds__(kThreads)
+quantize_fmt_kernel(const float* __restrict__ W, int64_t numel, int64_t nblocks, FmtArgs f,
+                    uint8_t* __restrict__ packed, void* __restrict__ scales,
+                    float* __restrict__ meta, int* __restrict__ nonfinite_flag, FmtTable tab) {
+    __shared__ float smid[16];
+    __shared__ float sabs[QLORA_GROUP];
+    __shared__ float sred[kThreads / 32];
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {                    // constant indices: no local copy of the table
+#pragma unroll
+        for (int q = 0; q < 15; ++q) smid[q] = tab.mid[q];
+        smid[15] = __int_as_float(0x7f800000);
+    }
+    __syncthreads();
+
+    const int lp = f.block >= 128 ? 32 : f.block / 4;        // lanes per block
+    const int bpw = 32 / lp;                                  // blocks per warp step
+    const int cpl = f.block / (4 * lp);                       // 16-byte pieces per lane
+    const int sub = lane % lp;
+    const int64_t group = blockIdx.x;
+    bool bad = false;
+
+    for (int blk = warp * bpw + lane / lp; blk < QLORA_GROUP; blk += (kThreads / 32) * bpw) {
+        const int64_t gblk = group * QLORA_GROUP + blk;
+        const int64_t ebase = gblk * f.block;
+        float a = 0.f;
+        for (int j = 0; j < cpl; ++j) {
+            const int64_t e0 = ebase + int64_t(j * lp + sub) * 4;
+            float4 v;
+            if (kFull) {
+                v = *reinterpret_cast<const float4*>(W + e0);
+            } else {
+                v.x = (e0 + 0 < numel) ? W[e0 + 0] : 0.f;
+                v.y = (e0 + 1 < numel) ? W[e0 + 1] : 0.f;
+                v.z = (e0 + 2 < numel) ? W[e0 + 2] : 0.f;
+                v.w = (e0 + 3 < numel) ? W[e0 + 3] : 0.f;
+            }
+            bad |= !(isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w));
+            a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+        }
+        for (int o = lp / 2; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        const bool live = kFull || gblk < nblocks;
+        for (int j = 0; j < cpl; ++j) {
+            const int64_t e0 = ebase + int64_t(j * lp + sub) * 4;
+            float4 v;
+            if (kFull) {
+                v = *reinterpret_cast<const float4*>(W + e0);
+            } else {
+                v.x = (e0 + 0 < numel) ? W[e0 + 0] : 0.f;
+                v.y = (e0 + 1 < numel) ? W[e0 + 1] : 0.f;
+                v.z = (e0 + 2 < numel) ? W[e0 + 2] : 0.f;
+                v.w = (e0 + 3 < numel) ? W[e0 + 3] : 0.f;
+            }
+            uint32_t q0 = tab.zero_index, q1 = tab.zero_index, q2 = tab.zero_index,
+                     q3 = tab.zero_index;
+            if (a > 0.f) {
+                q0 = nearest_code(__fdiv_rn(v.x, a), smid);
+                q1 = nearest_code(__fdiv_rn(v.y, a), smid);
+                q2 = nearest_code(__fdiv_rn(v.z, a), smid);
+                q3 = nearest_code(__fdiv_rn(v.w, a), smid);
+            }
+            if (live)
+                *reinterpret_cast<uint16_t*>(packed + e0 / 2) =
+                    static_cast<uint16_t>(q0 | (q1 << 4) | (q2 << 8) | (q3 << 12));
+        }
+        if (sub == 0) sabs[blk] = a;
+    }
+    if (bad && nonfinite_flag != nullptr) atomicOr(nonfinite_flag, 1);
+    __syncthreads();
+
+    const int64_t gblk = group * QLORA_GROUP + tid;
+    const bool live = kFull || gblk < nblocks;
+    const float c = sabs[tid];
+    if (f.scales_fp32) {
+        if (live) reinterpret_cast<float*>(scales)[gblk] = c;
+        return;
+    }
+    float m = c;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) sred[warp] = m;
+    __syncthreads();
+    float gmax = sred[0];
+#pragma unroll
+    for (int w = 1; w < kThreads / 32; ++w) gmax = fmaxf(gmax, sred[w]);
+    const float c2 = __fdiv_rn(gmax, 448.0f);
+    uint8_t code = 0;
+    if (c2 > 0.f)
+        code = static_cast<uint8_t>(__nv_cvt_float_to_fp8(__fdiv_rn(c, c2), __NV_SATFINITE, __NV_E4M3));
+    if (live) reinterpret_cast<uint8_t*>(scales)[gblk] = code;
+    if (tid == 0) meta[group] = c2;
+}
+
+__global__ void __launch_bounds__(kThreads)
+dequantize_fmt_kernel(const uint32_t* __restrict__ packed, const void* __restrict__ scales,
+                      const float* __restrict__ meta, int64_t numel, FmtArgs f,
+                      uint16_t* __restrict__ out, FmtTable tab) {
+    __shared__ float scode[16];
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int q = 0; q < 16; ++q) scode[q] = tab.code[q];
+    }
+    __syncthreads();
+    const int64_t nwords = (numel + 7) / 8;
+    for (int64_t u = blockIdx.x * int64_t(kThreads) + threadIdx.x; u < nwords;
+         u += int64_t(gridDim.x) * kThreads) {
+        const uint32_t v = packed[u];
+        const int64_t b = (u * 8) >> f.log2_block;
+        const float ct = f.scales_fp32
+                             ? reinterpret_cast<const float*>(scales)[b]
+                             : __fmul_rn(e4m3_to_float(reinterpret_cast<const uint8_t*>(scales)[b]),
+                                         meta[b >> 8]);
+        uint32_t r[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            r[j] = pack_bf16x2(__fmul_rn(scode[(v >> (8 * j)) & 15u], ct),
+                               __fmul_rn(scode[(v >> (8 * j + 4)) & 15u], ct));
+        const int64_t e = u * 8;
+        if (e + 8 <= numel) {
+            __stcs(reinterpret_cast<uint4*>(out + e), make_uint4(r[0], r[1], r[2], r[3]));
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (e + j < numel) out[e + j] = static_cast<uint16_t>(r[j >> 1] >> (16 * (j & 1)));
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_fmt(const float* W, int64_t numel, const FmtArgs& f, uint8_t* packed,
+                                void* scales, float* meta, int* nonfinite_flag,
+                                const FmtTable& tab, cudaStream_t stream) {
+    const int64_t nblocks = (numel + f.block - 1) / f.block;
+    const int64_t ngroups = (nblocks + QLORA_GROUP - 1) / QLORA_GROUP;
+    const int64_t group_elems = int64_t(QLORA_GROUP) * f.block;
+    const int64_t full = numel / group_elems;                // groups with no tail
+    if (full > 0) {
+        quantize_fmt_kernel<true><<<dim3(static_cast<unsigned>(full)), kThreads, 0, stream>>>(
+            W, numel, nblocks, f, packed, scales, meta, nonfinite_flag, tab);
+    }
+    if (ngroups > full) {
+        // the single trailing group, offset so blockIdx.x is its group index
+        const int64_t off = full * group_elems;
+        const int64_t blk_off = full * QLORA_GROUP;
+        void* sc = f.scales_fp32 ? static_cast<void*>(static_cast<float*>(scales) + blk_off)
+                                 : static_cast<void*>(static_cast<uint8_t*>(scales) + blk_off);
+        quantize_fmt_kernel<false><<<1, kThreads, 0, stream>>>(
+            W + off, numel - off, nblocks - blk_off, f, packed + off / 2, sc,
+            meta == nullptr ? nullptr : meta + full, nonfinite_flag, tab);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize_fmt(const uint8_t* packed, const void* scales, const float* meta,
+                                  int64_t numel, const FmtArgs& f, uint16_t* out,
+                                  const FmtTable& tab, int num_sms, cudaStream_t stream) {
+    const int64_t nwords = (numel + 7) / 8;
+    int64_t grid = (nwords + kThreads - 1) / kThreads;
+    const int64_t cap = int64_t(num_sms) * 8;
+    if (grid > cap) grid = cap;
+    if (grid < 1) grid = 1;
+    dequantize_fmt_kernel<<<dim3(static_cast<unsigned>(grid)), kThreads, 0, stream>>>(
+        reinterpret_cast<const uint32_t*>(packed), scales, meta, numel, f, out, tab);
+    return cudaGetLastError();
+}
+
+}  // namespace qnf4

@@ -20,6 +20,24 @@ cudaError_t launch_quantize_bf16(const uint16_t* W, int64_t numel, uint8_t* pack
                                  uint8_t* scale_codes, float* meta, int* nonfinite_flag,
                                  const Nf4Table& tab, cudaStream_t stream);
 
+// ------------------------------------------------- K1 / K6 format variants
+struct FmtTable {
+    float code[16];            // codebook (unused entries 0)
+    float mid[15];             // fp32 midpoints; +inf past the last code
+    uint32_t zero_index;       // index of the code nearest 0 (zero blocks, padding)
+};
+struct FmtArgs {
+    int block;                 // power of two, 16..4096
+    int log2_block;
+    int scales_fp32;           // 1: fp32 absmax per block; 0: E4M3 + fp32 per 256 blocks
+};
+cudaError_t launch_quantize_fmt(const float* W, int64_t numel, const FmtArgs& f, uint8_t* packed,
+                                void* scales, float* meta, int* nonfinite_flag,
+                                const FmtTable& tab, cudaStream_t stream);
+cudaError_t launch_dequantize_fmt(const uint8_t* packed, const void* scales, const float* meta,
+                                  int64_t numel, const FmtArgs& f, uint16_t* out,
+                                  const FmtTable& tab, int num_sms, cudaStream_t stream);
+
 // ---------------------------------------------------------------- K7 merge
 struct MergeArgs {
     const uint32_t* packed;      // N*K/8 words of packed indices

@@ -5,6 +5,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstring>
+#include <limits>
 #include <mutex>
 
 #include "kernels.cuh"
@@ -263,6 +264,41 @@ void gemm_schedule(GemmArgs& g, bool trans) {
     if (tiles > pairs) g.col_budget = cdiv(tiles, pairs) * tn;
 }
 
+// Format variants: validate a qlora_format and build the kernels' table.
+int check_format(const qlora_format* f, FmtTable* t, FmtArgs* a) {
+    if (!f) return QLORA_ERR_NULL;
+    const int b = f->block;
+    if (b < 16 || b > 4096 || (b & (b - 1)) != 0) return QLORA_ERR_UNSUPPORTED;
+    if (f->ncodes < 2 || f->ncodes > 16) return QLORA_ERR_UNSUPPORTED;
+    if (f->scales != QLORA_SCALES_FP32 && f->scales != QLORA_SCALES_E4M3) return QLORA_ERR_UNSUPPORTED;
+    for (int i = 0; i < f->ncodes; ++i) {
+        if (!std::isfinite(f->codes[i])) return QLORA_ERR_UNSUPPORTED;
+        if (i > 0 && !(f->codes[i] > f->codes[i - 1])) return QLORA_ERR_UNSUPPORTED;
+    }
+    if (t) {
+        std::memset(t, 0, sizeof(*t));
+        for (int i = 0; i < f->ncodes; ++i) t->code[i] = f->codes[i];
+        uint32_t z = 0;
+        for (int i = 0; i < 15; ++i) {
+            if (i < f->ncodes - 1) {
+                // exact average of two fp32 values (exact in double), rounded to fp32
+                t->mid[i] = static_cast<float>((double(f->codes[i]) + double(f->codes[i + 1])) / 2.0);
+                if (0.0f > t->mid[i]) ++z;
+            } else {
+                t->mid[i] = std::numeric_limits<float>::infinity();
+            }
+        }
+        t->zero_index = z;
+    }
+    if (a) {
+        a->block = b;
+        a->log2_block = 0;
+        while ((1 << a->log2_block) < b) ++a->log2_block;
+        a->scales_fp32 = f->scales == QLORA_SCALES_FP32 ? 1 : 0;
+    }
+    return QLORA_OK;
+}
+
 cudaError_t record(const qlora_events* ev, bool begin, cudaStream_t s) {
     if (!ev) return cudaSuccess;
     void* e = begin ? ev->gemm_begin : ev->gemm_end;
@@ -393,6 +429,55 @@ int qlora_quantize_bf16(const uint16_t* W, const qlora_nf4_tensor* out, int* d_n
     return cuda_status(launch_quantize_bf16(W, numel, out->packed, out->scale_codes,
                                             out->meta_scale, d_nonfinite_flag, table(),
                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int qlora_format_sizes(int64_t numel, const qlora_format* f, size_t* packed_bytes,
+                       size_t* scale_bytes, size_t* meta_bytes) {
+    if (!packed_bytes || !scale_bytes || !meta_bytes) return QLORA_ERR_NULL;
+    int st = check_format(f, nullptr, nullptr);
+    if (st != QLORA_OK) return st;
+    if (numel < 0) return QLORA_ERR_SHAPE;
+    const int64_t nblocks = cdiv(numel, f->block);
+    *packed_bytes = static_cast<size_t>(nblocks) * (f->block / 2);
+    if (f->scales == QLORA_SCALES_FP32) {
+        *scale_bytes = static_cast<size_t>(nblocks) * 4;
+        *meta_bytes = 0;
+    } else {
+        *scale_bytes = static_cast<size_t>(nblocks);
+        *meta_bytes = static_cast<size_t>(cdiv(nblocks, QLORA_GROUP)) * 4;
+    }
+    return QLORA_OK;
+}
+
+int qlora_quantize_fmt(const float* W, int64_t numel, const qlora_format* f, uint8_t* packed,
+                       void* scales, float* meta, int* d_nonfinite_flag, qlora_stream_t stream) {
+    FmtTable t;
+    FmtArgs a;
+    int st = check_format(f, &t, &a);
+    if (st != QLORA_OK) return st;
+    if (numel < 0) return QLORA_ERR_SHAPE;
+    if (numel == 0) return QLORA_OK;
+    if (!W || !packed || !scales || (!a.scales_fp32 && !meta)) return QLORA_ERR_NULL;
+    if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(scales, 4) || (meta && !aligned(meta, 4)))
+        return QLORA_ERR_ALIGN;
+    return cuda_status(launch_quantize_fmt(W, numel, a, packed, scales, meta, d_nonfinite_flag, t,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int qlora_dequantize_fmt(const uint8_t* packed, const void* scales, const float* meta,
+                         int64_t numel, const qlora_format* f, uint16_t* out,
+                         qlora_stream_t stream) {
+    FmtTable t;
+    FmtArgs a;
+    int st = check_format(f, &t, &a);
+    if (st != QLORA_OK) return st;
+    if (numel < 0) return QLORA_ERR_SHAPE;
+    if (numel == 0) return QLORA_OK;
+    if (!packed || !scales || !out || (!a.scales_fp32 && !meta)) return QLORA_ERR_NULL;
+    if (!aligned(packed, 16) || !aligned(out, 16) || !aligned(scales, 4) || (meta && !aligned(meta, 4)))
+        return QLORA_ERR_ALIGN;
+    return cuda_status(launch_dequantize_fmt(packed, scales, meta, numel, a, out, t, num_sms(),
+                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int qlora_merge(const qlora_nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r,

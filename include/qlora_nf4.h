@@ -155,6 +155,68 @@ QLORA_API int qlora_dequantize(const qlora_nf4_tensor* w, uint16_t* W_out,
                      qlora_stream_t stream);
 
 /*
+ * Format variants ("QLoRA, explained", "A toy run: how much does NF4 lose
+ * ..."): the same blockwise absmax quantisation with another codebook (the
+ * page compares E2M1 FP4 and a symmetric 15-level INT4 grid with NF4) and
+ * blocksize (16 and 4096 next to 64), with the block scales either kept as
+ * fp32 or double-quantised as in "Double quantisation".
+ * The stored layout generalises the NF4 one: nblocks = ceil(numel / block);
+ *   packed : nblocks * block / 2 bytes, two indices per byte, the even
+ *            element in the low nibble; a final partial block is padded with
+ *            the index of the code nearest 0.
+ *   scales : QLORA_SCALES_FP32 -- nblocks fp32, the block absmax c_b;
+ *            QLORA_SCALES_E4M3 -- nblocks bytes of FP8 E4M3 codes of c_b / c2,
+ *            with meta = ceil(nblocks / 256) fp32 constants c2 (as NF4).
+ * Index of a weight: the number of midpoints strictly below fp32(w / c_b),
+ * midpoint i being the exact average of codes i and i+1 rounded to fp32; a
+ * zero block takes the index of the code nearest 0.  Dequantisation:
+ * w~ = bf16_rne(fp32(codes[idx] * c~_b)), c~_b = c_b or fp32(e4m3 * c2).
+ * With the NF4 codebook, block 64 and E4M3 scales the layout and every byte
+ * equal those of qlora_quantize.
+ */
+typedef enum { QLORA_SCALES_FP32 = 0, QLORA_SCALES_E4M3 = 1 } qlora_scale_format;
+
+typedef struct {
+    int32_t block;       /* elements per block: a power of two, 16 ... 4096   */
+    int32_t ncodes;      /* 2 ... 16                                          */
+    float codes[16];     /* strictly ascending, finite; entries past ncodes   */
+                         /* are ignored                                       */
+    int32_t scales;      /* a qlora_scale_format                              */
+} qlora_format;
+
+/*
+ * qlora_format_sizes -- byte sizes of the packed, scale and meta buffers of
+ * numel weights in format f (meta is 0 bytes for fp32 scales).  Host only.
+ * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE (numel < 0), QLORA_ERR_UNSUPPORTED
+ * (a format field out of range, codes not strictly ascending or not finite).
+ */
+QLORA_API int qlora_format_sizes(int64_t numel, const qlora_format* f, size_t* packed_bytes,
+                                 size_t* scale_bytes, size_t* meta_bytes);
+
+/*
+ * qlora_quantize_fmt -- quantise numel fp32 weights (device, read) in format
+ * f (host struct, read) into packed, scales and meta (device, written, sized
+ * by qlora_format_sizes; meta may be NULL for fp32 scales).
+ * d_nonfinite_flag as in qlora_quantize.  numel = 0 launches nothing.
+ * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE, QLORA_ERR_UNSUPPORTED,
+ * QLORA_ERR_ALIGN (W and packed 16-byte aligned; scales and meta 4-byte),
+ * QLORA_ERR_CUDA.
+ */
+QLORA_API int qlora_quantize_fmt(const float* W, int64_t numel, const qlora_format* f,
+                                 uint8_t* packed, void* scales, float* meta,
+                                 int* d_nonfinite_flag, qlora_stream_t stream);
+
+/*
+ * qlora_dequantize_fmt -- w~ of numel weights stored in format f, written as
+ * bf16 bits to out (device, numel, 16-byte aligned).  Other buffers as
+ * qlora_quantize_fmt (read).  numel = 0 launches nothing.
+ * Errors as qlora_quantize_fmt.
+ */
+QLORA_API int qlora_dequantize_fmt(const uint8_t* packed, const void* scales, const float* meta,
+                                   int64_t numel, const qlora_format* f, uint16_t* out,
+                                   qlora_stream_t stream);
+
+/*
  * qlora_merge -- the fine-tuned weight for bf16 export,
  *     W_out = bf16_rne( W~ + scale * B A ).
  * "QLoRA, explained", "The forward pass and gradients": the model that was

@@ -132,6 +132,52 @@ def test_merge_and_bf16_quantize_argument_errors(q):
     assert L.qlora_quantize_bf16(fake, ctypes.byref(empty), None, None) == E.QLORA_OK
 
 
+def _books():
+    return {"nf4": tuple(o.nf4_codebook()[0]), "fp4": tuple(o.fp4_e2m1_codebook()),
+            "int4": tuple(o.int4_codebook())}
+
+
+@pytest.mark.parametrize("numel", [0, 1, 100, 4096 * 4096, 2 ** 20 + 17])
+@pytest.mark.parametrize("block", [16, 64, 4096])
+@pytest.mark.parametrize("scales", ["fp32", "e4m3"])
+def test_format_sizes_match_oracle(q, numel, block, scales):
+    f = q.Format(_books()["fp4"], block,
+                 q.QLORA_SCALES_FP32 if scales == "fp32" else q.QLORA_SCALES_E4M3)
+    assert q.qlora_format_sizes(numel, f) == o.format_nbytes(numel, block, scales)
+
+
+def test_format_validation_before_any_launch(q):
+    L = q.lib()
+    E = q._lib
+    fake = 0x40000
+    p, c, m = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+
+    def st(fmt, numel=1000):
+        f = fmt.c_struct()
+        return L.qlora_format_sizes(numel, ctypes.byref(f), ctypes.byref(p), ctypes.byref(c),
+                                    ctypes.byref(m))
+
+    good = q.Format(_books()["nf4"], 64, q.QLORA_SCALES_E4M3)
+    assert st(good) == E.QLORA_OK
+    for block in (8, 48, 8192, 0):
+        assert st(q.Format(good.codes, block)) == E.QLORA_ERR_UNSUPPORTED
+    assert st(q.Format((0.5,), 64)) == E.QLORA_ERR_UNSUPPORTED            # one code
+    assert st(q.Format((0.0, 0.5, 0.5), 64)) == E.QLORA_ERR_UNSUPPORTED   # not strictly ascending
+    assert st(q.Format((0.0, float("nan")), 64)) == E.QLORA_ERR_UNSUPPORTED
+    assert st(q.Format(good.codes, 64, 7)) == E.QLORA_ERR_UNSUPPORTED
+    assert st(good, -1) == E.QLORA_ERR_SHAPE
+    assert L.qlora_format_sizes(10, None, ctypes.byref(p), ctypes.byref(c), ctypes.byref(m)) == E.QLORA_ERR_NULL
+    f = good.c_struct()
+    assert L.qlora_quantize_fmt(None, 1000, ctypes.byref(f), fake, fake, fake, None, None) == E.QLORA_ERR_NULL
+    assert L.qlora_quantize_fmt(fake, 1000, ctypes.byref(f), fake, fake, None, None, None) == E.QLORA_ERR_NULL
+    assert L.qlora_quantize_fmt(fake + 4, 1000, ctypes.byref(f), fake, fake, fake, None, None) == E.QLORA_ERR_ALIGN
+    assert L.qlora_quantize_fmt(None, 0, ctypes.byref(f), None, None, None, None, None) == E.QLORA_OK
+    assert L.qlora_dequantize_fmt(fake, fake, fake, 1000, ctypes.byref(f), fake + 2, None) == E.QLORA_ERR_ALIGN
+    assert L.qlora_dequantize_fmt(fake, fake, fake, -5, ctypes.byref(f), fake, None) == E.QLORA_ERR_SHAPE
+    f32 = q.Format(good.codes, 16, q.QLORA_SCALES_FP32).c_struct()
+    assert L.qlora_dequantize_fmt(fake, None, None, 1000, ctypes.byref(f32), fake, None) == E.QLORA_ERR_NULL
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     import bit_nf4_quantised_b200._lib as L
     monkeypatch.setattr(L, "_LIB", None)

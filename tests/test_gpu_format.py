@@ -1,0 +1,117 @@
+"""GPU parity of the format variants (qlora_quantize_fmt / qlora_dequantize_fmt)
+against the oracle through the C-ABI: NF4, E2M1 FP4 and INT4 codebooks,
+blocksizes 16 to 4096, fp32 or double-quantised scales, bit-exact indices,
+scales and dequantised bf16; and the toy statistics of "A toy run ..."
+(relative MSE on 2^20 Gaussian weights) reproduced from the GPU's outputs."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import nf4_oracle as o
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def q():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    import bit_nf4_quantised_b200 as pkg
+    pkg.lib()
+    return pkg
+
+
+BOOKS = {"nf4": o.nf4_codebook()[0], "fp4": o.fp4_e2m1_codebook(), "int4": o.int4_codebook()}
+
+
+def _fmt(q, cb, block, scales):
+    return q.Format(tuple(float(c) for c in BOOKS[cb]), block,
+                    q.QLORA_SCALES_FP32 if scales == o.SCALES_FP32 else q.QLORA_SCALES_E4M3)
+
+
+CASES = [
+    ("nf4", 16, o.SCALES_FP32, 4096 * 64 + 40),
+    ("nf4", 16, o.SCALES_E4M3, 16 * 256 * 3 + 8),
+    ("fp4", 64, o.SCALES_E4M3, 64 * 256 * 2 + 100),
+    ("int4", 64, o.SCALES_FP32, 4096 * 7 + 3),
+    ("nf4", 128, o.SCALES_E4M3, 128 * 256 + 5000),
+    ("fp4", 512, o.SCALES_FP32, 512 * 300 + 1),
+    ("int4", 4096, o.SCALES_E4M3, 4096 * 256 + 4096 * 3 + 77),
+    ("nf4", 64, o.SCALES_E4M3, 1),
+]
+
+
+@pytest.mark.parametrize("cb,block,scales,numel", CASES)
+def test_format_matches_oracle(q, cb, block, scales, numel):
+    rng = np.random.default_rng(block + numel)
+    w = (rng.standard_normal(numel) * 0.02).astype(np.float32)
+    if numel > 100:
+        w[: block] = 0.0                                   # an all-zero block
+        w[rng.integers(0, numel, 20)] *= 10.0              # outliers
+    f = _fmt(q, cb, block, scales)
+    packed, sc, meta = q.qlora_quantize_fmt(torch.from_numpy(w).cuda(), f)
+    deq = q.qlora_dequantize_fmt(packed, sc, meta, numel, f)
+    torch.cuda.synchronize()
+    p0, s0, m0 = o.quantize_fmt(w, BOOKS[cb], block, scales)
+    assert np.array_equal(packed.cpu().numpy(), p0), "packed indices differ"
+    if scales == o.SCALES_FP32:
+        assert np.array_equal(sc.cpu().numpy().view(np.uint32), s0.view(np.uint32))
+        assert meta is None
+    else:
+        assert np.array_equal(sc.cpu().numpy(), s0)
+        assert np.array_equal(meta.cpu().numpy().view(np.uint32), m0.view(np.uint32))
+    ref = o.dequantize_fmt_bits(p0, s0, m0, numel, BOOKS[cb], block, scales)
+    assert np.array_equal(deq.view(torch.int16).cpu().numpy().view(np.uint16), ref)
+
+
+def test_nf4_format_is_the_stored_nf4_layout(q):
+    """NF4, block 64, E4M3 scales: byte for byte what qlora_quantize stores."""
+    rng = np.random.default_rng(3)
+    W = torch.from_numpy((rng.standard_normal((300, 4096)) * 0.02).astype(np.float32)).cuda()
+    w = q.qlora_quantize(W)
+    packed, sc, meta = q.qlora_quantize_fmt(W.reshape(-1), _fmt(q, "nf4", 64, o.SCALES_E4M3))
+    torch.cuda.synchronize()
+    assert torch.equal(packed, w.packed) and torch.equal(sc, w.scale_codes)
+    assert torch.equal(meta.view(torch.int32), w.meta_scale.view(torch.int32))
+
+
+def _golden_table():
+    import os
+    out = {}
+    with open(os.path.join(os.path.dirname(__file__), "golden", "toy_statistics.txt")) as fh:
+        for ln in fh:
+            if ln.strip() and not ln.startswith("#"):
+                k, v, tol = ln.split()
+                out[k] = (float(v), float(tol))
+    return out
+
+
+def test_toy_statistics_from_the_gpu(q):
+    """M1-M3: relative MSE of NF4 / FP4 / INT4 at blocksize 64 and NF4 at 16
+    and 4096 (fp32 scales, 2^20 N(0, 0.02^2) weights, seed 0) from the GPU's
+    bf16 dequantisation; tolerances widened by 0.0002 points for the bf16
+    rounding (at most 2^-18/3 of relative mean-square error)."""
+    t = _golden_table()
+    rng = np.random.default_rng(0)
+    w = rng.normal(0, 0.02, 2 ** 20).astype(np.float32)
+    wd = torch.from_numpy(w).cuda()
+    w64 = torch.from_numpy(w.astype(np.float64))
+    cases = {"gauss_nf4_b64": ("nf4", 64), "gauss_fp4_b64": ("fp4", 64),
+             "gauss_int4_b64": ("int4", 64), "gauss_nf4_b16": ("nf4", 16),
+             "gauss_nf4_b4096": ("nf4", 4096)}
+    got = {}
+    for key, (cb, block) in cases.items():
+        f = _fmt(q, cb, block, o.SCALES_FP32)
+        packed, sc, meta = q.qlora_quantize_fmt(wd, f)
+        rec = q.qlora_dequantize_fmt(packed, sc, meta, w.size, f).double().cpu()
+        got[key] = float(100 * torch.mean((rec - w64) ** 2) / torch.mean(w64 ** 2))
+        ref, tol = t[key]
+        assert abs(got[key] - ref) <= tol + 2e-4, (key, got[key], ref)
+    for cb in ("nf4", "fp4", "int4"):
+        sq = 10 * math.log10(100 / got[f"gauss_{cb}_b64"])
+        ref, tol = t[f"sqnr_{cb}_db"]
+        assert abs(sq - ref) <= tol + 2e-3, (cb, sq, ref)
