@@ -495,3 +495,53 @@ def format_nbytes(numel: int, block: int, scales: str) -> tuple[int, int, int]:
     if scales == SCALES_FP32:
         return nblocks * block // 2, 4 * nblocks, 0
     return nblocks * block // 2, nblocks, 4 * (-(-nblocks // GROUP))
+
+
+# ---------------------------------------------------------------------------
+# Layer chaining with gradient checkpointing.  "QLoRA, explained", "The
+# algorithm, step by step" (gradient checkpointing enabled) and "Compute and
+# memory cost" (checkpointing is effectively mandatory; a recomputed forward
+# dequantises every block a third time per step).  The chained block is the
+# MLP of the Llama-shaped workloads, y = down(silu(gate(x)) * up(x)), every
+# linear an adapted NF4 layer; the pages print no activation, so SwiGLU is
+# the reading taken from those shapes.  With checkpointing only x is kept
+# from the forward and the backward recomputes gate(x), up(x) and h.
+# ---------------------------------------------------------------------------
+def silu(z):
+    z = np.asarray(z, np.float64)
+    return z / (1.0 + np.exp(-z))
+
+
+def silu_grad(z):
+    """d silu / dz = s (1 + z (1 - s)), s the logistic sigmoid."""
+    z = np.asarray(z, np.float64)
+    s = 1.0 / (1.0 + np.exp(-z))
+    return s * (1.0 + z * (1.0 - s))
+
+
+def mlp_forward(X, layers, gamma):
+    """layers = {'gate': (Wt, A, B), 'up': ..., 'down': ...} with Wt = W~
+    [out, in].  -> (Y, saved) where saved = (G, U, H) are the activations a
+    non-checkpointed backward keeps."""
+    G, _ = linear_forward(X, *layers["gate"], gamma)
+    U, _ = linear_forward(X, *layers["up"], gamma)
+    H = silu(G) * U
+    Y, _ = linear_forward(H, *layers["down"], gamma)
+    return Y, (G, U, H)
+
+
+def mlp_backward(dY, X, layers, gamma, saved=None):
+    """-> (dX, {name: (dA, dB)}).  saved = None recomputes the forward from X
+    (gradient checkpointing: the third dequantisation of gate and up)."""
+    if saved is None:
+        _, saved = mlp_forward(X, layers, gamma)
+    G, U, H = saved
+    Wd, Ad, Bd = layers["down"]
+    dH, dAd, dBd, _ = linear_backward(dY, H, Wd, Ad, Bd, gamma)
+    dG = dH * U * silu_grad(G)
+    dU = dH * silu(G)
+    Wg, Ag, Bg = layers["gate"]
+    Wu, Au, Bu = layers["up"]
+    dXg, dAg, dBg, _ = linear_backward(dG, X, Wg, Ag, Bg, gamma)
+    dXu, dAu, dBu, _ = linear_backward(dU, X, Wu, Au, Bu, gamma)
+    return dXg + dXu, {"gate": (dAg, dBg), "up": (dAu, dBu), "down": (dAd, dBd)}

@@ -591,3 +591,79 @@ def test_format_nbytes():
     assert o.format_nbytes(4096 * 4096, 64, o.SCALES_E4M3) == o.quantized_nbytes(4096 * 4096)
     assert o.format_nbytes(100, 16, o.SCALES_FP32) == (56, 28, 0)
     assert o.format_nbytes(2 ** 20, 4096, o.SCALES_E4M3) == (2 ** 19, 256, 4)
+
+
+# --------------------------------------------------------------------------
+# Layer chaining with checkpoint recompute (SwiGLU MLP of adapted layers)
+# --------------------------------------------------------------------------
+def test_silu_grad_against_central_differences():
+    z = np.linspace(-8, 8, 97)
+    h = 1e-6
+    num = (o.silu(z + h) - o.silu(z - h)) / (2 * h)
+    assert np.allclose(o.silu_grad(z), num, atol=1e-8)
+    assert o.silu(0.0) == 0.0 and o.silu_grad(0.0) == 0.5
+
+
+def _tiny_mlp(seed=51, M=3, K=6, F=5, r=2):
+    rng = np.random.default_rng(seed)
+    mk = lambda n, k: (rng.normal(size=(n, k)), rng.normal(size=(r, k)), rng.normal(size=(n, r)))
+    layers = {"gate": mk(F, K), "up": mk(F, K), "down": mk(K, F)}
+    return rng.normal(size=(M, K)), layers, rng.normal(size=(M, K)), 0.75
+
+
+def test_mlp_forward_elementwise():
+    X, L, _, g = _tiny_mlp()
+    Y, (G, U, H) = o.mlp_forward(X, L, g)
+    m, f = 1, 3
+    lin = lambda x, name, j: (sum(x[k] * L[name][0][j, k] for k in range(x.size))
+                              + g * sum(sum(x[k] * L[name][1][i, k] for k in range(x.size))
+                                        * L[name][2][j, i] for i in range(L[name][1].shape[0])))
+    gv, uv = lin(X[m], "gate", f), lin(X[m], "up", f)
+    assert G[m, f] == pytest.approx(gv, abs=1e-12) and U[m, f] == pytest.approx(uv, abs=1e-12)
+    assert H[m, f] == pytest.approx(gv / (1 + math.exp(-gv)) * uv, abs=1e-12)
+    assert Y[m, 2] == pytest.approx(lin(H[m], "down", 2), abs=1e-12)
+
+
+def test_mlp_backward_finite_differences():
+    """Gradients of L = <dY, Y> by central differences, for X and every
+    adapter matrix of the three chained layers."""
+    X, L, dY, g = _tiny_mlp()
+    dX, dAB = o.mlp_backward(dY, X, L, g)
+
+    def loss(X_, L_):
+        return float(np.sum(dY * o.mlp_forward(X_, L_, g)[0]))
+
+    h = 1e-6
+    num = np.zeros_like(X)
+    for i in np.ndindex(X.shape):
+        p, m = X.copy(), X.copy()
+        p[i] += h
+        m[i] -= h
+        num[i] = (loss(p, L) - loss(m, L)) / (2 * h)
+    assert np.allclose(num, dX, atol=1e-5)
+    for name in ("gate", "up", "down"):
+        for which in (1, 2):                     # A, B
+            arr = L[name][which]
+            grad = dAB[name][which - 1]
+            num = np.zeros_like(arr)
+            for i in np.ndindex(arr.shape):
+                for sgn, store in ((1, "p"), (-1, "m")):
+                    a2 = arr.copy()
+                    a2[i] += sgn * h
+                    L2 = dict(L)
+                    t = list(L[name])
+                    t[which] = a2
+                    L2[name] = tuple(t)
+                    v = loss(X, L2)
+                    num[i] += sgn * v / (2 * h)
+            assert np.allclose(num, grad, atol=1e-5), (name, which)
+
+
+def test_checkpointed_backward_equals_stored_activations():
+    X, L, dY, g = _tiny_mlp(seed=52, M=4)
+    _, saved = o.mlp_forward(X, L, g)
+    dX1, d1 = o.mlp_backward(dY, X, L, g, saved=saved)
+    dX2, d2 = o.mlp_backward(dY, X, L, g, saved=None)
+    assert np.array_equal(dX1, dX2)
+    for k in d1:
+        assert all(np.array_equal(a, b) for a, b in zip(d1[k], d2[k]))
