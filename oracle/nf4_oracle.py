@@ -16,8 +16,7 @@ constants.  Every function names the passage of the pages it follows:
   * same page, section "Minimal implementation" (two indices per byte).
 
 Readings taken where the pages are silent or garbled (the displayed formulas
-and the codebook table did not survive extraction) are listed in the design doc and
-stated again at each function.
+and the codebook table did not survive extraction) are stated at each function.
 
 Pins (tests/test_oracle.py) tie every function here to something other than
 itself: printed codebook digits and the worked example, closed forms, two
