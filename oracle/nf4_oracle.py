@@ -544,3 +544,67 @@ def mlp_backward(dY, X, layers, gamma, saved=None):
     dXg, dAg, dBg, _ = linear_backward(dG, X, Wg, Ag, Bg, gamma)
     dXu, dAu, dBu, _ = linear_backward(dU, X, Wu, Au, Bu, gamma)
     return dXg + dXu, {"gate": (dAg, dBg), "up": (dAu, dBu), "down": (dAd, dBd)}
+
+
+# ---------------------------------------------------------------------------
+# Optimiser state for the adapter.  "QLoRA, explained", "The algorithm, step
+# by step" (AdamW over A and B only, 32-bit or 8-bit state) and "Hyperparameters
+# that matter" (the 8-bit variant quantises Adam's moments blockwise).  The
+# pages give no 8-bit format; the reading reuses the blockwise absmax scheme:
+# blocks of `block` consecutive state entries, an fp32 absmax c per block, the
+# first moment as a symmetric linear 8-bit code q = rint(127 m / c) in
+# [-127, 127], the second through its square root, q = rint(255 sqrt(v) / c)
+# in [0, 255] (ties to even); decoding is fp32(q * fp32(c / 127)) (or / 255,
+# then squared).  A linear code of v itself flushes every v below 1/510 of its
+# block's largest to zero while m is still non-zero, and the step m / (0 + eps)
+# then diverges; the square root keeps v's resolution on the scale of m's.
+# The update itself is AdamW in fp32 on the decoded state, after which the
+# state is re-encoded.
+# ---------------------------------------------------------------------------
+def adamw_step(p, g, m, v, t: int, lr: float, beta1: float, beta2: float, eps: float,
+               weight_decay: float):
+    """One AdamW step in fp32 (decoupled weight decay, bias-corrected moments).
+    Returns new (p, m, v); t counts from 1."""
+    f = np.float32
+    p, g, m, v = (np.asarray(a, np.float32) for a in (p, g, m, v))
+    p = (p * f(1.0 - lr * weight_decay)).astype(np.float32)
+    m = (f(beta1) * m + f(1.0 - beta1) * g).astype(np.float32)
+    v = (f(beta2) * v + f(1.0 - beta2) * g * g).astype(np.float32)
+    mhat = m / f(1.0 - beta1 ** t)
+    vhat = v / f(1.0 - beta2 ** t)
+    p = (p - f(lr) * mhat / (np.sqrt(vhat) + f(eps))).astype(np.float32)
+    return p, m, v
+
+
+def encode_state8(x: np.ndarray, signed: bool, block: int):
+    """(codes, absmax): codes int8 (signed) or uint8, absmax fp32 per block."""
+    x = np.asarray(x, np.float32).reshape(-1)
+    c = block_absmax(x, block)
+    levels = np.float32(127.0 if signed else 255.0)
+    nb = c.size
+    pad = np.zeros(nb * block, np.float32)
+    pad[: x.size] = x
+    safe = np.where(c == 0, np.float32(1.0), c).astype(np.float32).reshape(nb, 1)
+    q = np.rint((pad.reshape(nb, block) / safe).astype(np.float32) * levels)
+    q[(c == 0)] = 0
+    q = q.reshape(-1)[: x.size]
+    return (q.astype(np.int8) if signed else q.astype(np.uint8)), c
+
+
+def decode_state8(codes: np.ndarray, absmax: np.ndarray, signed: bool, block: int):
+    levels = np.float32(127.0 if signed else 255.0)
+    q = np.asarray(codes).astype(np.float32).reshape(-1)
+    step = (np.asarray(absmax, np.float32) / levels).astype(np.float32)
+    return (q * step[np.arange(q.size) // block]).astype(np.float32)
+
+
+def adamw8_step(p, g, m_state, v_state, t: int, lr: float, beta1: float, beta2: float,
+                eps: float, weight_decay: float, block: int = BLOCK):
+    """AdamW with 8-bit blockwise state: m_state = (int8 codes, absmax) of m,
+    v_state = (uint8 codes, absmax) of sqrt(v).  Returns (p, m_state, v_state)."""
+    m = decode_state8(*m_state, True, block).reshape(np.shape(p))
+    u = decode_state8(*v_state, False, block).reshape(np.shape(p))
+    v = (u * u).astype(np.float32)
+    p, m, v = adamw_step(p, g, m, v, t, lr, beta1, beta2, eps, weight_decay)
+    return (p, encode_state8(m, True, block),
+            encode_state8(np.sqrt(v).astype(np.float32), False, block))
