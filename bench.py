@@ -238,6 +238,44 @@ def _quantize_measure(q, syn, device, reps=5):
             "bytes_per_call": nbytes}
 
 
+def _merge_measure(q, syn, device, reps=10):
+    """Merge for export on the 28672 x 8192 decode weight (r = 16): the merge
+    kernel's CUDA-event time per launch, stored weights and bf16 outputs
+    rotated over two copies (2 x 590 MB > 2x L2), and GB/s of algorithmic
+    bytes (stored weight + adapter read, bf16 weight written); the plain
+    dequantisation of the same weight beside it."""
+    lin = syn.WORKLOADS[GEMV_WORKLOAD].layers[0]
+    W = torch.randn(lin.N, lin.K, device=device) * lin.sigma
+    ws = [q.qlora_quantize(W, check_finite=False) for _ in range(2)]
+    del W
+    A = (torch.randn(lin.r, lin.K, device=device) / lin.K ** 0.5).bfloat16()
+    B = (torch.randn(lin.N, lin.r, device=device) * 0.01).bfloat16()
+    outs = [torch.empty(lin.N, lin.K, dtype=torch.bfloat16, device=device) for _ in range(2)]
+
+    def timed(fn):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        for i in range(reps):
+            evs[i][0].record()
+            fn(i)
+            evs[i][1].record()
+        torch.cuda.synchronize()
+        return sum(b.elapsed_time(e) for b, e in evs) / reps * 1e3
+
+    mu = timed(lambda i: q.qlora_merge(ws[i % 2], A, B, lin.gamma, out=outs[i % 2]))
+    du = timed(lambda i: q.qlora_dequantize(ws[i % 2], out=outs[i % 2]))
+    stored = ws[0].nbytes
+    mb = stored + (lin.r * lin.K + lin.N * lin.r) * 2 + lin.N * lin.K * 2
+    db = stored + lin.N * lin.K * 2
+    del ws, outs
+    return {"workload": f"merge_{lin.N}x{lin.K}_r{lin.r}", "kernel_us": round(mu, 2),
+            "GBps": round(mb / mu / 1e3, 1), "algorithmic_bytes": mb,
+            "dequantize_us": round(du, 2), "dequantize_GBps": round(db / du / 1e3, 1)}
+
+
 def _format_measure(q, device, reps=10):
     """Format variants on a 28672 x 8192 weight (235 M weights, 940 MB fp32):
     quantise and bf16 dequantise throughput for NF4 / FP4 at blocksize 64 with
@@ -554,6 +592,11 @@ def run_gpu(args):
         ex = out["decoder"]["export"]
         for k in ("merge", "requantize", "dequantize"):
             ex[f"{k}_frac_hbm"] = round(ex[f"{k}_GBps"] / peaks["hbm_gbs"], 4)
+        try:
+            out["merge"] = _merge_measure(q, syn, device)
+            out["merge"]["frac_hbm"] = round(out["merge"]["GBps"] / peaks["hbm_gbs"], 4)
+        except Exception as exc:           # an extra measurement never sinks the bench line
+            out["merge"] = {"error": f"{type(exc).__name__}: {exc}"}
         try:
             out["formats"] = _format_measure(q, device)
             for row in out["formats"]:
