@@ -13,7 +13,8 @@
 // stay in L2.  The rank-r product B A is a contraction of depth r <= 128, done
 // on the warp-level tensor cores (mma.sync m16n8k16, bf16 in, fp32
 // accumulate): at r = 16 that is 16 MMAs per 1024 weights, a few per cent of
-// the issue slots, so the kernel's time is set by its stores.
+// the issue slots; the per-weight decode, the fused multiply-add and the two
+// roundings make up most of the instruction stream.
 //
 // Work unit: one CTA tile of 16 rows x 512 columns, each of the 8 warps
 // owning one 64-column strip (one NF4 block per row).  Units are ordered by
@@ -31,7 +32,8 @@
 // columns of each 8-wide n-tile.  The 8 n-tiles are mapped to the strip's
 // columns so that lane t of a quad owns columns 32i + 8t + (0..7) for i = 0, 1:
 // each quad then writes 64 contiguous bytes per store (full 32-byte sectors)
-// and reads its packed indices as one 32-bit word per row and i.  Logical
+// and needs one 32-bit word of packed indices per row and i (loaded by the
+// quad as one 32-byte sector and exchanged by shuffles).  Logical
 // column n (0..7) of n-tile nt is physical column
 //     32 (nt / 4) + 8 (n / 2) + 2 (nt % 4) + (n % 2),
 // and the slab stores A's columns in that logical order so that ldmatrix.trans
