@@ -184,3 +184,50 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(L, "LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(ImportError):
         L.lib()
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include "qlora_nf4.h"
+int main(void) {
+    float codes[16], mids[15];
+    if (nf4_build_codebook(codes, mids) != QLORA_OK) return 2;
+    size_t p = 0, c = 0, m = 0;
+    if (qlora_quantized_sizes(4096, 4096, &p, &c, &m) != QLORA_OK) return 3;
+    qlora_format f = {16, 16, {0}, QLORA_SCALES_FP32};
+    for (int i = 0; i < 16; ++i) f.codes[i] = codes[i];
+    size_t fp = 0, fs = 0, fm = 0;
+    if (qlora_format_sizes(100, &f, &fp, &fs, &fm) != QLORA_OK) return 4;
+    for (int i = 0; i < 16; ++i) printf("%a ", codes[i]);
+    printf("\n%zu %zu %zu %zu %zu %zu\n%s\n", p, c, m, fp, fs, fm, qlora_status_string(QLORA_ERR_ALIGN));
+    return 0;
+}
+"""
+
+
+def test_plain_c_client_links_and_runs(q, tmp_path):
+    """The boundary is a C ABI: a plain C99 program includes the header, links
+    the library and calls its host-only entry points."""
+    import shutil
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(q._lib.LIB_PATH)
+    import subprocess
+    cc = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                         "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                         "-L", libdir, "-lqlora_nf4", f"-Wl,-rpath,{libdir}"],
+                        capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, run.stderr
+    lines = run.stdout.strip().splitlines()
+    got = np.array([float.fromhex(t) for t in lines[0].split()], np.float32)
+    assert np.array_equal(got.view(np.uint32), o.nf4_codebook()[0].view(np.uint32))
+    sizes = tuple(int(t) for t in lines[1].split())
+    assert sizes[:3] == o.quantized_nbytes(4096 * 4096)
+    assert sizes[3:] == o.format_nbytes(100, 16, o.SCALES_FP32)
+    assert lines[2] == "misaligned pointer"
