@@ -8,13 +8,16 @@ from ._lib import (  # noqa: F401
     EXPORTED,
     QLORA_SCALES_E4M3,
     QLORA_SCALES_FP32,
+    Adam8State,
     Format,
+    adamw8_state,
     NF4Tensor,
     QloraError,
     device_error_word,
     empty_nf4,
     lib,
     nf4_build_codebook,
+    qlora_adamw8_step,
     qlora_dequantize,
     qlora_dequantize_fmt,
     qlora_format_sizes,

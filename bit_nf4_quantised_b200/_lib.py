@@ -46,6 +46,8 @@ EXPORTED = (
     "qlora_format_sizes",
     "qlora_quantize_fmt",
     "qlora_dequantize_fmt",
+    "qlora_adamw8_state_sizes",
+    "qlora_adamw8_step",
 )
 
 QLORA_SCALES_FP32 = 0
@@ -96,6 +98,12 @@ class _Format(ctypes.Structure):
     ]
 
 
+class _AdamConfig(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
+                ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float),
+                ("step", ctypes.c_int64)]
+
+
 _LIB = None
 
 
@@ -122,6 +130,9 @@ def lib() -> ctypes.CDLL:
         L.qlora_format_sizes.argtypes = [i64, fp, sz, sz, sz]
         L.qlora_quantize_fmt.argtypes = [vp, i64, fp, vp, vp, vp, vp, vp]
         L.qlora_dequantize_fmt.argtypes = [vp, vp, vp, i64, fp, vp, vp]
+        L.qlora_adamw8_state_sizes.argtypes = [i64, sz, sz]
+        L.qlora_adamw8_step.argtypes = [vp, vp, i64, vp, vp, vp, vp,
+                                        ctypes.POINTER(_AdamConfig), vp, vp]
         L.qlora_linear_workspace_size.argtypes = [i64, i64, i64, i32, sz]
         fwd = [vp, i64, tp, vp, vp, i32, f32, vp, vp, vp, ctypes.c_size_t, vp]
         bwd = [vp, vp, i64, tp, vp, vp, i32, f32, vp, vp, vp, vp, i32, vp, ctypes.c_size_t, vp]
@@ -317,6 +328,43 @@ def qlora_dequantize_fmt(packed: torch.Tensor, scales: torch.Tensor, meta, numel
                                       ctypes.byref(f), out.data_ptr(), _stream(stream)),
            "qlora_dequantize_fmt")
     return out
+
+
+@dataclass
+class Adam8State:
+    """8-bit blockwise AdamW state of n parameters (zeros = the initial state)."""
+    m_codes: torch.Tensor     # int8 [n]
+    m_absmax: torch.Tensor    # float32 [ceil(n/64)]
+    v_codes: torch.Tensor     # uint8 [n]
+    v_absmax: torch.Tensor    # float32 [ceil(n/64)]
+    step: int = 0
+
+
+def adamw8_state(n: int, device="cuda") -> Adam8State:
+    c, a = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().qlora_adamw8_state_sizes(n, ctypes.byref(c), ctypes.byref(a)),
+           "qlora_adamw8_state_sizes")
+    nb = a.value // 4
+    z = lambda k, dt: torch.zeros(max(k, 4), dtype=dt, device=device)[:k]
+    return Adam8State(z(n, torch.int8), z(nb, torch.float32), z(n, torch.uint8),
+                      z(nb, torch.float32))
+
+
+def qlora_adamw8_step(p: torch.Tensor, g: torch.Tensor, state: Adam8State, lr: float,
+                      beta1: float = 0.9, beta2: float = 0.999, eps: float = 1e-8,
+                      weight_decay: float = 0.0, p_bf16: torch.Tensor | None = None,
+                      stream=None) -> None:
+    """One AdamW step of the fp32 parameters p in place (state.step advances)."""
+    _need(p, torch.float32, "p")
+    _need(g, torch.float32, "g")
+    if p_bf16 is not None:
+        _need(p_bf16, torch.bfloat16, "p_bf16")
+    state.step += 1
+    cfg = _AdamConfig(lr, beta1, beta2, eps, weight_decay, state.step)
+    _check(lib().qlora_adamw8_step(p.data_ptr(), g.data_ptr(), p.numel(),
+                                   _ptr(state.m_codes), _ptr(state.m_absmax),
+                                   _ptr(state.v_codes), _ptr(state.v_absmax), ctypes.byref(cfg),
+                                   _ptr(p_bf16), _stream(stream)), "qlora_adamw8_step")
 
 
 def qlora_linear_workspace_size(M: int, N: int, K: int, r: int) -> int:

@@ -38,6 +38,23 @@ cudaError_t launch_dequantize_fmt(const uint8_t* packed, const void* scales, con
                                   int64_t numel, const FmtArgs& f, uint16_t* out,
                                   const FmtTable& tab, int num_sms, cudaStream_t stream);
 
+// -------------------------------------------- 8-bit optimiser state (AdamW)
+struct Adam8Args {
+    float* p;                  // fp32 parameters, updated in place
+    const float* g;            // fp32 gradients
+    int8_t* m_codes;           // first moment, linear code of m
+    float* m_absmax;
+    uint8_t* v_codes;          // second moment, linear code of sqrt(v)
+    float* v_absmax;
+    uint16_t* p_bf16;          // optional bf16 copy of the updated p
+    int64_t n;
+    float lr, beta1, beta2, eps;
+    float decay;               // fp32(1 - lr wd)
+    float one_m_beta1, one_m_beta2;
+    float bc1, bc2;            // fp32(1 - beta^t)
+};
+cudaError_t launch_adamw8(const Adam8Args& a, int num_sms, cudaStream_t stream);
+
 // ---------------------------------------------------------------- K7 merge
 struct MergeArgs {
     const uint32_t* packed;      // N*K/8 words of packed indices

@@ -480,6 +480,52 @@ int qlora_dequantize_fmt(const uint8_t* packed, const void* scales, const float*
                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int qlora_adamw8_state_sizes(int64_t n, size_t* code_bytes, size_t* absmax_bytes) {
+    if (!code_bytes || !absmax_bytes) return QLORA_ERR_NULL;
+    if (n < 0) return QLORA_ERR_SHAPE;
+    *code_bytes = static_cast<size_t>(n);
+    *absmax_bytes = static_cast<size_t>(cdiv(n, QLORA_BLOCK)) * 4;
+    return QLORA_OK;
+}
+
+int qlora_adamw8_step(float* p, const float* g, int64_t n, int8_t* m_codes, float* m_absmax,
+                      uint8_t* v_codes, float* v_absmax, const qlora_adamw_config* cfg,
+                      uint16_t* p_bf16, qlora_stream_t stream) {
+    if (!cfg) return QLORA_ERR_NULL;
+    if (n < 0) return QLORA_ERR_SHAPE;
+    if (cfg->step < 1 || !(cfg->beta1 >= 0.f && cfg->beta1 < 1.f) ||
+        !(cfg->beta2 >= 0.f && cfg->beta2 < 1.f) || !std::isfinite(cfg->lr) ||
+        !std::isfinite(cfg->eps) || !std::isfinite(cfg->weight_decay))
+        return QLORA_ERR_UNSUPPORTED;
+    if (n == 0) return QLORA_OK;
+    if (!p || !g || !m_codes || !m_absmax || !v_codes || !v_absmax) return QLORA_ERR_NULL;
+    if (!aligned(p, 16) || !aligned(g, 16) || !aligned(m_codes, 4) || !aligned(v_codes, 4) ||
+        !aligned(m_absmax, 4) || !aligned(v_absmax, 4) || (p_bf16 && !aligned(p_bf16, 8)))
+        return QLORA_ERR_ALIGN;
+    Adam8Args a{};
+    a.p = p;
+    a.g = g;
+    a.m_codes = m_codes;
+    a.m_absmax = m_absmax;
+    a.v_codes = v_codes;
+    a.v_absmax = v_absmax;
+    a.p_bf16 = p_bf16;
+    a.n = n;
+    // constants formed in double from the fp32 arguments, rounded once
+    const double lr = cfg->lr, b1 = cfg->beta1, b2 = cfg->beta2, wd = cfg->weight_decay;
+    const double t = static_cast<double>(cfg->step);
+    a.lr = cfg->lr;
+    a.beta1 = cfg->beta1;
+    a.beta2 = cfg->beta2;
+    a.eps = cfg->eps;
+    a.decay = static_cast<float>(1.0 - lr * wd);
+    a.one_m_beta1 = static_cast<float>(1.0 - b1);
+    a.one_m_beta2 = static_cast<float>(1.0 - b2);
+    a.bc1 = static_cast<float>(1.0 - std::pow(b1, t));
+    a.bc2 = static_cast<float>(1.0 - std::pow(b2, t));
+    return cuda_status(launch_adamw8(a, num_sms(), reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int qlora_merge(const qlora_nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r,
                 float scale, uint16_t* W_out, qlora_stream_t stream) {
     if (!w) return QLORA_ERR_NULL;

@@ -217,6 +217,46 @@ QLORA_API int qlora_dequantize_fmt(const uint8_t* packed, const void* scales, co
                                    qlora_stream_t stream);
 
 /*
+ * AdamW over an adapter matrix with 8-bit blockwise state ("QLoRA,
+ * explained", "The algorithm, step by step": AdamW over A and B only, 32- or
+ * 8-bit state; "Hyperparameters that matter": the 8-bit variant quantises
+ * Adam's moments blockwise).  The state of n parameters: blocks of 64, an
+ * fp32 absmax per block for each moment; m as int8 codes rint(127 m / c), v
+ * through its square root as uint8 codes rint(255 sqrt(v) / c).  Zero codes
+ * and absmax are the initial (zero) state.
+ */
+typedef struct {
+    float lr;
+    float beta1;          /* 0 <= beta1 < 1 */
+    float beta2;          /* 0 <= beta2 < 1 */
+    float eps;
+    float weight_decay;   /* decoupled: p *= 1 - lr weight_decay */
+    int64_t step;         /* t >= 1, for the bias corrections 1 - beta^t */
+} qlora_adamw_config;
+
+/* Byte sizes of one moment's codes (n) and absmax array (4 ceil(n/64)). */
+QLORA_API int qlora_adamw8_state_sizes(int64_t n, size_t* code_bytes, size_t* absmax_bytes);
+
+/*
+ * qlora_adamw8_step -- one AdamW step: decode the state, update in fp32
+ * (p *= fp32(1 - lr wd); m = b1 m + fp32(1 - b1) g; v = b2 v + (fp32(1 - b2) g) g;
+ * p -= (lr (m / fp32(1 - b1^t))) / (sqrt(v / fp32(1 - b2^t)) + eps), each
+ * operation rounded on its own), re-encode the state.
+ *   p (device, fp32, n, read and written); g (device, fp32, n, read);
+ *   m_codes, m_absmax, v_codes, v_absmax (device, read and written);
+ *   cfg (host, read); p_bf16 (device, bf16 bits, n, nullable, written): the
+ *   updated p rounded to bf16, for the layer's A or B.
+ * n = 0 launches nothing.
+ * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE, QLORA_ERR_UNSUPPORTED (a
+ * hyperparameter out of range), QLORA_ERR_ALIGN (p, g 16-byte aligned; codes
+ * and absmax 4-byte; p_bf16 8-byte), QLORA_ERR_CUDA.
+ */
+QLORA_API int qlora_adamw8_step(float* p, const float* g, int64_t n, int8_t* m_codes,
+                                float* m_absmax, uint8_t* v_codes, float* v_absmax,
+                                const qlora_adamw_config* cfg, uint16_t* p_bf16,
+                                qlora_stream_t stream);
+
+/*
  * qlora_merge -- the fine-tuned weight for bf16 export,
  *     W_out = bf16_rne( W~ + scale * B A ).
  * "QLoRA, explained", "The forward pass and gradients": the model that was

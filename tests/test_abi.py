@@ -178,6 +178,27 @@ def test_format_validation_before_any_launch(q):
     assert L.qlora_dequantize_fmt(fake, None, None, 1000, ctypes.byref(f32), fake, None) == E.QLORA_ERR_NULL
 
 
+def test_adamw8_argument_errors(q):
+    L = q.lib()
+    E = q._lib
+    fake = 0x40000
+    cfg = q._lib._AdamConfig(2e-4, 0.9, 0.999, 1e-8, 0.0, 1)
+    c, a = ctypes.c_size_t(), ctypes.c_size_t()
+    assert L.qlora_adamw8_state_sizes(130, ctypes.byref(c), ctypes.byref(a)) == E.QLORA_OK
+    assert (c.value, a.value) == (130, 12)
+    assert L.qlora_adamw8_state_sizes(-1, ctypes.byref(c), ctypes.byref(a)) == E.QLORA_ERR_SHAPE
+    step = lambda *args: L.qlora_adamw8_step(*args)
+    assert step(fake, fake, 100, fake, fake, fake, fake, None, None, None) == E.QLORA_ERR_NULL
+    assert step(None, fake, 100, fake, fake, fake, fake, ctypes.byref(cfg), None, None) == E.QLORA_ERR_NULL
+    assert step(fake + 4, fake, 100, fake, fake, fake, fake, ctypes.byref(cfg), None, None) == E.QLORA_ERR_ALIGN
+    assert step(fake, fake, -1, fake, fake, fake, fake, ctypes.byref(cfg), None, None) == E.QLORA_ERR_SHAPE
+    assert step(None, None, 0, None, None, None, None, ctypes.byref(cfg), None, None) == E.QLORA_OK
+    for bad in (q._lib._AdamConfig(2e-4, 1.0, 0.999, 1e-8, 0.0, 1),
+                q._lib._AdamConfig(2e-4, 0.9, 0.999, 1e-8, 0.0, 0),
+                q._lib._AdamConfig(float("nan"), 0.9, 0.999, 1e-8, 0.0, 1)):
+        assert step(fake, fake, 100, fake, fake, fake, fake, ctypes.byref(bad), None, None) == E.QLORA_ERR_UNSUPPORTED
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     import bit_nf4_quantised_b200._lib as L
     monkeypatch.setattr(L, "_LIB", None)
