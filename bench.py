@@ -276,6 +276,32 @@ def _merge_measure(q, syn, device, reps=10):
             "dequantize_us": round(du, 2), "dequantize_GBps": round(db / du / 1e3, 1)}
 
 
+def _adam8_measure(q, syn, device, reps=10):
+    """AdamW with 8-bit state over every adapter of the 32-layer decoder
+    (r = 16: 40 M parameters as one flat fp32 tensor), one launch per step
+    with the bf16 copy written; GB/s of algorithmic bytes per parameter:
+    p 4 + 4, g 4, two 1-byte codes read and written, bf16 copy 2 (18 B)."""
+    lins = syn.WORKLOADS["llama7b_decoder_32layers_m4096_r16"].layers
+    n = sum(l.r * (l.K + l.N) for l in lins)
+    p = torch.randn(n, device=device) * 0.02
+    g = torch.randn(n, device=device)
+    pb = torch.empty(n, dtype=torch.bfloat16, device=device)
+    st = q.adamw8_state(n, device)
+    for _ in range(3):
+        q.qlora_adamw8_step(p, g, st, 2e-4, weight_decay=0.01, p_bf16=pb)
+    torch.cuda.synchronize()
+    b, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b.record()
+    for _ in range(reps):
+        q.qlora_adamw8_step(p, g, st, 2e-4, weight_decay=0.01, p_bf16=pb)
+    e.record()
+    torch.cuda.synchronize()
+    us = b.elapsed_time(e) / reps * 1e3
+    nbytes = n * 18 + 2 * 2 * 4 * ((n + 63) // 64)
+    return {"params": n, "kernel_us": round(us, 2), "GBps": round(nbytes / us / 1e3, 1),
+            "bytes_per_step": nbytes}
+
+
 def _format_measure(q, device, reps=10):
     """Format variants on a 28672 x 8192 weight (235 M weights, 940 MB fp32):
     quantise and bf16 dequantise throughput for NF4 / FP4 at blocksize 64 with
@@ -597,6 +623,11 @@ def run_gpu(args):
             out["merge"]["frac_hbm"] = round(out["merge"]["GBps"] / peaks["hbm_gbs"], 4)
         except Exception as exc:           # an extra measurement never sinks the bench line
             out["merge"] = {"error": f"{type(exc).__name__}: {exc}"}
+        try:
+            out["adamw8"] = _adam8_measure(q, syn, device)
+            out["adamw8"]["frac_hbm"] = round(out["adamw8"]["GBps"] / peaks["hbm_gbs"], 4)
+        except Exception as exc:           # an extra measurement never sinks the bench line
+            out["adamw8"] = {"error": f"{type(exc).__name__}: {exc}"}
         try:
             out["formats"] = _format_measure(q, device)
             for row in out["formats"]:
