@@ -12,12 +12,14 @@
 // The update is AdamW in fp32 in a fixed operation order, every product,
 // quotient and sum rounded on its own (no contraction into fused
 // multiply-adds): p *= 1 - lr wd; m = b1 m + (1 - b1) g; v = b2 v + ((1 - b2)
-// g) g; p -= (lr m / (1 - b1^t)) ... see the kernel for the exact order.
+// g) g; p -= (lr (m / (1 - b1^t))) / (sqrt(v / (1 - b2^t)) + eps).
 //
-// HBM-bound elementwise work: per entry 4 B of p and 4 B of g read, 4 B of p
-// written, 1 + 1 B of codes read and written (+ the bf16 copy of p if asked).
-// A half-warp covers one block of 64 (four entries per lane, 16-byte loads),
-// reducing each block's new absmax values with four shuffles.
+// Elementwise work: per entry 4 B of p and 4 B of g read, 4 B of p written,
+// 1 + 1 B of codes read and written (+ the bf16 copy of p if asked).  The
+// five correctly rounded divisions and two square roots per entry cost more
+// issue slots than the memory traffic needs time.  A half-warp covers one
+// block of 64 (four entries per lane, 16-byte loads), reducing each block's
+// new absmax values with four shuffles.
 #include "kernels.cuh"
 
 namespace qnf4 {
