@@ -216,6 +216,24 @@ def e4m3_encode(x: np.ndarray) -> np.ndarray:
     return out
 
 
+def e4m3_encode_sorted(x: np.ndarray) -> np.ndarray:
+    """The same encoding as e4m3_encode, written for whole arrays: the 127
+    values are ascending in code order, so a binary search (np.searchsorted)
+    finds each element's two neighbours lo <= x <= hi; the nearer one wins,
+    an exact tie takes the even code, and anything at or above 448 takes
+    0x7E."""
+    x = np.asarray(x, dtype=np.float32).astype(np.float64).reshape(-1)
+    if np.any(x < 0) or not np.all(np.isfinite(x)):
+        raise ValueError("e4m3_encode_sorted takes finite non-negative values")
+    hi = np.clip(np.searchsorted(_E4M3, x, side="left"), 1, 126)
+    lo = hi - 1
+    d_lo = x - _E4M3[lo]
+    d_hi = _E4M3[hi] - x
+    even = np.where(lo % 2 == 0, lo, hi)
+    code = np.where(d_lo < d_hi, lo, np.where(d_hi < d_lo, hi, even))
+    return np.where(x >= E4M3_MAX, 0x7E, code).astype(np.uint8)
+
+
 def e4m3_decode(code: np.ndarray) -> np.ndarray:
     c = np.asarray(code, dtype=np.uint8).reshape(-1)
     if np.any(c == 0x7F) or np.any(c >= 0x80):
@@ -238,11 +256,11 @@ def double_quantize(absmax: np.ndarray, group: int = GROUP
     padded[:nblocks] = c
     padded = padded.reshape(ngroups, group)
     meta = (padded.max(axis=1) / np.float32(E4M3_MAX)).astype(np.float32)
-    codes = np.zeros((ngroups, group), dtype=np.uint8)
-    for g in range(ngroups):
-        if meta[g] > 0:
-            ratio = (padded[g] / meta[g]).astype(np.float32)
-            codes[g] = e4m3_encode(ratio)
+    live = meta > 0
+    safe = np.where(live, meta, np.float32(1.0)).astype(np.float32)
+    ratio = (padded / safe.reshape(ngroups, 1)).astype(np.float32)
+    codes = e4m3_encode_sorted(ratio).reshape(ngroups, group)
+    codes[~live] = 0
     return codes.reshape(-1)[:nblocks], meta
 
 
@@ -552,9 +570,10 @@ def mlp_backward(dY, X, layers, gamma, saved=None):
 # that matter" (the 8-bit variant quantises Adam's moments blockwise).  The
 # pages give no 8-bit format; the reading reuses the blockwise absmax scheme:
 # blocks of `block` consecutive state entries, an fp32 absmax c per block, the
-# first moment as a symmetric linear 8-bit code q = rint(127 m / c) in
-# [-127, 127], the second through its square root, q = rint(255 sqrt(v) / c)
-# in [0, 255] (ties to even); decoding is fp32(q * fp32(c / 127)) (or / 255,
+# first moment as a symmetric linear 8-bit code q = rint(fp32(m / c) * 127) in
+# [-127, 127], the second through its square root, q = rint(fp32(sqrt(v) / c)
+# * 255) in [0, 255] (the quotient rounded to fp32, then the product, ties to
+# even); decoding is fp32(q * fp32(c / 127)) (or / 255,
 # then squared).  A linear code of v itself flushes every v below 1/510 of its
 # block's largest to zero while m is still non-zero, and the step m / (0 + eps)
 # then diverges; the square root keeps v's resolution on the scale of m's.

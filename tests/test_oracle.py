@@ -241,6 +241,56 @@ def test_e4m3_encode_matches_torch_cast():
     assert o.e4m3_encode(np.array([465.0, 1e30], np.float32)).tolist() == [0x7E, 0x7E]
 
 
+def _e4m3_probe_values(n_random):
+    """Every E4M3 value, every midpoint between neighbours and its two fp32
+    neighbours, values above the top code, and random values over the whole
+    range (uniform and log-uniform)."""
+    rng = np.random.default_rng(11)
+    tab = o.e4m3_value_table()
+    mids = ((tab[:-1] + tab[1:]) / 2).astype(np.float32)
+    return np.concatenate([
+        tab.astype(np.float32), mids,
+        np.nextafter(mids, np.float32(np.inf)), np.nextafter(mids, np.float32(0)),
+        np.array([448.0, 455.9, 460.0, 464.0, 1e3, 1e30], np.float32),
+        rng.uniform(0, 464, n_random // 2).astype(np.float32),
+        (2.0 ** rng.uniform(-16, 8.8, n_random // 2)).astype(np.float32),
+    ])
+
+
+def test_e4m3_encode_sorted_equals_enumeration():
+    vals = _e4m3_probe_values(200_000)
+    assert np.array_equal(o.e4m3_encode_sorted(vals), o.e4m3_encode(vals))
+
+
+def test_e4m3_encode_sorted_matches_torch_cast():
+    vals = _e4m3_probe_values(2_000_000)
+    vals = vals[vals <= 464.0]                      # torch's cast saturates only up to there
+    ours = o.e4m3_encode_sorted(vals)
+    theirs = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert vals.size > 1_000_000 and np.array_equal(ours, theirs)
+    assert o.e4m3_encode_sorted(np.array([465.0, 1e30], np.float32)).tolist() == [0x7E, 0x7E]
+    with pytest.raises(ValueError):
+        o.e4m3_encode_sorted(np.array([-1.0], np.float32))
+
+
+def test_double_quantize_matches_per_group_enumeration():
+    """The whole-array double quantisation equals the group-by-group one with
+    the enumerating encoder (all-zero groups, a partial last group)."""
+    rng = np.random.default_rng(12)
+    c = np.abs(rng.standard_normal(256 * 9 + 77)).astype(np.float32) * np.float32(0.05)
+    c[256:512] = 0.0
+    c[600] = 0.0
+    sc, meta = o.double_quantize(c)
+    ngroups = -(-c.size // 256)
+    for g in range(ngroups):
+        part = c[g * 256:(g + 1) * 256]
+        m = np.float32(part.max() / np.float32(448.0))
+        assert meta[g] == m
+        want = (o.e4m3_encode((part / m).astype(np.float32)) if m > 0
+                else np.zeros(part.size, np.uint8))
+        assert np.array_equal(sc[g * 256:g * 256 + part.size], want)
+
+
 def test_e4m3_decode_matches_torch():
     c = np.arange(127, dtype=np.uint8)
     theirs = torch.from_numpy(c).view(torch.float8_e4m3fn).to(torch.float32).numpy()
