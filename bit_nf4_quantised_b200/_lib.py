@@ -41,6 +41,7 @@ EXPORTED = (
     "qlora_linear_forward_ex",
     "qlora_linear_backward_ex",
     "qlora_linear_forward_noalloc",
+    "qlora_linear_forward_noalloc_error_word",
     "qlora_merge",
     "qlora_quantize_bf16",
     "qlora_format_sizes",
@@ -214,18 +215,16 @@ def empty_nf4(rows: int, cols: int, device="cuda") -> NF4Tensor:
 
 def qlora_quantize(W: torch.Tensor, out: NF4Tensor | None = None, check_finite: bool = True,
                    stream=None) -> NF4Tensor:
-    """Quantise a fp32 [rows, cols] CUDA tensor.  With check_finite the call
-    synchronises the stream and raises QloraError(QLORA_ERR_NONFINITE) if the
-    kernel saw a NaN or an infinity."""
+    """Quantise a fp32 [rows, cols] CUDA tensor.  With check_finite the
+    library synchronises the stream and the call raises
+    QloraError(QLORA_ERR_NONFINITE) if the kernel saw a NaN or an infinity."""
     _need(W, torch.float32, "W")
     rows, cols = (W.shape[0], W.shape[1]) if W.dim() == 2 else (1, W.numel())
     out = out if out is not None else empty_nf4(rows, cols, W.device)
-    flag = torch.zeros(1, dtype=torch.int32, device=W.device) if check_finite else None
+    flag = torch.empty(1, dtype=torch.int32, device=W.device) if check_finite else None
     st = out.c_struct()
     _check(lib().qlora_quantize(W.data_ptr(), ctypes.byref(st), _ptr(flag), _stream(stream)),
            "qlora_quantize")
-    if check_finite and int(flag.item()) != 0:
-        raise QloraError(QLORA_ERR_NONFINITE, "qlora_quantize")
     return out
 
 
@@ -246,12 +245,10 @@ def qlora_quantize_bf16(W: torch.Tensor, out: NF4Tensor | None = None, check_fin
     _need(W, torch.bfloat16, "W")
     rows, cols = (W.shape[0], W.shape[1]) if W.dim() == 2 else (1, W.numel())
     out = out if out is not None else empty_nf4(rows, cols, W.device)
-    flag = torch.zeros(1, dtype=torch.int32, device=W.device) if check_finite else None
+    flag = torch.empty(1, dtype=torch.int32, device=W.device) if check_finite else None
     st = out.c_struct()
     _check(lib().qlora_quantize_bf16(W.data_ptr(), ctypes.byref(st), _ptr(flag), _stream(stream)),
            "qlora_quantize_bf16")
-    if check_finite and int(flag.item()) != 0:
-        raise QloraError(QLORA_ERR_NONFINITE, "qlora_quantize_bf16")
     return out
 
 
@@ -310,12 +307,10 @@ def qlora_quantize_fmt(W: torch.Tensor, fmt: Format, check_finite: bool = True, 
     else:
         scales = torch.empty(max(sb, 4), dtype=torch.uint8, device=dev)[:sb]
         meta = torch.empty(max(mb // 4, 1), dtype=torch.float32, device=dev)[: mb // 4]
-    flag = torch.zeros(1, dtype=torch.int32, device=dev) if check_finite else None
+    flag = torch.empty(1, dtype=torch.int32, device=dev) if check_finite else None
     f = fmt.c_struct()
     _check(lib().qlora_quantize_fmt(W.data_ptr(), n, ctypes.byref(f), _ptr(packed), _ptr(scales),
                                     _ptr(meta), _ptr(flag), _stream(stream)), "qlora_quantize_fmt")
-    if check_finite and int(flag.item()) != 0:
-        raise QloraError(QLORA_ERR_NONFINITE, "qlora_quantize_fmt")
     return packed, scales, meta
 
 

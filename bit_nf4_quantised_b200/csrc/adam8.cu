@@ -5,8 +5,9 @@
 // variant quantises Adam's moments blockwise).  The pages give no 8-bit
 // format; the reading reuses the blockwise absmax scheme: blocks of 64 state
 // entries with an fp32 absmax each, the first moment as the symmetric linear
-// code rint(127 m / c), the second through its square root, rint(255 sqrt(v)
-// / c) (a linear code of v flushes small v to zero while m is not, and the
+// code rint(fp32(m / c) * 127), the second through its square root,
+// rint(fp32(sqrt(v) / c) * 255) (the quotient rounded to fp32 first, then the
+// product; a linear code of v flushes small v to zero while m is not, and the
 // step then diverges).  Decoding is q * fp32(c / 127) (or / 255, squared).
 //
 // The update is AdamW in fp32 in a fixed operation order, every product,

@@ -20,6 +20,12 @@
 // rest, so the contents left by the previous call do no harm.  All calls on
 // a device share the one array: calls that can overlap on the GPU (different
 // streams with no ordering between them) race on it and must not be issued.
+//
+// The ordinary forward reports kernel-side failures (a bounded wait that
+// expired, a shared-memory plan or tile schedule that did not fit) in the
+// first 4 bytes of the caller's workspace.  Here that word lives in the
+// library's array, which the caller cannot address, so
+// qlora_linear_forward_noalloc_error_word copies it out.
 #include <mutex>
 
 #include "kernels.cuh"
@@ -70,4 +76,16 @@ extern "C" QLORA_API int qlora_linear_forward_noalloc(const uint16_t* X, int64_t
     if (st != QLORA_OK) return st;
     return qlora_linear_forward(X, M, w, A, B, r, scale, Y, T_save, ws, kNoAllocScratchBytes,
                                 stream);
+}
+
+extern "C" QLORA_API int qlora_linear_forward_noalloc_error_word(int* h_word,
+                                                                qlora_stream_t stream) {
+    if (!h_word) return QLORA_ERR_NULL;
+    void* ws = nullptr;
+    const int st = scratch_on_current_device(&ws);
+    if (st != QLORA_OK) return st;
+    return cudaMemcpyAsync(h_word, ws, sizeof(int), cudaMemcpyDeviceToHost,
+                           reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? QLORA_OK
+               : QLORA_ERR_CUDA;
 }

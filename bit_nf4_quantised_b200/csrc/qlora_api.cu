@@ -307,6 +307,23 @@ cudaError_t record(const qlora_events* ev, bool begin, cudaStream_t s) {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA; }
 
+// The quantisers' optional non-finite check.  When the caller passes a flag,
+// the call clears it ahead of its kernels, and afterwards waits for the
+// stream and returns QLORA_ERR_NONFINITE if a kernel raised it.
+int begin_checked(int* d_flag, cudaStream_t s) {
+    if (!d_flag) return QLORA_OK;
+    return cuda_status(cudaMemsetAsync(d_flag, 0, sizeof(int), s));
+}
+
+int end_checked(int status, int* d_flag, cudaStream_t s) {
+    if (status != QLORA_OK || !d_flag) return status;
+    int h = 0;
+    if (cudaMemcpyAsync(&h, d_flag, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return QLORA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return QLORA_ERR_CUDA;
+    return h != 0 ? QLORA_ERR_NONFINITE : QLORA_OK;
+}
+
 #define QTRY(expr)                                   \
     do {                                             \
         cudaError_t _e = (expr);                     \
@@ -401,9 +418,12 @@ int qlora_quantize(const float* W, const qlora_nf4_tensor* out, int* d_nonfinite
     if (!aligned(W, 16)) return QLORA_ERR_ALIGN;
     const int64_t numel = out->rows * out->cols;
     if (numel == 0) return QLORA_OK;
-    return cuda_status(launch_quantize(W, numel, out->packed, out->scale_codes, out->meta_scale,
-                                       d_nonfinite_flag, table(),
-                                       reinterpret_cast<cudaStream_t>(stream)));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    st = begin_checked(d_nonfinite_flag, s);
+    if (st != QLORA_OK) return st;
+    st = cuda_status(launch_quantize(W, numel, out->packed, out->scale_codes, out->meta_scale,
+                                     d_nonfinite_flag, table(), s));
+    return end_checked(st, d_nonfinite_flag, s);
 }
 
 int qlora_dequantize(const qlora_nf4_tensor* w, uint16_t* W_out, qlora_stream_t stream) {
@@ -426,9 +446,12 @@ int qlora_quantize_bf16(const uint16_t* W, const qlora_nf4_tensor* out, int* d_n
     if (!aligned(W, 16)) return QLORA_ERR_ALIGN;
     const int64_t numel = out->rows * out->cols;
     if (numel == 0) return QLORA_OK;
-    return cuda_status(launch_quantize_bf16(W, numel, out->packed, out->scale_codes,
-                                            out->meta_scale, d_nonfinite_flag, table(),
-                                            reinterpret_cast<cudaStream_t>(stream)));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    st = begin_checked(d_nonfinite_flag, s);
+    if (st != QLORA_OK) return st;
+    st = cuda_status(launch_quantize_bf16(W, numel, out->packed, out->scale_codes,
+                                          out->meta_scale, d_nonfinite_flag, table(), s));
+    return end_checked(st, d_nonfinite_flag, s);
 }
 
 int qlora_format_sizes(int64_t numel, const qlora_format* f, size_t* packed_bytes,
@@ -460,8 +483,11 @@ int qlora_quantize_fmt(const float* W, int64_t numel, const qlora_format* f, uin
     if (!W || !packed || !scales || (!a.scales_fp32 && !meta)) return QLORA_ERR_NULL;
     if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(scales, 4) || (meta && !aligned(meta, 4)))
         return QLORA_ERR_ALIGN;
-    return cuda_status(launch_quantize_fmt(W, numel, a, packed, scales, meta, d_nonfinite_flag, t,
-                                           reinterpret_cast<cudaStream_t>(stream)));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    st = begin_checked(d_nonfinite_flag, s);
+    if (st != QLORA_OK) return st;
+    st = cuda_status(launch_quantize_fmt(W, numel, a, packed, scales, meta, d_nonfinite_flag, t, s));
+    return end_checked(st, d_nonfinite_flag, s);
 }
 
 int qlora_dequantize_fmt(const uint8_t* packed, const void* scales, const float* meta,
@@ -493,9 +519,14 @@ int qlora_adamw8_step(float* p, const float* g, int64_t n, int8_t* m_codes, floa
                       uint16_t* p_bf16, qlora_stream_t stream) {
     if (!cfg) return QLORA_ERR_NULL;
     if (n < 0) return QLORA_ERR_SHAPE;
+    // eps > 0 keeps every division finite (a block whose gradient and moments
+    // are all zero divides 0 by eps); lr >= 0, wd >= 0 and lr wd < 1 keep the
+    // decoupled decay factor 1 - lr wd in (0, 1]
     if (cfg->step < 1 || !(cfg->beta1 >= 0.f && cfg->beta1 < 1.f) ||
         !(cfg->beta2 >= 0.f && cfg->beta2 < 1.f) || !std::isfinite(cfg->lr) ||
-        !std::isfinite(cfg->eps) || !std::isfinite(cfg->weight_decay))
+        !std::isfinite(cfg->eps) || !std::isfinite(cfg->weight_decay) || !(cfg->eps > 0.f) ||
+        !(cfg->lr >= 0.f) || !(cfg->weight_decay >= 0.f) ||
+        !(double(cfg->lr) * double(cfg->weight_decay) < 1.0))
         return QLORA_ERR_UNSUPPORTED;
     if (n == 0) return QLORA_OK;
     if (!p || !g || !m_codes || !m_absmax || !v_codes || !v_absmax) return QLORA_ERR_NULL;

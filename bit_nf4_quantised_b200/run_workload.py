@@ -2,17 +2,19 @@
 profilers such as ncu, which want a short process around the kernels).
 
   python -m bit_nf4_quantised_b200.run_workload --workload NAME [--calls 2]
-         [--forward-only | --merge]
+         [--forward-only | --merge | --quantize]
 
 NAME is a key of synthetic.WORKLOADS; for a multi-layer workload only its
 first layer runs.  Each call is one forward (and, unless --forward-only, one
 backward) of that layer on cuda:0; with --merge, one merge of the layer's
-weight and adapter into a bf16 weight instead.
+weight and adapter into a bf16 weight instead; with --quantize, one
+quantisation of the layer's fp32 weight.
 """
 from __future__ import annotations
 
 import argparse
 
+import numpy as np
 import torch
 
 from . import _lib as q
@@ -25,8 +27,17 @@ def main() -> None:
     ap.add_argument("--calls", type=int, default=2)
     ap.add_argument("--forward-only", action="store_true")
     ap.add_argument("--merge", action="store_true")
+    ap.add_argument("--quantize", action="store_true")
     args = ap.parse_args()
     lin = syn.WORKLOADS[args.workload].layers[0]
+    if args.quantize:
+        rng = np.random.default_rng(lin.seed)
+        W = torch.from_numpy(syn.make_weight(lin, rng)).cuda()
+        for _ in range(args.calls):
+            q.qlora_quantize(W)
+        torch.cuda.synchronize()
+        print(f"{args.workload}: {args.calls} quantise call(s)")
+        return
     d = syn.make_layer(lin, with_grad=not (args.forward_only or args.merge))
     w = q.qlora_quantize(torch.from_numpy(d["W"]).cuda())
     g = {k: v.cuda() for k, v in d.items() if isinstance(v, torch.Tensor)}

@@ -130,13 +130,18 @@ QLORA_API int qlora_quantized_sizes(int64_t rows, int64_t cols, size_t* packed_b
  *   W     (device, fp32, rows*cols, read): the weight, row-major.
  *   out   (host struct, read): rows, cols and the three device buffers to
  *         write, sized by qlora_quantized_sizes.  All of them are written.
- *   d_nonfinite_flag (device int, nullable): if given, the kernel stores a
- *         non-zero value there when any element of W is NaN or +-Inf (it
- *         never clears it; zero it first).  Outputs are then unspecified.
- *         The host call cannot see device data, so it still returns
- *         QLORA_OK; read the flag after synchronising the stream.
+ *   d_nonfinite_flag (device int, nullable): the caller's request for the
+ *         non-finite check (a NaN or infinity leaves its block's absmax scale
+ *         meaningless; "Failure modes", "Loss spikes and NaNs", asks for NaNs
+ *         to be detected).  If given, the call zeroes it, enqueues
+ *         the kernels (which set it when any element of W is NaN or +-Inf),
+ *         then synchronises `stream` and returns QLORA_ERR_NONFINITE if it
+ *         was set; the outputs are then unspecified.  If NULL, nothing is
+ *         checked and the call returns as soon as the kernels are enqueued.
+ *         rows * cols = 0 launches nothing and leaves the flag untouched.
  * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE, QLORA_ERR_ALIGN (W, packed not
- * 16-byte aligned; scale_codes, meta_scale not 4-byte aligned), QLORA_ERR_CUDA.
+ * 16-byte aligned; scale_codes, meta_scale not 4-byte aligned),
+ * QLORA_ERR_NONFINITE (only when d_nonfinite_flag is given), QLORA_ERR_CUDA.
  */
 QLORA_API int qlora_quantize(const float* W, const qlora_nf4_tensor* out,
                    int* d_nonfinite_flag, qlora_stream_t stream);
@@ -197,10 +202,11 @@ QLORA_API int qlora_format_sizes(int64_t numel, const qlora_format* f, size_t* p
  * qlora_quantize_fmt -- quantise numel fp32 weights (device, read) in format
  * f (host struct, read) into packed, scales and meta (device, written, sized
  * by qlora_format_sizes; meta may be NULL for fp32 scales).
- * d_nonfinite_flag as in qlora_quantize.  numel = 0 launches nothing.
+ * d_nonfinite_flag as in qlora_quantize (given: the call synchronises the
+ * stream and reports QLORA_ERR_NONFINITE).  numel = 0 launches nothing.
  * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE, QLORA_ERR_UNSUPPORTED,
  * QLORA_ERR_ALIGN (W and packed 16-byte aligned; scales and meta 4-byte),
- * QLORA_ERR_CUDA.
+ * QLORA_ERR_NONFINITE, QLORA_ERR_CUDA.
  */
 QLORA_API int qlora_quantize_fmt(const float* W, int64_t numel, const qlora_format* f,
                                  uint8_t* packed, void* scales, float* meta,
@@ -221,9 +227,11 @@ QLORA_API int qlora_dequantize_fmt(const uint8_t* packed, const void* scales, co
  * explained", "The algorithm, step by step": AdamW over A and B only, 32- or
  * 8-bit state; "Hyperparameters that matter": the 8-bit variant quantises
  * Adam's moments blockwise).  The state of n parameters: blocks of 64, an
- * fp32 absmax per block for each moment; m as int8 codes rint(127 m / c), v
- * through its square root as uint8 codes rint(255 sqrt(v) / c).  Zero codes
- * and absmax are the initial (zero) state.
+ * fp32 absmax per block for each moment; m as int8 codes
+ * rint(fp32(m / c) * 127), v through its square root as uint8 codes
+ * rint(fp32(sqrt(v) / c) * 255) (quotient rounded to fp32, then the product
+ * rounded to the nearest integer, ties to even).  Zero codes and absmax are
+ * the initial (zero) state.
  */
 typedef struct {
     float lr;
@@ -247,9 +255,14 @@ QLORA_API int qlora_adamw8_state_sizes(int64_t n, size_t* code_bytes, size_t* ab
  *   cfg (host, read); p_bf16 (device, bf16 bits, n, nullable, written): the
  *   updated p rounded to bf16, for the layer's A or B.
  * n = 0 launches nothing.
+ * Non-finite values are not detected: a NaN or infinite gradient leaves p and
+ * the state of its block unspecified (the block maximum that sets the new
+ * absmax skips NaN).  Check gradients before the step if they may overflow.
  * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE, QLORA_ERR_UNSUPPORTED (a
- * hyperparameter out of range), QLORA_ERR_ALIGN (p, g 16-byte aligned; codes
- * and absmax 4-byte; p_bf16 8-byte), QLORA_ERR_CUDA.
+ * hyperparameter out of range: beta1 or beta2 outside [0, 1), step < 1,
+ * eps <= 0, lr < 0, weight_decay < 0, lr * weight_decay >= 1, or any of them
+ * not finite), QLORA_ERR_ALIGN (p, g 16-byte aligned; codes and absmax 4-byte;
+ * p_bf16 8-byte), QLORA_ERR_CUDA.
  */
 QLORA_API int qlora_adamw8_step(float* p, const float* g, int64_t n, int8_t* m_codes,
                                 float* m_absmax, uint8_t* v_codes, float* v_absmax,
@@ -292,7 +305,8 @@ QLORA_API int qlora_merge(const qlora_nf4_tensor* w, const uint16_t* A, const ui
  * deployment ("QLoRA" (finetunellm.com), "What it costs you": merging into
  * 4-bit weights means merging in bf16 and quantising again, a second
  * rounding).  Same result as qlora_quantize given the fp32 values of W.
- *   W (device, bf16 bits, rows*cols, read); other arguments as qlora_quantize.
+ *   W (device, bf16 bits, rows*cols, read); other arguments as qlora_quantize,
+ *   d_nonfinite_flag included (given: synchronise and report).
  * Errors: as qlora_quantize (W 16-byte aligned).
  */
 QLORA_API int qlora_quantize_bf16(const uint16_t* W, const qlora_nf4_tensor* out,
@@ -421,6 +435,21 @@ QLORA_API int qlora_linear_forward_noalloc(const uint16_t* X, int64_t M,
                                            const qlora_nf4_tensor* w, const uint16_t* A,
                                            const uint16_t* B, int r, float scale, uint16_t* Y,
                                            float* T_save, qlora_stream_t stream);
+
+/*
+ * qlora_linear_forward_noalloc_error_word -- the kernels' error word of the
+ * last qlora_linear_forward_noalloc call on the current device (the word
+ * qlora_linear_forward leaves in the first 4 bytes of a caller's workspace:
+ * 0 = none, bits as documented there).  That word lives in the library's
+ * scratch array, which callers cannot address, so this call enqueues a copy
+ * of it on `stream` into *h_word (host memory; pinned memory keeps the copy
+ * asynchronous).  The value is valid once `stream` has reached the copy;
+ * order the copy after the forward call whose word it should report.  Like
+ * the forward it allocates nothing; its first call on a device performs the
+ * same address look-up.  The paper has no counterpart to this call.
+ * Errors: QLORA_ERR_NULL (h_word NULL), QLORA_ERR_CUDA.
+ */
+QLORA_API int qlora_linear_forward_noalloc_error_word(int* h_word, qlora_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -193,10 +193,23 @@ def test_adamw8_argument_errors(q):
     assert step(fake + 4, fake, 100, fake, fake, fake, fake, ctypes.byref(cfg), None, None) == E.QLORA_ERR_ALIGN
     assert step(fake, fake, -1, fake, fake, fake, fake, ctypes.byref(cfg), None, None) == E.QLORA_ERR_SHAPE
     assert step(None, None, 0, None, None, None, None, ctypes.byref(cfg), None, None) == E.QLORA_OK
-    for bad in (q._lib._AdamConfig(2e-4, 1.0, 0.999, 1e-8, 0.0, 1),
-                q._lib._AdamConfig(2e-4, 0.9, 0.999, 1e-8, 0.0, 0),
-                q._lib._AdamConfig(float("nan"), 0.9, 0.999, 1e-8, 0.0, 1)):
+    C = q._lib._AdamConfig
+    for bad in (C(2e-4, 1.0, 0.999, 1e-8, 0.0, 1),
+                C(2e-4, 0.9, 0.999, 1e-8, 0.0, 0),
+                C(float("nan"), 0.9, 0.999, 1e-8, 0.0, 1),
+                C(2e-4, 0.9, 0.999, 0.0, 0.0, 1),          # eps = 0: 0 / 0 on an all-zero block
+                C(2e-4, 0.9, 0.999, -1e-8, 0.0, 1),
+                C(-2e-4, 0.9, 0.999, 1e-8, 0.0, 1),        # negative learning rate
+                C(2e-4, 0.9, 0.999, 1e-8, -0.1, 1),        # negative weight decay
+                C(2.0, 0.9, 0.999, 1e-8, 0.5, 1)):         # lr * wd >= 1: decay factor <= 0
         assert step(fake, fake, 100, fake, fake, fake, fake, ctypes.byref(bad), None, None) == E.QLORA_ERR_UNSUPPORTED
+    ok = C(2e-4, 0.9, 0.999, 1e-8, 0.01, 1)
+    assert step(None, None, 0, None, None, None, None, ctypes.byref(ok), None, None) == E.QLORA_OK
+
+
+def test_noalloc_error_word_argument_errors(q):
+    L = q.lib()
+    assert L.qlora_linear_forward_noalloc_error_word(None, None) == q._lib.QLORA_ERR_NULL
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

@@ -117,6 +117,31 @@ def test_decode_weight_sampled_groups(q):
         assert np.array_equal(got, ref)
 
 
+def test_nonfinite_status_from_the_c_call(q):
+    """The C entry point itself returns QLORA_ERR_NONFINITE when the caller
+    passes a flag (it synchronises the stream); without a flag it returns
+    QLORA_OK at once and checks nothing."""
+    import ctypes
+    L = q._lib.lib()
+    W = torch.ones(4, 128, device="cuda")
+    W[1, 70] = float("-inf")
+    w = q._lib.empty_nf4(4, 128)
+    st = w.c_struct()
+    flag = torch.full((1,), 123, dtype=torch.int32, device="cuda")   # stale value: cleared
+    s = torch.cuda.current_stream().cuda_stream
+    assert L.qlora_quantize(W.data_ptr(), ctypes.byref(st), flag.data_ptr(), s) == \
+        q._lib.QLORA_ERR_NONFINITE
+    assert L.qlora_quantize(W.data_ptr(), ctypes.byref(st), None, s) == q._lib.QLORA_OK
+    W[1, 70] = 2.0
+    flag.fill_(123)
+    assert L.qlora_quantize(W.data_ptr(), ctypes.byref(st), flag.data_ptr(), s) == q._lib.QLORA_OK
+    assert flag.item() == 0
+    Wb = W.bfloat16()
+    Wb[3, 3] = float("nan")
+    assert L.qlora_quantize_bf16(Wb.data_ptr(), ctypes.byref(st), flag.data_ptr(), s) == \
+        q._lib.QLORA_ERR_NONFINITE
+
+
 def test_nonfinite_is_reported(q):
     W = torch.ones(4, 128, device="cuda")
     W[2, 5] = float("nan")

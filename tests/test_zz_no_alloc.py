@@ -49,7 +49,13 @@ def test_noalloc_forward_matches_workspace_forward_twice():
         Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
         T = torch.full((M, r), float("nan"), dtype=torch.float32, device="cuda")
         assert _noalloc(L, q, X, w, A, B, 2.0, Y, T) == 0
+        # the kernels' error word of this call, read from the library's array
+        word = ctypes.c_int(-1)
+        L.qlora_linear_forward_noalloc_error_word.argtypes = [ctypes.POINTER(ctypes.c_int), vp]
+        assert L.qlora_linear_forward_noalloc_error_word(
+            ctypes.byref(word), torch.cuda.current_stream().cuda_stream) == 0
         torch.cuda.synchronize()
+        assert word.value == 0, f"device error word {word.value}"
         assert_close("Y", Y, Y_ref.double().cpu().numpy())
         assert_close("T", T, T_ref.double().cpu().numpy())
 
