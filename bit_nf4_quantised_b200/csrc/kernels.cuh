@@ -7,8 +7,22 @@
 namespace qnf4 {
 
 // ---------------------------------------------------------------- K1 / K6
+// Nearest-code table of the quantiser.  A normalised value x in [-1, 1] is
+// bucketed by y = max(x + 3, 2) in [2, 4]: bucket b = (bits of y >> 18) -
+// 0x1000 (the top five mantissa bits; b = 32 only at x = 1, entries past it
+// are padding).  Each bucket is 1/16 wide in x, narrower than the closest two
+// NF4 midpoints, so it holds at most one: base[b] = the number of midpoints
+// below the bucket (counted 2^-22 below its lower edge, past the rounding of
+// x + 3) and thr[b] = the bits of midpoint number base[b] (+inf when base is
+// 15).  The code index of any x in bucket b is base[b] + (x > thr[b]).
+constexpr int kNf4LutEntries = 64;
+struct Nf4IndexLut {
+    uint32_t thr[kNf4LutEntries];
+    uint32_t base[kNf4LutEntries];
+};
+
 cudaError_t launch_quantize(const float* W, int64_t numel, uint8_t* packed, uint8_t* scale_codes,
-                            float* meta, int* nonfinite_flag, const Nf4Table& tab,
+                            float* meta, int* nonfinite_flag, const Nf4IndexLut& lut,
                             cudaStream_t stream);
 
 cudaError_t launch_dequantize(const uint8_t* packed, const uint8_t* scale_codes, const float* meta,
@@ -18,7 +32,7 @@ cudaError_t launch_dequantize(const uint8_t* packed, const uint8_t* scale_codes,
 // K1 on a bf16 weight (the re-quantisation of a merged export).
 cudaError_t launch_quantize_bf16(const uint16_t* W, int64_t numel, uint8_t* packed,
                                  uint8_t* scale_codes, float* meta, int* nonfinite_flag,
-                                 const Nf4Table& tab, cudaStream_t stream);
+                                 const Nf4IndexLut& lut, cudaStream_t stream);
 
 // ------------------------------------------------- K1 / K6 format variants
 struct FmtTable {

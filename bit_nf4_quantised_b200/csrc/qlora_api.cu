@@ -62,6 +62,34 @@ const Nf4Table& table() {
     return t;
 }
 
+// The quantiser's bucket table (kernels.cuh): bucket b covers x + 3 in
+// [2 + b/16, 2 + (b+1)/16); base = the number of midpoints below
+// 2 + b/16 - 3 - 2^-22, thr = midpoint number base (+inf past the last).
+// Returns false unless every bucket spans at most one midpoint (true for the
+// NF4 codes, whose midpoints lie at least 0.08 apart).
+bool build_index_lut(const float mids[15], Nf4IndexLut* lut) {
+    for (int i = 0; i + 1 < 15; ++i)
+        if (!(double(mids[i + 1]) - double(mids[i]) > 1.0 / 16.0 + std::ldexp(1.0, -20))) return false;
+    for (int b = 0; b < kNf4LutEntries; ++b) {
+        const double lo = 2.0 + b / 16.0 - 3.0 - std::ldexp(1.0, -22);
+        uint32_t base = 0;
+        for (int i = 0; i < 15; ++i) base += double(mids[i]) < lo ? 1u : 0u;
+        const float thr = base < 15 ? mids[base] : std::numeric_limits<float>::infinity();
+        std::memcpy(&lut->thr[b], &thr, 4);
+        lut->base[b] = base;
+    }
+    return true;
+}
+
+// nullptr if the table could not be built
+const Nf4IndexLut* index_lut() {
+    static Nf4IndexLut lut;
+    static bool ok = false;
+    static std::once_flag once;
+    std::call_once(once, [] { ok = build_index_lut(table().mid, &lut); });
+    return ok ? &lut : nullptr;
+}
+
 // ---------------------------------------------------------------- TMA
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -421,8 +449,10 @@ int qlora_quantize(const float* W, const qlora_nf4_tensor* out, int* d_nonfinite
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     st = begin_checked(d_nonfinite_flag, s);
     if (st != QLORA_OK) return st;
+    const Nf4IndexLut* lut = index_lut();
+    if (!lut) return QLORA_ERR_UNSUPPORTED;
     st = cuda_status(launch_quantize(W, numel, out->packed, out->scale_codes, out->meta_scale,
-                                     d_nonfinite_flag, table(), s));
+                                     d_nonfinite_flag, *lut, s));
     return end_checked(st, d_nonfinite_flag, s);
 }
 
@@ -449,8 +479,10 @@ int qlora_quantize_bf16(const uint16_t* W, const qlora_nf4_tensor* out, int* d_n
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     st = begin_checked(d_nonfinite_flag, s);
     if (st != QLORA_OK) return st;
+    const Nf4IndexLut* lut = index_lut();
+    if (!lut) return QLORA_ERR_UNSUPPORTED;
     st = cuda_status(launch_quantize_bf16(W, numel, out->packed, out->scale_codes,
-                                          out->meta_scale, d_nonfinite_flag, table(), s));
+                                          out->meta_scale, d_nonfinite_flag, *lut, s));
     return end_checked(st, d_nonfinite_flag, s);
 }
 

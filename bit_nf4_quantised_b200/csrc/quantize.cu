@@ -8,160 +8,240 @@
 // max(c1 over the group) / 448, code = E4M3 round-to-nearest-even of c1 / c2,
 // saturated to 448; an all-zero group stores c2 = 0 and codes 0.
 //
-// One CTA of 256 threads owns one group of 256 blocks (16384 weights, 64 KiB of
-// fp32).  Each warp streams two blocks per step with fully coalesced 16-byte
-// loads (lanes 0-15 on one block, 16-31 on the next), reduces the absmax with
-// four shuffles, divides with a correctly rounded fp32 division (__fdiv_rn, as
-// the method's normalisation is an fp32 quotient), finds the code by binary
-// search over the midpoints in shared memory, and writes its four nibbles as
-// one 16-bit store, so a warp writes 64 contiguous bytes.  The block scales
-// stay in shared memory for the group-level FP8 pass at the end.
+// One CTA of 512 threads owns one group of 256 blocks (16384 weights, 64 KiB
+// of fp32); eight lanes cover a block, each lane the block's 32 consecutive
+// bytes 32 s .. 32 s + 31 (s = lane mod 8), so a warp takes four blocks per
+// step and a thread issues its four steps' loads (eight 16-byte loads) before
+// using any: the whole group is in flight at once, and at 64 registers two
+// CTAs (32 warps) share an SM.  (Layouts with four lanes per block, and
+// persistent CTAs streaming groups through shared memory by bulk copies, were
+// measured slower.)  Per block:
+//   - absmax by three shuffles of NaN-propagating maxima (one test of the
+//     result catches NaN and infinities);
+//   - x = fp32(w / c) without a division per element: with r = RN(1/c)
+//     computed once, q = RN(w r) is within one unit in the last place of
+//     w / c, the fused multiply-add w - q c is then exact, and
+//     RN(q + (w - q c) r) is the correctly rounded quotient (Markstein's
+//     theorem); blocks whose absmax lies outside [2^-90, 2^90], where the
+//     theorem's range conditions could fail, take the correctly rounded
+//     division instead (clamped to [-1, 1], which also sends the NaN of an
+//     infinite weight into range);
+//   - the nearest code, the number of midpoints strictly below x (a value on
+//     a midpoint takes the lower code): y = x + 3 lies in [2, 4], and the top
+//     five mantissa bits of y cut [-1, 1] into buckets 1/16 wide, narrower
+//     than the closest two midpoints (0.08 apart), so no bucket holds two.
+//     A bucket's entry gives base = the number of midpoints below it (taken
+//     2^-22 below, past the rounding of x + 3) and thr = midpoint number
+//     base; every x of the bucket has base or base + 1 midpoints below it,
+//     and idx = base + (x > thr) picks the right one.  The table (64 entries,
+//     the top ones unused) is replicated per lane in shared memory, so the
+//     lookups are free of bank conflicts;
+//   - the lane's eight indices packed into one 32-bit store (a warp writes
+//     128 contiguous bytes).
+// The block scales stay in shared memory for the group-level FP8 pass.
 //
 // The same kernel also takes a bf16 weight (a merged export being
-// re-quantised): each lane then loads 8 bytes, widened exactly to fp32.
+// re-quantised): each lane then loads 32 bytes per block, widened exactly.
+#include <cfloat>
+
 #include "kernels.cuh"
 
 namespace qnf4 {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kGroupElems = QLORA_BLOCK * QLORA_GROUP;   // 16384
+constexpr int kThreads = 512;
+constexpr int kLanesPerBlock = 8;
+constexpr int kPerLane = QLORA_BLOCK / kLanesPerBlock;                             // 8
+constexpr int kBlocksPerWarpStep = 32 / kLanesPerBlock;                            // 4
+constexpr int kSteps = QLORA_GROUP / (kThreads / 32 * kBlocksPerWarpStep);         // 4
+constexpr int kGroupElems = QLORA_BLOCK * QLORA_GROUP;                             // 16384
+constexpr int kLutBytes = kNf4LutEntries * 32 * 8;                                  // 16 KiB
 
-__device__ __forceinline__ uint32_t nearest_code(float x, const float* smid) {
-    // number of midpoints strictly below x (ties to the lower code)
-    uint32_t i = 0;
-    i += (x > smid[i + 7]) ? 8u : 0u;
-    i += (x > smid[i + 3]) ? 4u : 0u;
-    i += (x > smid[i + 1]) ? 2u : 0u;
-    i += (x > smid[i + 0]) ? 1u : 0u;
-    return i;
+// eight consecutive weights of one lane
+struct W8 {
+    float v[kPerLane];
+};
+__device__ __forceinline__ W8 load8(const float* W, int64_t e0) {
+    const float4 a = __ldcs(reinterpret_cast<const float4*>(W + e0));
+    const float4 b = __ldcs(reinterpret_cast<const float4*>(W + e0 + 4));
+    return W8{{a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w}};
 }
-
-// Four consecutive weights as fp32: fp32 input directly, bf16 input widened
-// exactly (a bf16 value is the top half of its fp32).
-__device__ __forceinline__ float4 load4(const float* W, int64_t e0) {
-    return __ldcs(reinterpret_cast<const float4*>(W + e0));
-}
-__device__ __forceinline__ float4 load4(const uint16_t* W, int64_t e0) {
-    const uint2 u = __ldcs(reinterpret_cast<const uint2*>(W + e0));
-    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
-                       __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+__device__ __forceinline__ W8 load8(const uint16_t* W, int64_t e0) {
+    const uint4 u = __ldcs(reinterpret_cast<const uint4*>(W + e0));   // bf16 = top half of fp32
+    return W8{{__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+               __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u),
+               __uint_as_float(u.z << 16), __uint_as_float(u.z & 0xffff0000u),
+               __uint_as_float(u.w << 16), __uint_as_float(u.w & 0xffff0000u)}};
 }
 __device__ __forceinline__ float load1(const float* W, int64_t e) { return W[e]; }
 __device__ __forceinline__ float load1(const uint16_t* W, int64_t e) {
     return __uint_as_float(uint32_t(W[e]) << 16);
 }
+template <typename Tin>
+__device__ __forceinline__ W8 load8_tail(const Tin* W, int64_t e0, int64_t numel) {
+    W8 r;
+#pragma unroll
+    for (int j = 0; j < kPerLane; ++j) r.v[j] = e0 + j < numel ? load1(W, e0 + j) : 0.f;
+    return r;
+}
+
+// max that returns NaN when either operand is NaN
+__device__ __forceinline__ float max_nan(float a, float b) {
+    float d;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+    return d;
+}
+
+// fp32(w / c), correctly rounded, from r = RN(1/c) (c in [2^-90, 2^90], |w| <= c)
+__device__ __forceinline__ float quotient(float w, float c, float r) {
+    const float q = __fmul_rn(w, r);
+    const float rem = __fmaf_rn(-q, c, w);
+    return __fmaf_rn(rem, r, q);
+}
+
+// Number of midpoints strictly below x in [-1, 1], from the bucket table.
+// lane_lut is this lane's column of the table, minus the offset of key
+// 0x1000 (the bucket of y = 2).
+__device__ __forceinline__ uint32_t code_index(float x, uint32_t lane_lut) {
+    const uint32_t key = __float_as_uint(__fadd_rn(x, 3.0f)) >> 18;   // 0x1000 + bucket
+    uint32_t thr, base;
+    asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(thr), "=r"(base) : "r"(lane_lut + (key << 8)));
+    return base + (x > __uint_as_float(thr) ? 1u : 0u);
+}
 
 template <bool kFull, typename Tin>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 quantize_kernel(const Tin* __restrict__ W, int64_t numel, int64_t nblocks,
                 uint8_t* __restrict__ packed, uint8_t* __restrict__ scale_codes,
-                float* __restrict__ meta, int* __restrict__ nonfinite_flag, Nf4Table tab) {
-    __shared__ float smid[16];
+                float* __restrict__ meta, int* __restrict__ nonfinite_flag, Nf4IndexLut lut) {
+    extern __shared__ __align__(16) uint8_t smem[];                // the per-lane table
     __shared__ float sabs[QLORA_GROUP];
-    __shared__ float sred[kThreads / 32];
+    __shared__ float sred[QLORA_GROUP / 32];
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    if (tid < 15) smid[tid] = tab.mid[tid];
-    __syncthreads();
-
+    const int sub = lane & (kLanesPerBlock - 1), bq = lane / kLanesPerBlock;
     const int64_t group = blockIdx.x;
     const int64_t gbase = group * kGroupElems;
-    const int half = lane >> 4, sub = lane & 15;
-    bool bad = false;
 
-    // 32 blocks per warp, two per step.
-#pragma unroll 4
-    for (int step = 0; step < 16; ++step) {
-        const int blk = warp * 32 + step * 2 + half;          // block within group
-        const int64_t e0 = gbase + int64_t(blk) * QLORA_BLOCK + sub * 4;
-        float4 v;
-        if (kFull) {
-            v = load4(W, e0);
-        } else {
-            v.x = (e0 + 0 < numel) ? load1(W, e0 + 0) : 0.f;
-            v.y = (e0 + 1 < numel) ? load1(W, e0 + 1) : 0.f;
-            v.z = (e0 + 2 < numel) ? load1(W, e0 + 2) : 0.f;
-            v.w = (e0 + 3 < numel) ? load1(W, e0 + 3) : 0.f;
-        }
-        bad |= !(isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w));
-        float a = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+    // every load of the group first
+    W8 v[kSteps];
 #pragma unroll
-        for (int o = 8; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-        // a = c_b for this half-warp's block
-        uint32_t q0 = 7, q1 = 7, q2 = 7, q3 = 7;               // zero block -> code 0
+    for (int step = 0; step < kSteps; ++step) {
+        const int blk = (step * (kThreads / 32) + warp) * kBlocksPerWarpStep + bq;
+        const int64_t e0 = gbase + int64_t(blk) * QLORA_BLOCK + sub * kPerLane;
+        v[step] = kFull ? load8(W, e0) : load8_tail(W, e0, numel);
+    }
+    // table entry e for lane l at byte 256 e + 8 l: thread t writes entry
+    // t / 8 for lanes 4 (t mod 8) .. + 3
+    {
+        const int e = tid >> 3, l0 = (tid & 7) * 4;
+        const uint32_t a = smem_u32(smem) + e * 256 + l0 * 8;
+        const uint32_t t = lut.thr[e], b = lut.base[e];
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %1, %2};" ::"r"(a), "r"(t), "r"(b) : "memory");
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %1, %2};" ::"r"(a + 16), "r"(t), "r"(b) : "memory");
+    }
+    __syncthreads();
+    const uint32_t lane_lut = smem_u32(smem) + lane * 8 - (0x1000u << 8);
+    uint32_t* packed_w = reinterpret_cast<uint32_t*>(packed + group * (kGroupElems / 2));
+
+    bool bad = false;
+#pragma unroll
+    for (int step = 0; step < kSteps; ++step) {
+        const int blk = (step * (kThreads / 32) + warp) * kBlocksPerWarpStep + bq;
+        const float* f = v[step].v;
+        float a = max_nan(max_nan(max_nan(fabsf(f[0]), fabsf(f[1])), max_nan(fabsf(f[2]), fabsf(f[3]))),
+                          max_nan(max_nan(fabsf(f[4]), fabsf(f[5])), max_nan(fabsf(f[6]), fabsf(f[7]))));
+#pragma unroll
+        for (int o = 4; o >= 1; o >>= 1) a = max_nan(a, __shfl_xor_sync(0xffffffffu, a, o));
+        bad |= !(a <= FLT_MAX);                                // NaN or infinity in the block
+        // a = c_b for this block
+        uint32_t word = 0x77777777u;                            // zero block -> code 0
         if (a > 0.f) {
-            q0 = nearest_code(__fdiv_rn(v.x, a), smid);
-            q1 = nearest_code(__fdiv_rn(v.y, a), smid);
-            q2 = nearest_code(__fdiv_rn(v.z, a), smid);
-            q3 = nearest_code(__fdiv_rn(v.w, a), smid);
+            word = 0;
+            if (a >= 0x1p-90f && a <= 0x1p90f) {
+                const float r = __frcp_rn(a);
+#pragma unroll
+                for (int j = 0; j < kPerLane; ++j) word += code_index(quotient(f[j], a, r), lane_lut) << (4 * j);
+            } else {
+#pragma unroll
+                for (int j = 0; j < kPerLane; ++j)
+                    word += code_index(fminf(fmaxf(__fdiv_rn(f[j], a), -1.0f), 1.0f), lane_lut) << (4 * j);
+            }
         }
-        const int64_t gblk = group * QLORA_GROUP + blk;
-        if (kFull || gblk < nblocks) {
-            const uint16_t nib = static_cast<uint16_t>(q0 | (q1 << 4) | (q2 << 8) | (q3 << 12));
-            reinterpret_cast<uint16_t*>(packed + gblk * (QLORA_BLOCK / 2))[sub] = nib;
-        }
+        if (kFull || group * QLORA_GROUP + blk < nblocks) packed_w[blk * (QLORA_BLOCK / 8) + sub] = word;
         if (sub == 0) sabs[blk] = a;
     }
-    if (bad && nonfinite_flag != nullptr) atomicOr(nonfinite_flag, 1);
+    if (bad && sub == 0 && nonfinite_flag != nullptr) atomicOr(nonfinite_flag, 1);
     __syncthreads();
 
-    // Double quantisation of this group's 256 scales.
-    const float c = sabs[tid];
-    float m = c;
+    // Double quantisation of this group's 256 scales (the first 8 warps).
+    if (tid < QLORA_GROUP) {
+        const float c = sabs[tid];
+        float m = c;
 #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) sred[warp] = m;
-    __syncthreads();
-    float gmax = sred[0];
+        for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) sred[warp] = m;
+        asm volatile("bar.sync 1, %0;" ::"n"(QLORA_GROUP) : "memory");
+        float gmax = sred[0];
 #pragma unroll
-    for (int w = 1; w < kThreads / 32; ++w) gmax = fmaxf(gmax, sred[w]);
-    const float c2 = __fdiv_rn(gmax, 448.0f);
-    uint8_t code = 0;
-    if (c2 > 0.f) {
-        code = static_cast<uint8_t>(
-            __nv_cvt_float_to_fp8(__fdiv_rn(c, c2), __NV_SATFINITE, __NV_E4M3));
+        for (int w = 1; w < QLORA_GROUP / 32; ++w) gmax = fmaxf(gmax, sred[w]);
+        const float c2 = __fdiv_rn(gmax, 448.0f);
+        uint8_t code = 0;
+        if (c2 > 0.f) {
+            code = static_cast<uint8_t>(
+                __nv_cvt_float_to_fp8(__fdiv_rn(c, c2), __NV_SATFINITE, __NV_E4M3));
+        }
+        const int64_t gblk = group * QLORA_GROUP + tid;
+        if (kFull || gblk < nblocks) scale_codes[gblk] = code;
+        if (tid == 0) meta[group] = c2;
     }
-    const int64_t gblk = group * QLORA_GROUP + tid;
-    if (kFull || gblk < nblocks) scale_codes[gblk] = code;
-    if (tid == 0) meta[group] = c2;
+}
+
+template <bool kFull, typename Tin>
+cudaError_t launch_one(unsigned grid, const Tin* W, int64_t numel, int64_t nblocks, uint8_t* packed,
+                       uint8_t* scale_codes, float* meta, int* nonfinite_flag,
+                       const Nf4IndexLut& lut, cudaStream_t stream) {
+    quantize_kernel<kFull, Tin><<<grid, kThreads, kLutBytes, stream>>>(
+        W, numel, nblocks, packed, scale_codes, meta, nonfinite_flag, lut);
+    return cudaGetLastError();
 }
 
 template <typename Tin>
 cudaError_t quantize_any(const Tin* W, int64_t numel, uint8_t* packed, uint8_t* scale_codes,
-                         float* meta, int* nonfinite_flag, const Nf4Table& tab,
+                         float* meta, int* nonfinite_flag, const Nf4IndexLut& lut,
                          cudaStream_t stream) {
     const int64_t nblocks = (numel + QLORA_BLOCK - 1) / QLORA_BLOCK;
     const int64_t ngroups = (nblocks + QLORA_GROUP - 1) / QLORA_GROUP;
     const int64_t full = numel / kGroupElems;                  // groups with no tail
     if (full > 0) {
-        quantize_kernel<true, Tin><<<dim3(static_cast<unsigned>(full)), kThreads, 0, stream>>>(
-            W, numel, nblocks, packed, scale_codes, meta, nonfinite_flag, tab);
+        const cudaError_t e = launch_one<true>(static_cast<unsigned>(full), W, numel, nblocks, packed,
+                                               scale_codes, meta, nonfinite_flag, lut, stream);
+        if (e != cudaSuccess) return e;
     }
     if (ngroups > full) {
         // the single trailing group, offset so blockIdx.x is its group index
         const int64_t off = full * kGroupElems;
-        quantize_kernel<false, Tin><<<1, kThreads, 0, stream>>>(
-            W + off, numel - off, nblocks - full * QLORA_GROUP, packed + full * (kGroupElems / 2),
-            scale_codes + full * QLORA_GROUP, meta + full, nonfinite_flag, tab);
+        return launch_one<false>(1u, W + off, numel - off, nblocks - full * QLORA_GROUP,
+                                 packed + full * (kGroupElems / 2), scale_codes + full * QLORA_GROUP,
+                                 meta + full, nonfinite_flag, lut, stream);
     }
-    return cudaGetLastError();
+    return cudaSuccess;
 }
 
 }  // namespace
 
 cudaError_t launch_quantize(const float* W, int64_t numel, uint8_t* packed, uint8_t* scale_codes,
-                            float* meta, int* nonfinite_flag, const Nf4Table& tab,
+                            float* meta, int* nonfinite_flag, const Nf4IndexLut& lut,
                             cudaStream_t stream) {
-    return quantize_any(W, numel, packed, scale_codes, meta, nonfinite_flag, tab, stream);
+    return quantize_any(W, numel, packed, scale_codes, meta, nonfinite_flag, lut, stream);
 }
 
 cudaError_t launch_quantize_bf16(const uint16_t* W, int64_t numel, uint8_t* packed,
                                  uint8_t* scale_codes, float* meta, int* nonfinite_flag,
-                                 const Nf4Table& tab, cudaStream_t stream) {
-    return quantize_any(W, numel, packed, scale_codes, meta, nonfinite_flag, tab, stream);
+                                 const Nf4IndexLut& lut, cudaStream_t stream) {
+    return quantize_any(W, numel, packed, scale_codes, meta, nonfinite_flag, lut, stream);
 }
 
 }  // namespace qnf4
