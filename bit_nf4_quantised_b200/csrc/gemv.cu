@@ -1,37 +1,44 @@
 // K5: bandwidth-bound dequant-GEMV for decode-sized token counts (M <= 16):
 //   Y = X W~^T + gamma (X A^T) B^T
 // ("QLoRA, explained": serving the adapter unmerged on the 4-bit base).  The
-// packed weight is streamed from HBM exactly once.
+// packed weight is streamed from HBM exactly once, and every weight enters
+// the product as the W~ the page's dDQ defines, bf16_rne(fp32(q[idx] * c~)),
+// the same value the dequantise kernel writes and the GEMM multiplies.
 //
 // One persistent CTA per SM: a producer warp and 16 consumer warps.
-//   producer   pulls work units (16 rows of W x one contraction slice) from an
-//              atomic counter and streams each unit as tiles of 16 rows x 32
-//              NF4 blocks (16 rows x 1024 contiguous bytes) with one 3-D TMA
-//              box per tile into a 4-stage ring (128-byte swizzle).  Its other
-//              lanes read the tile's FP8 scale codes and fp32 meta scales and
-//              publish c~ = e4m3(code) * c2 for every (row, block) of the
-//              tile next to it, so consumers do no global loads at all.
-//   consumers  each take 2 of the tile's 32 blocks for all 16 rows: swap-AB
-//              mma.sync m16n8k16 with W rows on the MMA's M side and tokens on
-//              its N side (one n8 tile for M <= 8, two for M <= 16).  A lane
-//              turns each packed byte into the bf16 pair (q[lo], q[hi]) with
-//              one byte permute and one shared-memory load from a
-//              byte->bf16x2 table replicated per lane: table rows are 256
-//              bytes apart from a 64 KiB-aligned base, so the permute drops the
-//              byte straight into bits 8..15 of the lane's address.  Inside a
-//              block the contraction order is permuted identically on both
-//              operands (lane c of a row group covers k = 16c .. 16c+15), the
-//              block's MMAs accumulate into fresh registers, and the block
-//              partial is scaled by its c~ once.  At the end of a unit the 16
-//              warps' partials are summed through shared memory.
+//   producer   pulls work units (R rows of W x one contraction slice) from an
+//              atomic counter and streams each unit as tiles of R rows x D
+//              256-wide chunks (R D = 256, 32 KiB of packed indices) with one
+//              3-D TMA box per tile into a ring of stages (128-byte swizzle);
+//              its lanes copy the tile's FP8 scale codes and each row's meta
+//              scales next to it (cp.async), so consumers do no global loads.
+//   consumers  warp w takes the tile's 16-row group w / D of chunk w % D: a
+//              swap-AB mma.sync m16n8k16 with W rows on the MMA's M side and
+//              tokens on its N side (one n8 tile for M <= 8, two for M <= 16).
+//              The contraction order inside the chunk is permuted identically
+//              on both operands so that lane (g, c) of the warp holds, over
+//              the chunk's 16 MMAs, all 64 weights of NF4 block c of rows g
+//              and g + 8 (MMA j feeds the block's positions 4j .. 4j + 3).
+//              Each packed byte addresses a per-lane table of fp32 code pairs
+//              (q[lo], q[hi]) in shared memory (one permute drops the byte
+//              into the lane's address; one 8-byte load); the pair is
+//              multiplied by the block's c~ in fp32 and rounded to a bf16 pair
+//              (RNE): exactly bf16_rne(fp32(q * c~)), the A operand of the
+//              MMA.  The activations sit in shared memory with 8-byte units
+//              XOR-swizzled by block and token, so that a warp's 8-byte
+//              fragment loads are free of bank conflicts.
+//              At the end of a unit the D warps of each row group sum their
+//              partials through shared memory.
 // The first few CTAs of each slice also compute a share of T = X A^T.  Slices
 // and T shares write fp32 partials; the finalize kernel sums them, adds
 // gamma T B^T and rounds Y to bf16.
 //
-// Deviation from the dequantise kernel, stated: the table holds bf16(q[i])
-// rather than bf16(q[i] * c~), so each weight enters as bf16(q) * c~ in fp32;
-// the difference from bf16_rne(q * c~) is below one bf16 ulp per weight, far
-// inside the layer tolerance.
+// Per two weights the expansion costs one permute, one 8-byte shared load
+// (two wavefronts per warp), two fp32 multiplies and one paired rounding.
+// Measured alternatives that built each block's 16-entry bf16 table in
+// registers and expanded nibbles with byte permutes (about 2.5 integer-pipe
+// instructions per weight, entirely or for part of the rows) were slower: the
+// integer pipe runs 64 such instructions per clock per SM on this GPU.
 //
 // Every mbarrier wait is bounded (common.cuh); a timeout sets the workspace
 // error word and the kernel winds down.
@@ -45,21 +52,19 @@ namespace {
 
 constexpr int kConsumerWarps = 16;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;   // + producer warp
-constexpr int kLutBytes = 256 * 256;                  // 256 rows of 256 bytes
 constexpr int kSmemBytes = 227 * 1024;
 constexpr int kMaxStages = 6;
-// A weight tile is 16 KiB: R rows x D chunks of 256 contraction positions
-// (128 packed bytes), R D = 128, D in {1, 2, 4, 8} chosen per launch so that
-// a contraction slice is a whole number of tiles.  A work unit is R rows x the
-// whole slice.
-constexpr int kTileBytes = 16384;
+// A weight tile is 32 KiB: R rows x D chunks of 256 contraction positions
+// (128 packed bytes), R D = 256, D in {1, 2, 4, 8} chosen per launch so that
+// a contraction slice is a whole number of tiles; the 16 consumer warps take
+// its 16 (16-row group, chunk) pieces.  A work unit is R rows x the whole
+// slice.
+constexpr int kTileBytes = 32768;
 // Raw scale data of a tile, copied next to it by the producer: the FP8 codes
-// [R rows][4 D + 4 bytes] (the pitch puts the 8 rows a consumer load reads on
-// distinct banks), then the meta scales [R rows][2] fp32 of each row's first
-// and last block (a row's blocks in a tile span at most two groups of 256
-// scales).  At most 512 + 12 R <= 2048 bytes.
-constexpr int kScaleBytes = 2048;
-
+// [R rows][4 D + 4 bytes], then the meta scales [R rows][2] fp32 of each row's
+// first and last block (a row's blocks in a tile span at most two groups of
+// 256 scales).  1024 + 12 R <= 4096 bytes.
+constexpr int kScaleBytes = 4096;
 __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, bool valid) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(valid ? 4 : 0)
                  : "memory");
@@ -98,11 +103,6 @@ __device__ __forceinline__ uint32_t opaque_zero() {
 
 __device__ __forceinline__ void keep_before(float v) { asm volatile("" ::"f"(v)); }
 
-__device__ __forceinline__ uint32_t lds32_nv(uint32_t addr) {
-    uint32_t v;
-    asm("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
-    return v;
-}
 
 __device__ __forceinline__ uint32_t lds16_nv(uint32_t addr) {
     uint16_t v;
@@ -136,12 +136,6 @@ __device__ __forceinline__ void mma16816_nv(float (&d)[4], uint32_t a0, uint32_t
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// bf16 pair of byte k of w: lane_reg = table base + 4*lane, bits 8..15 clear.
-template <int k>
-__device__ __forceinline__ uint32_t lut_pair(uint32_t w, uint32_t lane_reg) {
-    return lds32_nv(prmt(w, lane_reg, 0x7604u | (k << 4)));
-}
-
 __device__ __forceinline__ void tma_load_3d(uint32_t smem_dst, const CUtensorMap* map, int32_t c0,
                                             int32_t c1, int32_t c2, uint64_t* bar) {
     asm volatile(
@@ -151,12 +145,16 @@ __device__ __forceinline__ void tma_load_3d(uint32_t smem_dst, const CUtensorMap
         : "memory");
 }
 
-// Shared-memory plan: the table sits at the first 64 KiB boundary; everything
-// else is placed first-fit in the space before it, then after it.  The host
-// evaluates the same plan to pick the stage count; the kernel re-checks it
-// against its real shared-memory base and reports a misfit.
+// Shared-memory plan.  The code-pair table sits at the first 64 KiB boundary
+// (its addresses are formed by dropping a byte into bits 8-15 of the lane's
+// base, so bits 8-15 of the base must be clear); everything else is placed
+// first-fit in the space before it, then after it.  The host evaluates the
+// same plan to pick the stage count; the kernel re-checks it against its real
+// shared-memory base and reports a misfit.
+constexpr int kLutBytes = 256 * 256;      // 256 byte values x 32 lanes x 8 bytes
+
 struct SmemPlan {
-    uint32_t lut, ring, scales, units, red, x, bars;
+    uint32_t lut, ring, scales, units, red, x, zero, bars;
     bool ok;
 };
 
@@ -168,7 +166,7 @@ __host__ __device__ inline SmemPlan plan_smem(uint32_t start, int stages, uint32
     const uint32_t lo_end = p.lut;                             // region before the table
     uint32_t hi = p.lut + kLutBytes;
     const uint32_t hi_end = start + kSmemBytes;
-    p.ok = true;
+    p.ok = hi <= hi_end;
     auto take = [&](uint32_t bytes, uint32_t align) -> uint32_t {
         uint32_t at = (lo + align - 1) & ~(align - 1);
         if (at + bytes <= lo_end) {
@@ -186,26 +184,39 @@ __host__ __device__ inline SmemPlan plan_smem(uint32_t start, int stages, uint32
     p.ring = take(stages * kTileBytes, 1024);
     p.scales = take(stages * kScaleBytes, 16);
     p.red = take(red_bytes, 16);
-    p.x = take(x_bytes, 16);
+    p.x = take(x_bytes, 128);
+    p.zero = take(128, 128);                       // zero activations for absent tokens
     p.units = take(stages * 8, 8);
     p.bars = take((2 * stages + 4) * 8 + 8, 8);   // full, empty, rdone[2], rfree[2], flag
     return p;
 }
 
-// Activation slab bytes (rows 16-byte aligned, pitch 16 mod 128 bytes) and
-// reduction-buffer bytes (two [warp][16 rows][M] fp32 buffers, which also
-// hold the [M][r] reduction of T) for M tokens over a kslab-wide slice.
+// Activation slab bytes (M rows of kslab bf16, a row a whole number of 128-byte
+// lines) and reduction-buffer bytes (two [warp][16 rows][M] fp32 buffers,
+// which also hold the [M][r] reduction of T) for M tokens over a kslab-wide
+// slice.
 __host__ __device__ inline uint32_t gemv_x_bytes(int64_t M, int64_t kslab) {
-    return static_cast<uint32_t>(M * (kslab * 2 + 16));
+    return static_cast<uint32_t>(M * kslab * 2);
 }
 __host__ __device__ inline uint32_t gemv_red_bytes(int64_t M) {
     return static_cast<uint32_t>(2 * kConsumerWarps * 16 * M * 4);
 }
 
+// Byte offset of activation (token m, slice position k) in the slab, k a
+// multiple of 2: rows of kslab bf16; within each 64-position block the
+// 8-byte units (4 positions) are permuted by u -> u ^ (4 (block mod 4) +
+// (m mod 4)), so that the 16 lanes of a half-warp, which read unit j of
+// blocks 0-3 for tokens 0-3 (or 4-7), hit 16 different bank pairs.
+__device__ __forceinline__ uint32_t x_off(int m, int k, uint32_t x_pitch) {
+    const int blk = k >> 6;
+    const int u = ((k & 63) >> 2) ^ (((blk & 3) << 2) | (m & 3));
+    return static_cast<uint32_t>(m) * x_pitch + static_cast<uint32_t>(blk * 128 + u * 8 + (k & 3) * 2);
+}
+
 template <int NT, int kStages, int D>
 __global__ void __launch_bounds__(kThreads, 1)
 gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t start = smem_u32(smem);
     const int slice = blockIdx.y;
@@ -215,12 +226,12 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
     const int kslab = static_cast<int>(k_end - k_beg);
     const int nblk = kslab / QLORA_BLOCK;
     // D: 256-wide chunks per tile (= a.tile_chunks)
-    constexpr int R = 128 / D;                   // rows per tile and unit
+    constexpr int R = 256 / D;                   // rows per tile and unit
     constexpr int bpr = 4 * D;                   // blocks per tile row
     constexpr int code_pitch = bpr + 4;
     constexpr int meta_off = R * code_pitch;     // a multiple of 16
     const int tiles_per_unit = (nblk + bpr - 1) / bpr;
-    const uint32_t x_pitch = static_cast<uint32_t>(kslab * 2 + 16);   // as gemv_x_bytes
+    const uint32_t x_pitch = static_cast<uint32_t>(kslab * 2);        // as gemv_x_bytes
     const int xrows = static_cast<int>(a.M);
     const uint32_t red_half = gemv_red_bytes(a.M) / 2;
     const SmemPlan sp = plan_smem(start, kStages, gemv_x_bytes(a.M, kslab), 2u * red_half);
@@ -245,23 +256,30 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
         fence_barrier_init();
         prefetch_tensormap(&tm_packed);
     }
-    // lookup table: byte -> (bf16 q[lo nibble], bf16 q[hi nibble]), one copy
-    // per lane, written four lanes' copies at a time
-    for (int e = tid; e < 256 * 8; e += kThreads) {
-        const int b = e >> 3, l4 = e & 7;
-        const uint32_t v = pack_bf16x2(a.tab.code[b & 15], a.tab.code[b >> 4]);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(sp.lut + b * 256 + l4 * 16), "r"(v)
-                     : "memory");
+    // code-pair table: entry e (a packed byte) of lane l at lut + 256 e + 8 l
+    // holds the fp32 codes (q[e & 15], q[e >> 4]); each thread writes two
+    // lanes' copies of an entry at a time
+    if (sp.ok) {
+        for (int i = tid; i < 256 * 16; i += kThreads) {
+            const int e = i >> 4, l2 = (i & 15) * 2;
+            const float q0 = a.tab.code[e & 15], q1 = a.tab.code[e >> 4];
+            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %1, %2};" ::"r"(sp.lut + e * 256 + l2 * 8),
+                         "f"(q0), "f"(q1)
+                         : "memory");
+        }
     }
-    // activation slice, M rows; the pitch is 16 mod 128 bytes so that the
-    // consumers' 16-byte fragment loads (8 lanes a phase) hit distinct banks
-    const int vec_per_row = kslab / 8;
-    for (int q = tid; q < xrows * vec_per_row; q += kThreads) {
-        const int m = q / vec_per_row, v = q % vec_per_row;
-        const uint4 val = *reinterpret_cast<const uint4*>(a.X + m * a.K + k_beg + v * 8);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sp.x + m * x_pitch + v * 16),
-                     "r"(val.x), "r"(val.y), "r"(val.z), "r"(val.w)
-                     : "memory");
+    // activation slice, M rows of 8-byte units, swizzled (x_off); a zero
+    // line stands in for tokens past M and blocks past the slice
+    if (sp.ok) {
+        if (tid < 32) asm volatile("st.shared.b32 [%0], %1;" ::"r"(sp.zero + tid * 4), "r"(0u) : "memory");
+        const int units_per_row = kslab / 4;
+        for (int q = tid; q < xrows * units_per_row; q += kThreads) {
+            const int m = q / units_per_row, u = q % units_per_row;
+            const uint2 val = *reinterpret_cast<const uint2*>(a.X + m * a.K + k_beg + u * 4);
+            asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(sp.x + x_off(m, u * 4, x_pitch)),
+                         "r"(val.x), "r"(val.y)
+                         : "memory");
+        }
     }
     __syncthreads();
     if (*abort_flag) return;
@@ -274,7 +292,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
     if (warp == kConsumerWarps) {
         // -------------------------------------------------------- producer
         // Per work item (unit, tile), once its stage is free: lane 0 starts
-        // the tile's TMA load; the lanes copy the tile's FP8 scale codes (four
+        // the tile's TMA load; the lanes copy the tile's FP8 scale codes (8
         // 4-byte groups each, cp.async, zeros past the slice or the matrix)
         // and each row's two meta scales into the stage's scale area, and
         // arrive on the stage's full barrier when their copies land.  Units
@@ -321,15 +339,14 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
                 const int bs_row = t * bpr;                    // each row's first block
                 const int cnt_full = max(0, min(bpr, nblk - bs_row));
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const int gi = lane + 32 * q4;             // 128 groups: R rows x D
+                for (int q8 = 0; q8 < 8; ++q8) {
+                    const int gi = lane + 32 * q8;             // 256 groups: R rows x D
                     const int row = gi / D, grp = gi % D;
                     const int64_t n = int64_t(u) * R + row;
                     const bool live = n < a.N && 4 * grp < cnt_full;
                     cp_async4(area + row * code_pitch + 4 * grp,
                               a.scale_codes + (live ? n * nkb + kb_beg + bs_row + 4 * grp : 0), live);
                 }
-#pragma unroll
                 for (int mi = lane; mi < 2 * R; mi += 32) {
                     const int row = mi >> 1, last = mi & 1;
                     const int64_t n = int64_t(u) * R + row;
@@ -374,10 +391,10 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
             for (int j = 0; j < 4; ++j) tacc[j][0] = tacc[j][1] = tacc[j][2] = tacc[j][3] = 0.f;
             for (int st = s0 + warp; st < s1; st += kConsumerWarps) {
                 const int kk = st * 16 + 2 * c;
-                const uint32_t a0 = g < xrows ? lds32(sp.x + g * x_pitch + kk * 2) : 0u;
-                const uint32_t a2 = g < xrows ? lds32(sp.x + g * x_pitch + (kk + 8) * 2) : 0u;
-                const uint32_t a1 = g + 8 < xrows ? lds32(sp.x + (g + 8) * x_pitch + kk * 2) : 0u;
-                const uint32_t a3 = g + 8 < xrows ? lds32(sp.x + (g + 8) * x_pitch + (kk + 8) * 2) : 0u;
+                const uint32_t a0 = g < xrows ? lds32(sp.x + x_off(g, kk, x_pitch)) : 0u;
+                const uint32_t a2 = g < xrows ? lds32(sp.x + x_off(g, kk + 8, x_pitch)) : 0u;
+                const uint32_t a1 = g + 8 < xrows ? lds32(sp.x + x_off(g + 8, kk, x_pitch)) : 0u;
+                const uint32_t a3 = g + 8 < xrows ? lds32(sp.x + x_off(g + 8, kk + 8, x_pitch)) : 0u;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     if ((jg + j) * 8 < a.r) {
@@ -414,19 +431,19 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
         asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
     }
 
-    // main loop: 2 blocks of every tile, all 16 rows.  MMA row g (and g + 8)
-    // holds tile row rg (and rg + 8), rg = 2 (g mod 4) + g / 4: the half-warp
-    // that a 64-bit shared load serves then reads rows 0, 2, 4, 6 (or 1, 3,
-    // 5, 7), whose swizzled 16-byte units cover all 32 banks.
-    const int rg = 2 * (g & 3) + (g >> 2);
-    // this warp's pairs 2 warp, 2 warp + 1 of (block, 16-row group): blocks
-    // btw, btw + 1 of rows ra = 16 rq + rg and rb = ra + 8 of every tile
-    const int rq = (2 * warp) / bpr, btw = (2 * warp) % bpr;
-    const int ra = rq * 16 + rg, rb = ra + 8;
+    // Main loop.  Warp w takes row group rq = w / D (tile rows 16 rq + g and
+    // 16 rq + g + 8 for MMA rows g, g + 8) of chunk cw = w % D; lane (g, c)
+    // owns NF4 block bt = 4 cw + c of its two rows.  MMA j multiplies block
+    // positions 4j .. 4j + 3: A fragment a0 / a2 = row g's positions
+    // 4j, 4j+1 / 4j+2, 4j+3 (a1 / a3 the same of row g + 8), B fragment
+    // b0, b1 = token g's activations at the same four positions.
+    const int rq = warp / D, cw = warp % D;
+    const int ra = rq * 16 + g, rb = ra + 8;
+    const int bt = cw * 4 + c;
+    const uint32_t lane_lut = sp.lut + lane * 8;       // bits 8-15 clear
     float acc[NT][4];
 #pragma unroll
     for (int t = 0; t < NT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-    const uint32_t lane_reg = sp.lut + lane * 4;
     float* part = a.part + int64_t(slice) * a.M * a.N;
     uint32_t it = 0, units_done = 0;
     for (;;) {
@@ -439,100 +456,70 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
         const uint32_t z = opaque_zero();
         const uint32_t ring = sp.ring + s * kTileBytes + z;
         const uint32_t scl = sp.scales + s * kScaleBytes + z;
-        // operands of both blocks first, then the lookups and MMAs
-        uint32_t wa[2][2], wb[2][2], xk[2];
-        float ct[2][2];
-        // this warp's two blocks of rows rg and rg + 8: FP8 codes (16 bits
-        // per row) and the rows' meta scales; a row's blocks before `split`
-        // belong to its first block's group of 256 scales
-        const uint32_t cra = lds16_nv(scl + ra * code_pitch + btw);
-        const uint32_t crb = lds16_nv(scl + rb * code_pitch + btw);
-        const float2 mra = lds64f_nv(scl + meta_off + ra * 8);
-        const float2 mrb = lds64f_nv(scl + meta_off + rb * 8);
-        const float2 va = e4m3x2_to_float2(cra), vb = e4m3x2_to_float2(crb);
+        const int bs = tile * bpr + bt;                       // block within the slice
+        // Blocks past the slice (only in a zero-filled last tile) take
+        // c~ = 0 and zero activations, so they add nothing.
+        const bool valid = bs < nblk;
+        // c~ = fp32(e4m3 code * meta scale), one rounding; a row's blocks
+        // before `split` belong to its first block's group of 256 scales
         // (the low 8 bits of the row's first scale index; 32-bit wrap-around
         // keeps them exact)
         const uint32_t ci_lo = static_cast<uint32_t>(unit) * static_cast<uint32_t>(R) * static_cast<uint32_t>(nkb) +
                                static_cast<uint32_t>(kb_beg + tile * bpr);
         const int split_a = 256 - static_cast<int>((ci_lo + ra * static_cast<uint32_t>(nkb)) & 255u);
         const int split_b = 256 - static_cast<int>((ci_lo + rb * static_cast<uint32_t>(nkb)) & 255u);
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int bt = btw + j;                           // block within the tile row
-            const int bs = tile * bpr + bt;                   // block within the slice
-            // Blocks past the slice carry c~ = 0 and finite table values;
-            // their activations are taken as zero so they add nothing.
-            const bool valid = bs < nblk;
-            // tile layout [chunk of 4 blocks][R rows][128 bytes], 16-byte
-            // units swizzled by (row & 7); lane (g, c) reads 8 bytes of rows
-            // ra and rb (both = rg mod 8)
-            const int within = (bt & 3) * 32 + c * 8;
-            const uint32_t unit16 = static_cast<uint32_t>(within >> 4);
-            const uint32_t chunk = ring + (bt >> 2) * (R * 128) + (within & 15) +
-                                   ((unit16 ^ static_cast<uint32_t>(rg & 7)) << 4);
-            asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(wa[j][0]), "=r"(wa[j][1]) : "r"(chunk + ra * 128));
-            asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(wb[j][0]), "=r"(wb[j][1]) : "r"(chunk + rb * 128));
-            // c~ = fp32(e4m3 code * meta scale), one rounding
-            ct[j][0] = __fmul_rn(j == 0 ? va.x : va.y, bt < split_a ? mra.x : mra.y);
-            ct[j][1] = __fmul_rn(j == 0 ? vb.x : vb.y, bt < split_b ? mrb.x : mrb.y);
-            xk[j] = valid ? sp.x + z + static_cast<uint32_t>((bs * 64 + c * 16) * 2) : 0u;
+        const float2 mra = lds64f_nv(scl + meta_off + ra * 8);
+        const float2 mrb = lds64f_nv(scl + meta_off + rb * 8);
+        const uint32_t cab = lds16_nv(scl + ra * code_pitch + (bt & ~1)) >> (8 * (bt & 1));
+        const uint32_t cbb = lds16_nv(scl + rb * code_pitch + (bt & ~1)) >> (8 * (bt & 1));
+        const float2 va = e4m3x2_to_float2(cab & 0xffu), vb = e4m3x2_to_float2(cbb & 0xffu);
+        const float cta = valid ? __fmul_rn(va.x, bt < split_a ? mra.x : mra.y) : 0.f;
+        const float ctb = valid ? __fmul_rn(vb.x, bt < split_b ? mrb.x : mrb.y) : 0.f;
+        // this lane's 32 packed bytes of each row: tile layout [chunk][R
+        // rows][128 bytes], 16-byte units swizzled by (row & 7); block c is
+        // units 2c, 2c + 1
+        const uint32_t chunk = ring + cw * (R * 128);
+        uint32_t wa[8], wb[8];
+        {
+            const uint32_t ua = chunk + ra * 128, ub = chunk + rb * 128;
+            const uint32_t u0 = static_cast<uint32_t>((2 * c) ^ (ra & 7)) << 4;
+            const uint32_t u1 = static_cast<uint32_t>((2 * c + 1) ^ (ra & 7)) << 4;
+            asm("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(wa[0]), "=r"(wa[1]), "=r"(wa[2]), "=r"(wa[3]) : "r"(ua + u0));
+            asm("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(wa[4]), "=r"(wa[5]), "=r"(wa[6]), "=r"(wa[7]) : "r"(ua + u1));
+            asm("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(wb[0]), "=r"(wb[1]), "=r"(wb[2]), "=r"(wb[3]) : "r"(ub + u0));
+            asm("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(wb[4]), "=r"(wb[5]), "=r"(wb[6]), "=r"(wb[7]) : "r"(ub + u1));
         }
-        float blk[2][NT][4];
+        // activations of this lane's token(s) for block bs: the block's
+        // 128-byte line of the slab (or the zero line past the slice or the
+        // batch); unit j of it sits at line ^ ((j ^ key) << 3) (x_off)
+        uint32_t xk[NT];
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
+        for (int t = 0; t < NT; ++t) {
+            const int tok = g + 8 * t;
+            const uint32_t line = valid && tok < xrows ? sp.x + tok * x_pitch + bs * 128 : sp.zero;
+            xk[t] = (line + z) | static_cast<uint32_t>((((bs & 3) << 2) | (tok & 3)) << 3);
+        }
 #pragma unroll
-            for (int t = 0; t < NT; ++t) blk[j][t][0] = blk[j][t][1] = blk[j][t][2] = blk[j][t][3] = 0.f;
-        // one token tile: the two blocks' steps interleave; two token tiles:
-        // block after block, which keeps fewer activation registers live
-        uint32_t xb[2][NT][8];
+        for (int w = 0; w < 8; ++w) {
+            // each packed byte -> its two fp32 codes from the lane's pair
+            // table -> fp32 products with c~ -> one bf16 pair (RNE): exactly
+            // bf16_rne(fp32(q * c~)) for both elements
+            uint32_t oa[4], ob[4];
 #pragma unroll
-        for (int o = 0; o < 8; ++o) {
-            const int st = NT == 1 ? (o >> 1) : (o & 3);
-            const int j = NT == 1 ? (o & 1) : (o >> 2);
-            if (st == 0) {
-                // activations of lane c's 16 contraction positions, two
-                // 16-byte loads (zero for a block past the slice)
-#pragma unroll
-                for (int t = 0; t < NT; ++t) {
-                    const int tok = g + 8 * t;
-#pragma unroll
-                    for (int h = 0; h < 8; ++h) xb[j][t][h] = 0u;
-                    if (xk[j] != 0u && tok < xrows) {
-                        const uint32_t xa = xk[j] + tok * x_pitch;
-                        asm("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                            : "=r"(xb[j][t][0]), "=r"(xb[j][t][1]), "=r"(xb[j][t][2]), "=r"(xb[j][t][3])
-                            : "r"(xa));
-                        asm("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                            : "=r"(xb[j][t][4]), "=r"(xb[j][t][5]), "=r"(xb[j][t][6]), "=r"(xb[j][t][7])
-                            : "r"(xa + 16));
-                    }
-                }
-            }
-            const uint32_t wA = wa[j][st >> 1];
-            const uint32_t wB = wb[j][st >> 1];
-            uint32_t a0, a1, a2, a3;
-            if (st & 1) {
-                a0 = lut_pair<2>(wA, lane_reg);
-                a2 = lut_pair<3>(wA, lane_reg);
-                a1 = lut_pair<2>(wB, lane_reg);
-                a3 = lut_pair<3>(wB, lane_reg);
-            } else {
-                a0 = lut_pair<0>(wA, lane_reg);
-                a2 = lut_pair<1>(wA, lane_reg);
-                a1 = lut_pair<0>(wB, lane_reg);
-                a3 = lut_pair<1>(wB, lane_reg);
+            for (int k = 0; k < 4; ++k) {
+                const float2 qa = lds64f_nv(prmt(wa[w], lane_lut, 0x7604u | (k << 4)));
+                const float2 qb = lds64f_nv(prmt(wb[w], lane_lut, 0x7604u | (k << 4)));
+                oa[k] = pack_bf16x2(__fmul_rn(qa.x, cta), __fmul_rn(qa.y, cta));
+                ob[k] = pack_bf16x2(__fmul_rn(qb.x, ctb), __fmul_rn(qb.y, ctb));
             }
 #pragma unroll
-            for (int t = 0; t < NT; ++t)
-                mma16816_nv(blk[j][t], a0, a1, a2, a3, xb[j][t][2 * st], xb[j][t][2 * st + 1]);
-            if (st == 3) {
-                // the block is done: scale its sums into the accumulators
+            for (int h = 0; h < 2; ++h) {
+                const int j = 2 * w + h;                          // MMA: positions 4j .. 4j + 3
 #pragma unroll
                 for (int t = 0; t < NT; ++t) {
-                    acc[t][0] = fmaf(ct[j][0], blk[j][t][0], acc[t][0]);
-                    acc[t][1] = fmaf(ct[j][0], blk[j][t][1], acc[t][1]);
-                    acc[t][2] = fmaf(ct[j][1], blk[j][t][2], acc[t][2]);
-                    acc[t][3] = fmaf(ct[j][1], blk[j][t][3], acc[t][3]);
+                    uint32_t b0, b1;
+                    asm("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(b0), "=r"(b1) : "r"(xk[t] ^ (j << 3)));
+                    mma16816_nv(acc[t], oa[2 * h], ob[2 * h], oa[2 * h + 1], ob[2 * h + 1], b0, b1);
                 }
             }
         }
@@ -549,8 +536,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
         if (tile == tiles_per_unit - 1) {
             // The unit is complete.  Each warp writes its 16 rows x M
             // partials; then min(M, 16) warps, a different run of warps for
-            // each unit, share the 256 M additions (each output adds the
-            // partials of the bpr / 2 warps of its row group, in warp order).
+            // each unit, share the R M additions (each output adds the
+            // partials of the D warps of its row group, in warp order).
             // Buffer p is reused every second unit; rfree[p] says the summing
             // warps have read its last contents.
             const int p = units_done & 1;
@@ -562,8 +549,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
                 const int tok = 8 * t + 2 * c;
-                const uint32_t r0 = base + (rg * xrows + tok) * 4;
-                const uint32_t r1 = base + ((rg + 8) * xrows + tok) * 4;
+                const uint32_t r0 = base + (g * xrows + tok) * 4;
+                const uint32_t r1 = base + ((g + 8) * xrows + tok) * 4;
                 if (tok < xrows) {
                     asm volatile("st.shared.f32 [%0], %1;" ::"r"(r0), "f"(acc[t][0]) : "memory");
                     asm volatile("st.shared.f32 [%0], %1;" ::"r"(r1), "f"(acc[t][2]) : "memory");
@@ -580,12 +567,11 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
             const int idx = (warp - unit * nsum) & (kConsumerWarps - 1);
             if (idx < nsum) {
                 if (!mbar_wait(&rdone[p], use & 1, abort_flag, a.err)) break;
-                const int wpg = bpr / 2;                      // warps per row group
                 for (int e = idx * 32 + lane; e < R * xrows; e += nsum * 32) {
                     const int row = e / xrows, tok = e % xrows;
-                    const int w0 = (row >> 4) * wpg, r16 = row & 15;
+                    const int w0 = (row >> 4) * D, r16 = row & 15;
                     float sum = 0.f;
-                    for (int w = w0; w < w0 + wpg; ++w)
+                    for (int w = w0; w < w0 + D; ++w)
                         sum += __uint_as_float(lds32(red + ((w * 16 + r16) * xrows + tok) * 4));
                     const int64_t n = int64_t(unit) * R + row;
                     if (n < a.N) part[int64_t(tok) * a.N + n] = sum;
@@ -673,7 +659,7 @@ gemv_finalize_kernel(GemvFinalizeArgs a) {
 int gemv_stages(int64_t M, int64_t kslab) {
     // dynamic shared memory starts after the 1 KiB the driver reserves; the
     // plan must also hold for a base 1 KiB either side of that
-    for (int st = kMaxStages; st >= 4; st -= 2) {
+    for (int st = kMaxStages; st >= 3; --st) {
         bool ok = true;
         for (uint32_t start : {0u, 1024u, 2048u})
             ok = ok && plan_smem(start, st, gemv_x_bytes(M, kslab), gemv_red_bytes(M)).ok;
@@ -708,9 +694,20 @@ cudaError_t launch_gemv(const CUtensorMap& tm_packed, const GemvArgs& a, int num
     dim3 grid(per_slice, static_cast<unsigned>(a.splits));
     const int st = gemv_stages(a.M, std::min<int64_t>(a.K, a.k_per_split));
     if (st == 0) return cudaErrorInvalidConfiguration;
-    if (a.M > 8) return st == 6 ? launch_depth<2, 6>(grid, tm_packed, a, stream)
-                                : launch_depth<2, 4>(grid, tm_packed, a, stream);
-    return st == 6 ? launch_depth<1, 6>(grid, tm_packed, a, stream) : launch_depth<1, 4>(grid, tm_packed, a, stream);
+    if (a.M > 8) {
+        switch (st) {
+            case 6: return launch_depth<2, 6>(grid, tm_packed, a, stream);
+            case 5: return launch_depth<2, 5>(grid, tm_packed, a, stream);
+            case 4: return launch_depth<2, 4>(grid, tm_packed, a, stream);
+            default: return launch_depth<2, 3>(grid, tm_packed, a, stream);
+        }
+    }
+    switch (st) {
+        case 6: return launch_depth<1, 6>(grid, tm_packed, a, stream);
+        case 5: return launch_depth<1, 5>(grid, tm_packed, a, stream);
+        case 4: return launch_depth<1, 4>(grid, tm_packed, a, stream);
+        default: return launch_depth<1, 3>(grid, tm_packed, a, stream);
+    }
 }
 
 cudaError_t launch_gemv_finalize(const GemvFinalizeArgs& a, cudaStream_t stream) {

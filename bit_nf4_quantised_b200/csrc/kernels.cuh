@@ -175,7 +175,7 @@ struct GemvArgs {
     int64_t M, N, K;
     int splits;
     int64_t k_per_split;  // multiple of 256 (or K)
-    int tile_chunks;      // D: 256-wide chunks per weight tile (1, 2, 4, 8); tiles are 128 / D rows
+    int tile_chunks;      // D: 256-wide chunks per weight tile (1, 2, 4, 8); tiles are 256 / D rows
     int t_ctas;           // CTAs of each slice that compute a share of T
     Nf4Table tab;
 };
@@ -183,7 +183,7 @@ struct GemvArgs {
 // contraction slice (0: its activations do not fit in shared memory).
 int gemv_stages(int64_t M, int64_t kslab);
 // tm_packed: 3-D view of the packed weight {128 bytes, N rows, K/256 chunks},
-// strides {K/2, 128} bytes, box {128, 128 / D rows, D chunks}, 128-byte
+// strides {K/2, 128} bytes, box {128, 256 / D rows, D chunks}, 128-byte
 // swizzle, D = a.tile_chunks.
 cudaError_t launch_gemv(const CUtensorMap& tm_packed, const GemvArgs& a, int num_sms,
                         cudaStream_t stream);

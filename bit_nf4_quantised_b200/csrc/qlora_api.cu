@@ -125,13 +125,13 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uin
 }
 
 // Packed weight seen as {128 bytes, N rows, K/256 chunks of 128 bytes}; box
-// {128, 16, 8} = 16 rows x 1024 contiguous bytes, 128-byte swizzle.
+// {128, 256 / chunks, chunks} = a 32 KiB tile, 128-byte swizzle.
 bool make_map_3d_packed(CUtensorMap* map, const void* packed, int64_t N, int64_t K, int chunks) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(K / 256)};
     const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K / 2), 128};
-    const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(128 / chunks), static_cast<cuuint32_t>(chunks)};
+    const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(256 / chunks), static_cast<cuuint32_t>(chunks)};
     const cuuint32_t estr[3] = {1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(packed), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

@@ -343,8 +343,10 @@ QLORA_API int qlora_linear_workspace_size(int64_t M, int64_t N, int64_t K, int r
  *          schedule broke its width rules; with any bit set the outputs
  *          are unspecified).
  *   M <= 16 with K % 256 == 0 runs the bandwidth-bound dequant-GEMV kernel,
- *   every other shape the tensor-core dequant-GEMM; both compute the same
- *   function.
+ *   every other shape the tensor-core dequant-GEMM; both multiply the same
+ *   W~ (each weight bf16_rne(fp32(q[idx] * c~_b)), as qlora_dequantize
+ *   writes it) in fp32 accumulation, so they differ only in the order of
+ *   their fp32 additions.
  * Shape rules: K % 64 == 0, N % 8 == 0, K >= 64, N >= 8.
  * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE, QLORA_ERR_ALIGN (every tensor
  * 16-byte aligned, except scale_codes and meta_scale: 4-byte),
