@@ -216,22 +216,29 @@ def e4m3_encode(x: np.ndarray) -> np.ndarray:
     return out
 
 
-def e4m3_encode_sorted(x: np.ndarray) -> np.ndarray:
-    """The same encoding as e4m3_encode, written for whole arrays: the 127
-    values are ascending in code order, so a binary search (np.searchsorted)
-    finds each element's two neighbours lo <= x <= hi; the nearer one wins,
-    an exact tie takes the even code, and anything at or above 448 takes
-    0x7E."""
+def _encode_sorted(x: np.ndarray, table: np.ndarray, what: str) -> np.ndarray:
+    """Nearest value of an ascending table of a float format's non-negative
+    finite values (code i has value table[i]): a binary search
+    (np.searchsorted) finds each element's two neighbours lo <= x <= hi; the
+    nearer one wins, an exact tie takes the even code, and anything at or
+    above the largest value takes the largest code (saturation)."""
     x = np.asarray(x, dtype=np.float32).astype(np.float64).reshape(-1)
     if np.any(x < 0) or not np.all(np.isfinite(x)):
-        raise ValueError("e4m3_encode_sorted takes finite non-negative values")
-    hi = np.clip(np.searchsorted(_E4M3, x, side="left"), 1, 126)
+        raise ValueError(f"{what} takes finite non-negative values")
+    top = table.size - 1
+    hi = np.clip(np.searchsorted(table, x, side="left"), 1, top)
     lo = hi - 1
-    d_lo = x - _E4M3[lo]
-    d_hi = _E4M3[hi] - x
+    d_lo = x - table[lo]
+    d_hi = table[hi] - x
     even = np.where(lo % 2 == 0, lo, hi)
     code = np.where(d_lo < d_hi, lo, np.where(d_hi < d_lo, hi, even))
-    return np.where(x >= E4M3_MAX, 0x7E, code).astype(np.uint8)
+    return np.where(x >= table[top], top, code).astype(np.uint8)
+
+
+def e4m3_encode_sorted(x: np.ndarray) -> np.ndarray:
+    """The same encoding as e4m3_encode, written for whole arrays (the 127
+    values ascend in code order; at or above 448 -> 0x7E)."""
+    return _encode_sorted(x, _E4M3, "e4m3_encode_sorted")
 
 
 def e4m3_decode(code: np.ndarray) -> np.ndarray:
@@ -241,36 +248,101 @@ def e4m3_decode(code: np.ndarray) -> np.ndarray:
     return _E4M3[c].astype(np.float32)
 
 
-def double_quantize(absmax: np.ndarray, group: int = GROUP
+# The other 8-bit scale encodings ("Double quantisation" names only "8-bit
+# floats"; "A toy run ..." measures what the choice costs): OCP FP8 E5M2
+# (bias 15, two mantissa bits, largest finite 57344) and a linear unsigned
+# 8-bit code (c2 = max / 255, code = rint(fp32(c_b / c2)), ties to even).
+E5M2_MAX = 57344.0
+U8_MAX = 255.0
+
+
+def e5m2_value_table() -> np.ndarray:
+    """Values of the 124 non-negative finite E5M2 codes 0x00..0x7B (fp64).
+
+    Code c = eeeee mm: exponent field 0 is subnormal, m/4 * 2^-14; otherwise
+    (1 + m/4) * 2^(e - 15).  0x7C is +inf and 0x7D..0x7F are NaN, never
+    produced."""
+    vals = np.empty(124, dtype=np.float64)
+    for c in range(124):
+        e, m = c >> 2, c & 3
+        vals[c] = (m / 4.0) * 2.0 ** -14 if e == 0 else (1.0 + m / 4.0) * 2.0 ** (e - 15)
+    return vals
+
+
+_E5M2 = e5m2_value_table()
+
+
+def e5m2_encode(x: np.ndarray) -> np.ndarray:
+    """Non-negative fp32 -> E5M2 code, nearest with ties to the even code,
+    at or above 57344 saturated to 0x7B."""
+    return _encode_sorted(x, _E5M2, "e5m2_encode")
+
+
+def e5m2_decode(code: np.ndarray) -> np.ndarray:
+    c = np.asarray(code, dtype=np.uint8).reshape(-1)
+    if np.any(c >= 0x7C):
+        raise ValueError("only non-negative finite E5M2 codes are produced")
+    return _E5M2[c].astype(np.float32)
+
+
+def u8_encode(x: np.ndarray) -> np.ndarray:
+    """Non-negative fp32 x (the ratio c_b / c2, at most about 255) -> the
+    linear code rint(x), ties to even, clamped to 255."""
+    x = np.asarray(x, dtype=np.float32).reshape(-1)
+    if np.any(x < 0) or not np.all(np.isfinite(x)):
+        raise ValueError("u8_encode takes finite non-negative values")
+    return np.minimum(np.rint(x), np.float32(U8_MAX)).astype(np.uint8)
+
+
+SCALE_CODES = {"e4m3": (E4M3_MAX, e4m3_encode_sorted),
+               "e5m2": (E5M2_MAX, e5m2_encode),
+               "u8": (U8_MAX, u8_encode)}
+
+
+def decode_scale_codes(codes: np.ndarray, fmt: str = "e4m3") -> np.ndarray:
+    """fp32 value of each 8-bit scale code (exact in every format)."""
+    if fmt == "e4m3":
+        return e4m3_decode(codes)
+    if fmt == "e5m2":
+        return e5m2_decode(codes)
+    if fmt == "u8":
+        return np.asarray(codes, dtype=np.uint8).astype(np.float32).reshape(-1)
+    raise ValueError(fmt)
+
+
+def double_quantize(absmax: np.ndarray, group: int = GROUP, fmt: str = "e4m3"
                     ) -> tuple[np.ndarray, np.ndarray]:
     """(scale_codes u8[nblocks], meta fp32[ngroups]).
 
-    c2_g = fp32(max_{b in g} c_b / 448); code_b = E4M3(fp32(c_b / c2_g)).
-    An all-zero group has c2 = 0 and codes 0.  A final partial group is padded
-    with zero scales, which cannot change its max.
+    c2_g = fp32(max_{b in g} c_b / TOP); code_b = ENC(fp32(c_b / c2_g)), with
+    TOP and ENC those of the 8-bit format (E4M3: 448 and round-to-nearest-even
+    E4M3; E5M2: 57344 and E5M2; u8: 255 and rint).  An all-zero group has
+    c2 = 0 and codes 0.  A final partial group is padded with zero scales,
+    which cannot change its max.
     """
+    top, encode = SCALE_CODES[fmt]
     c = np.asarray(absmax, dtype=np.float32).reshape(-1)
     nblocks = c.size
     ngroups = -(-nblocks // group)
     padded = np.zeros(ngroups * group, dtype=np.float32)
     padded[:nblocks] = c
     padded = padded.reshape(ngroups, group)
-    meta = (padded.max(axis=1) / np.float32(E4M3_MAX)).astype(np.float32)
+    meta = (padded.max(axis=1) / np.float32(top)).astype(np.float32)
     live = meta > 0
     safe = np.where(live, meta, np.float32(1.0)).astype(np.float32)
     ratio = (padded / safe.reshape(ngroups, 1)).astype(np.float32)
-    codes = e4m3_encode_sorted(ratio).reshape(ngroups, group)
+    codes = encode(ratio).reshape(ngroups, group)
     codes[~live] = 0
     return codes.reshape(-1)[:nblocks], meta
 
 
 def dequantize_scales(scale_codes: np.ndarray, meta: np.ndarray,
-                      group: int = GROUP) -> np.ndarray:
+                      group: int = GROUP, fmt: str = "e4m3") -> np.ndarray:
     """First step of dDQ ("The forward pass and gradients"): c~_b = fp32(
     decode(code_b) * c2_g), a single correctly rounded fp32 product."""
     codes = np.asarray(scale_codes, dtype=np.uint8).reshape(-1)
     g = np.arange(codes.size) // group
-    return (e4m3_decode(codes) * np.asarray(meta, dtype=np.float32)[g]).astype(np.float32)
+    return (decode_scale_codes(codes, fmt) * np.asarray(meta, dtype=np.float32)[g]).astype(np.float32)
 
 
 # ---------------------------------------------------------------------------
@@ -470,6 +542,8 @@ def merge(packed, scale_codes, meta, rows: int, cols: int, A, B, gamma):
 # ---------------------------------------------------------------------------
 SCALES_FP32 = "fp32"
 SCALES_E4M3 = "e4m3"
+SCALES_E5M2 = "e5m2"
+SCALES_U8 = "u8"
 
 
 def midpoints_of(codes: np.ndarray) -> np.ndarray:
@@ -479,8 +553,8 @@ def midpoints_of(codes: np.ndarray) -> np.ndarray:
 
 def quantize_fmt(W: np.ndarray, codes: np.ndarray, block: int, scales: str):
     """W (flattened, fp32) -> (packed, scales, meta).  scales 'fp32': one fp32
-    absmax per block and meta None; 'e4m3': FP8 codes and fp32 constants per
-    256 blocks, as quantize()."""
+    absmax per block and meta None; 'e4m3' (as quantize()), 'e5m2' or 'u8':
+    8-bit codes and fp32 constants per 256 blocks (double_quantize)."""
     w = np.asarray(W, dtype=np.float32).reshape(-1)
     if not np.all(np.isfinite(w)):
         raise NonFiniteWeight("weights must be finite")
@@ -490,16 +564,16 @@ def quantize_fmt(W: np.ndarray, codes: np.ndarray, block: int, scales: str):
     packed = pack_nibbles(idx)
     if scales == SCALES_FP32:
         return packed, absmax.astype(np.float32), None
-    sc, meta = double_quantize(absmax)
+    sc, meta = double_quantize(absmax, fmt=scales)
     return packed, sc, meta
 
 
 def dequantize_fmt_bits(packed, scale_data, meta, numel: int, codes: np.ndarray, block: int,
                         scales: str) -> np.ndarray:
     """bf16 bits of w~ = bf16_rne(fp32(q[idx] * c~_b)), c~_b the fp32 absmax
-    ('fp32') or fp32(e4m3 * c2) ('e4m3')."""
+    ('fp32') or fp32(decode(code) * c2) (the 8-bit formats)."""
     c = (np.asarray(scale_data, dtype=np.float32) if scales == SCALES_FP32
-         else dequantize_scales(scale_data, meta))
+         else dequantize_scales(scale_data, meta, fmt=scales))
     nblocks = c.size
     idx = unpack_nibbles(packed, nblocks * block).reshape(nblocks, block)
     prod = (np.asarray(codes, dtype=np.float32)[idx] * c.reshape(nblocks, 1)).astype(np.float32)

@@ -291,6 +291,85 @@ def test_double_quantize_matches_per_group_enumeration():
         assert np.array_equal(sc[g * 256:g * 256 + part.size], want)
 
 
+def _e5m2_probe_values(n_random):
+    rng = np.random.default_rng(13)
+    tab = o.e5m2_value_table()
+    mids = ((tab[:-1] + tab[1:]) / 2).astype(np.float32)
+    return np.concatenate([
+        tab.astype(np.float32), mids,
+        np.nextafter(mids, np.float32(np.inf)), np.nextafter(mids, np.float32(0)),
+        np.array([57344.0, 60000.0, 61439.0], np.float32),
+        rng.uniform(0, 61000, n_random // 2).astype(np.float32),
+        (2.0 ** rng.uniform(-18, 15.8, n_random // 2)).astype(np.float32),
+    ])
+
+
+def test_e5m2_encode_matches_torch_cast():
+    """The E5M2 scale code is torch's float8_e5m2 cast (round to nearest,
+    ties to even) wherever that cast is finite; above, it saturates."""
+    vals = _e5m2_probe_values(1_000_000)
+    vals = vals[vals < 61440.0]                # torch's cast overflows to inf from here
+    ours = o.e5m2_encode(vals)
+    theirs = torch.from_numpy(vals).to(torch.float8_e5m2).view(torch.uint8).numpy()
+    assert vals.size > 500_000 and np.array_equal(ours, theirs)
+    assert o.e5m2_encode(np.array([61440.0, 1e30], np.float32)).tolist() == [0x7B, 0x7B]
+
+
+def test_e5m2_decode_matches_torch():
+    c = np.arange(0x7C, dtype=np.uint8)
+    theirs = torch.from_numpy(c).view(torch.float8_e5m2).to(torch.float32).numpy()
+    assert np.array_equal(o.e5m2_decode(c), theirs)
+    assert o.e5m2_decode(np.array([0x7B], np.uint8))[0] == 57344.0
+
+
+def test_u8_scale_code_is_the_nearest_level():
+    """Linear 8-bit scale codes: the group's largest scale takes 255, every
+    dequantised scale lies within half a step (plus fp32 rounding) of the
+    true one, no other of the 256 levels is nearer, and scales that are
+    exact multiples of the step come back exactly."""
+    rng = np.random.default_rng(14)
+    c = np.abs(rng.standard_normal(256 * 40)).astype(np.float32) * np.float32(0.03)
+    c[256 * 3:256 * 4] = 0.0                                   # an all-zero group
+    step = np.float32(0.001)
+    c[256 * 5:256 * 6] = (np.arange(256) % 256).astype(np.float32) * step
+    c[256 * 5 + 255] = np.float32(255) * step                  # the group max
+    sc, meta = o.double_quantize(c, fmt="u8")
+    g = np.arange(c.size) // 256
+    for k in range(40):
+        part = c[k * 256:(k + 1) * 256]
+        if part.max() > 0:
+            assert sc[k * 256 + int(np.argmax(part))] == 255
+    ct = o.dequantize_scales(sc, meta, fmt="u8").astype(np.float64)
+    c2 = meta[g].astype(np.float64)
+    err = np.abs(ct - c.astype(np.float64))
+    slack = ct * 2.0 ** -23 + c2 * 2.0 ** -18           # fp32 roundings of c / c2 and code * c2
+    assert np.all(err <= c2 * 0.5 + slack + 1e-30)
+    levels = np.arange(256)[None, :] * c2[:, None]
+    best = np.abs(levels - c.astype(np.float64)[:, None]).min(axis=1)
+    assert np.all(err <= best + slack + 1e-30)
+    exact = slice(256 * 5, 256 * 6)
+    assert np.array_equal(sc[exact], np.arange(256, dtype=np.uint8))
+
+
+def test_scale_formats_cost_on_the_toy():
+    """The page's toy (2^20 N(0, 0.02^2) weights, NF4, blocks of 64): fp32
+    scales give the printed 0.845 %; a linear 8-bit code of the scales adds
+    almost nothing, E4M3 about 0.08 points, E5M2 (two mantissa bits) more
+    again; every 8-bit format stays within its scale step of fp32."""
+    rng = np.random.default_rng(0)
+    w = (rng.standard_normal(2 ** 20) * 0.02).astype(np.float32)
+    codes, _ = o.nf4_codebook()
+    rel = {}
+    for fmt in ("fp32", "u8", "e4m3", "e5m2"):
+        p, s_, m = o.quantize_fmt(w, codes, 64, fmt)
+        rec = o.bf16_bits_to_float(o.dequantize_fmt_bits(p, s_, m, w.size, codes, 64, fmt))
+        rel[fmt] = float(np.sum((rec.astype(np.float64) - w) ** 2) / np.sum(w.astype(np.float64) ** 2))
+    assert abs(rel["fp32"] - 0.00845) < 0.00002
+    assert rel["fp32"] < rel["u8"] < rel["fp32"] + 0.00002
+    assert rel["u8"] < rel["e4m3"] < rel["e5m2"]
+    assert 0.0090 < rel["e4m3"] < 0.0095 and 0.0110 < rel["e5m2"] < 0.0120
+
+
 def test_e4m3_decode_matches_torch():
     c = np.arange(127, dtype=np.uint8)
     theirs = torch.from_numpy(c).view(torch.float8_e4m3fn).to(torch.float32).numpy()
