@@ -610,32 +610,49 @@ def silu_grad(z):
     return s * (1.0 + z * (1.0 - s))
 
 
-def mlp_forward(X, layers, gamma):
+def _bf16_of(x):
+    """fp64 -> the nearest bf16 value (ties to even), as fp64."""
+    return bf16_bits_to_float(bf16_rne_f64(x)).astype(np.float64)
+
+
+def mlp_forward(X, layers, gamma, bf16_activations: bool = False):
     """layers = {'gate': (Wt, A, B), 'up': ..., 'down': ...} with Wt = W~
     [out, in].  -> (Y, saved) where saved = (G, U, H) are the activations a
-    non-checkpointed backward keeps."""
+    non-checkpointed backward keeps.
+
+    bf16_activations: the activations that pass between the block's steps
+    (the outputs of gate, up and down, and h) are rounded to bf16, the compute
+    type the pages fix ("Failure modes", "Loss spikes and NaNs": use bf16
+    compute; "Minimal implementation": bnb_4bit_compute_dtype bf16); each
+    step itself stays exact in fp64."""
+    rnd = _bf16_of if bf16_activations else (lambda a: a)
     G, _ = linear_forward(X, *layers["gate"], gamma)
     U, _ = linear_forward(X, *layers["up"], gamma)
-    H = silu(G) * U
+    G, U = rnd(G), rnd(U)
+    H = rnd(silu(G) * U)
     Y, _ = linear_forward(H, *layers["down"], gamma)
-    return Y, (G, U, H)
+    return rnd(Y), (G, U, H)
 
 
-def mlp_backward(dY, X, layers, gamma, saved=None):
+def mlp_backward(dY, X, layers, gamma, saved=None, bf16_activations: bool = False):
     """-> (dX, {name: (dA, dB)}).  saved = None recomputes the forward from X
-    (gradient checkpointing: the third dequantisation of gate and up)."""
+    (gradient checkpointing: the third dequantisation of gate and up).
+    bf16_activations as mlp_forward, for dH, dG, dU and each linear's input
+    gradient (the two parts of dX rounded, then their sum)."""
+    rnd = _bf16_of if bf16_activations else (lambda a: a)
     if saved is None:
-        _, saved = mlp_forward(X, layers, gamma)
+        _, saved = mlp_forward(X, layers, gamma, bf16_activations)
     G, U, H = saved
     Wd, Ad, Bd = layers["down"]
     dH, dAd, dBd, _ = linear_backward(dY, H, Wd, Ad, Bd, gamma)
-    dG = dH * U * silu_grad(G)
-    dU = dH * silu(G)
+    dH = rnd(dH)
+    dG = rnd(dH * U * silu_grad(G))
+    dU = rnd(dH * silu(G))
     Wg, Ag, Bg = layers["gate"]
     Wu, Au, Bu = layers["up"]
     dXg, dAg, dBg, _ = linear_backward(dG, X, Wg, Ag, Bg, gamma)
     dXu, dAu, dBu, _ = linear_backward(dU, X, Wu, Au, Bu, gamma)
-    return dXg + dXu, {"gate": (dAg, dBg), "up": (dAu, dBu), "down": (dAd, dBd)}
+    return rnd(rnd(dXg) + rnd(dXu)), {"gate": (dAg, dBg), "up": (dAu, dBu), "down": (dAd, dBd)}
 
 
 # ---------------------------------------------------------------------------

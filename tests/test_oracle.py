@@ -798,6 +798,32 @@ def test_checkpointed_backward_equals_stored_activations():
         assert all(np.array_equal(a, b) for a, b in zip(d1[k], d2[k]))
 
 
+def test_mlp_bf16_activations():
+    """With bf16 activations every activation passed between the steps is a
+    bf16 value, equal to bf16_rne of the same step's exact value computed from
+    the rounded inputs (checked by redoing one element by hand, with torch's
+    bf16 cast as the rounding), and the block's results stay within a few
+    bf16 roundings of the exact chain."""
+    X, L, dY, g = _tiny_mlp(seed=53, M=5, K=8, F=7)
+    Y0, _ = o.mlp_forward(X, L, g)
+    Y1, (G, U, H) = o.mlp_forward(X, L, g, bf16_activations=True)
+    tb = lambda a: torch.tensor(a, dtype=torch.float64).to(torch.bfloat16).double().item()
+    for arr in (G, U, H, Y1):
+        assert np.array_equal(o._bf16_of(arr), arr)
+    m, f = 2, 4
+    gx = float(X[m] @ L["gate"][0][f] + g * (X[m] @ L["gate"][1].T) @ L["gate"][2][f])
+    assert G[m, f] == tb(gx)
+    assert H[m, f] == tb(G[m, f] / (1 + math.exp(-G[m, f])) * U[m, f])
+    assert np.linalg.norm(Y1 - Y0) / np.linalg.norm(Y0) < 2 ** -6
+    dX0, d0 = o.mlp_backward(dY, X, L, g)
+    dX1, d1 = o.mlp_backward(dY, X, L, g, bf16_activations=True)
+    assert np.array_equal(o._bf16_of(dX1), dX1)
+    assert np.linalg.norm(dX1 - dX0) / np.linalg.norm(dX0) < 2 ** -5
+    for k in d0:
+        for a, b in zip(d0[k], d1[k]):
+            assert np.linalg.norm(a - b) / np.linalg.norm(a) < 2 ** -5
+
+
 # --------------------------------------------------------------------------
 # Optimiser state for the adapter (AdamW, fp32 and 8-bit blockwise)
 # --------------------------------------------------------------------------
