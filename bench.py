@@ -63,7 +63,7 @@ def _source_sha():
 
 class Clocks:
     """SM clock and clock-event reasons, read through NVML (read-only queries)
-    every 2 ms by a host thread with host timestamps.  mark() brackets the
+    as fast as NVML answers by a host thread with host timestamps.  mark() brackets the
     timed region; stop() summarises the samples inside it (falling back to
     all samples, and saying so, when the region was shorter than a few
     sampling periods).  nvidia-smi reads the same counters."""
@@ -94,15 +94,20 @@ class Clocks:
             return
 
         def run():
+            # the clock on every pass, the event reasons on every fourth (each
+            # NVML query takes a sizeable fraction of a millisecond)
             nv = self._nvml
+            rs, k = 0, 0
             while not self._stop:
                 try:
                     mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
-                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                    if k % 4 == 0:
+                        rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                    k += 1
                     self.samples.append((time.perf_counter(), mhz, rs))
                 except Exception:
                     pass
-                time.sleep(0.002)
+                time.sleep(0.0001)
 
         self._thread = threading.Thread(target=run, daemon=True)
         self._thread.start()
@@ -213,9 +218,10 @@ def _gemv_measure(q, syn, device, reps=20):
     call_ms = call_b.elapsed_time(call_e) / reps
     wbytes = copies[0].nbytes
     act = lin.M * lin.K * 2 + lin.r * lin.K * 2 + lin.N * lin.r * 2 + lin.M * lin.N * 2
+    # one byte count for both rates: the stored weight, X, A, B and Y
     return {"workload": GEMV_WORKLOAD, "kernel_us": kern_ms * 1e3, "call_us": call_ms * 1e3,
             "algorithmic_bytes": wbytes + act,
-            "kernel_GBps": (wbytes + lin.M * lin.K * 2) / (kern_ms * 1e-3) / 1e9,
+            "kernel_GBps": (wbytes + act) / (kern_ms * 1e-3) / 1e9,
             "call_GBps": (wbytes + act) / (call_ms * 1e-3) / 1e9}
 
 
@@ -514,6 +520,106 @@ def _export_measure(q, lins, ws, act, kind, device, reps=3):
             "dequantize_GBps": round(d_bytes / (d_ms * 1e-3) / 1e9, 1)}
 
 
+def _mlp_measure(q, syn, device, reps=6):
+    """Llama-7B MLP (gate, up 4096 -> 11008, down 11008 -> 4096, 8192 tokens,
+    r = 64, alpha = 16): each linear's forward + backward on its own (CUDA
+    events around the step and around its two dequant-GEMM launches), and the
+    chained SwiGLU block through qlora_mlp_forward / qlora_mlp_backward, whose
+    backward recomputes gate and up (checkpointing).  Weights and activations
+    are drawn on the GPU (timing does not depend on the values)."""
+    lins = syn.WORKLOADS["llama7b_mlp_m8192_r64"].layers
+    gen = torch.Generator(device=device).manual_seed(5)
+    M, r, gamma = lins[0].M, lins[0].r, lins[0].gamma
+    D, F = lins[0].K, lins[0].N
+    store, A, B = {}, {}, {}
+    for lin, name in zip(lins, ("gate", "up", "down")):
+        W = torch.randn(lin.N, lin.K, device=device, generator=gen) * lin.sigma
+        store[name] = q.qlora_quantize(W, check_finite=False)
+        del W
+        A[name] = (torch.randn(r, lin.K, device=device, generator=gen) / lin.K ** 0.5).bfloat16()
+        B[name] = (torch.randn(lin.N, r, device=device, generator=gen) * 0.01).bfloat16()
+    X = torch.randn(M, D, device=device, generator=gen).bfloat16()
+    dY = torch.randn(M, D, device=device, generator=gen).bfloat16()
+    dYf = torch.randn(M, F, device=device, generator=gen).bfloat16()
+    Hin = torch.randn(M, F, device=device, generator=gen).bfloat16()
+    peaks, _ = _peaks()
+    rows = []
+    total_flops, total_ms = 0, 0.0
+    for lin, name in zip(lins, ("gate", "up", "down")):
+        x = X if name != "down" else Hin
+        dy = dYf if name != "down" else dY
+        ws = q.workspace(M, lin.N, lin.K, r, device)
+        bufs = {"Y": torch.empty(M, lin.N, dtype=torch.bfloat16, device=device),
+                "T": torch.empty(M, r, dtype=torch.float32, device=device),
+                "dX": torch.empty(M, lin.K, dtype=torch.bfloat16, device=device),
+                "dA": torch.empty(r, lin.K, dtype=torch.float32, device=device),
+                "dB": torch.empty(lin.N, r, dtype=torch.float32, device=device)}
+        g = {"X": x, "A": A[name], "B": B[name], "dY": dy}
+        for _ in range(3):
+            _step(q, lin, store[name], g, bufs, ws)
+        torch.cuda.synchronize()
+        b, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        b.record()
+        for _ in range(reps):
+            _step(q, lin, store[name], g, bufs, ws)
+        e.record()
+        torch.cuda.synchronize()
+        ms = b.elapsed_time(e) / reps
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(reps)]
+        for i in range(reps):
+            _step(q, lin, store[name], g, bufs, ws, evs[i])
+        torch.cuda.synchronize()
+        if q.device_error_word(ws) != 0:
+            raise RuntimeError(f"device error word set in the {name} linear")
+        fwd = sum(v[0].elapsed_time(v[1]) for v in evs) / reps
+        dx = sum(v[2].elapsed_time(v[3]) for v in evs) / reps
+        f_gemm = 2 * M * lin.N * lin.K * 2 + 2 * M * r * (lin.N + lin.K)
+        flops = lin.fwd_bwd_flops()
+        total_flops += flops
+        total_ms += ms
+        rows.append({"linear": name, "N": lin.N, "K": lin.K, "ms": round(ms, 4),
+                     "TFLOPs": round(flops / (ms * 1e-3) / 1e12, 1),
+                     "gemm_fwd_us": round(fwd * 1e3, 1), "gemm_dx_us": round(dx * 1e3, 1),
+                     "gemm_TFLOPs": round(f_gemm / ((fwd + dx) * 1e-3) / 1e12, 1),
+                     "gemm_frac_bf16": round(f_gemm / ((fwd + dx) * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)})
+    mlp = q.MLP(store["gate"], store["up"], store["down"], A["gate"], B["gate"], A["up"], B["up"],
+                A["down"], B["down"])
+    ws = q.mlp_workspace(M, mlp, device)
+    Y = torch.empty(M, D, dtype=torch.bfloat16, device=device)
+    dX = torch.empty(M, D, dtype=torch.bfloat16, device=device)
+    grads = {}
+    for lin, name in zip(lins, ("gate", "up", "down")):
+        grads[f"dA_{name}"] = torch.empty(r, lin.K, dtype=torch.float32, device=device)
+        grads[f"dB_{name}"] = torch.empty(lin.N, r, dtype=torch.float32, device=device)
+
+    def chained():
+        q.qlora_mlp_forward(X, mlp, gamma, Y=Y, ws=ws)
+        q.qlora_mlp_backward(dY, X, mlp, gamma, dX=dX, grads=grads, ws=ws)
+
+    for _ in range(3):
+        chained()
+    torch.cuda.synchronize()
+    b, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b.record()
+    for _ in range(reps):
+        chained()
+    e.record()
+    torch.cuda.synchronize()
+    if q.device_error_word(ws) != 0:
+        raise RuntimeError("device error word set in the chained MLP")
+    cms = b.elapsed_time(e) / reps
+    recompute = sum(l.fwd_flops() for l in lins[:2])
+    return {"workload": "llama7b_mlp_m8192_r64", "per_linear": rows,
+            "independent_ms": round(total_ms, 3),
+            "independent_TFLOPs": round(total_flops / (total_ms * 1e-3) / 1e12, 1),
+            "independent_frac_bf16": round(total_flops / (total_ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+            "chained": {"step": "forward, then backward recomputing gate(x), up(x) and h",
+                        "ms": round(cms, 3), "algorithmic_flops": total_flops,
+                        "recompute_flops": recompute,
+                        "TFLOPs": round(total_flops / (cms * 1e-3) / 1e12, 1),
+                        "TFLOPs_with_recompute": round((total_flops + recompute) / (cms * 1e-3) / 1e12, 1)}}
+
+
 def run_gpu(args):
     import bit_nf4_quantised_b200 as q
     from bit_nf4_quantised_b200 import synthetic as syn
@@ -629,6 +735,10 @@ def run_gpu(args):
         except Exception as exc:           # an extra measurement never sinks the bench line
             out["adamw8"] = {"error": f"{type(exc).__name__}: {exc}"}
         try:
+            out["mlp"] = _mlp_measure(q, syn, device)
+        except Exception as exc:           # an extra measurement never sinks the bench line
+            out["mlp"] = {"error": f"{type(exc).__name__}: {exc}"}
+        try:
             out["formats"] = _format_measure(q, device)
             for row in out["formats"]:
                 row["dequantize_frac_hbm"] = round(row["dequantize_GBps"] / peaks["hbm_gbs"], 4)
@@ -714,19 +824,71 @@ class _OracleLayer:
         o.linear_backward(self.dY, self.X, Wt, self.A, self.B, lin.gamma)
 
 
-def _cpu_baseline(seconds: float = 10.0, sample_tokens: int = 256):
-    layer = _OracleLayer(sample_tokens)
-    layer.step()                                               # warm
+def _timed_passes(layer, seconds):
     n, t = 0, 0.0
     while t < seconds or n < 2:
         t0 = time.perf_counter()
         layer.step()
         t += time.perf_counter() - t0
         n += 1
-    return {"value": round(layer.flops * n / t / 1e12, 5), "unit": "TFLOP/s",
-            "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"{sample_tokens} of {layer.lin.M} tokens per pass, W dequantised once "
-                      f"per pass, fwd+bwd in fp64 numpy; {n} passes, {t:.1f} s"}
+    return n, t
+
+
+def _cpu_shape_rates(sample_tokens: int = 128):
+    """The oracle's rate on each distinct linear shape of the MLP and decoder
+    workloads (one pass over a token sample, W dequantised once), and the
+    times those rates give for the whole workloads, labelled extrapolated."""
+    from bit_nf4_quantised_b200 import synthetic as syn
+    from oracle import nf4_oracle as o
+    shapes = [("mlp.gate/up", 11008, 4096, 64, 8192, 2), ("mlp.down", 4096, 11008, 64, 8192, 1),
+              ("dec.qkvo", 4096, 4096, 16, 4096, 128), ("dec.gate/up", 11008, 4096, 16, 4096, 64),
+              ("dec.down", 4096, 11008, 16, 4096, 32)]
+    stores = {}
+    rows = []
+    totals = {"mlp": 0.0, "dec": 0.0}
+    for name, N, K, r, M_full, count in shapes:
+        lin = syn.Linear(name, sample_tokens, N, K, r, 2.0 * r, 0.02, False, N + K)
+        d = syn.make_layer(lin)
+        if (N, K) not in stores:
+            stores[(N, K)] = o.quantize(d["W"])
+        X, A, B, dY = (syn.as_f64(d[k]) for k in ("X", "A", "B", "dY"))
+        t0 = time.perf_counter()
+        Wt = o.dequantize(*stores[(N, K)], N, K).astype(np.float64)
+        o.linear_forward(X, Wt, A, B, lin.gamma)
+        o.linear_backward(dY, X, Wt, A, B, lin.gamma)
+        dt = time.perf_counter() - t0
+        rate = lin.fwd_bwd_flops() / dt
+        full = syn.Linear(name, M_full, N, K, r, 2.0 * r).fwd_bwd_flops() * count
+        totals[name.split(".")[0]] += full / rate
+        rows.append({"shape": f"{N}x{K}", "r": r, "role": name, "tokens_sampled": sample_tokens,
+                     "GFLOPs": round(rate / 1e9, 2)})
+    return rows, {"llama7b_mlp_m8192_r64_s": round(totals["mlp"], 1),
+                  "llama7b_decoder_32layers_m4096_r16_s": round(totals["dec"], 1),
+                  "label": "extrapolated: workload flops divided by the per-shape rates measured "
+                           f"on {sample_tokens}-token samples"}
+
+
+def _cpu_baseline(seconds: float = 10.0, sample_tokens: int = 256):
+    layer = _OracleLayer(sample_tokens)
+    layer.step()                                               # warm
+    n, t = _timed_passes(layer, seconds)
+    out = {"value": round(layer.flops * n / t / 1e12, 5), "unit": "TFLOP/s",
+           "cores": _blas_threads(), "kind": "oracle",
+           "sample": f"{sample_tokens} of {layer.lin.M} tokens per pass, W dequantised once "
+                     f"per pass, fwd+bwd in fp64 numpy; {n} passes, {t:.1f} s"}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1, user_api="blas"):
+            n1, t1 = _timed_passes(layer, seconds / 3)
+        out["one_thread"] = {"value": round(layer.flops * n1 / t1 / 1e12, 5), "cores": 1,
+                             "sample": f"the same pass on one BLAS thread; {n1} passes, {t1:.1f} s"}
+    except Exception as exc:               # an extra measurement never sinks the bench line
+        out["one_thread"] = {"error": f"{type(exc).__name__}: {exc}"}
+    try:
+        out["per_shape"], out["extrapolated"] = _cpu_shape_rates()
+    except Exception as exc:
+        out["per_shape"] = {"error": f"{type(exc).__name__}: {exc}"}
+    return out
 
 
 def run_reference(args):

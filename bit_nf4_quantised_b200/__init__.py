@@ -7,15 +7,19 @@ synthetic workload generator (``synthetic``).
 from ._lib import (  # noqa: F401
     EXPORTED,
     QLORA_SCALES_E4M3,
+    QLORA_SCALES_E5M2,
     QLORA_SCALES_FP32,
+    QLORA_SCALES_U8,
     Adam8State,
     Format,
+    MLP,
     adamw8_state,
     NF4Tensor,
     QloraError,
     device_error_word,
     empty_nf4,
     lib,
+    mlp_workspace,
     nf4_build_codebook,
     qlora_adamw8_step,
     qlora_dequantize,
@@ -25,6 +29,9 @@ from ._lib import (  # noqa: F401
     qlora_linear_forward,
     qlora_linear_workspace_size,
     qlora_merge,
+    qlora_mlp_backward,
+    qlora_mlp_forward,
+    qlora_mlp_workspace_size,
     qlora_quantize,
     qlora_quantize_bf16,
     qlora_quantize_fmt,

@@ -49,10 +49,15 @@ EXPORTED = (
     "qlora_dequantize_fmt",
     "qlora_adamw8_state_sizes",
     "qlora_adamw8_step",
+    "qlora_mlp_workspace_size",
+    "qlora_mlp_forward",
+    "qlora_mlp_backward",
 )
 
 QLORA_SCALES_FP32 = 0
 QLORA_SCALES_E4M3 = 1
+QLORA_SCALES_E5M2 = 2
+QLORA_SCALES_U8 = 3
 
 
 class QloraError(RuntimeError):
@@ -99,6 +104,19 @@ class _Format(ctypes.Structure):
     ]
 
 
+class _Mlp(ctypes.Structure):
+    _fields_ = [("gate", _Tensor), ("up", _Tensor), ("down", _Tensor),
+                ("A_gate", ctypes.c_void_p), ("B_gate", ctypes.c_void_p),
+                ("A_up", ctypes.c_void_p), ("B_up", ctypes.c_void_p),
+                ("A_down", ctypes.c_void_p), ("B_down", ctypes.c_void_p),
+                ("r", ctypes.c_int)]
+
+
+class _MlpGrads(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("dA_gate", "dB_gate", "dA_up", "dB_up", "dA_down", "dB_down")]
+
+
 class _AdamConfig(ctypes.Structure):
     _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
                 ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float),
@@ -135,6 +153,11 @@ def lib() -> ctypes.CDLL:
         L.qlora_adamw8_step.argtypes = [vp, vp, i64, vp, vp, vp, vp,
                                         ctypes.POINTER(_AdamConfig), vp, vp]
         L.qlora_linear_workspace_size.argtypes = [i64, i64, i64, i32, sz]
+        mp = ctypes.POINTER(_Mlp)
+        L.qlora_mlp_workspace_size.argtypes = [i64, mp, sz]
+        L.qlora_mlp_forward.argtypes = [vp, i64, mp, f32, vp, vp, ctypes.c_size_t, vp]
+        L.qlora_mlp_backward.argtypes = [vp, vp, i64, mp, f32, vp, ctypes.POINTER(_MlpGrads), i32,
+                                         vp, ctypes.c_size_t, vp]
         fwd = [vp, i64, tp, vp, vp, i32, f32, vp, vp, vp, ctypes.c_size_t, vp]
         bwd = [vp, vp, i64, tp, vp, vp, i32, f32, vp, vp, vp, vp, i32, vp, ctypes.c_size_t, vp]
         L.qlora_linear_forward.argtypes = fwd
@@ -270,7 +293,8 @@ def qlora_merge(w: NF4Tensor, A: torch.Tensor, B: torch.Tensor, scale: float,
 @dataclass
 class Format:
     """A quantisation format: codebook (ascending, up to 16 codes), blocksize
-    (power of two, 16..4096) and scale storage (QLORA_SCALES_FP32 or _E4M3)."""
+    (power of two, 16..4096) and scale storage (QLORA_SCALES_FP32, or an 8-bit
+    code: _E4M3, _E5M2 or _U8)."""
     codes: tuple
     block: int = BLOCK
     scales: int = QLORA_SCALES_E4M3
@@ -436,3 +460,82 @@ def device_error_word(ws: torch.Tensor) -> int:
     """The kernels' error word (first 4 bytes of the workspace); 0 = no error,
     bit 0 = a bounded wait inside the GEMM expired."""
     return int(ws[:4].view(torch.int32).item())
+
+
+# --------------------------------------------------------------------------
+@dataclass
+class MLP:
+    """The SwiGLU MLP of adapted NF4 linears: stored gate, up (F x D) and
+    down (D x F) weights and their bf16 adapters (A r x in, B out x r)."""
+    gate: NF4Tensor
+    up: NF4Tensor
+    down: NF4Tensor
+    A_gate: torch.Tensor
+    B_gate: torch.Tensor
+    A_up: torch.Tensor
+    B_up: torch.Tensor
+    A_down: torch.Tensor
+    B_down: torch.Tensor
+
+    @property
+    def r(self) -> int:
+        return self.A_gate.shape[0]
+
+    def c_struct(self) -> _Mlp:
+        for name in ("A_gate", "B_gate", "A_up", "B_up", "A_down", "B_down"):
+            _need(getattr(self, name), torch.bfloat16, name)
+        return _Mlp(self.gate.c_struct(), self.up.c_struct(), self.down.c_struct(),
+                    self.A_gate.data_ptr(), self.B_gate.data_ptr(), self.A_up.data_ptr(),
+                    self.B_up.data_ptr(), self.A_down.data_ptr(), self.B_down.data_ptr(), self.r)
+
+
+def qlora_mlp_workspace_size(M: int, mlp: MLP) -> int:
+    b = ctypes.c_size_t()
+    st = mlp.c_struct()
+    _check(lib().qlora_mlp_workspace_size(M, ctypes.byref(st), ctypes.byref(b)),
+           "qlora_mlp_workspace_size")
+    return b.value
+
+
+def mlp_workspace(M: int, mlp: MLP, device="cuda") -> torch.Tensor:
+    return torch.empty(max(qlora_mlp_workspace_size(M, mlp), 256), dtype=torch.uint8, device=device)
+
+
+def qlora_mlp_forward(X: torch.Tensor, mlp: MLP, scale: float, Y: torch.Tensor | None = None,
+                      ws: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y = down(silu(gate(X)) * up(X)); X [M, D] bf16."""
+    _need(X, torch.bfloat16, "X")
+    M, D = X.shape
+    Y = Y if Y is not None else torch.empty(M, D, dtype=torch.bfloat16, device=X.device)
+    _need(Y, torch.bfloat16, "Y")
+    ws = ws if ws is not None else mlp_workspace(M, mlp, X.device)
+    st = mlp.c_struct()
+    _check(lib().qlora_mlp_forward(X.data_ptr(), M, ctypes.byref(st), float(scale), Y.data_ptr(),
+                                   ws.data_ptr(), ws.numel(), _stream(stream)), "qlora_mlp_forward")
+    return Y
+
+
+def qlora_mlp_backward(dY: torch.Tensor, X: torch.Tensor, mlp: MLP, scale: float,
+                       dX: torch.Tensor | None = None, grads: dict | None = None,
+                       accumulate: bool = False, ws: torch.Tensor | None = None, stream=None):
+    """(dX, grads) of the MLP, recomputing its forward (checkpointing); grads
+    maps dA_gate, dB_gate, dA_up, dB_up, dA_down, dB_down to fp32 tensors."""
+    _need(dY, torch.bfloat16, "dY")
+    _need(X, torch.bfloat16, "X")
+    M, D = X.shape
+    dev = X.device
+    dX = dX if dX is not None else torch.empty(M, D, dtype=torch.bfloat16, device=dev)
+    if grads is None:
+        grads = {}
+        for lin, name in ((mlp.gate, "gate"), (mlp.up, "up"), (mlp.down, "down")):
+            grads[f"dA_{name}"] = torch.empty(mlp.r, lin.cols, dtype=torch.float32, device=dev)
+            grads[f"dB_{name}"] = torch.empty(lin.rows, mlp.r, dtype=torch.float32, device=dev)
+    g = _MlpGrads(*(grads[n].data_ptr() for n in
+                    ("dA_gate", "dB_gate", "dA_up", "dB_up", "dA_down", "dB_down")))
+    ws = ws if ws is not None else mlp_workspace(M, mlp, dev)
+    st = mlp.c_struct()
+    _check(lib().qlora_mlp_backward(dY.data_ptr(), X.data_ptr(), M, ctypes.byref(st), float(scale),
+                                    dX.data_ptr(), ctypes.byref(g), int(bool(accumulate)),
+                                    ws.data_ptr(), ws.numel(), _stream(stream)),
+           "qlora_mlp_backward")
+    return dX, grads

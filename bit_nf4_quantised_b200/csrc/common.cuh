@@ -389,4 +389,10 @@ __device__ __forceinline__ float e4m3_to_float(uint8_t code) {
     return __half2float(__half(h));
 }
 
+// Exact E5M2 -> fp32: E5M2 is the top byte of an fp16.
+__device__ __forceinline__ float e5m2_to_float(uint8_t code) {
+    __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(code), __NV_E5M2);
+    return __half2float(__half(h));
+}
+
 }  // namespace qnf4

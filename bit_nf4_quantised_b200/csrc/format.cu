@@ -1,6 +1,7 @@
 // K1 / K6 format variants: blockwise absmax quantisation with any codebook of
 // up to 16 codes, blocksizes 16 to 4096, and the block scales kept as fp32 or
-// double-quantised to FP8 E4M3 with one fp32 constant per 256 blocks.
+// double-quantised to an 8-bit code (FP8 E4M3 or E5M2, or a linear code)
+// with one fp32 constant per 256 blocks.
 //
 // "QLoRA, explained", "A toy run: how much does NF4 lose ...": the same scheme
 // with the E2M1 FP4 and symmetric INT4 codebooks and blocksizes 16 and 4096
@@ -10,7 +11,7 @@
 // it (a zero block and the padding of a final partial block take the index
 // nearest to 0), two indices per byte with the even element in the low
 // nibble; w~ = bf16_rne(fp32(q[idx] * c~_b)) with c~_b the fp32 absmax or
-// fp32(e4m3 * c2).
+// fp32(decode(code) * c2).
 //
 // Quantise: one CTA per group of 256 blocks.  A block is covered by
 // min(32, B/4) lanes that each load 16-byte pieces; the lanes reduce the
@@ -112,7 +113,7 @@ quantize_fmt_kernel(const float* __restrict__ W, int64_t numel, int64_t nblocks,
     const int64_t gblk = group * QLORA_GROUP + tid;
     const bool live = kFull || gblk < nblocks;
     const float c = sabs[tid];
-    if (f.scales_fp32) {
+    if (f.scale_fmt == QLORA_SCALES_FP32) {
         if (live) reinterpret_cast<float*>(scales)[gblk] = c;
         return;
     }
@@ -124,10 +125,20 @@ quantize_fmt_kernel(const float* __restrict__ W, int64_t numel, int64_t nblocks,
     float gmax = sred[0];
 #pragma unroll
     for (int w = 1; w < kThreads / 32; ++w) gmax = fmaxf(gmax, sred[w]);
-    const float c2 = __fdiv_rn(gmax, 448.0f);
+    // the format's largest code value: E4M3 448, E5M2 57344, linear 255
+    const float top = f.scale_fmt == QLORA_SCALES_E4M3 ? 448.0f
+                    : f.scale_fmt == QLORA_SCALES_E5M2 ? 57344.0f : 255.0f;
+    const float c2 = __fdiv_rn(gmax, top);
     uint8_t code = 0;
-    if (c2 > 0.f)
-        code = static_cast<uint8_t>(__nv_cvt_float_to_fp8(__fdiv_rn(c, c2), __NV_SATFINITE, __NV_E4M3));
+    if (c2 > 0.f) {
+        const float x = __fdiv_rn(c, c2);
+        if (f.scale_fmt == QLORA_SCALES_E4M3)
+            code = static_cast<uint8_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3));
+        else if (f.scale_fmt == QLORA_SCALES_E5M2)
+            code = static_cast<uint8_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E5M2));
+        else
+            code = static_cast<uint8_t>(fminf(rintf(x), 255.0f));       // ties to even
+    }
     if (live) reinterpret_cast<uint8_t*>(scales)[gblk] = code;
     if (tid == 0) meta[group] = c2;
 }
@@ -147,10 +158,16 @@ dequantize_fmt_kernel(const uint32_t* __restrict__ packed, const void* __restric
          u += int64_t(gridDim.x) * kThreads) {
         const uint32_t v = packed[u];
         const int64_t b = (u * 8) >> f.log2_block;
-        const float ct = f.scales_fp32
-                             ? reinterpret_cast<const float*>(scales)[b]
-                             : __fmul_rn(e4m3_to_float(reinterpret_cast<const uint8_t*>(scales)[b]),
-                                         meta[b >> 8]);
+        float ct;
+        if (f.scale_fmt == QLORA_SCALES_FP32) {
+            ct = reinterpret_cast<const float*>(scales)[b];
+        } else {
+            const uint8_t code = reinterpret_cast<const uint8_t*>(scales)[b];
+            const float d = f.scale_fmt == QLORA_SCALES_E4M3 ? e4m3_to_float(code)
+                          : f.scale_fmt == QLORA_SCALES_E5M2 ? e5m2_to_float(code)
+                                                            : static_cast<float>(code);
+            ct = __fmul_rn(d, meta[b >> 8]);
+        }
         uint32_t r[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j)
@@ -184,8 +201,9 @@ cudaError_t launch_quantize_fmt(const float* W, int64_t numel, const FmtArgs& f,
         // the single trailing group, offset so blockIdx.x is its group index
         const int64_t off = full * group_elems;
         const int64_t blk_off = full * QLORA_GROUP;
-        void* sc = f.scales_fp32 ? static_cast<void*>(static_cast<float*>(scales) + blk_off)
-                                 : static_cast<void*>(static_cast<uint8_t*>(scales) + blk_off);
+        void* sc = f.scale_fmt == QLORA_SCALES_FP32
+                       ? static_cast<void*>(static_cast<float*>(scales) + blk_off)
+                       : static_cast<void*>(static_cast<uint8_t*>(scales) + blk_off);
         quantize_fmt_kernel<false><<<1, kThreads, 0, stream>>>(
             W + off, numel - off, nblocks - blk_off, f, packed + off / 2, sc,
             meta == nullptr ? nullptr : meta + full, nonfinite_flag, tab);

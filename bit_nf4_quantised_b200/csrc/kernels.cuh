@@ -43,7 +43,8 @@ struct FmtTable {
 struct FmtArgs {
     int block;                 // power of two, 16..4096
     int log2_block;
-    int scales_fp32;           // 1: fp32 absmax per block; 0: E4M3 + fp32 per 256 blocks
+    int scale_fmt;             // a qlora_scale_format: fp32 absmax per block, or an 8-bit
+                               // code (E4M3, E5M2, linear) + an fp32 constant per 256 blocks
 };
 cudaError_t launch_quantize_fmt(const float* W, int64_t numel, const FmtArgs& f, uint8_t* packed,
                                 void* scales, float* meta, int* nonfinite_flag,
@@ -203,5 +204,17 @@ struct GemvFinalizeArgs {
     int64_t M, N;
 };
 cudaError_t launch_gemv_finalize(const GemvFinalizeArgs& a, cudaStream_t stream);
+
+// ----------------------------------------------- chained SwiGLU MLP (f3)
+// n = elements, a multiple of 8; H = bf16(silu(G) U); (G, U) <- (dG, dU);
+// C = bf16(A + B); dst = (accumulate ? dst : 0) | *a | *b | *c.
+cudaError_t launch_swiglu_forward(const uint16_t* G, const uint16_t* U, uint16_t* H, int64_t n,
+                                  int num_sms, cudaStream_t s);
+cudaError_t launch_swiglu_backward(uint16_t* G, uint16_t* U, const uint16_t* dH, int64_t n,
+                                   int num_sms, cudaStream_t s);
+cudaError_t launch_add_bf16(const uint16_t* A, const uint16_t* B, uint16_t* C, int64_t n,
+                            int num_sms, cudaStream_t s);
+cudaError_t launch_or_words(int* dst, const int* a, const int* b, const int* c, bool accumulate,
+                            cudaStream_t s);
 
 }  // namespace qnf4

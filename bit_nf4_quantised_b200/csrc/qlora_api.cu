@@ -298,7 +298,9 @@ int check_format(const qlora_format* f, FmtTable* t, FmtArgs* a) {
     const int b = f->block;
     if (b < 16 || b > 4096 || (b & (b - 1)) != 0) return QLORA_ERR_UNSUPPORTED;
     if (f->ncodes < 2 || f->ncodes > 16) return QLORA_ERR_UNSUPPORTED;
-    if (f->scales != QLORA_SCALES_FP32 && f->scales != QLORA_SCALES_E4M3) return QLORA_ERR_UNSUPPORTED;
+    if (f->scales != QLORA_SCALES_FP32 && f->scales != QLORA_SCALES_E4M3 &&
+        f->scales != QLORA_SCALES_E5M2 && f->scales != QLORA_SCALES_U8)
+        return QLORA_ERR_UNSUPPORTED;
     for (int i = 0; i < f->ncodes; ++i) {
         if (!std::isfinite(f->codes[i])) return QLORA_ERR_UNSUPPORTED;
         if (i > 0 && !(f->codes[i] > f->codes[i - 1])) return QLORA_ERR_UNSUPPORTED;
@@ -322,7 +324,7 @@ int check_format(const qlora_format* f, FmtTable* t, FmtArgs* a) {
         a->block = b;
         a->log2_block = 0;
         while ((1 << a->log2_block) < b) ++a->log2_block;
-        a->scales_fp32 = f->scales == QLORA_SCALES_FP32 ? 1 : 0;
+        a->scale_fmt = f->scales;
     }
     return QLORA_OK;
 }
@@ -512,7 +514,7 @@ int qlora_quantize_fmt(const float* W, int64_t numel, const qlora_format* f, uin
     if (st != QLORA_OK) return st;
     if (numel < 0) return QLORA_ERR_SHAPE;
     if (numel == 0) return QLORA_OK;
-    if (!W || !packed || !scales || (!a.scales_fp32 && !meta)) return QLORA_ERR_NULL;
+    if (!W || !packed || !scales || (a.scale_fmt != QLORA_SCALES_FP32 && !meta)) return QLORA_ERR_NULL;
     if (!aligned(W, 16) || !aligned(packed, 16) || !aligned(scales, 4) || (meta && !aligned(meta, 4)))
         return QLORA_ERR_ALIGN;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -531,7 +533,7 @@ int qlora_dequantize_fmt(const uint8_t* packed, const void* scales, const float*
     if (st != QLORA_OK) return st;
     if (numel < 0) return QLORA_ERR_SHAPE;
     if (numel == 0) return QLORA_OK;
-    if (!packed || !scales || !out || (!a.scales_fp32 && !meta)) return QLORA_ERR_NULL;
+    if (!packed || !scales || !out || (a.scale_fmt != QLORA_SCALES_FP32 && !meta)) return QLORA_ERR_NULL;
     if (!aligned(packed, 16) || !aligned(out, 16) || !aligned(scales, 4) || (meta && !aligned(meta, 4)))
         return QLORA_ERR_ALIGN;
     return cuda_status(launch_dequantize_fmt(packed, scales, meta, numel, a, out, t, num_sms(),
@@ -841,6 +843,178 @@ int qlora_linear_backward(const uint16_t* dY, const uint16_t* X, int64_t M,
                           int accumulate, void* ws, size_t ws_bytes, qlora_stream_t stream) {
     return qlora_linear_backward_ex(dY, X, M, w, A, B, r, scale, T_saved, dX, dA, dB, accumulate,
                                     ws, ws_bytes, stream, nullptr);
+}
+
+// ------------------------------------------------ chained SwiGLU MLP (f3)
+}  // extern "C"
+
+namespace {
+
+struct MlpPlan {
+    int64_t D, F;
+    size_t lin;                          // one linear call's workspace
+    // linear calls' workspaces, each keeping its own error word: [0] gate
+    // and [1] up forward (or recompute), [2] down, [3] gate and [4] up backward
+    int64_t off_lin[5], off_g, off_u, off_h, off_dh, off_dxg, off_tg, off_tu, total;
+};
+
+int mlp_plan(int64_t M, const qlora_mlp* m, MlpPlan* p) {
+    if (!m) return QLORA_ERR_NULL;
+    int st = check_tensor(&m->gate);
+    if (st == QLORA_OK) st = check_tensor(&m->up);
+    if (st == QLORA_OK) st = check_tensor(&m->down);
+    if (st != QLORA_OK) return st;
+    const int64_t F = m->gate.rows, D = m->gate.cols;
+    if (m->up.rows != F || m->up.cols != D || m->down.rows != D || m->down.cols != F)
+        return QLORA_ERR_SHAPE;
+    if (M < 0) return QLORA_ERR_SHAPE;
+    st = check_linear_shapes(M, F, D, m->r);
+    if (st == QLORA_OK) st = check_linear_shapes(M, D, F, m->r);
+    if (st != QLORA_OK) return st;
+    p->D = D;
+    p->F = F;
+    p->lin = static_cast<size_t>(std::max(make_plan(M, F, D, m->r).total, make_plan(M, D, F, m->r).total));
+    int64_t o = kAlign;                                   // header: the call's error word
+    for (int i = 0; i < 5; ++i) {
+        p->off_lin[i] = o;
+        o += up(static_cast<int64_t>(p->lin), kAlign);
+    }
+    const int64_t mf = up(M * F * 2, kAlign);
+    p->off_g = o;   o += mf;
+    p->off_u = o;   o += mf;
+    p->off_h = o;   o += mf;
+    p->off_dh = o;  o += mf;
+    p->off_dxg = o; o += up(M * D * 2, kAlign);
+    p->off_tg = o;  o += up(M * m->r * 4, kAlign);
+    p->off_tu = o;  o += up(M * m->r * 4, kAlign);
+    p->total = o;
+    return QLORA_OK;
+}
+
+int check_mlp_adapters(const qlora_mlp* m) {
+    if (!m->A_gate || !m->B_gate || !m->A_up || !m->B_up || !m->A_down || !m->B_down)
+        return QLORA_ERR_NULL;
+    return QLORA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qlora_mlp_workspace_size(int64_t M, const qlora_mlp* mlp, size_t* bytes) {
+    if (!bytes) return QLORA_ERR_NULL;
+    MlpPlan p;
+    const int st = mlp_plan(M, mlp, &p);
+    if (st != QLORA_OK) return st;
+    *bytes = static_cast<size_t>(p.total);
+    return QLORA_OK;
+}
+
+int qlora_mlp_forward(const uint16_t* X, int64_t M, const qlora_mlp* mlp, float scale, uint16_t* Y,
+                      void* ws, size_t ws_bytes, qlora_stream_t stream) {
+    MlpPlan p;
+    int st = mlp_plan(M, mlp, &p);
+    if (st != QLORA_OK) return st;
+    st = check_mlp_adapters(mlp);
+    if (st != QLORA_OK) return st;
+    if (M != 0 && (!X || !Y)) return QLORA_ERR_NULL;
+    if (!aligned(X, 16) || !aligned(Y, 16)) return QLORA_ERR_ALIGN;
+    if (!ws || ws_bytes < static_cast<size_t>(p.total)) return QLORA_ERR_WORKSPACE;
+    if (!aligned(ws, kAlign)) return QLORA_ERR_ALIGN;
+    if (M == 0) return QLORA_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint16_t* G = at<uint16_t>(ws, p.off_g);
+    uint16_t* U = at<uint16_t>(ws, p.off_u);
+    uint16_t* H = at<uint16_t>(ws, p.off_h);
+    const int r = mlp->r;
+    void* w0 = at<void>(ws, p.off_lin[0]);
+    void* w1 = at<void>(ws, p.off_lin[1]);
+    void* w2 = at<void>(ws, p.off_lin[2]);
+    st = qlora_linear_forward(X, M, &mlp->gate, mlp->A_gate, mlp->B_gate, r, scale, G, nullptr, w0,
+                              p.lin, stream);
+    if (st == QLORA_OK)
+        st = qlora_linear_forward(X, M, &mlp->up, mlp->A_up, mlp->B_up, r, scale, U, nullptr, w1,
+                                  p.lin, stream);
+    if (st != QLORA_OK) return st;
+    QTRY(launch_swiglu_forward(G, U, H, M * p.F, num_sms(), s));
+    st = qlora_linear_forward(H, M, &mlp->down, mlp->A_down, mlp->B_down, r, scale, Y, nullptr, w2,
+                              p.lin, stream);
+    if (st != QLORA_OK) return st;
+    QTRY(launch_or_words(at<int>(ws, 0), at<int>(ws, p.off_lin[0]), at<int>(ws, p.off_lin[1]),
+                         at<int>(ws, p.off_lin[2]), false, s));
+    return QLORA_OK;
+}
+
+int qlora_mlp_backward(const uint16_t* dY, const uint16_t* X, int64_t M, const qlora_mlp* mlp,
+                       float scale, uint16_t* dX, const qlora_mlp_grads* g, int accumulate,
+                       void* ws, size_t ws_bytes, qlora_stream_t stream) {
+    MlpPlan p;
+    int st = mlp_plan(M, mlp, &p);
+    if (st != QLORA_OK) return st;
+    st = check_mlp_adapters(mlp);
+    if (st != QLORA_OK) return st;
+    if (!g || !g->dA_gate || !g->dB_gate || !g->dA_up || !g->dB_up || !g->dA_down || !g->dB_down)
+        return QLORA_ERR_NULL;
+    if (M != 0 && (!dY || !X || !dX)) return QLORA_ERR_NULL;
+    if (!aligned(dY, 16) || !aligned(X, 16) || !aligned(dX, 16)) return QLORA_ERR_ALIGN;
+    if (!ws || ws_bytes < static_cast<size_t>(p.total)) return QLORA_ERR_WORKSPACE;
+    if (!aligned(ws, kAlign)) return QLORA_ERR_ALIGN;
+    const int r = mlp->r;
+    void* w0 = at<void>(ws, p.off_lin[0]);
+    void* w1 = at<void>(ws, p.off_lin[1]);
+    void* w2 = at<void>(ws, p.off_lin[2]);
+    void* w3 = at<void>(ws, p.off_lin[3]);
+    void* w4 = at<void>(ws, p.off_lin[4]);
+    if (M == 0) {
+        // empty batch: the linear backwards write zero gradients (or leave
+        // them when accumulating)
+        st = qlora_linear_backward(nullptr, nullptr, 0, &mlp->down, mlp->A_down, mlp->B_down, r,
+                                   scale, nullptr, nullptr, g->dA_down, g->dB_down, accumulate, w2,
+                                   p.lin, stream);
+        if (st == QLORA_OK)
+            st = qlora_linear_backward(nullptr, nullptr, 0, &mlp->gate, mlp->A_gate, mlp->B_gate, r,
+                                       scale, nullptr, nullptr, g->dA_gate, g->dB_gate, accumulate,
+                                       w0, p.lin, stream);
+        if (st == QLORA_OK)
+            st = qlora_linear_backward(nullptr, nullptr, 0, &mlp->up, mlp->A_up, mlp->B_up, r, scale,
+                                       nullptr, nullptr, g->dA_up, g->dB_up, accumulate, w1, p.lin,
+                                       stream);
+        return st;
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint16_t* G = at<uint16_t>(ws, p.off_g);
+    uint16_t* U = at<uint16_t>(ws, p.off_u);
+    uint16_t* H = at<uint16_t>(ws, p.off_h);
+    uint16_t* dH = at<uint16_t>(ws, p.off_dh);
+    uint16_t* dXg = at<uint16_t>(ws, p.off_dxg);
+    float* Tg = at<float>(ws, p.off_tg);
+    float* Tu = at<float>(ws, p.off_tu);
+    // recompute (checkpointing): gate(x), up(x) with their T = X A^T, h
+    st = qlora_linear_forward(X, M, &mlp->gate, mlp->A_gate, mlp->B_gate, r, scale, G, Tg, w0, p.lin,
+                              stream);
+    if (st == QLORA_OK)
+        st = qlora_linear_forward(X, M, &mlp->up, mlp->A_up, mlp->B_up, r, scale, U, Tu, w1, p.lin,
+                                  stream);
+    if (st != QLORA_OK) return st;
+    QTRY(launch_swiglu_forward(G, U, H, M * p.F, num_sms(), s));
+    // down: dH, dA_down, dB_down (its T recomputed from h)
+    st = qlora_linear_backward(dY, H, M, &mlp->down, mlp->A_down, mlp->B_down, r, scale, nullptr, dH,
+                               g->dA_down, g->dB_down, accumulate, w2, p.lin, stream);
+    if (st != QLORA_OK) return st;
+    // SwiGLU backward: (G, U) <- (dG, dU)
+    QTRY(launch_swiglu_backward(G, U, dH, M * p.F, num_sms(), s));
+    st = qlora_linear_backward(G, X, M, &mlp->gate, mlp->A_gate, mlp->B_gate, r, scale, Tg, dXg,
+                               g->dA_gate, g->dB_gate, accumulate, w3, p.lin, stream);
+    if (st == QLORA_OK)
+        st = qlora_linear_backward(U, X, M, &mlp->up, mlp->A_up, mlp->B_up, r, scale, Tu, dX,
+                                   g->dA_up, g->dB_up, accumulate, w4, p.lin, stream);
+    if (st != QLORA_OK) return st;
+    QTRY(launch_add_bf16(dX, dXg, dX, M * p.D, num_sms(), s));
+    QTRY(launch_or_words(at<int>(ws, 0), at<int>(ws, p.off_lin[0]), at<int>(ws, p.off_lin[1]),
+                         at<int>(ws, p.off_lin[2]), false, s));
+    QTRY(launch_or_words(at<int>(ws, 0), at<int>(ws, p.off_lin[3]), at<int>(ws, p.off_lin[4]),
+                         at<int>(ws, p.off_lin[4]), true, s));
+    return QLORA_OK;
 }
 
 }  // extern "C"

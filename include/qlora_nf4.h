@@ -164,22 +164,33 @@ QLORA_API int qlora_dequantize(const qlora_nf4_tensor* w, uint16_t* W_out,
  * ..."): the same blockwise absmax quantisation with another codebook (the
  * page compares E2M1 FP4 and a symmetric 15-level INT4 grid with NF4) and
  * blocksize (16 and 4096 next to 64), with the block scales either kept as
- * fp32 or double-quantised as in "Double quantisation".
+ * fp32 or double-quantised as in "Double quantisation" ("8-bit floats", no
+ * format named: E4M3, E5M2, or a linear 8-bit code).
  * The stored layout generalises the NF4 one: nblocks = ceil(numel / block);
  *   packed : nblocks * block / 2 bytes, two indices per byte, the even
  *            element in the low nibble; a final partial block is padded with
  *            the index of the code nearest 0.
  *   scales : QLORA_SCALES_FP32 -- nblocks fp32, the block absmax c_b;
- *            QLORA_SCALES_E4M3 -- nblocks bytes of FP8 E4M3 codes of c_b / c2,
- *            with meta = ceil(nblocks / 256) fp32 constants c2 (as NF4).
+ *            otherwise nblocks bytes of 8-bit codes of c_b / c2, with meta =
+ *            ceil(nblocks / 256) fp32 constants c2 = fp32(max c_b / TOP):
+ *            QLORA_SCALES_E4M3 -- FP8 E4M3 (as NF4), TOP = 448;
+ *            QLORA_SCALES_E5M2 -- FP8 E5M2, TOP = 57344;
+ *            QLORA_SCALES_U8   -- linear, code = rint(fp32(c_b / c2)) (ties to
+ *                                 even), TOP = 255.
+ *            The FP8 codes round to nearest even and saturate at TOP.
  * Index of a weight: the number of midpoints strictly below fp32(w / c_b),
  * midpoint i being the exact average of codes i and i+1 rounded to fp32; a
  * zero block takes the index of the code nearest 0.  Dequantisation:
- * w~ = bf16_rne(fp32(codes[idx] * c~_b)), c~_b = c_b or fp32(e4m3 * c2).
+ * w~ = bf16_rne(fp32(codes[idx] * c~_b)), c~_b = c_b or fp32(decode(code) * c2).
  * With the NF4 codebook, block 64 and E4M3 scales the layout and every byte
  * equal those of qlora_quantize.
  */
-typedef enum { QLORA_SCALES_FP32 = 0, QLORA_SCALES_E4M3 = 1 } qlora_scale_format;
+typedef enum {
+    QLORA_SCALES_FP32 = 0,
+    QLORA_SCALES_E4M3 = 1,
+    QLORA_SCALES_E5M2 = 2,
+    QLORA_SCALES_U8 = 3
+} qlora_scale_format;
 
 typedef struct {
     int32_t block;       /* elements per block: a power of two, 16 ... 4096   */
@@ -385,6 +396,86 @@ QLORA_API int qlora_linear_backward(const uint16_t* dY, const uint16_t* X, int64
                           const float* T_saved, uint16_t* dX, float* dA,
                           float* dB, int accumulate, void* ws, size_t ws_bytes,
                           qlora_stream_t stream);
+
+/*
+ * Layer chaining with gradient checkpointing: the SwiGLU MLP of adapted NF4
+ * linears, y = down(silu(gate(x)) * up(x)) ("QLoRA, explained", "The
+ * algorithm, step by step": the training step runs with gradient
+ * checkpointing enabled; "Compute and memory cost": checkpointing is
+ * effectively mandatory, and the recomputed forward dequantises every block
+ * a third time per step).  The pages print no block structure; this is the
+ * MLP of the Llama-shaped models.  gate and up are F x D stored weights, down
+ * is D x F, each with its own LoRA adapter of rank r, all with the same
+ * scale gamma.  silu(z) = z / (1 + exp(-z)).
+ */
+typedef struct {
+    qlora_nf4_tensor gate, up, down;   /* F x D, F x D, D x F               */
+    const uint16_t* A_gate;            /* bf16 r x D (device, read)         */
+    const uint16_t* B_gate;            /* bf16 F x r                        */
+    const uint16_t* A_up;              /* bf16 r x D                        */
+    const uint16_t* B_up;              /* bf16 F x r                        */
+    const uint16_t* A_down;            /* bf16 r x F                        */
+    const uint16_t* B_down;            /* bf16 D x r                        */
+    int r;                             /* 8 <= r <= 128, r % 8 == 0         */
+} qlora_mlp;
+
+/* Adapter gradients of the MLP (device fp32, written or accumulated):
+ * dA_* r x (input features), dB_* (output features) x r. */
+typedef struct {
+    float* dA_gate;
+    float* dB_gate;
+    float* dA_up;
+    float* dB_up;
+    float* dA_down;
+    float* dB_down;
+} qlora_mlp_grads;
+
+/*
+ * qlora_mlp_workspace_size -- bytes of device workspace qlora_mlp_forward and
+ * qlora_mlp_backward need for M tokens (the intermediate activations gate(x),
+ * up(x), h and dh in bf16, M x F each, plus each linear call's own
+ * workspace).  Host only.
+ * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE (negative M, or the three weights'
+ * shapes not F x D, F x D, D x F), QLORA_ERR_ALIGN, QLORA_ERR_UNSUPPORTED (a
+ * linear's shape rules, D and F both taking the roles of N and K).
+ */
+QLORA_API int qlora_mlp_workspace_size(int64_t M, const qlora_mlp* mlp, size_t* bytes);
+
+/*
+ * qlora_mlp_forward -- Y = down(silu(gate(X)) * up(X)), every linear the
+ * adapted layer of qlora_linear_forward; gate(x) and up(x) are rounded to
+ * bf16, h = bf16(silu(g) * u) in fp32 from them.
+ *   X (device, bf16, M x D, read); Y (device, bf16, M x D, written); nothing
+ *   else is kept for the backward (checkpointing: it recomputes from X).
+ *   ws: >= qlora_mlp_workspace_size bytes, 256-byte aligned; its first 4
+ *   bytes then hold the OR of the linear calls' error words (as
+ *   qlora_linear_forward documents).
+ * M = 0 launches nothing.
+ * Errors: those of qlora_mlp_workspace_size and qlora_linear_forward.
+ */
+QLORA_API int qlora_mlp_forward(const uint16_t* X, int64_t M, const qlora_mlp* mlp, float scale,
+                                uint16_t* Y, void* ws, size_t ws_bytes, qlora_stream_t stream);
+
+/*
+ * qlora_mlp_backward -- gradients of the MLP with the stored weights frozen,
+ * recomputing the forward (the third dequantisation of gate and up):
+ *   g = gate(X), u = up(X) (with their X A^T), h = silu(g) * u;
+ *   dh, dA_down, dB_down from the down layer's backward at input h;
+ *   dg = dh * u * silu'(g), du = dh * silu(g)  (silu' = s (1 + z (1 - s)),
+ *   s the logistic sigmoid), rounded to bf16;
+ *   dX = (dg's backward through gate) + (du's through up), each bf16, summed
+ *   in fp32 and rounded; dA, dB of gate and up.
+ *   dY (device, bf16, M x D, read); X (device, bf16, M x D, read);
+ *   dX (device, bf16, M x D, written); grads (host struct of device
+ *   pointers); accumulate != 0 adds to the adapter gradients.
+ *   ws as qlora_mlp_forward (error word: OR over every linear call).
+ * M = 0 writes zero adapter gradients (or leaves them when accumulating).
+ * Errors: those of qlora_mlp_forward and qlora_linear_backward.
+ */
+QLORA_API int qlora_mlp_backward(const uint16_t* dY, const uint16_t* X, int64_t M,
+                                 const qlora_mlp* mlp, float scale, uint16_t* dX,
+                                 const qlora_mlp_grads* grads, int accumulate, void* ws,
+                                 size_t ws_bytes, qlora_stream_t stream);
 
 /*
  * Profiling variants.  Identical to qlora_linear_forward / _backward, plus

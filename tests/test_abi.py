@@ -139,10 +139,11 @@ def _books():
 
 @pytest.mark.parametrize("numel", [0, 1, 100, 4096 * 4096, 2 ** 20 + 17])
 @pytest.mark.parametrize("block", [16, 64, 4096])
-@pytest.mark.parametrize("scales", ["fp32", "e4m3"])
+@pytest.mark.parametrize("scales", ["fp32", "e4m3", "e5m2", "u8"])
 def test_format_sizes_match_oracle(q, numel, block, scales):
-    f = q.Format(_books()["fp4"], block,
-                 q.QLORA_SCALES_FP32 if scales == "fp32" else q.QLORA_SCALES_E4M3)
+    enum = {"fp32": q.QLORA_SCALES_FP32, "e4m3": q.QLORA_SCALES_E4M3,
+            "e5m2": q.QLORA_SCALES_E5M2, "u8": q.QLORA_SCALES_U8}[scales]
+    f = q.Format(_books()["fp4"], block, enum)
     assert q.qlora_format_sizes(numel, f) == o.format_nbytes(numel, block, scales)
 
 
@@ -165,6 +166,9 @@ def test_format_validation_before_any_launch(q):
     assert st(q.Format((0.0, 0.5, 0.5), 64)) == E.QLORA_ERR_UNSUPPORTED   # not strictly ascending
     assert st(q.Format((0.0, float("nan")), 64)) == E.QLORA_ERR_UNSUPPORTED
     assert st(q.Format(good.codes, 64, 7)) == E.QLORA_ERR_UNSUPPORTED
+    assert st(q.Format(good.codes, 64, 4)) == E.QLORA_ERR_UNSUPPORTED
+    for enc in (q.QLORA_SCALES_E5M2, q.QLORA_SCALES_U8):
+        assert st(q.Format(good.codes, 64, enc)) == E.QLORA_OK
     assert st(good, -1) == E.QLORA_ERR_SHAPE
     assert L.qlora_format_sizes(10, None, ctypes.byref(p), ctypes.byref(c), ctypes.byref(m)) == E.QLORA_ERR_NULL
     f = good.c_struct()

@@ -1,6 +1,7 @@
 """GPU parity of the format variants (qlora_quantize_fmt / qlora_dequantize_fmt)
 against the oracle through the C-ABI: NF4, E2M1 FP4 and INT4 codebooks,
-blocksizes 16 to 4096, fp32 or double-quantised scales, bit-exact indices,
+blocksizes 16 to 4096, fp32 scales or scales double-quantised to E4M3, E5M2
+or a linear 8-bit code, bit-exact indices,
 scales and dequantised bf16; and the toy statistics of "A toy run ..."
 (relative MSE on 2^20 Gaussian weights) reproduced from the GPU's outputs."""
 from __future__ import annotations
@@ -29,8 +30,9 @@ BOOKS = {"nf4": o.nf4_codebook()[0], "fp4": o.fp4_e2m1_codebook(), "int4": o.int
 
 
 def _fmt(q, cb, block, scales):
-    return q.Format(tuple(float(c) for c in BOOKS[cb]), block,
-                    q.QLORA_SCALES_FP32 if scales == o.SCALES_FP32 else q.QLORA_SCALES_E4M3)
+    enum = {o.SCALES_FP32: q.QLORA_SCALES_FP32, o.SCALES_E4M3: q.QLORA_SCALES_E4M3,
+            o.SCALES_E5M2: q.QLORA_SCALES_E5M2, o.SCALES_U8: q.QLORA_SCALES_U8}[scales]
+    return q.Format(tuple(float(c) for c in BOOKS[cb]), block, enum)
 
 
 CASES = [
@@ -42,6 +44,11 @@ CASES = [
     ("fp4", 512, o.SCALES_FP32, 512 * 300 + 1),
     ("int4", 4096, o.SCALES_E4M3, 4096 * 256 + 4096 * 3 + 77),
     ("nf4", 64, o.SCALES_E4M3, 1),
+    # the other 8-bit encodings of the double-quantised scales
+    ("nf4", 64, o.SCALES_E5M2, 64 * 256 * 3 + 130),
+    ("nf4", 64, o.SCALES_U8, 64 * 256 * 3 + 130),
+    ("fp4", 16, o.SCALES_E5M2, 16 * 256 * 2 + 9),
+    ("int4", 1024, o.SCALES_U8, 1024 * 256 + 1024 * 5 + 3),
 ]
 
 
@@ -115,3 +122,24 @@ def test_toy_statistics_from_the_gpu(q):
         sq = 10 * math.log10(100 / got[f"gauss_{cb}_b64"])
         ref, tol = t[f"sqnr_{cb}_db"]
         assert abs(sq - ref) <= tol + 2e-3, (cb, sq, ref)
+
+
+def test_scale_encodings_on_the_toy_from_the_gpu(q):
+    """NF4 at blocksize 64 on the toy's 2^20 N(0, 0.02^2) weights with each
+    8-bit scale encoding: the GPU's dequantised weights equal the oracle's
+    bit for bit, and the relative errors order fp32 < linear < E4M3 < E5M2."""
+    rng = np.random.default_rng(0)
+    w = rng.normal(0, 0.02, 2 ** 20).astype(np.float32)
+    wd = torch.from_numpy(w).cuda()
+    w64 = w.astype(np.float64)
+    rel = {}
+    for scales in (o.SCALES_FP32, o.SCALES_U8, o.SCALES_E4M3, o.SCALES_E5M2):
+        f = _fmt(q, "nf4", 64, scales)
+        packed, sc, meta = q.qlora_quantize_fmt(wd, f)
+        bits = q.qlora_dequantize_fmt(packed, sc, meta, w.size, f).view(torch.int16).cpu().numpy()
+        p0, s0, m0 = o.quantize_fmt(w, BOOKS["nf4"], 64, scales)
+        ref = o.dequantize_fmt_bits(p0, s0, m0, w.size, BOOKS["nf4"], 64, scales)
+        assert np.array_equal(bits.view(np.uint16), ref), scales
+        rec = o.bf16_bits_to_float(ref).astype(np.float64)
+        rel[scales] = float(np.sum((rec - w64) ** 2) / np.sum(w64 ** 2))
+    assert rel[o.SCALES_FP32] < rel[o.SCALES_U8] < rel[o.SCALES_E4M3] < rel[o.SCALES_E5M2]
