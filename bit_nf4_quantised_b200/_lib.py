@@ -49,6 +49,7 @@ EXPORTED = (
     "qlora_dequantize_fmt",
     "qlora_adamw8_state_sizes",
     "qlora_adamw8_step",
+    "qlora_set_gemm_wait_limit_us",
     "qlora_mlp_workspace_size",
     "qlora_mlp_forward",
     "qlora_mlp_backward",
@@ -153,6 +154,7 @@ def lib() -> ctypes.CDLL:
         L.qlora_adamw8_step.argtypes = [vp, vp, i64, vp, vp, vp, vp,
                                         ctypes.POINTER(_AdamConfig), vp, vp]
         L.qlora_linear_workspace_size.argtypes = [i64, i64, i64, i32, sz]
+        L.qlora_set_gemm_wait_limit_us.argtypes = [i64]
         mp = ctypes.POINTER(_Mlp)
         L.qlora_mlp_workspace_size.argtypes = [i64, mp, sz]
         L.qlora_mlp_forward.argtypes = [vp, i64, mp, f32, vp, vp, ctypes.c_size_t, vp]

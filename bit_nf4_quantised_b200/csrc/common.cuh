@@ -71,18 +71,39 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking test of the phase (try_wait may suspend the thread inside the
+// instruction until the phase completes or a system-defined time passes).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait until the phase with the given parity has completed.  Gives up (and
-// returns false) when *abort_flag becomes non-zero or after kWaitLimitNs; a
-// timeout sets kErrWaitTimeout in *err and raises *abort_flag.
+// returns false) when *abort_flag becomes non-zero or after limit_ns; a
+// timeout sets kErrWaitTimeout in *err and raises *abort_flag.  A limit
+// below the default polls with the non-blocking test, checks after every
+// poll and counts SM clock cycles (%globaltimer may tick far more coarsely
+// than a microsecond), so that even a limit of a microsecond is honoured:
+// limit_ns cycles, at most limit_ns nanoseconds at SM clocks of 1 GHz and up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile int* abort_flag, int* err) {
-    if (mbar_try_wait(bar, parity)) return true;
+                                          volatile int* abort_flag, int* err,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
+    const bool poll = limit_ns < kWaitLimitNs;
+    if (poll ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
+    const long long c0 = clock64();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0) {
+        if (poll ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
+        if (poll || (it & 63u) == 0) {
             if (abort_flag != nullptr && *abort_flag) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (poll ? clock64() - c0 > static_cast<long long>(limit_ns) : globaltimer_ns() - t0 > limit_ns) {
                 if (err != nullptr) atomicOr(err, kErrWaitTimeout);
                 if (abort_flag != nullptr) *abort_flag = 1;
                 return false;
@@ -267,16 +288,31 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
     return ok != 0;
 }
 
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // As mbar_wait, with cluster-scope acquire (arrivals may come from the peer).
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort_flag, int* err) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
+                                                  volatile int* abort_flag, int* err,
+                                                  unsigned long long limit_ns = kWaitLimitNs) {
+    const bool poll = limit_ns < kWaitLimitNs;
+    if (poll ? mbar_test_wait_cluster(bar, parity) : mbar_try_wait_cluster(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
+    const long long c0 = clock64();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait_cluster(bar, parity)) return true;
-        if ((it & 63u) == 0) {
+        if (poll ? mbar_test_wait_cluster(bar, parity) : mbar_try_wait_cluster(bar, parity)) return true;
+        if (poll || (it & 63u) == 0) {
             if (abort_flag != nullptr && *abort_flag) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (poll ? clock64() - c0 > static_cast<long long>(limit_ns) : globaltimer_ns() - t0 > limit_ns) {
                 if (err != nullptr) atomicOr(err, kErrWaitTimeout);
                 if (abort_flag != nullptr) *abort_flag = 1;
                 return false;

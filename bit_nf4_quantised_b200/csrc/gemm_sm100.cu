@@ -219,7 +219,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
                 for (int step = 0; step < total_steps; ++step, ++gstep) {
                     const int s = gstep % kStages;
                     const uint32_t ph = (gstep / kStages) & 1;
-                    if (!mbar_wait(&bars->empty[s], ph ^ 1, abort_flag, a.err)) {
+                    if (!mbar_wait(&bars->empty[s], ph ^ 1, abort_flag, a.err, a.wait_ns)) {
                         ok = false;
                         break;
                     }
@@ -282,7 +282,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
                 // the accumulators are free once both CTAs' epilogues of the
                 // previous tile have read them
                 if (tile > 0) {
-                    ok = mbar_wait_cluster(&bars->acc_empty, (tile - 1) & 1, abort_flag, a.err);
+                    ok = mbar_wait_cluster(&bars->acc_empty, (tile - 1) & 1, abort_flag, a.err, a.wait_ns);
                     if (!ok) break;
                     tc_fence_after();
                 }
@@ -291,9 +291,9 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
                     const int s = gstep % kStages;
                     const uint32_t ph = (gstep / kStages) & 1;
                     const bool main = step < a.main_steps;
-                    ok = mbar_wait_cluster(&bars->a_full[s], ph, abort_flag, a.err);
+                    ok = mbar_wait_cluster(&bars->a_full[s], ph, abort_flag, a.err, a.wait_ns);
                     // (deq_full takes a phase on LoRA steps too, with no expansion)
-                    if (ok) ok = mbar_wait_cluster(&bars->deq_full[s], ph, abort_flag, a.err);
+                    if (ok) ok = mbar_wait_cluster(&bars->deq_full[s], ph, abort_flag, a.err, a.wait_ns);
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t a_base = smem_u32(smem + s * kStageBytes);
@@ -394,7 +394,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
                 const uint32_t gs = gbase + static_cast<uint32_t>(step);
                 const int s = gs % kStages;
                 const uint32_t ph = (gs / kStages) & 1;
-                if (!mbar_wait(&bars->pk_full[s], ph, abort_flag, a.err)) {
+                if (!mbar_wait(&bars->pk_full[s], ph, abort_flag, a.err, a.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -429,7 +429,7 @@ qlora_gemm_kernel(const __grid_constant__ CUtensorMap tm_act,    // X or dY   [M
             // need not be a multiple of kGroups), and a parity wait is only
             // sound when the waiter is at most one phase ahead of the last
             // completed phase, so no group may start the next tile earlier.
-            if (!mbar_wait(&bars->acc_full, tile & 1, abort_flag, a.err)) break;
+            if (!mbar_wait(&bars->acc_full, tile & 1, abort_flag, a.err, a.wait_ns)) break;
 
             // ---------------------------------------------- epilogue
             if (epi) {

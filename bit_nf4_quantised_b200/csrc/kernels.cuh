@@ -107,6 +107,8 @@ struct GemmArgs {
     int64_t cols_lin;
     int64_t col_budget;
     int* err;             // device error word
+    unsigned long long wait_ns;   // bound of every operational mbarrier wait (teardown
+                                  // drains keep kWaitLimitNs)
     Nf4Table tab;
 };
 

@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstring>
 #include <limits>
+#include <atomic>
 #include <mutex>
 
 #include "kernels.cuh"
@@ -329,6 +330,9 @@ int check_format(const qlora_format* f, FmtTable* t, FmtArgs* a) {
     return QLORA_OK;
 }
 
+// Bound of the tensor-core GEMM's operational waits (qlora_set_gemm_wait_limit_us).
+std::atomic<unsigned long long> g_gemm_wait_ns{kWaitLimitNs};
+
 cudaError_t record(const qlora_events* ev, bool begin, cudaStream_t s) {
     if (!ev) return cudaSuccess;
     void* e = begin ? ev->gemm_begin : ev->gemm_end;
@@ -416,6 +420,13 @@ const char* qlora_status_string(int status) {
         case QLORA_ERR_WORKSPACE: return "workspace missing or too small";
         default: return "unknown status";
     }
+}
+
+int qlora_set_gemm_wait_limit_us(int64_t us) {
+    if (us < 0 || us > 10000000) return QLORA_ERR_UNSUPPORTED;
+    g_gemm_wait_ns.store(us == 0 ? kWaitLimitNs : static_cast<unsigned long long>(us) * 1000ull,
+                         std::memory_order_relaxed);
+    return QLORA_OK;
 }
 
 int nf4_build_codebook(float codes[16], float midpoints[15]) {
@@ -713,6 +724,7 @@ int qlora_linear_forward_ex(const uint16_t* X, int64_t M, const qlora_nf4_tensor
     g.m_tiles = static_cast<int>(cdiv(M, gemm_tile_m()));
     gemm_schedule(g, false);
     g.err = err;
+    g.wait_ns = g_gemm_wait_ns.load(std::memory_order_relaxed);
     g.tab = table();
     // an event record between the two kernels would serialise them fully
     QTRY(record(ev, true, s));
@@ -813,6 +825,7 @@ int qlora_linear_backward_ex(const uint16_t* dY, const uint16_t* X, int64_t M,
         g.m_tiles = static_cast<int>(cdiv(M, gemm_tile_m()));
         gemm_schedule(g, true);
         g.err = err;
+        g.wait_ns = g_gemm_wait_ns.load(std::memory_order_relaxed);
         g.tab = table();
         QTRY(record(ev, true, s));
         QTRY(launch_gemm(true, m_act, m_packed, m_la, m_lb, m_out, g, ev == nullptr, s));

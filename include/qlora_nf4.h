@@ -23,7 +23,8 @@
  *     the host before anything is launched and leave every output untouched.
  *     QLORA_ERR_CUDA reports a failed launch (cudaGetLastError()).
  *   - The only global state is the scratch array of
- *     qlora_linear_forward_noalloc.  Calls on different streams with
+ *     qlora_linear_forward_noalloc and the wait limit that
+ *     qlora_set_gemm_wait_limit_us sets.  Calls on different streams with
  *     disjoint outputs and workspaces may run concurrently.
  *   - Within a call, some kernels are launched as programmatic dependents of
  *     the kernel before them (they may start before it finishes and wait for
@@ -476,6 +477,24 @@ QLORA_API int qlora_mlp_backward(const uint16_t* dY, const uint16_t* X, int64_t 
                                  const qlora_mlp* mlp, float scale, uint16_t* dX,
                                  const qlora_mlp_grads* grads, int accumulate, void* ws,
                                  size_t ws_bytes, qlora_stream_t stream);
+
+/*
+ * qlora_set_gemm_wait_limit_us -- the bound, in microseconds, of every wait of
+ * the tensor-core dequant-GEMM (the forward and dX kernel of
+ * qlora_linear_forward / _backward) on its pipeline barriers, for GEMMs
+ * launched after the call; 0 restores the default of 2 seconds.  A wait that
+ * runs out sets bit 0 of the call's error word, and the kernel lets its
+ * in-flight copies and MMAs land (those waits keep the default bound),
+ * frees its tensor memory and returns; the call's outputs are then
+ * unspecified and later calls are unaffected.  Under a limit below the
+ * default the waits poll the barriers without blocking and count SM clock
+ * cycles (1000 per microsecond of the limit: at most the stated time at
+ * clocks of 1 GHz and above), so that even a microsecond is honoured.  This is a failure-detection control: a
+ * healthy wait lasts microseconds, and a limit at or below that makes waits
+ * run out on purpose.  Process-wide; host only.
+ * Errors: QLORA_ERR_UNSUPPORTED (us < 0 or above 10 seconds).
+ */
+QLORA_API int qlora_set_gemm_wait_limit_us(int64_t us);
 
 /*
  * Profiling variants.  Identical to qlora_linear_forward / _backward, plus
