@@ -59,16 +59,17 @@ skinny_kernel(SkinnyArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
     // a dependent tensor-core GEMM may start streaming its weight tiles now;
     // it waits for this grid only before it reads this kernel's output
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // the call's error word is cleared before a dependent may start
+    if (a.err_zero != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *a.err_zero = 0;
     if (a.trigger_dependents) launch_dependents();
     cg::cluster_group cluster = cg::this_cluster();
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t i0 = int64_t(blockIdx.x) * TI;
     const int split = blockIdx.y;
     const int64_t c_beg = int64_t(split) * a.c_per_split;
     const int64_t c_end = min(a.C, c_beg + a.c_per_split);
     const int nchunks = c_end > c_beg ? static_cast<int>((c_end - c_beg + TC - 1) / TC) : 0;
     const uint32_t sbase = smem_u32(smem);
-    if (a.err_zero != nullptr && blockIdx.x == 0 && split == 0 && tid == 0) *a.err_zero = 0;
 
     auto load_stage = [&](int chunk, int st) {
         const int64_t c0 = c_beg + int64_t(chunk) * TC;
