@@ -34,7 +34,7 @@
 // gamma T B^T and rounds Y to bf16.
 //
 // Per two weights the expansion costs one permute, one 8-byte shared load
-// (two wavefronts per warp), two fp32 multiplies and one paired rounding.
+// (two wavefronts per warp), one paired fp32 multiply and one paired rounding.
 // Measured alternatives that built each block's 16-entry bf16 table in
 // registers and expanded nibbles with byte permutes (about 2.5 integer-pipe
 // instructions per weight, entirely or for part of the rows) were slower: the
@@ -114,6 +114,31 @@ __device__ __forceinline__ float2 lds64f_nv(uint32_t addr) {
     float2 v;
     asm("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
     return v;
+}
+
+__device__ __forceinline__ uint64_t lds64_nv(uint32_t addr) {
+    uint64_t v;
+    asm("ld.shared.b64 %0, [%1];" : "=l"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint64_t splat_f32x2(float x) {
+    uint64_t v;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(v) : "f"(x));
+    return v;
+}
+
+// Both fp32 lanes of q times those of c (each rounded to nearest, as two
+// __fmul_rn), then rounded to one bf16 pair (RNE), low lane in the low half.
+__device__ __forceinline__ uint32_t mul_f32x2_to_bf16x2(uint64_t q, uint64_t c) {
+    uint32_t out;
+    asm("{\n\t.reg .b64 p;\n\t.reg .f32 lo, hi;\n\t"
+        "mul.rn.f32x2 p, %1, %2;\n\t"
+        "mov.b64 {lo, hi}, p;\n\t"
+        "cvt.rn.bf16x2.f32 %0, hi, lo;\n\t}"
+        : "=r"(out)
+        : "l"(q), "l"(c));
+    return out;
 }
 
 // Two FP8 E4M3 codes (low byte first) to their exact fp32 values: E4M3 is a
@@ -475,6 +500,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
         const float2 va = e4m3x2_to_float2(cab & 0xffu), vb = e4m3x2_to_float2(cbb & 0xffu);
         const float cta = valid ? __fmul_rn(va.x, bt < split_a ? mra.x : mra.y) : 0.f;
         const float ctb = valid ? __fmul_rn(vb.x, bt < split_b ? mrb.x : mrb.y) : 0.f;
+        const uint64_t cta2 = splat_f32x2(cta), ctb2 = splat_f32x2(ctb);
         // this lane's 32 packed bytes of each row: tile layout [chunk][R
         // rows][128 bytes], 16-byte units swizzled by (row & 7); block c is
         // units 2c, 2c + 1
@@ -502,15 +528,13 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
 #pragma unroll
         for (int w = 0; w < 8; ++w) {
             // each packed byte -> its two fp32 codes from the lane's pair
-            // table -> fp32 products with c~ -> one bf16 pair (RNE): exactly
-            // bf16_rne(fp32(q * c~)) for both elements
+            // table -> fp32 products with c~ (one paired multiply) -> one
+            // bf16 pair (RNE): exactly bf16_rne(fp32(q * c~)) for both
             uint32_t oa[4], ob[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const float2 qa = lds64f_nv(prmt(wa[w], lane_lut, 0x7604u | (k << 4)));
-                const float2 qb = lds64f_nv(prmt(wb[w], lane_lut, 0x7604u | (k << 4)));
-                oa[k] = pack_bf16x2(__fmul_rn(qa.x, cta), __fmul_rn(qa.y, cta));
-                ob[k] = pack_bf16x2(__fmul_rn(qb.x, ctb), __fmul_rn(qb.y, ctb));
+                oa[k] = mul_f32x2_to_bf16x2(lds64_nv(prmt(wa[w], lane_lut, 0x7604u | (k << 4))), cta2);
+                ob[k] = mul_f32x2_to_bf16x2(lds64_nv(prmt(wb[w], lane_lut, 0x7604u | (k << 4))), ctb2);
             }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {

@@ -179,10 +179,15 @@ Split skinny_split(int64_t C) {
     return {static_cast<int>(cdiv(std::max<int64_t>(C, 1), per)), per, 0};
 }
 
-// Contraction slices for the GEMV: as wide as the activations allow in shared
-// memory, but at least enough slices for ~8 16-row units per SM.  Tiles are D
-// chunks deep with D dividing the slice width (so no tile reads a neighbour's
-// columns) -- except with a single slice, where a tile past K is zero-filled.
+// Contraction slices for the GEMV.  Each slice's activations must fit in
+// shared memory (cap); among the slice widths that do, the one with the
+// shortest estimated makespan is taken, in weight-tile times per CTA: the
+// slice's units (R = 256 / D rows x the slice) are dealt to its CTAs in
+// waves, so a CTA streams waves x ceil(chunks / D) tiles, and every slice
+// adds M x N fp32 partials that are written and read again (counted as
+// 32 KiB tiles spread over all CTAs).  D, the chunks per tile, is the
+// largest power of two up to 8 that divides the slice's 256-wide chunks
+// (8 for a single slice, whose last tile past K is zero-filled).
 Split gemv_split(int64_t M, int64_t N, int64_t K) {
     int64_t cap = 256;
     for (int64_t c = std::min<int64_t>(K, 32768) / 256 * 256; c >= 256; c -= 256)
@@ -190,38 +195,33 @@ Split gemv_split(int64_t M, int64_t N, int64_t K) {
             cap = c;
             break;
         }
-    const int64_t units = cdiv(N, 16);
-    int64_t s = std::max(cdiv(K, cap), cdiv(8 * 148, units));
-    s = std::min(s, std::max<int64_t>(1, K / 256));
-    int64_t per = up(cdiv(K, s), 256);
-    while (per > cap) per = up(cdiv(K, ++s), 256);
-    Split r;
-    if (per >= K) {
-        r.splits = 1;
-        r.per = K;
-    } else {
-        r.splits = static_cast<int>(cdiv(K, per));
-        r.per = per;
-    }
-    // prefer deeper tiles: widen the slice to a multiple of 2048 (or 1024,
-    // 512) when that keeps the slice count and fits the activation budget
-    if (r.splits > 1) {
-        for (int64_t q : {2048, 1024, 512}) {
-            const int64_t wide = up(r.per, q);
-            if (wide <= cap && cdiv(K, wide) == r.splits) {
-                r.per = wide;
-                break;
+    const int64_t sms = std::max(1, num_sms());
+    Split best{0, 0, 0};
+    double best_cost = 0.0;
+    const int64_t s_max = std::min<int64_t>(kMaxGemvSlices, std::max<int64_t>(1, K / 256));
+    for (int64_t s = std::max<int64_t>(1, cdiv(K, cap)); s <= s_max; ++s) {
+        for (int64_t q : {256, 512, 1024, 2048}) {
+            const int64_t per = up(cdiv(K, s), q);
+            if (per > cap || cdiv(K, per) != s) continue;
+            const int64_t chunks = per / 256;
+            int d = 1;
+            if (s == 1 && chunks >= 8) {
+                d = 8;
+            } else {
+                while (d < 8 && chunks % (2 * d) == 0) d *= 2;
+            }
+            const int64_t units = cdiv(N, 256 / d);
+            const int64_t ctas = std::max<int64_t>(1, sms / s);
+            const double cost = double(cdiv(units, ctas) * cdiv(chunks, d)) +
+                                double(s * M * N * 8) / 32768.0 / double(ctas * s);
+            if (best.splits == 0 || cost < best_cost - 1e-9) {
+                best = {static_cast<int>(s), s == 1 ? K : per, d};
+                best_cost = cost;
             }
         }
     }
-    const int64_t chunks = r.per / 256;
-    if (r.splits == 1 && chunks >= 8) {
-        r.chunks = 8;
-    } else {
-        r.chunks = 1;
-        while (r.chunks < 8 && chunks % (2 * r.chunks) == 0) r.chunks *= 2;
-    }
-    return r;
+    if (best.splits == 0) best = {static_cast<int>(cdiv(K, 256)), 256, 1};   // one chunk per slice
+    return best;
 }
 
 // M <= 16 with K % 256 == 0 runs the bandwidth-bound GEMV (its 3-D weight view
