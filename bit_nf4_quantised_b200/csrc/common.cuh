@@ -85,25 +85,55 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// The same test with cluster-scope acquire (arrivals may come from the peer).
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// A wait under a limit shorter than the default (qlora_set_gemm_wait_limit_us):
+// it polls with the non-blocking test, whose thread is never suspended inside
+// the instruction, and checks after every poll against SM clock cycles
+// (%globaltimer may tick far more coarsely than a microsecond), so that even
+// a limit of a microsecond is honoured: limit_ns cycles, at most limit_ns
+// nanoseconds at SM clocks of 1 GHz and up.  Kept out of line so that the
+// inlined waits of the pipelines stay as short as the default path needs.
+static __device__ __noinline__ bool mbar_wait_short(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                             int* err, unsigned long long limit_ns, bool cluster) {
+    const long long c0 = clock64();
+    for (;;) {
+        if (cluster ? mbar_test_wait_cluster(bar, parity) : mbar_test_wait(bar, parity)) return true;
+        if (abort_flag != nullptr && *abort_flag) return false;
+        if (clock64() - c0 > static_cast<long long>(limit_ns)) {
+            if (err != nullptr) atomicOr(err, kErrWaitTimeout);
+            if (abort_flag != nullptr) *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
 // Wait until the phase with the given parity has completed.  Gives up (and
 // returns false) when *abort_flag becomes non-zero or after limit_ns; a
-// timeout sets kErrWaitTimeout in *err and raises *abort_flag.  A limit
-// below the default polls with the non-blocking test, checks after every
-// poll and counts SM clock cycles (%globaltimer may tick far more coarsely
-// than a microsecond), so that even a limit of a microsecond is honoured:
-// limit_ns cycles, at most limit_ns nanoseconds at SM clocks of 1 GHz and up.
+// timeout sets kErrWaitTimeout in *err and raises *abort_flag.  A limit below
+// the default goes to mbar_wait_short once the first test fails.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           volatile int* abort_flag, int* err,
                                           unsigned long long limit_ns = kWaitLimitNs) {
-    const bool poll = limit_ns < kWaitLimitNs;
-    if (poll ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
+    if (limit_ns < kWaitLimitNs) return mbar_wait_short(bar, parity, abort_flag, err, limit_ns, false);
     const unsigned long long t0 = globaltimer_ns();
-    const long long c0 = clock64();
     for (uint32_t it = 1;; ++it) {
-        if (poll ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
-        if (poll || (it & 63u) == 0) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 0) {
             if (abort_flag != nullptr && *abort_flag) return false;
-            if (poll ? clock64() - c0 > static_cast<long long>(limit_ns) : globaltimer_ns() - t0 > limit_ns) {
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
                 if (err != nullptr) atomicOr(err, kErrWaitTimeout);
                 if (abort_flag != nullptr) *abort_flag = 1;
                 return false;
@@ -288,31 +318,18 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
     return ok != 0;
 }
 
-__device__ __forceinline__ bool mbar_test_wait_cluster(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 // As mbar_wait, with cluster-scope acquire (arrivals may come from the peer).
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
                                                   volatile int* abort_flag, int* err,
                                                   unsigned long long limit_ns = kWaitLimitNs) {
-    const bool poll = limit_ns < kWaitLimitNs;
-    if (poll ? mbar_test_wait_cluster(bar, parity) : mbar_try_wait_cluster(bar, parity)) return true;
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (limit_ns < kWaitLimitNs) return mbar_wait_short(bar, parity, abort_flag, err, limit_ns, true);
     const unsigned long long t0 = globaltimer_ns();
-    const long long c0 = clock64();
     for (uint32_t it = 1;; ++it) {
-        if (poll ? mbar_test_wait_cluster(bar, parity) : mbar_try_wait_cluster(bar, parity)) return true;
-        if (poll || (it & 63u) == 0) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if ((it & 63u) == 0) {
             if (abort_flag != nullptr && *abort_flag) return false;
-            if (poll ? clock64() - c0 > static_cast<long long>(limit_ns) : globaltimer_ns() - t0 > limit_ns) {
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
                 if (err != nullptr) atomicOr(err, kErrWaitTimeout);
                 if (abort_flag != nullptr) *abort_flag = 1;
                 return false;

@@ -41,7 +41,8 @@
 // The block scales stay in shared memory for the group-level FP8 pass.
 //
 // The same kernel also takes a bf16 weight (a merged export being
-// re-quantised): each lane then loads 32 bytes per block, widened exactly.
+// re-quantised): each lane then loads its 8 weights as 16 bytes, widened
+// exactly.
 #include <cfloat>
 
 #include "kernels.cuh"
