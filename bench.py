@@ -41,9 +41,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the saved T), dB product, dequant-GEMM dX, dA product).
 LAUNCHES_PER_STEP = 2 + 4
 # ncu DRAM traffic (read + write bytes) of one dequant-GEMM launch of this
-# workload, valid only for the source it was captured on.
-GEMM_TRAFFIC = {"source_sha": "4c197ac7a6e2f9bb", "fwd_bytes": (44.354816 + 7.093248) * 1e6,
-                "dx_bytes": (44.429568 + 7.148032) * 1e6}
+# workload, valid only for the sources it was captured on (_source_sha).
+GEMM_TRAFFIC = {"source_sha": "b8581179eda348e5", "fwd_bytes": (44.550144 + 8.004608) * 1e6,
+                "dx_bytes": (44.379648 + 6.835968) * 1e6}
 
 
 def _peaks():
@@ -56,9 +56,12 @@ def _peaks():
 
 
 def _source_sha():
-    p = os.path.join(ROOT, "bit_nf4_quantised_b200", "csrc", "gemm_sm100.cu")
-    with open(p, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """sha256 prefix over the sources the dequant-GEMM kernel is compiled from."""
+    h = hashlib.sha256()
+    for name in ("gemm_sm100.cu", "common.cuh", "kernels.cuh"):
+        with open(os.path.join(ROOT, "bit_nf4_quantised_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 class Clocks:
