@@ -682,8 +682,10 @@ gemv_finalize_kernel(GemvFinalizeArgs a) {
 
 int gemv_stages(int64_t M, int64_t kslab) {
     // dynamic shared memory starts after the 1 KiB the driver reserves; the
-    // plan must also hold for a base 1 KiB either side of that
-    for (int st = kMaxStages; st >= 3; --st) {
+    // plan must also hold for a base 1 KiB either side of that.  Two stages
+    // (64 KiB in flight per SM) still outrun what the consumers take; the
+    // slice choice uses them to fit wider activation slabs.
+    for (int st = kMaxStages; st >= 2; --st) {
         bool ok = true;
         for (uint32_t start : {0u, 1024u, 2048u})
             ok = ok && plan_smem(start, st, gemv_x_bytes(M, kslab), gemv_red_bytes(M)).ok;
@@ -723,14 +725,16 @@ cudaError_t launch_gemv(const CUtensorMap& tm_packed, const GemvArgs& a, int num
             case 6: return launch_depth<2, 6>(grid, tm_packed, a, stream);
             case 5: return launch_depth<2, 5>(grid, tm_packed, a, stream);
             case 4: return launch_depth<2, 4>(grid, tm_packed, a, stream);
-            default: return launch_depth<2, 3>(grid, tm_packed, a, stream);
+            case 3: return launch_depth<2, 3>(grid, tm_packed, a, stream);
+            default: return launch_depth<2, 2>(grid, tm_packed, a, stream);
         }
     }
     switch (st) {
         case 6: return launch_depth<1, 6>(grid, tm_packed, a, stream);
         case 5: return launch_depth<1, 5>(grid, tm_packed, a, stream);
         case 4: return launch_depth<1, 4>(grid, tm_packed, a, stream);
-        default: return launch_depth<1, 3>(grid, tm_packed, a, stream);
+        case 3: return launch_depth<1, 3>(grid, tm_packed, a, stream);
+        default: return launch_depth<1, 2>(grid, tm_packed, a, stream);
     }
 }
 
