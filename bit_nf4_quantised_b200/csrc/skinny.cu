@@ -5,9 +5,9 @@
 // output side (r <= 128): HBM-bound streams over X or dY.  One kernel covers
 // the four operand layouts.  A CTA of 4 warps owns 64 rows of the long output
 // side and all r columns of one contraction slice, streams the slice through
-// a 3-stage cp.async ring and feeds mma.sync m16n8k16 (bf16 in, fp32
-// accumulate) through ldmatrix (.trans where the stored layout is the
-// transpose).  The slices of a row block form one thread-block cluster (up to
+// a 3-stage cp.async ring (one barrier per stage) and feeds mma.sync
+// m16n8k16 (bf16 in, fp32 accumulate) through ldmatrix (.trans where the
+// stored layout is the transpose).  The slices of a row block form one thread-block cluster (up to
 // 8 CTAs): each parks its fp32 partial in shared memory, then every CTA sums
 // one slice of the rows over all partials through distributed shared memory
 // and writes the finished result -- scaled fp32 (optionally transposed or
@@ -122,10 +122,14 @@ skinny_kernel(SkinnyArgs a) {
     }
     for (int chunk = 0; chunk < nchunks; ++chunk) {
         const int st = chunk % kStages;
+        // this chunk's copies have landed (the kStages - 2 later ones may
+        // still fly); after the barrier every warp is also done with the
+        // previous chunk's stage, which the next prefetch overwrites, so one
+        // barrier per chunk suffices
+        cp_async_wait<kStages - 2>();
+        __syncthreads();
         if (chunk + kStages - 1 < nchunks) load_stage(chunk + kStages - 1, (chunk + kStages - 1) % kStages);
         cp_async_commit();
-        cp_async_wait<kStages - 1>();
-        __syncthreads();
         const uint32_t sp = sbase + st * Tl::kStage;
         const uint32_t sq = sp + Tl::kPBytes;
         const int mi = lane >> 3, r8 = lane & 7;
@@ -157,7 +161,6 @@ skinny_kernel(SkinnyArgs a) {
                 mma_bf16_16816(acc[jt][1], a0, a1, a2, a3, b2, b3);
             }
         }
-        __syncthreads();
     }
     cp_async_wait<0>();
     __syncthreads();
