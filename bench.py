@@ -759,38 +759,72 @@ def run_gpu(args):
 
 def _e2e(q, syn, lin, device, steps, world=1):
     """Same step through the public API with host buffers: pinned host X and
-    dY copied in, Y, dX, dA, dB copied out, all inside the timed region."""
+    dY copied in, Y, dX, dA, dB copied out, every step, all inside the timed
+    region.  The copies run on their own streams with device inputs and
+    outputs double-buffered, so that step i+1's inputs go in and step i-1's
+    results come out (PCIe is full duplex) while step i computes; events order
+    each buffer's reuse after its last reader."""
     d = syn.make_layer(lin)
     w = q.qlora_quantize(torch.from_numpy(d["W"]).to(device))
     host_in = {k: d[k].pin_memory() for k in ("X", "dY")}
-    g = {k: d[k].to(device) for k in ("X", "A", "B", "dY")}
-    bufs = _bufs(lin, device)
-    host_out = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in bufs.items()
+    gs = [{k: d[k].to(device) for k in ("X", "A", "B", "dY")} for _ in range(2)]
+    bufs = [_bufs(lin, device) for _ in range(2)]
+    host_out = {k: torch.empty_like(v, device="cpu").pin_memory() for k, v in bufs[0].items()
                 if k != "T"}
     ws = q.workspace(lin.M, lin.N, lin.K, lin.r, device)
+    s_in, s_cmp, s_out = (torch.cuda.Stream(device) for _ in range(3))
+    ev = lambda: torch.cuda.Event()
+    in_done = [ev(), ev()]       # inputs of buffer set b landed
+    cmp_done = [ev(), ev()]      # step on buffer set b finished (inputs free, outputs ready)
+    out_done = [ev(), ev()]      # results of buffer set b copied out (outputs free)
+    started = [False, False]
 
-    def one():
-        g["X"].copy_(host_in["X"], non_blocking=True)
-        g["dY"].copy_(host_in["dY"], non_blocking=True)
-        _step(q, lin, w, g, bufs, ws)
-        for k, v in host_out.items():
-            v.copy_(bufs[k], non_blocking=True)
+    def one(i):
+        b = i % 2
+        g, o = gs[b], bufs[b]
+        with torch.cuda.stream(s_in):
+            if started[b]:
+                s_in.wait_event(cmp_done[b])          # the step that read these inputs is done
+            g["X"].copy_(host_in["X"], non_blocking=True)
+            g["dY"].copy_(host_in["dY"], non_blocking=True)
+            in_done[b].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(in_done[b])
+            if started[b]:
+                s_cmp.wait_event(out_done[b])         # these outputs have been copied out
+            _step(q, lin, w, g, o, ws)
+            cmp_done[b].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(cmp_done[b])
+            for k, v in host_out.items():
+                v.copy_(o[k], non_blocking=True)
+            out_done[b].record(s_out)
+        started[b] = True
 
-    for _ in range(2):
-        one()
+    for i in range(2):
+        one(i)
+    torch.cuda.synchronize()
     _barrier(world)
-    b, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    b.record()
-    for _ in range(steps):
-        one()
-    e.record()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cur = torch.cuda.current_stream(device)
+    t0.record(cur)
+    for s in (s_in, s_cmp, s_out):
+        s.wait_event(t0)
+    for i in range(steps):
+        one(i)
+    for s in (s_in, s_cmp, s_out):
+        e = ev()
+        e.record(s)
+        cur.wait_event(e)
+    t1.record(cur)
     _barrier(world)
-    ms = _max_over_ranks(b.elapsed_time(e), world) / steps
+    ms = _max_over_ranks(t0.elapsed_time(t1), world) / steps
     h2d = sum(v.numel() * v.element_size() for v in host_in.values())
     d2h = sum(v.numel() * v.element_size() for v in host_out.values())
     return {"value": round(world * lin.fwd_bwd_flops() / (ms * 1e-3) / 1e12, 2),
             "unit": "TFLOP/s", "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h}
+            "d2h_bytes_per_step": d2h,
+            "overlap": "copy-in, compute and copy-out on three streams, device buffers doubled"}
 
 
 # --------------------------------------------------------------- CPU oracle
