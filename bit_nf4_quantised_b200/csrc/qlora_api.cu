@@ -172,9 +172,17 @@ struct Split {
 };
 
 // contraction slices of a LoRA side product: one cluster of up to 8 CTAs
-Split skinny_split(int64_t C) {
+// Contraction slices of a skinny product with `rows` output rows (64 per
+// CTA): enough slices for about 128 CTAs, at most 8 (one cluster) and at most
+// one per 64-wide chunk.  With the deep ring, fewer and longer slices keep
+// more bytes in flight per CTA; measured on the 4096-token layer, 2 slices
+// (128 CTAs) beat 4 and 8, and leave SMs free for the GEMM that follows.
+constexpr int64_t kSkinnyTargetCtas = 128;
+Split skinny_split(int64_t C, int64_t rows) {
     const int64_t chunks = std::max<int64_t>(1, cdiv(C, 64));
-    const int64_t s = std::min<int64_t>(kMaxSkinnySplits, chunks);
+    const int64_t row_tiles = std::max<int64_t>(1, cdiv(rows, 64));
+    const int64_t want = std::max<int64_t>(1, cdiv(kSkinnyTargetCtas, row_tiles));
+    const int64_t s = std::min<int64_t>({int64_t(kMaxSkinnySplits), chunks, want});
     const int64_t per = cdiv(chunks, s) * 64;
     return {static_cast<int>(cdiv(std::max<int64_t>(C, 1), per)), per, 0};
 }
@@ -379,7 +387,7 @@ SkinnyArgs skinny_args(const uint16_t* P, const uint16_t* Q, int64_t I, int64_t 
     a.C = C;
     a.ldp = ldp;
     a.ldq = ldq;
-    const Split sp = skinny_split(C);
+    const Split sp = skinny_split(C, I);
     a.splits = sp.splits;
     a.c_per_split = sp.per;
     a.alpha = 1.0f;

@@ -5,7 +5,8 @@
 // output side (r <= 128): HBM-bound streams over X or dY.  One kernel covers
 // the four operand layouts.  A CTA of 4 warps owns 64 rows of the long output
 // side and all r columns of one contraction slice, streams the slice through
-// a 3-stage cp.async ring (one barrier per stage) and feeds mma.sync
+// a deep cp.async ring (8 stages of 64 contraction positions for r <= 64: a
+// CTA keeps 7 chunks in flight; one barrier per stage) and feeds mma.sync
 // m16n8k16 (bf16 in, fp32 accumulate) through ldmatrix (.trans where the
 // stored layout is the transpose).  The slices of a row block form one thread-block cluster (up to
 // 8 CTAs): each parks its fp32 partial in shared memory, then every CTA sums
@@ -27,7 +28,6 @@ namespace {
 constexpr int kThreads = 128;
 constexpr int TI = 64;           // output rows per CTA
 constexpr int TC = 64;           // contraction per stage
-constexpr int kStages = 3;
 constexpr int kPitchK = TC * 2 + 16;   // bytes per 64-wide row (+16 against bank conflicts)
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
@@ -48,8 +48,12 @@ struct SkinnyTile {
     static constexpr int kQPitch = QK ? kPitchK : (JP * 2 + 16);
     static constexpr int kQBytes = QK ? JP * kPitchK : TC * kQPitch;
     static constexpr int kStage = kPBytes + kQBytes;
+    // ring depth: 8 stages (7 chunks in flight per CTA), fewer where a stage
+    // is large (r > 64) so that the ring stays within 200 KiB
+    static constexpr int kStages = (200 * 1024 / kStage) < 8 ? (200 * 1024 / kStage) : 8;
     static constexpr int kRedBytes = TI * JP * 4;                       // fp32 partial tile
     static constexpr int kSmem = (kStages * kStage > kRedBytes) ? kStages * kStage : kRedBytes;
+    static_assert(kStages >= 3, "skinny ring depth");
 };
 
 template <bool PK, bool QK, int JT16>
@@ -116,6 +120,7 @@ skinny_kernel(SkinnyArgs a) {
             for (int e = 0; e < 4; ++e) acc[j][t][e] = 0.f;
 
 #pragma unroll
+    constexpr int kStages = Tl::kStages;
     for (int st = 0; st < kStages - 1; ++st) {
         if (st < nchunks) load_stage(st, st);
         cp_async_commit();
