@@ -281,32 +281,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
         fence_barrier_init();
         prefetch_tensormap(&tm_packed);
     }
-    // code-pair table: entry e (a packed byte) of lane l at lut + 256 e + 8 l
-    // holds the fp32 codes (q[e & 15], q[e >> 4]); each thread writes two
-    // lanes' copies of an entry at a time
-    if (sp.ok) {
-        for (int i = tid; i < 256 * 16; i += kThreads) {
-            const int e = i >> 4, l2 = (i & 15) * 2;
-            const float q0 = a.tab.code[e & 15], q1 = a.tab.code[e >> 4];
-            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %1, %2};" ::"r"(sp.lut + e * 256 + l2 * 8),
-                         "f"(q0), "f"(q1)
-                         : "memory");
-        }
-    }
-    // activation slice, M rows of 8-byte units, swizzled (x_off); a zero
-    // line stands in for tokens past M and blocks past the slice
-    if (sp.ok) {
-        if (tid < 32) asm volatile("st.shared.b32 [%0], %1;" ::"r"(sp.zero + tid * 4), "r"(0u) : "memory");
-        const int units_per_row = kslab / 4;
-        for (int q = tid; q < xrows * units_per_row; q += kThreads) {
-            const int m = q / units_per_row, u = q % units_per_row;
-            const uint2 val = *reinterpret_cast<const uint2*>(a.X + m * a.K + k_beg + u * 4);
-            asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(sp.x + x_off(m, u * 4, x_pitch)),
-                         "r"(val.x), "r"(val.y)
-                         : "memory");
-        }
-    }
-    __syncthreads();
+    __syncthreads();                             // barriers initialised, plan checked
     if (*abort_flag) return;
 
     const int64_t nkb = a.K / QLORA_BLOCK;
@@ -396,6 +371,32 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
     }
 
     // ---------------------------------------------------------- consumers
+    // While the producer's first tiles stream in, the consumer warps fill the
+    // code-pair table and the activation slab, then meet on a named barrier.
+    // Code-pair table: entry e (a packed byte) of lane l at lut + 256 e + 8 l
+    // holds the fp32 codes (q[e & 15], q[e >> 4]); each thread writes two
+    // lanes' copies of an entry at a time.
+    for (int i = tid; i < 256 * 16; i += kConsumerWarps * 32) {
+        const int e = i >> 4, l2 = (i & 15) * 2;
+        const float q0 = a.tab.code[e & 15], q1 = a.tab.code[e >> 4];
+        asm volatile("st.shared.v4.f32 [%0], {%1, %2, %1, %2};" ::"r"(sp.lut + e * 256 + l2 * 8),
+                     "f"(q0), "f"(q1)
+                     : "memory");
+    }
+    // Activation slice, M rows of 8-byte units, swizzled (x_off); a zero line
+    // stands in for tokens past M and blocks past the slice.
+    if (tid < 32) asm volatile("st.shared.b32 [%0], %1;" ::"r"(sp.zero + tid * 4), "r"(0u) : "memory");
+    {
+        const int units_per_row = kslab / 4;
+        for (int q = tid; q < xrows * units_per_row; q += kConsumerWarps * 32) {
+            const int m = q / units_per_row, u = q % units_per_row;
+            const uint2 val = *reinterpret_cast<const uint2*>(a.X + m * a.K + k_beg + u * 4);
+            asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(sp.x + x_off(m, u * 4, x_pitch)),
+                         "r"(val.x), "r"(val.y)
+                         : "memory");
+        }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
     if (blockIdx.x < a.t_ctas) {
         // a share of this slice's T = X A^T: CTA x of the first t_ctas takes
         // an equal run of the slice's 16-wide k-steps, spread over its warps;
