@@ -16,8 +16,13 @@
 // Quantise: one CTA per group of 256 blocks.  A block is covered by
 // min(32, B/4) lanes that each load 16-byte pieces; the lanes reduce the
 // absmax with shuffles and then re-read their pieces (from L1/L2) to write the
-// indices, four per 16-bit store.  The group's scales stay in shared memory
-// for the FP8 pass, as in K1.  Dequantise: as K6, one packed word (8 weights)
+// indices, four per 16-bit store.  As in K1, x = fp32(w / c_b) comes from one
+// correctly rounded reciprocal per block and two fused multiply-adds (exact,
+// with a guarded fallback), and when the codebook's midpoints lie more than
+// 1/16 apart (NF4, FP4, INT4) the index comes from K1's bucket table, one
+// conflict-free shared-memory load per weight; other codebooks take a 4-step
+// search over the midpoints.  The group's scales stay in shared memory for
+// the FP8 pass, as in K1.  Dequantise: as K6, one packed word (8 weights)
 // per thread and one 16-byte store; the block index is a shift.
 #include "kernels.cuh"
 
@@ -26,6 +31,31 @@ namespace qnf4 {
 namespace {
 
 constexpr int kThreads = 256;
+
+// The correctly rounded a / b, given r = RN(1 / b): q = RN(a r) is within an
+// ulp of a / b, the fused a - q b is then exact, and RN(q + (a - q b) r) is
+// the correctly rounded quotient (Markstein's theorem), as long as no step
+// overflows or underflows: a, b and q in [2^-100, 2^100] in magnitude.
+// Elsewhere (zeros with their signs, NaN, infinities, extreme ranges) the
+// plain correctly rounded division.  Both give the same bits.
+__device__ __forceinline__ float div_rn_by(float a, float b, float r) {
+    const float q = __fmul_rn(a, r);
+    const float aa = fabsf(a), ab = fabsf(b), aq = fabsf(q);
+    if (aa >= 0x1p-100f && aa <= 0x1p100f && ab >= 0x1p-100f && ab <= 0x1p100f && aq >= 0x1p-100f &&
+        aq <= 0x1p100f)
+        return __fmaf_rn(__fmaf_rn(-q, b, a), r, q);
+    return __fdiv_rn(a, b);
+}
+
+// Number of midpoints strictly below x in [-1, 1], from K1's bucket table:
+// bucket key = the top bits of x + 3; lane_lut is this lane's column of the
+// table minus the offset of key 0x1000 (the bucket of x + 3 = 2).
+__device__ __forceinline__ uint32_t bucket_code(float x, uint32_t lane_lut) {
+    const uint32_t key = __float_as_uint(__fadd_rn(x, 3.0f)) >> 18;
+    uint32_t thr, base;
+    asm("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(thr), "=r"(base) : "r"(lane_lut + (key << 8)));
+    return base + (x > __uint_as_float(thr) ? 1u : 0u);
+}
 
 __device__ __forceinline__ uint32_t nearest_code(float x, const float* smid) {
     // number of midpoints strictly below x; unused midpoints are +inf
@@ -45,6 +75,7 @@ quantize_fmt_kernel(const float* __restrict__ W, int64_t numel, int64_t nblocks,
     __shared__ float smid[16];
     __shared__ float sabs[QLORA_GROUP];
     __shared__ float sred[kThreads / 32];
+    __shared__ __align__(16) uint2 slut[kNf4LutEntries * 32];   // entry b of lane l at 256 b + 8 l
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -53,7 +84,12 @@ quantize_fmt_kernel(const float* __restrict__ W, int64_t numel, int64_t nblocks,
         for (int q = 0; q < 15; ++q) smid[q] = tab.mid[q];
         smid[15] = __int_as_float(0x7f800000);
     }
+    if (tab.use_lut) {
+        for (int i = tid; i < kNf4LutEntries * 32; i += kThreads)
+            slut[i] = make_uint2(tab.lut.thr[i >> 5], tab.lut.base[i >> 5]);
+    }
     __syncthreads();
+    const uint32_t lane_lut = smem_u32(slut) + lane * 8 - (0x1000u << 8);
 
     const int lp = f.block >= 128 ? 32 : f.block / 4;        // lanes per block
     const int bpw = 32 / lp;                                  // blocks per warp step
@@ -81,6 +117,7 @@ quantize_fmt_kernel(const float* __restrict__ W, int64_t numel, int64_t nblocks,
             a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
         }
         for (int o = lp / 2; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        const float r = __frcp_rn(a);
         const bool live = kFull || gblk < nblocks;
         for (int j = 0; j < cpl; ++j) {
             const int64_t e0 = ebase + int64_t(j * lp + sub) * 4;
@@ -96,10 +133,23 @@ quantize_fmt_kernel(const float* __restrict__ W, int64_t numel, int64_t nblocks,
             uint32_t q0 = tab.zero_index, q1 = tab.zero_index, q2 = tab.zero_index,
                      q3 = tab.zero_index;
             if (a > 0.f) {
-                q0 = nearest_code(__fdiv_rn(v.x, a), smid);
-                q1 = nearest_code(__fdiv_rn(v.y, a), smid);
-                q2 = nearest_code(__fdiv_rn(v.z, a), smid);
-                q3 = nearest_code(__fdiv_rn(v.w, a), smid);
+                // |w| <= c_b, so x lies in [-1, 1]; the clamp only sends the NaN
+                // of a non-finite weight (flagged above) into the table's range
+                const float x0 = fminf(fmaxf(div_rn_by(v.x, a, r), -1.0f), 1.0f);
+                const float x1 = fminf(fmaxf(div_rn_by(v.y, a, r), -1.0f), 1.0f);
+                const float x2 = fminf(fmaxf(div_rn_by(v.z, a, r), -1.0f), 1.0f);
+                const float x3 = fminf(fmaxf(div_rn_by(v.w, a, r), -1.0f), 1.0f);
+                if (tab.use_lut) {
+                    q0 = bucket_code(x0, lane_lut);
+                    q1 = bucket_code(x1, lane_lut);
+                    q2 = bucket_code(x2, lane_lut);
+                    q3 = bucket_code(x3, lane_lut);
+                } else {
+                    q0 = nearest_code(x0, smid);
+                    q1 = nearest_code(x1, smid);
+                    q2 = nearest_code(x2, smid);
+                    q3 = nearest_code(x3, smid);
+                }
             }
             if (live)
                 *reinterpret_cast<uint16_t*>(packed + e0 / 2) =

@@ -39,6 +39,8 @@ struct FmtTable {
     float code[16];            // codebook (unused entries 0)
     float mid[15];             // fp32 midpoints; +inf past the last code
     uint32_t zero_index;       // index of the code nearest 0 (zero blocks, padding)
+    uint32_t use_lut;          // the finite midpoints are more than 1/16 apart: the
+    Nf4IndexLut lut;           // bucket table gives the code index (else a search)
 };
 struct FmtArgs {
     int block;                 // power of two, 16..4096

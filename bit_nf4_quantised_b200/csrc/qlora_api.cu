@@ -69,7 +69,9 @@ const Nf4Table& table() {
 // Returns false unless every bucket spans at most one midpoint (true for the
 // NF4 codes, whose midpoints lie at least 0.08 apart).
 bool build_index_lut(const float mids[15], Nf4IndexLut* lut) {
-    for (int i = 0; i + 1 < 15; ++i)
+    // consecutive finite midpoints (a codebook of fewer than 16 codes pads
+    // its midpoints with +inf) must be more than a bucket apart
+    for (int i = 0; i + 1 < 15 && std::isfinite(mids[i + 1]); ++i)
         if (!(double(mids[i + 1]) - double(mids[i]) > 1.0 / 16.0 + std::ldexp(1.0, -20))) return false;
     for (int b = 0; b < kNf4LutEntries; ++b) {
         const double lo = 2.0 + b / 16.0 - 3.0 - std::ldexp(1.0, -22);
@@ -328,6 +330,7 @@ int check_format(const qlora_format* f, FmtTable* t, FmtArgs* a) {
             }
         }
         t->zero_index = z;
+        t->use_lut = build_index_lut(t->mid, &t->lut) ? 1u : 0u;
     }
     if (a) {
         a->block = b;
