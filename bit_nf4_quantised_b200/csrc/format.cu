@@ -67,7 +67,12 @@ __device__ __forceinline__ uint32_t nearest_code(float x, const float* smid) {
     return i;
 }
 
-template <bool kFull>
+// kLP > 0 (full groups of blocks of 4 kLP <= 32 weights): kLP lanes cover a
+// block, one 16-byte piece each, and a lane issues the loads of all its
+// pieces of the group (4 kLP floats) before using any, keeping them in
+// registers for the index pass; otherwise pieces are loaded block by block
+// and re-read for the index pass.
+template <bool kFull, int kLP>
 __global__ void __launch_bounds__(kThreads)
 quantize_fmt_kernel(const float* __restrict__ W, int64_t numel, int64_t nblocks, FmtArgs f,
                     uint8_t* __restrict__ packed, void* __restrict__ scales,
@@ -91,54 +96,36 @@ quantize_fmt_kernel(const float* __restrict__ W, int64_t numel, int64_t nblocks,
     __syncthreads();
     const uint32_t lane_lut = smem_u32(slut) + lane * 8 - (0x1000u << 8);
 
-    const int lp = f.block >= 128 ? 32 : f.block / 4;        // lanes per block
-    const int bpw = 32 / lp;                                  // blocks per warp step
-    const int cpl = f.block / (4 * lp);                       // 16-byte pieces per lane
-    const int sub = lane % lp;
     const int64_t group = blockIdx.x;
     bool bad = false;
-
-    for (int blk = warp * bpw + lane / lp; blk < QLORA_GROUP; blk += (kThreads / 32) * bpw) {
-        const int64_t gblk = group * QLORA_GROUP + blk;
-        const int64_t ebase = gblk * f.block;
-        float a = 0.f;
-        for (int j = 0; j < cpl; ++j) {
-            const int64_t e0 = ebase + int64_t(j * lp + sub) * 4;
-            float4 v;
-            if (kFull) {
-                v = *reinterpret_cast<const float4*>(W + e0);
-            } else {
-                v.x = (e0 + 0 < numel) ? W[e0 + 0] : 0.f;
-                v.y = (e0 + 1 < numel) ? W[e0 + 1] : 0.f;
-                v.z = (e0 + 2 < numel) ? W[e0 + 2] : 0.f;
-                v.w = (e0 + 3 < numel) ? W[e0 + 3] : 0.f;
-            }
-            bad |= !(isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w));
-            a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+    if constexpr (kLP > 0) {
+        constexpr int kBpw = 32 / kLP;                            // blocks per warp step
+        constexpr int kIt = QLORA_GROUP / ((kThreads / 32) * kBpw);   // = kLP
+        const int sub = lane % kLP;
+        float4 v[kIt];
+#pragma unroll
+        for (int it = 0; it < kIt; ++it) {
+            const int blk = warp * kBpw + lane / kLP + it * (kThreads / 32) * kBpw;
+            const int64_t e0 = (group * QLORA_GROUP + blk) * (4 * kLP) + sub * 4;
+            v[it] = __ldcs(reinterpret_cast<const float4*>(W + e0));
         }
-        for (int o = lp / 2; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-        const float r = __frcp_rn(a);
-        const bool live = kFull || gblk < nblocks;
-        for (int j = 0; j < cpl; ++j) {
-            const int64_t e0 = ebase + int64_t(j * lp + sub) * 4;
-            float4 v;
-            if (kFull) {
-                v = *reinterpret_cast<const float4*>(W + e0);
-            } else {
-                v.x = (e0 + 0 < numel) ? W[e0 + 0] : 0.f;
-                v.y = (e0 + 1 < numel) ? W[e0 + 1] : 0.f;
-                v.z = (e0 + 2 < numel) ? W[e0 + 2] : 0.f;
-                v.w = (e0 + 3 < numel) ? W[e0 + 3] : 0.f;
-            }
+#pragma unroll
+        for (int it = 0; it < kIt; ++it) {
+            const int blk = warp * kBpw + lane / kLP + it * (kThreads / 32) * kBpw;
+            const int64_t e0 = (group * QLORA_GROUP + blk) * (4 * kLP) + sub * 4;
+            const float4 w = v[it];
+            bad |= !(isfinite(w.x) && isfinite(w.y) && isfinite(w.z) && isfinite(w.w));
+            float a = fmaxf(fmaxf(fabsf(w.x), fabsf(w.y)), fmaxf(fabsf(w.z), fabsf(w.w)));
+#pragma unroll
+            for (int o = kLP / 2; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+            const float r = __frcp_rn(a);
             uint32_t q0 = tab.zero_index, q1 = tab.zero_index, q2 = tab.zero_index,
                      q3 = tab.zero_index;
             if (a > 0.f) {
-                // |w| <= c_b, so x lies in [-1, 1]; the clamp only sends the NaN
-                // of a non-finite weight (flagged above) into the table's range
-                const float x0 = fminf(fmaxf(div_rn_by(v.x, a, r), -1.0f), 1.0f);
-                const float x1 = fminf(fmaxf(div_rn_by(v.y, a, r), -1.0f), 1.0f);
-                const float x2 = fminf(fmaxf(div_rn_by(v.z, a, r), -1.0f), 1.0f);
-                const float x3 = fminf(fmaxf(div_rn_by(v.w, a, r), -1.0f), 1.0f);
+                const float x0 = fminf(fmaxf(div_rn_by(w.x, a, r), -1.0f), 1.0f);
+                const float x1 = fminf(fmaxf(div_rn_by(w.y, a, r), -1.0f), 1.0f);
+                const float x2 = fminf(fmaxf(div_rn_by(w.z, a, r), -1.0f), 1.0f);
+                const float x3 = fminf(fmaxf(div_rn_by(w.w, a, r), -1.0f), 1.0f);
                 if (tab.use_lut) {
                     q0 = bucket_code(x0, lane_lut);
                     q1 = bucket_code(x1, lane_lut);
@@ -151,11 +138,75 @@ quantize_fmt_kernel(const float* __restrict__ W, int64_t numel, int64_t nblocks,
                     q3 = nearest_code(x3, smid);
                 }
             }
-            if (live)
-                *reinterpret_cast<uint16_t*>(packed + e0 / 2) =
-                    static_cast<uint16_t>(q0 | (q1 << 4) | (q2 << 8) | (q3 << 12));
+            *reinterpret_cast<uint16_t*>(packed + e0 / 2) =
+                static_cast<uint16_t>(q0 | (q1 << 4) | (q2 << 8) | (q3 << 12));
+            if (sub == 0) sabs[blk] = a;
         }
-        if (sub == 0) sabs[blk] = a;
+    } else {
+        const int lp = f.block >= 128 ? 32 : f.block / 4;        // lanes per block
+        const int bpw = 32 / lp;                                  // blocks per warp step
+        const int cpl = f.block / (4 * lp);                       // 16-byte pieces per lane
+        const int sub = lane % lp;
+
+        for (int blk = warp * bpw + lane / lp; blk < QLORA_GROUP; blk += (kThreads / 32) * bpw) {
+            const int64_t gblk = group * QLORA_GROUP + blk;
+            const int64_t ebase = gblk * f.block;
+            float a = 0.f;
+            for (int j = 0; j < cpl; ++j) {
+                const int64_t e0 = ebase + int64_t(j * lp + sub) * 4;
+                float4 v;
+                if (kFull) {
+                    v = *reinterpret_cast<const float4*>(W + e0);
+                } else {
+                    v.x = (e0 + 0 < numel) ? W[e0 + 0] : 0.f;
+                    v.y = (e0 + 1 < numel) ? W[e0 + 1] : 0.f;
+                    v.z = (e0 + 2 < numel) ? W[e0 + 2] : 0.f;
+                    v.w = (e0 + 3 < numel) ? W[e0 + 3] : 0.f;
+                }
+                bad |= !(isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w));
+                a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+            }
+            for (int o = lp / 2; o >= 1; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+            const float r = __frcp_rn(a);
+            const bool live = kFull || gblk < nblocks;
+            for (int j = 0; j < cpl; ++j) {
+                const int64_t e0 = ebase + int64_t(j * lp + sub) * 4;
+                float4 v;
+                if (kFull) {
+                    v = *reinterpret_cast<const float4*>(W + e0);
+                } else {
+                    v.x = (e0 + 0 < numel) ? W[e0 + 0] : 0.f;
+                    v.y = (e0 + 1 < numel) ? W[e0 + 1] : 0.f;
+                    v.z = (e0 + 2 < numel) ? W[e0 + 2] : 0.f;
+                    v.w = (e0 + 3 < numel) ? W[e0 + 3] : 0.f;
+                }
+                uint32_t q0 = tab.zero_index, q1 = tab.zero_index, q2 = tab.zero_index,
+                         q3 = tab.zero_index;
+                if (a > 0.f) {
+                    // |w| <= c_b, so x lies in [-1, 1]; the clamp only sends the NaN
+                    // of a non-finite weight (flagged above) into the table's range
+                    const float x0 = fminf(fmaxf(div_rn_by(v.x, a, r), -1.0f), 1.0f);
+                    const float x1 = fminf(fmaxf(div_rn_by(v.y, a, r), -1.0f), 1.0f);
+                    const float x2 = fminf(fmaxf(div_rn_by(v.z, a, r), -1.0f), 1.0f);
+                    const float x3 = fminf(fmaxf(div_rn_by(v.w, a, r), -1.0f), 1.0f);
+                    if (tab.use_lut) {
+                        q0 = bucket_code(x0, lane_lut);
+                        q1 = bucket_code(x1, lane_lut);
+                        q2 = bucket_code(x2, lane_lut);
+                        q3 = bucket_code(x3, lane_lut);
+                    } else {
+                        q0 = nearest_code(x0, smid);
+                        q1 = nearest_code(x1, smid);
+                        q2 = nearest_code(x2, smid);
+                        q3 = nearest_code(x3, smid);
+                    }
+                }
+                if (live)
+                    *reinterpret_cast<uint16_t*>(packed + e0 / 2) =
+                        static_cast<uint16_t>(q0 | (q1 << 4) | (q2 << 8) | (q3 << 12));
+            }
+            if (sub == 0) sabs[blk] = a;
+        }
     }
     if (bad && nonfinite_flag != nullptr) atomicOr(nonfinite_flag, 1);
     __syncthreads();
@@ -244,8 +295,16 @@ cudaError_t launch_quantize_fmt(const float* W, int64_t numel, const FmtArgs& f,
     const int64_t group_elems = int64_t(QLORA_GROUP) * f.block;
     const int64_t full = numel / group_elems;                // groups with no tail
     if (full > 0) {
-        quantize_fmt_kernel<true><<<dim3(static_cast<unsigned>(full)), kThreads, 0, stream>>>(
-            W, numel, nblocks, f, packed, scales, meta, nonfinite_flag, tab);
+        const dim3 grid(static_cast<unsigned>(full));
+        if (f.block == 16)
+            quantize_fmt_kernel<true, 4><<<grid, kThreads, 0, stream>>>(W, numel, nblocks, f, packed, scales,
+                                                                       meta, nonfinite_flag, tab);
+        else if (f.block == 32)
+            quantize_fmt_kernel<true, 8><<<grid, kThreads, 0, stream>>>(W, numel, nblocks, f, packed, scales,
+                                                                       meta, nonfinite_flag, tab);
+        else  // at B = 64 a lane would hold 64 floats; block by block measured faster there
+            quantize_fmt_kernel<true, 0><<<grid, kThreads, 0, stream>>>(W, numel, nblocks, f, packed, scales,
+                                                                       meta, nonfinite_flag, tab);
     }
     if (ngroups > full) {
         // the single trailing group, offset so blockIdx.x is its group index
@@ -254,7 +313,7 @@ cudaError_t launch_quantize_fmt(const float* W, int64_t numel, const FmtArgs& f,
         void* sc = f.scale_fmt == QLORA_SCALES_FP32
                        ? static_cast<void*>(static_cast<float*>(scales) + blk_off)
                        : static_cast<void*>(static_cast<uint8_t*>(scales) + blk_off);
-        quantize_fmt_kernel<false><<<1, kThreads, 0, stream>>>(
+        quantize_fmt_kernel<false, 0><<<1, kThreads, 0, stream>>>(
             W + off, numel - off, nblocks - blk_off, f, packed + off / 2, sc,
             meta == nullptr ? nullptr : meta + full, nonfinite_flag, tab);
     }

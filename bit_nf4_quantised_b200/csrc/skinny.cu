@@ -119,8 +119,8 @@ skinny_kernel(SkinnyArgs a) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) acc[j][t][e] = 0.f;
 
-#pragma unroll
     constexpr int kStages = Tl::kStages;
+#pragma unroll
     for (int st = 0; st < kStages - 1; ++st) {
         if (st < nchunks) load_stage(st, st);
         cp_async_commit();
