@@ -442,6 +442,22 @@ __device__ __forceinline__ float e4m3_to_float(uint8_t code) {
     return __half2float(__half(h));
 }
 
+// Double quantisation of a group's block scales into 8-bit codes: the
+// largest code value (E4M3 448, E5M2 57344, linear 255) the group constant
+// c2 = max / top maps onto, and a scale's code of x = fp32(c / c2): E4M3 and
+// E5M2 by the hardware's saturating round-to-nearest-even conversion, the
+// linear code as min(rint(x), 255) (ties to even).
+__device__ __forceinline__ float scale8_top(int fmt) {
+    return fmt == QLORA_SCALES_E4M3 ? 448.0f : fmt == QLORA_SCALES_E5M2 ? 57344.0f : 255.0f;
+}
+__device__ __forceinline__ uint8_t scale8_encode(float x, int fmt) {
+    if (fmt == QLORA_SCALES_E4M3)
+        return static_cast<uint8_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3));
+    if (fmt == QLORA_SCALES_E5M2)
+        return static_cast<uint8_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E5M2));
+    return static_cast<uint8_t>(fminf(rintf(x), 255.0f));
+}
+
 // Exact E5M2 -> fp32: E5M2 is the top byte of an fp16.
 __device__ __forceinline__ float e5m2_to_float(uint8_t code) {
     __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(code), __NV_E5M2);

@@ -226,20 +226,8 @@ quantize_fmt_kernel(const float* __restrict__ W, int64_t numel, int64_t nblocks,
     float gmax = sred[0];
 #pragma unroll
     for (int w = 1; w < kThreads / 32; ++w) gmax = fmaxf(gmax, sred[w]);
-    // the format's largest code value: E4M3 448, E5M2 57344, linear 255
-    const float top = f.scale_fmt == QLORA_SCALES_E4M3 ? 448.0f
-                    : f.scale_fmt == QLORA_SCALES_E5M2 ? 57344.0f : 255.0f;
-    const float c2 = __fdiv_rn(gmax, top);
-    uint8_t code = 0;
-    if (c2 > 0.f) {
-        const float x = __fdiv_rn(c, c2);
-        if (f.scale_fmt == QLORA_SCALES_E4M3)
-            code = static_cast<uint8_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3));
-        else if (f.scale_fmt == QLORA_SCALES_E5M2)
-            code = static_cast<uint8_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E5M2));
-        else
-            code = static_cast<uint8_t>(fminf(rintf(x), 255.0f));       // ties to even
-    }
+    const float c2 = __fdiv_rn(gmax, scale8_top(f.scale_fmt));
+    const uint8_t code = c2 > 0.f ? scale8_encode(__fdiv_rn(c, c2), f.scale_fmt) : uint8_t(0);
     if (live) reinterpret_cast<uint8_t*>(scales)[gblk] = code;
     if (tid == 0) meta[group] = c2;
 }
@@ -294,6 +282,9 @@ cudaError_t launch_quantize_fmt(const float* W, int64_t numel, const FmtArgs& f,
     const int64_t ngroups = (nblocks + QLORA_GROUP - 1) / QLORA_GROUP;
     const int64_t group_elems = int64_t(QLORA_GROUP) * f.block;
     const int64_t full = numel / group_elems;                // groups with no tail
+    if (f.block == 64 && tab.use_lut)      // K1's kernel, with this codebook and scale format
+        return launch_quantize_b64(W, numel, packed, scales, meta, nonfinite_flag, tab.lut,
+                                   tab.zero_index, f.scale_fmt, stream);
     if (full > 0) {
         const dim3 grid(static_cast<unsigned>(full));
         if (f.block == 16)

@@ -29,6 +29,13 @@ cudaError_t launch_dequantize(const uint8_t* packed, const uint8_t* scale_codes,
                               int64_t numel, uint16_t* out, const Nf4Table& tab, int num_sms,
                               cudaStream_t stream);
 
+// K1 with another codebook of the same blocksize (64): its bucket table, the
+// index of a zero block, and the scales as fp32 (QLORA_SCALES_FP32: c_b per
+// block, meta unused) or an 8-bit code with one fp32 constant per 256 blocks.
+cudaError_t launch_quantize_b64(const float* W, int64_t numel, uint8_t* packed, void* scales,
+                                float* meta, int* nonfinite_flag, const Nf4IndexLut& lut,
+                                uint32_t zero_index, int scale_fmt, cudaStream_t stream);
+
 // K1 on a bf16 weight (the re-quantisation of a merged export).
 cudaError_t launch_quantize_bf16(const uint16_t* W, int64_t numel, uint8_t* packed,
                                  uint8_t* scale_codes, float* meta, int* nonfinite_flag,

@@ -114,8 +114,9 @@ __device__ __forceinline__ uint32_t code_index(float x, uint32_t lane_lut) {
 template <bool kFull, typename Tin>
 __global__ void __launch_bounds__(kThreads, 2)
 quantize_kernel(const Tin* __restrict__ W, int64_t numel, int64_t nblocks,
-                uint8_t* __restrict__ packed, uint8_t* __restrict__ scale_codes,
-                float* __restrict__ meta, int* __restrict__ nonfinite_flag, Nf4IndexLut lut) {
+                uint8_t* __restrict__ packed, void* __restrict__ scales,
+                float* __restrict__ meta, int* __restrict__ nonfinite_flag, Nf4IndexLut lut,
+                uint32_t zero_word, int scale_fmt) {
     extern __shared__ __align__(16) uint8_t smem[];                // the per-lane table
     __shared__ float sabs[QLORA_GROUP];
     __shared__ float sred[QLORA_GROUP / 32];
@@ -158,7 +159,7 @@ quantize_kernel(const Tin* __restrict__ W, int64_t numel, int64_t nblocks,
         for (int o = 4; o >= 1; o >>= 1) a = max_nan(a, __shfl_xor_sync(0xffffffffu, a, o));
         bad |= !(a <= FLT_MAX);                                // NaN or infinity in the block
         // a = c_b for this block
-        uint32_t word = 0x77777777u;                            // zero block -> code 0
+        uint32_t word = zero_word;                              // zero block -> the code of 0
         if (a > 0.f) {
             word = 0;
             if (a >= 0x1p-90f && a <= 0x1p90f) {
@@ -177,9 +178,15 @@ quantize_kernel(const Tin* __restrict__ W, int64_t numel, int64_t nblocks,
     if (bad && sub == 0 && nonfinite_flag != nullptr) atomicOr(nonfinite_flag, 1);
     __syncthreads();
 
-    // Double quantisation of this group's 256 scales (the first 8 warps).
+    // Double quantisation of this group's 256 scales (the first 8 warps), or
+    // the fp32 scales themselves.
     if (tid < QLORA_GROUP) {
         const float c = sabs[tid];
+        const int64_t gblk = group * QLORA_GROUP + tid;
+        if (scale_fmt == QLORA_SCALES_FP32) {
+            if (kFull || gblk < nblocks) reinterpret_cast<float*>(scales)[gblk] = c;
+            return;
+        }
         float m = c;
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -188,45 +195,49 @@ quantize_kernel(const Tin* __restrict__ W, int64_t numel, int64_t nblocks,
         float gmax = sred[0];
 #pragma unroll
         for (int w = 1; w < QLORA_GROUP / 32; ++w) gmax = fmaxf(gmax, sred[w]);
-        const float c2 = __fdiv_rn(gmax, 448.0f);
-        uint8_t code = 0;
-        if (c2 > 0.f) {
-            code = static_cast<uint8_t>(
-                __nv_cvt_float_to_fp8(__fdiv_rn(c, c2), __NV_SATFINITE, __NV_E4M3));
-        }
-        const int64_t gblk = group * QLORA_GROUP + tid;
-        if (kFull || gblk < nblocks) scale_codes[gblk] = code;
+        const float c2 = __fdiv_rn(gmax, scale8_top(scale_fmt));
+        const uint8_t code = c2 > 0.f ? scale8_encode(__fdiv_rn(c, c2), scale_fmt) : uint8_t(0);
+        if (kFull || gblk < nblocks) reinterpret_cast<uint8_t*>(scales)[gblk] = code;
         if (tid == 0) meta[group] = c2;
     }
 }
 
+// index of the exact zero among the NF4 codes: a zero block's word
+constexpr uint32_t kNf4ZeroWord = 0x77777777u;
+
 template <bool kFull, typename Tin>
 cudaError_t launch_one(unsigned grid, const Tin* W, int64_t numel, int64_t nblocks, uint8_t* packed,
-                       uint8_t* scale_codes, float* meta, int* nonfinite_flag,
-                       const Nf4IndexLut& lut, cudaStream_t stream) {
+                       void* scales, float* meta, int* nonfinite_flag, const Nf4IndexLut& lut,
+                       uint32_t zero_word, int scale_fmt, cudaStream_t stream) {
     quantize_kernel<kFull, Tin><<<grid, kThreads, kLutBytes, stream>>>(
-        W, numel, nblocks, packed, scale_codes, meta, nonfinite_flag, lut);
+        W, numel, nblocks, packed, scales, meta, nonfinite_flag, lut, zero_word, scale_fmt);
     return cudaGetLastError();
 }
 
 template <typename Tin>
-cudaError_t quantize_any(const Tin* W, int64_t numel, uint8_t* packed, uint8_t* scale_codes,
-                         float* meta, int* nonfinite_flag, const Nf4IndexLut& lut,
-                         cudaStream_t stream) {
+cudaError_t quantize_any(const Tin* W, int64_t numel, uint8_t* packed, void* scales, float* meta,
+                         int* nonfinite_flag, const Nf4IndexLut& lut, uint32_t zero_word,
+                         int scale_fmt, cudaStream_t stream) {
     const int64_t nblocks = (numel + QLORA_BLOCK - 1) / QLORA_BLOCK;
     const int64_t ngroups = (nblocks + QLORA_GROUP - 1) / QLORA_GROUP;
     const int64_t full = numel / kGroupElems;                  // groups with no tail
     if (full > 0) {
         const cudaError_t e = launch_one<true>(static_cast<unsigned>(full), W, numel, nblocks, packed,
-                                               scale_codes, meta, nonfinite_flag, lut, stream);
+                                               scales, meta, nonfinite_flag, lut, zero_word,
+                                               scale_fmt, stream);
         if (e != cudaSuccess) return e;
     }
     if (ngroups > full) {
         // the single trailing group, offset so blockIdx.x is its group index
         const int64_t off = full * kGroupElems;
-        return launch_one<false>(1u, W + off, numel - off, nblocks - full * QLORA_GROUP,
-                                 packed + full * (kGroupElems / 2), scale_codes + full * QLORA_GROUP,
-                                 meta + full, nonfinite_flag, lut, stream);
+        const int64_t blk_off = full * QLORA_GROUP;
+        void* sc = scale_fmt == QLORA_SCALES_FP32
+                       ? static_cast<void*>(static_cast<float*>(scales) + blk_off)
+                       : static_cast<void*>(static_cast<uint8_t*>(scales) + blk_off);
+        return launch_one<false>(1u, W + off, numel - off, nblocks - blk_off,
+                                 packed + full * (kGroupElems / 2), sc,
+                                 meta == nullptr ? nullptr : meta + full, nonfinite_flag, lut,
+                                 zero_word, scale_fmt, stream);
     }
     return cudaSuccess;
 }
@@ -236,13 +247,22 @@ cudaError_t quantize_any(const Tin* W, int64_t numel, uint8_t* packed, uint8_t* 
 cudaError_t launch_quantize(const float* W, int64_t numel, uint8_t* packed, uint8_t* scale_codes,
                             float* meta, int* nonfinite_flag, const Nf4IndexLut& lut,
                             cudaStream_t stream) {
-    return quantize_any(W, numel, packed, scale_codes, meta, nonfinite_flag, lut, stream);
+    return quantize_any(W, numel, packed, scale_codes, meta, nonfinite_flag, lut, kNf4ZeroWord,
+                        QLORA_SCALES_E4M3, stream);
+}
+
+cudaError_t launch_quantize_b64(const float* W, int64_t numel, uint8_t* packed, void* scales,
+                                float* meta, int* nonfinite_flag, const Nf4IndexLut& lut,
+                                uint32_t zero_index, int scale_fmt, cudaStream_t stream) {
+    return quantize_any(W, numel, packed, scales, meta, nonfinite_flag, lut, zero_index * 0x11111111u,
+                        scale_fmt, stream);
 }
 
 cudaError_t launch_quantize_bf16(const uint16_t* W, int64_t numel, uint8_t* packed,
                                  uint8_t* scale_codes, float* meta, int* nonfinite_flag,
                                  const Nf4IndexLut& lut, cudaStream_t stream) {
-    return quantize_any(W, numel, packed, scale_codes, meta, nonfinite_flag, lut, stream);
+    return quantize_any(W, numel, packed, scale_codes, meta, nonfinite_flag, lut, kNf4ZeroWord,
+                        QLORA_SCALES_E4M3, stream);
 }
 
 }  // namespace qnf4
