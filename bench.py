@@ -42,8 +42,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 LAUNCHES_PER_STEP = 2 + 4
 # ncu DRAM traffic (read + write bytes) of one dequant-GEMM launch of this
 # workload, valid only for the sources it was captured on (_source_sha).
-GEMM_TRAFFIC = {"source_sha": "b8581179eda348e5", "fwd_bytes": (44.550144 + 8.004608) * 1e6,
-                "dx_bytes": (44.379648 + 6.835968) * 1e6}
+GEMM_TRAFFIC = {"source_sha": "e1cb81df73c9acac", "fwd_bytes": (44.599552 + 6.562304) * 1e6,
+                "dx_bytes": (44.409344 + 3.521536) * 1e6}
 
 
 def _peaks():
@@ -962,7 +962,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
