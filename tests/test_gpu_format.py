@@ -1,6 +1,6 @@
 """GPU parity of the format variants (qlora_quantize_fmt / qlora_dequantize_fmt)
-against the oracle through the C-ABI: NF4, E2M1 FP4 and INT4 codebooks,
-blocksizes 16 to 4096, fp32 scales or scales double-quantised to E4M3, E5M2
+against the oracle through the C-ABI: NF4, E2M1 FP4 and INT4 codebooks and
+one too dense for the quantiser's bucket table, blocksizes 16 to 4096, fp32 scales or scales double-quantised to E4M3, E5M2
 or a linear 8-bit code, bit-exact indices,
 scales and dequantised bf16; and the toy statistics of "A toy run ..."
 (relative MSE on 2^20 Gaussian weights) reproduced from the GPU's outputs."""
@@ -26,7 +26,11 @@ def q():
     return pkg
 
 
-BOOKS = {"nf4": o.nf4_codebook()[0], "fp4": o.fp4_e2m1_codebook(), "int4": o.int4_codebook()}
+# "dense": codes 0.01 apart near 0, closer than the 1/16 buckets of the
+# quantiser's index table, so the kernel takes its search over the midpoints
+BOOKS = {"nf4": o.nf4_codebook()[0], "fp4": o.fp4_e2m1_codebook(), "int4": o.int4_codebook(),
+         "dense": np.array([-1.0, -0.5, -0.2, -0.1, -0.05, -0.02, -0.01, 0.0, 0.01, 0.02, 0.05,
+                            0.1, 0.2, 0.5, 0.75, 1.0], np.float32)}
 
 
 def _fmt(q, cb, block, scales):
@@ -44,6 +48,12 @@ CASES = [
     ("fp4", 512, o.SCALES_FP32, 512 * 300 + 1),
     ("int4", 4096, o.SCALES_E4M3, 4096 * 256 + 4096 * 3 + 77),
     ("nf4", 64, o.SCALES_E4M3, 1),
+    # blocksize 32 (a lane's share of the group held in registers)
+    ("nf4", 32, o.SCALES_E5M2, 32 * 256 * 4),
+    ("fp4", 32, o.SCALES_U8, 32 * 256 * 2 + 31),
+    # a codebook too dense for the index table: the search over the midpoints
+    ("dense", 64, o.SCALES_E4M3, 64 * 256 * 2 + 33),
+    ("dense", 32, o.SCALES_FP32, 32 * 256 * 3 + 17),
     # the other 8-bit encodings of the double-quantised scales
     ("nf4", 64, o.SCALES_E5M2, 64 * 256 * 3 + 130),
     ("nf4", 64, o.SCALES_U8, 64 * 256 * 3 + 130),
