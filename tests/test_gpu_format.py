@@ -30,7 +30,10 @@ def q():
 # quantiser's index table, so the kernel takes its search over the midpoints
 BOOKS = {"nf4": o.nf4_codebook()[0], "fp4": o.fp4_e2m1_codebook(), "int4": o.int4_codebook(),
          "dense": np.array([-1.0, -0.5, -0.2, -0.1, -0.05, -0.02, -0.01, 0.0, 0.01, 0.02, 0.05,
-                            0.1, 0.2, 0.5, 0.75, 1.0], np.float32)}
+                            0.1, 0.2, 0.5, 0.75, 1.0], np.float32),
+         # 8 codes with no exact zero: 0 lies on a midpoint and takes the lower
+         # code (index 3), so zero blocks and padding do not take index 7
+         "grid8": np.linspace(-1.0, 1.0, 8).astype(np.float32)}
 
 
 def _fmt(q, cb, block, scales):
@@ -51,6 +54,9 @@ CASES = [
     # blocksize 32 (a lane's share of the group held in registers)
     ("nf4", 32, o.SCALES_E5M2, 32 * 256 * 4),
     ("fp4", 32, o.SCALES_U8, 32 * 256 * 2 + 31),
+    # fewer than 15 codes (several +inf midpoints), zero index 3
+    ("grid8", 64, o.SCALES_E4M3, 64 * 256 * 2 + 70),
+    ("grid8", 16, o.SCALES_FP32, 16 * 256 + 5),
     # a codebook too dense for the index table: the search over the midpoints
     ("dense", 64, o.SCALES_E4M3, 64 * 256 * 2 + 33),
     ("dense", 32, o.SCALES_FP32, 32 * 256 * 3 + 17),
