@@ -468,9 +468,10 @@ def _decoder_measure(q, syn, device, steps=2):
 def _export_measure(q, lins, ws, act, kind, device, reps=3):
     """Export of the whole fine-tuned decoder: every one of the 224 stored
     weights merged with its adapter into its own slice of one bf16 buffer
-    (13 GB, far beyond L2), timed with CUDA events over the 224 launches;
-    then the same buffer re-quantised to NF4, and, for comparison, the plain
-    dequantisation of every weight.  GB/s are algorithmic bytes: the stored
+    (13 GB, far beyond L2) by one qlora_merge_many call (16 weights per
+    launch), timed with CUDA events, and beside it the same merges as 224
+    qlora_merge calls; then the same buffer re-quantised to NF4, and, for
+    comparison, the plain dequantisation of every weight.  GB/s are algorithmic bytes: the stored
     weight read, the adapter read and the bf16 weight written (merge), the
     bf16 read and the stored weight written (re-quantise)."""
     params = sum(l.N * l.K for l in lins)
@@ -495,6 +496,10 @@ def _export_measure(q, lins, ws, act, kind, device, reps=3):
         return b.elapsed_time(e) / reps
 
     def merge_all():
+        q.qlora_merge_many([(w, act[kind(l)]["A"], act[kind(l)]["B"], l.gamma, v)
+                            for l, w, v in zip(lins, ws, views)])
+
+    def merge_each():
         for l, w, v in zip(lins, ws, views):
             a = act[kind(l)]
             q.qlora_merge(w, a["A"], a["B"], l.gamma, out=v)
@@ -508,6 +513,7 @@ def _export_measure(q, lins, ws, act, kind, device, reps=3):
             q.qlora_dequantize(w, out=v)
 
     m_ms = timed(merge_all)
+    m1_ms = timed(merge_each)
     r_ms = timed(requant_all)
     d_ms = timed(dequant_all)
     m_bytes = stored + adapter + params * 2
@@ -517,6 +523,8 @@ def _export_measure(q, lins, ws, act, kind, device, reps=3):
     return {"linears": len(lins), "params": params,
             "merge_ms": round(m_ms, 3), "merge_GBps": round(m_bytes / (m_ms * 1e-3) / 1e9, 1),
             "merge_bytes": m_bytes,
+            "merge_one_by_one_ms": round(m1_ms, 3),
+            "merge_one_by_one_GBps": round(m_bytes / (m1_ms * 1e-3) / 1e9, 1),
             "requantize_ms": round(r_ms, 3),
             "requantize_GBps": round(r_bytes / (r_ms * 1e-3) / 1e9, 1),
             "dequantize_ms": round(d_ms, 3),
@@ -725,7 +733,7 @@ def run_gpu(args):
         out["decoder"] = _decoder_measure(q, syn, device)
         out["decoder"]["frac_bf16"] = round(out["decoder"]["fwd_bwd_TFLOPs"] / peak, 4)
         ex = out["decoder"]["export"]
-        for k in ("merge", "requantize", "dequantize"):
+        for k in ("merge", "merge_one_by_one", "requantize", "dequantize"):
             ex[f"{k}_frac_hbm"] = round(ex[f"{k}_GBps"] / peaks["hbm_gbs"], 4)
         try:
             out["merge"] = _merge_measure(q, syn, device)

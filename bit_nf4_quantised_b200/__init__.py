@@ -29,6 +29,7 @@ from ._lib import (  # noqa: F401
     qlora_linear_forward,
     qlora_linear_workspace_size,
     qlora_merge,
+    qlora_merge_many,
     qlora_mlp_backward,
     qlora_mlp_forward,
     qlora_mlp_workspace_size,

@@ -43,6 +43,7 @@ EXPORTED = (
     "qlora_linear_forward_noalloc",
     "qlora_linear_forward_noalloc_error_word",
     "qlora_merge",
+    "qlora_merge_many",
     "qlora_quantize_bf16",
     "qlora_format_sizes",
     "qlora_quantize_fmt",
@@ -84,6 +85,17 @@ def _events(events):
             ev.record()
         handles.append(ev.cuda_event)
     return ctypes.byref(_Events(*handles))
+
+
+class _MergeJob(ctypes.Structure):
+    _fields_ = [
+        ("w", ctypes.c_void_p),          # const qlora_nf4_tensor*
+        ("A", ctypes.c_void_p),
+        ("B", ctypes.c_void_p),
+        ("r", ctypes.c_int),
+        ("scale", ctypes.c_float),
+        ("W_out", ctypes.c_void_p),
+    ]
 
 
 class _Tensor(ctypes.Structure):
@@ -146,6 +158,7 @@ def lib() -> ctypes.CDLL:
         L.qlora_dequantize.argtypes = [tp, vp, vp]
         L.qlora_quantize_bf16.argtypes = [vp, tp, vp, vp]
         L.qlora_merge.argtypes = [tp, vp, vp, i32, f32, vp, vp]
+        L.qlora_merge_many.argtypes = [ctypes.POINTER(_MergeJob), i32, vp]
         fp = ctypes.POINTER(_Format)
         L.qlora_format_sizes.argtypes = [i64, fp, sz, sz, sz]
         L.qlora_quantize_fmt.argtypes = [vp, i64, fp, vp, vp, vp, vp, vp]
@@ -290,6 +303,27 @@ def qlora_merge(w: NF4Tensor, A: torch.Tensor, B: torch.Tensor, scale: float,
     _check(lib().qlora_merge(ctypes.byref(st), A.data_ptr(), B.data_ptr(), r, float(scale),
                              out.data_ptr(), _stream(stream)), "qlora_merge")
     return out
+
+
+def qlora_merge_many(jobs, stream=None) -> list:
+    """qlora_merge of several weights in as few launches as the library needs.
+    jobs: sequence of (w, A, B, scale, out) with out None or a bf16 [rows,
+    cols] tensor; returns the outputs in order."""
+    outs, structs = [], []
+    for w, A, B, scale, out in jobs:
+        _need(A, torch.bfloat16, "A")
+        _need(B, torch.bfloat16, "B")
+        out = out if out is not None else torch.empty(w.rows, w.cols, dtype=torch.bfloat16,
+                                                      device=w.packed.device)
+        _need(out, torch.bfloat16, "out")
+        outs.append(out)
+        structs.append((w.c_struct(), A, B, float(scale), out))
+    arr = (_MergeJob * max(1, len(structs)))()
+    for i, (st, A, B, scale, out) in enumerate(structs):
+        arr[i] = _MergeJob(ctypes.addressof(st), A.data_ptr(), B.data_ptr(), A.shape[0], scale,
+                           out.data_ptr())
+    _check(lib().qlora_merge_many(arr, len(structs), _stream(stream)), "qlora_merge_many")
+    return outs
 
 
 @dataclass

@@ -94,7 +94,11 @@ struct MergeArgs {
     int64_t tiles;               // CTA units of 16 rows x 512 columns (set by launch_merge)
 };
 int merge_smem_bytes(int r);
-cudaError_t launch_merge(const MergeArgs& a, const Nf4Table& tab, int num_sms, cudaStream_t stream);
+// Up to kMaxMergeJobs weights merged by one launch: their CTA units form one
+// sequence (job 0's first), dealt to the CTAs in equal runs.
+constexpr int kMaxMergeJobs = 16;
+cudaError_t launch_merge(const MergeArgs* jobs, int n, const Nf4Table& tab, int num_sms,
+                         cudaStream_t stream);
 
 // ---------------------------------------------------------------- K2 / K3
 struct GemmArgs {

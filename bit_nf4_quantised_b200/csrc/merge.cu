@@ -71,12 +71,22 @@ struct WeightRegs {
     float mt[2];
 };
 
+// The weights of one launch: their units in sequence (first[j] = the index of
+// job j's first unit, first[n] = the total), the slabs sized for the largest
+// rank among them.
+struct MergeBatch {
+    MergeArgs job[kMaxMergeJobs];
+    int64_t first[kMaxMergeJobs + 1];
+    int n;
+    int rp_max;
+};
+
 __global__ void __launch_bounds__(kThreads)
-merge_kernel(MergeArgs a, Nf4Table tab) {
+merge_kernel(const __grid_constant__ MergeBatch bt, Nf4Table tab) {
     extern __shared__ __align__(16) uint8_t smem[];
     float* scode = reinterpret_cast<float*>(smem + kCodesOff);            // 16 codes
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint16_t* slab = reinterpret_cast<uint16_t*>(smem + kSlabOff + warp * slab_bytes(a.rp));
+    uint16_t* slab = reinterpret_cast<uint16_t*>(smem + kSlabOff + warp * slab_bytes(bt.rp_max));
     if (threadIdx.x == 0) {            // constant indices: no local copy of the table
 #pragma unroll
         for (int q = 0; q < 16; ++q) scode[q] = tab.code[q];
@@ -96,11 +106,11 @@ merge_kernel(MergeArgs a, Nf4Table tab) {
     const int g = lane >> 2, tq = lane & 3;
     // N and K are below 2^31 (checked on the host); products of a row and K
     // are formed in 64 bits.
-    const int N = static_cast<int>(a.N), K = static_cast<int>(a.K);
-    const int row_tiles = (N + kTileRows - 1) / kTileRows;
-    const int kblocks = K / kStrip;            // NF4 blocks (strips) per row
-    const int64_t u_begin = a.tiles * blockIdx.x / gridDim.x;
-    const int64_t u_end = a.tiles * (blockIdx.x + 1) / gridDim.x;
+    const int64_t total = bt.first[bt.n];
+    const int64_t u_begin = total * blockIdx.x / gridDim.x;
+    const int64_t u_end = total * (blockIdx.x + 1) / gridDim.x;
+    auto rows_of = [&](int j) { return (static_cast<int>(bt.job[j].N) + kTileRows - 1) / kTileRows; };
+    auto cblocks_of = [&](int j) { return (static_cast<int>(bt.job[j].K) / kStrip + kWarps - 1) / kWarps; };
 
     // The slab position lane l fills: A's physical columns 2l, 2l+1 are
     // logical columns p0, p0 + 1 of the strip (see the column map above).
@@ -119,8 +129,12 @@ merge_kernel(MergeArgs a, Nf4Table tab) {
     const int qbase = lane & ~3;
     const int src_a = qbase + (tq >> 1), src_b = qbase + 2 + (tq >> 1);
 
-    // Unit (column block cb, row tile rt); units advance row tile first.
-    auto load_unit = [&](int cb, int rt, WeightRegs& wr) {
+    // Unit (job j, column block cb, row tile rt); units advance row tile
+    // first, then column block, then job.
+    auto load_unit = [&](int j, int cb, int rt, WeightRegs& wr) {
+        const MergeArgs& a = bt.job[j];
+        const int N = static_cast<int>(a.N), K = static_cast<int>(a.K);
+        const int kblocks = K / kStrip;
         const int strip = cb * kWarps + warp;
 #pragma unroll
         for (int s = 0; s < 2; ++s) {
@@ -151,20 +165,40 @@ merge_kernel(MergeArgs a, Nf4Table tab) {
         }
     };
 
-    int cb = static_cast<int>(u_begin / row_tiles);
-    int rt = static_cast<int>(u_begin - int64_t(cb) * row_tiles);
-    int ncb = cb, nrt = rt + 1;
-    if (nrt == row_tiles) { nrt = 0; ++ncb; }
+    int j = 0;
+    while (j + 1 < bt.n && bt.first[j + 1] <= u_begin) ++j;
+    int cb, rt;
+    {
+        const int64_t local = u_begin - bt.first[j];
+        const int rtj = rows_of(j);
+        cb = static_cast<int>(local / rtj);
+        rt = static_cast<int>(local - int64_t(cb) * rtj);
+    }
+    // the unit after (j, cb, rt)
+    auto advance = [&](int& jj, int& cc, int& rr) {
+        if (++rr == rows_of(jj)) {
+            rr = 0;
+            if (++cc == cblocks_of(jj)) {
+                cc = 0;
+                ++jj;
+            }
+        }
+    };
+    int nj = j, ncb = cb, nrt = rt;
+    advance(nj, ncb, nrt);
     WeightRegs cur, nxt;
-    if (u_begin < u_end) load_unit(cb, rt, cur);
-    int cur_cb = -1;
+    if (u_begin < u_end) load_unit(j, cb, rt, cur);
+    int cur_j = -1, cur_cb = -1;
     for (int64_t u = u_begin; u < u_end; ++u) {
-        if (u + 1 < u_end) load_unit(ncb, nrt, nxt);
+        if (u + 1 < u_end) load_unit(nj, ncb, nrt, nxt);
         exchange(cur);
+        const MergeArgs& a = bt.job[j];
+        const int N = static_cast<int>(a.N), K = static_cast<int>(a.K);
+        const int kblocks = K / kStrip;
         const int strip = cb * kWarps + warp;
         if (strip < kblocks) {
             const int c0 = strip * kStrip;
-            if (cb != cur_cb) {
+            if (cb != cur_cb || j != cur_j) {
                 __syncwarp();
                 for (int k = 0; k < a.rp; ++k) {
                     uint32_t v = 0u;
@@ -173,6 +207,7 @@ merge_kernel(MergeArgs a, Nf4Table tab) {
                 }
                 __syncwarp();
                 cur_cb = cb;
+                cur_j = j;
             }
             const int n0 = rt * kTileRows;
 
@@ -230,9 +265,10 @@ merge_kernel(MergeArgs a, Nf4Table tab) {
             }
         }
         cur = nxt;
+        j = nj;
         cb = ncb;
         rt = nrt;
-        if (++nrt == row_tiles) { nrt = 0; ++ncb; }
+        if (u + 1 < u_end) advance(nj, ncb, nrt);
     }
 }
 
@@ -243,14 +279,28 @@ int merge_smem_bytes(int r) {
     return kSlabOff + kWarps * slab_bytes(rp);
 }
 
-cudaError_t launch_merge(const MergeArgs& args, const Nf4Table& tab, int num_sms,
+cudaError_t launch_merge(const MergeArgs* jobs, int n, const Nf4Table& tab, int num_sms,
                          cudaStream_t stream) {
-    MergeArgs a = args;
-    a.rp = (a.r + 15) / 16 * 16;
-    const int64_t col_blocks = (a.K / kStrip + kWarps - 1) / kWarps;
-    a.tiles = col_blocks * ((a.N + kTileRows - 1) / kTileRows);      // CTA units
-    if (a.tiles == 0) return cudaSuccess;
-    const int smem = merge_smem_bytes(a.r);
+    if (n < 1 || n > kMaxMergeJobs) return cudaErrorInvalidValue;
+    MergeBatch bt{};
+    bt.n = 0;
+    bt.rp_max = 16;
+    int64_t total = 0;
+    for (int i = 0; i < n; ++i) {
+        MergeArgs a = jobs[i];
+        a.rp = (a.r + 15) / 16 * 16;
+        const int64_t col_blocks = (a.K / kStrip + kWarps - 1) / kWarps;
+        a.tiles = col_blocks * ((a.N + kTileRows - 1) / kTileRows);   // CTA units
+        if (a.tiles == 0) continue;
+        bt.job[bt.n] = a;
+        bt.first[bt.n] = total;
+        total += a.tiles;
+        if (a.rp > bt.rp_max) bt.rp_max = a.rp;
+        ++bt.n;
+    }
+    bt.first[bt.n] = total;
+    if (total == 0) return cudaSuccess;
+    const int smem = merge_smem_bytes(bt.rp_max);
     cudaError_t e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          smem);
     if (e != cudaSuccess) return e;
@@ -259,8 +309,8 @@ cudaError_t launch_merge(const MergeArgs& args, const Nf4Table& tab, int num_sms
     if (e != cudaSuccess) return e;
     if (per_sm < 1) per_sm = 1;
     int64_t grid = int64_t(num_sms) * per_sm;
-    if (grid > a.tiles) grid = a.tiles;                           // at least one unit per CTA
-    merge_kernel<<<dim3(static_cast<unsigned>(grid)), kThreads, smem, stream>>>(a, tab);
+    if (grid > total) grid = total;                               // at least one unit per CTA
+    merge_kernel<<<dim3(static_cast<unsigned>(grid)), kThreads, smem, stream>>>(bt, tab);
     return cudaGetLastError();
 }
 

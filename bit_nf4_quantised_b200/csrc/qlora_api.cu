@@ -613,31 +613,81 @@ int qlora_adamw8_step(float* p, const float* g, int64_t n, int8_t* m_codes, floa
     return cuda_status(launch_adamw8(a, num_sms(), reinterpret_cast<cudaStream_t>(stream)));
 }
 
-int qlora_merge(const qlora_nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r,
-                float scale, uint16_t* W_out, qlora_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Checks one merge and fills its kernel arguments; *skip = true when the
+// weight is empty (nothing read or written).
+int merge_job_args(const qlora_nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r,
+                   float scale, uint16_t* W_out, MergeArgs* a, bool* skip) {
+    *skip = false;
     if (!w) return QLORA_ERR_NULL;
     const int64_t N = w->rows, K = w->cols;
     if (N < 0 || K < 0 || (K > 0 && N > INT64_MAX / K)) return QLORA_ERR_SHAPE;
     if (K % QLORA_BLOCK != 0) return QLORA_ERR_UNSUPPORTED;
     if (r < 8 || r > QLORA_MAX_RANK || r % 8 != 0) return QLORA_ERR_UNSUPPORTED;
     if (N > (int64_t(1) << 31) - 1 || K > (int64_t(1) << 31) - 1) return QLORA_ERR_UNSUPPORTED;
-    if (N == 0 || K == 0) return QLORA_OK;              // nothing read or written
+    if (N == 0 || K == 0) {
+        *skip = true;
+        return QLORA_OK;
+    }
     int st = check_tensor(w);
     if (st != QLORA_OK) return st;
     if (!A || !B || !W_out) return QLORA_ERR_NULL;
     if (!aligned(A, 16) || !aligned(B, 16) || !aligned(W_out, 16)) return QLORA_ERR_ALIGN;
-    MergeArgs a{};
-    a.packed = reinterpret_cast<const uint32_t*>(w->packed);
-    a.scale_codes = w->scale_codes;
-    a.meta = w->meta_scale;
-    a.A = A;
-    a.B = B;
-    a.out = W_out;
-    a.N = N;
-    a.K = K;
-    a.r = r;
-    a.gamma = scale;
-    return cuda_status(launch_merge(a, table(), num_sms(), reinterpret_cast<cudaStream_t>(stream)));
+    *a = MergeArgs{};
+    a->packed = reinterpret_cast<const uint32_t*>(w->packed);
+    a->scale_codes = w->scale_codes;
+    a->meta = w->meta_scale;
+    a->A = A;
+    a->B = B;
+    a->out = W_out;
+    a->N = N;
+    a->K = K;
+    a->r = r;
+    a->gamma = scale;
+    return QLORA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qlora_merge(const qlora_nf4_tensor* w, const uint16_t* A, const uint16_t* B, int r,
+                float scale, uint16_t* W_out, qlora_stream_t stream) {
+    MergeArgs a;
+    bool skip = false;
+    const int st = merge_job_args(w, A, B, r, scale, W_out, &a, &skip);
+    if (st != QLORA_OK || skip) return st;
+    return cuda_status(launch_merge(&a, 1, table(), num_sms(), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int qlora_merge_many(const qlora_merge_job* jobs, int n, qlora_stream_t stream) {
+    if (n < 0) return QLORA_ERR_SHAPE;
+    if (n > 0 && !jobs) return QLORA_ERR_NULL;
+    // every job is checked before anything is launched
+    for (int i = 0; i < n; ++i) {
+        MergeArgs a;
+        bool skip = false;
+        const int st = merge_job_args(jobs[i].w, jobs[i].A, jobs[i].B, jobs[i].r, jobs[i].scale,
+                                      jobs[i].W_out, &a, &skip);
+        if (st != QLORA_OK) return st;
+    }
+    MergeArgs batch[kMaxMergeJobs];
+    int k = 0;
+    for (int i = 0; i < n; ++i) {
+        bool skip = false;
+        merge_job_args(jobs[i].w, jobs[i].A, jobs[i].B, jobs[i].r, jobs[i].scale, jobs[i].W_out,
+                       &batch[k], &skip);
+        if (skip) continue;
+        if (++k == kMaxMergeJobs) {
+            QTRY(launch_merge(batch, k, table(), num_sms(), reinterpret_cast<cudaStream_t>(stream)));
+            k = 0;
+        }
+    }
+    if (k > 0) QTRY(launch_merge(batch, k, table(), num_sms(), reinterpret_cast<cudaStream_t>(stream)));
+    return QLORA_OK;
 }
 
 int qlora_linear_workspace_size(int64_t M, int64_t N, int64_t K, int r, size_t* bytes) {

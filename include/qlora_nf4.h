@@ -312,6 +312,32 @@ QLORA_API int qlora_merge(const qlora_nf4_tensor* w, const uint16_t* A, const ui
                           int r, float scale, uint16_t* W_out, qlora_stream_t stream);
 
 /*
+ * qlora_merge_many -- qlora_merge of several weights, e.g. every adapted
+ * linear of a model at export, with up to 16 of them per kernel launch: a
+ * launch deals the weights' units of work to the GPU as one sequence, so
+ * small weights do not each pay a launch's ramp and tail.  Each job's result
+ * is bit for bit what qlora_merge gives for it.
+ *   jobs  (host array of n qlora_merge_job, read): one merge each, with the
+ *         arguments and rules of qlora_merge; the jobs' W_out must not
+ *         overlap one another or any job's inputs.  Ranks may differ.
+ *   n     >= 0 (0 launches nothing).
+ * Every job is checked before anything is launched; the first failing job's
+ * status is returned and nothing runs.
+ * Errors: those of qlora_merge; QLORA_ERR_NULL (jobs NULL with n > 0),
+ * QLORA_ERR_SHAPE (n < 0).
+ */
+typedef struct {
+    const qlora_nf4_tensor* w;   /* host struct, read */
+    const uint16_t* A;           /* device, bf16, r x K */
+    const uint16_t* B;           /* device, bf16, N x r */
+    int r;
+    float scale;
+    uint16_t* W_out;             /* device, bf16, N x K */
+} qlora_merge_job;
+
+QLORA_API int qlora_merge_many(const qlora_merge_job* jobs, int n, qlora_stream_t stream);
+
+/*
  * qlora_quantize_bf16 -- qlora_quantize of a bf16 weight (each value widened
  * exactly to fp32 first), the re-quantisation of a merged weight for a 4-bit
  * deployment ("QLoRA" (finetunellm.com), "What it costs you": merging into

@@ -137,6 +137,31 @@ def _books():
             "int4": tuple(o.int4_codebook())}
 
 
+def test_merge_many_checks_every_job_before_any_launch(q):
+    """qlora_merge_many validates all its jobs on the host first: one bad job
+    (rank 12, a misaligned output, a null adapter) fails the whole call with
+    that job's status and nothing is launched (the fake device pointers are
+    never touched); an empty list and empty weights launch nothing."""
+    L = q.lib()
+    E = q._lib
+    T, J = q._lib._Tensor, q._lib._MergeJob
+    good = T(0x10000, 0x20000, 0x30000, 256, 512)
+    empty = T(0x10000, 0x20000, 0x30000, 0, 512)
+    fake = 0x40000
+    ok = lambda: J(ctypes.addressof(good), fake, fake, 16, 2.0, fake)
+    assert L.qlora_merge_many(None, 0, None) == E.QLORA_OK
+    assert L.qlora_merge_many(None, 2, None) == E.QLORA_ERR_NULL
+    assert L.qlora_merge_many(None, -1, None) == E.QLORA_ERR_SHAPE
+    for bad, status in ((J(ctypes.addressof(good), fake, fake, 12, 2.0, fake), E.QLORA_ERR_UNSUPPORTED),
+                        (J(ctypes.addressof(good), fake, fake, 16, 2.0, fake + 2), E.QLORA_ERR_ALIGN),
+                        (J(ctypes.addressof(good), None, fake, 16, 2.0, fake), E.QLORA_ERR_NULL),
+                        (J(None, fake, fake, 16, 2.0, fake), E.QLORA_ERR_NULL)):
+        arr = (J * 20)(*([ok()] * 17 + [bad] + [ok()] * 2))
+        assert L.qlora_merge_many(arr, 20, None) == status
+    only_empty = (J * 3)(*([J(ctypes.addressof(empty), None, None, 16, 2.0, None)] * 3))
+    assert L.qlora_merge_many(only_empty, 3, None) == E.QLORA_OK
+
+
 @pytest.mark.parametrize("numel", [0, 1, 100, 4096 * 4096, 2 ** 20 + 17])
 @pytest.mark.parametrize("block", [16, 64, 4096])
 @pytest.mark.parametrize("scales", ["fp32", "e4m3", "e5m2", "u8"])

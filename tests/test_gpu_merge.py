@@ -154,6 +154,30 @@ def test_merge_stream_and_empty(q):
     q.qlora_merge(e, d["A"].cuda(), d["B"].cuda()[:0], lin.gamma, out=out)
 
 
+def test_merge_many_equals_one_by_one(q):
+    """qlora_merge_many over 21 weights of different shapes and ranks (two
+    launches of at most 16, one empty weight among them): every output equals
+    qlora_merge's for that weight bit for bit, and qlora_merge is checked
+    against the oracle above."""
+    shapes = [CASES[i % len(CASES)][:3] for i in range(20)] + [(4096, 1024, 16)]
+    jobs, singles = [], []
+    for i, (N, K, r) in enumerate(shapes):
+        lin, d = _layer(N, K, r, 100 + i)
+        w = q.qlora_quantize(torch.from_numpy(d["W"]).cuda())
+        A, B = d["A"].cuda(), d["B"].cuda()
+        jobs.append((w, A, B, lin.gamma, None))
+        singles.append(q.qlora_merge(w, A, B, lin.gamma))
+    e = q.empty_nf4(0, 256)
+    jobs.insert(7, (e, jobs[0][1][:, :256].contiguous(), jobs[0][2][:0], 2.0,
+                    torch.empty(0, 256, dtype=torch.bfloat16, device="cuda")))
+    outs = q.qlora_merge_many(jobs)
+    torch.cuda.synchronize()
+    outs.pop(7)
+    assert len(outs) == len(singles)
+    for i, (got, ref) in enumerate(zip(outs, singles)):
+        assert torch.equal(got.view(torch.int16), ref.view(torch.int16)), f"job {i} {shapes[i]}"
+
+
 @pytest.mark.parametrize("N,K,seed", [(4096, 4096, 11), (40, 768, 12), (3, 100, 13), (1, 1, 14)])
 def test_quantize_bf16_matches_oracle(q, N, K, seed):
     """Re-quantisation of a bf16 weight: bit-exact with the oracle's quantiser
