@@ -415,6 +415,11 @@ def _decoder_measure(q, syn, device, steps=2):
         q.qlora_quantize(src[kind(l)], out=w, check_finite=False)
     e.record()
     torch.cuda.synchronize()
+    q1_ms = b.elapsed_time(e)
+    b.record()
+    q.qlora_quantize_many([(src[kind(l)], w) for l, w in zip(lins, ws)], check_finite=False)
+    e.record()
+    torch.cuda.synchronize()
     q_ms = b.elapsed_time(e)
     params = sum(l.N * l.K for l in lins)
     q_bytes = params * 4 + sum(w.nbytes for w in ws)
@@ -456,7 +461,9 @@ def _decoder_measure(q, syn, device, steps=2):
     out = {"workload": "llama7b_decoder_32layers_m4096_r16", "linears": len(lins),
            "fwd_bwd_ms": round(ms, 3), "fwd_bwd_TFLOPs": round(flops / (ms * 1e-3) / 1e12, 2),
            "quantize_ms": round(q_ms, 3), "quantize_params": params,
-           "quantize_GBps": round(q_bytes / (q_ms * 1e-3) / 1e9, 1)}
+           "quantize_GBps": round(q_bytes / (q_ms * 1e-3) / 1e9, 1),
+           "quantize_one_by_one_ms": round(q1_ms, 3),
+           "quantize_one_by_one_GBps": round(q_bytes / (q1_ms * 1e-3) / 1e9, 1)}
     del Ts, wsp
     for a in act.values():
         for k in ("X", "dY", "Y", "dX", "dA", "dB"):
@@ -473,7 +480,8 @@ def _export_measure(q, lins, ws, act, kind, device, reps=3):
     qlora_merge calls; then the same buffer re-quantised to NF4, and, for
     comparison, the plain dequantisation of every weight.  GB/s are algorithmic bytes: the stored
     weight read, the adapter read and the bf16 weight written (merge), the
-    bf16 read and the stored weight written (re-quantise)."""
+    bf16 read and the stored weight written (re-quantise: one
+    qlora_quantize_many call, and 224 qlora_quantize_bf16 calls beside it)."""
     params = sum(l.N * l.K for l in lins)
     buf = torch.empty(params, dtype=torch.bfloat16, device=device)
     views, o = [], 0
@@ -505,6 +513,9 @@ def _export_measure(q, lins, ws, act, kind, device, reps=3):
             q.qlora_merge(w, a["A"], a["B"], l.gamma, out=v)
 
     def requant_all():
+        q.qlora_quantize_many(list(zip(views, re_ws)), check_finite=False)
+
+    def requant_each():
         for w, v in zip(re_ws, views):
             q.qlora_quantize_bf16(v, out=w, check_finite=False)
 
@@ -515,6 +526,7 @@ def _export_measure(q, lins, ws, act, kind, device, reps=3):
     m_ms = timed(merge_all)
     m1_ms = timed(merge_each)
     r_ms = timed(requant_all)
+    r1_ms = timed(requant_each)
     d_ms = timed(dequant_all)
     m_bytes = stored + adapter + params * 2
     r_bytes = params * 2 + sum(w.nbytes for w in re_ws)
@@ -527,6 +539,8 @@ def _export_measure(q, lins, ws, act, kind, device, reps=3):
             "merge_one_by_one_GBps": round(m_bytes / (m1_ms * 1e-3) / 1e9, 1),
             "requantize_ms": round(r_ms, 3),
             "requantize_GBps": round(r_bytes / (r_ms * 1e-3) / 1e9, 1),
+            "requantize_one_by_one_ms": round(r1_ms, 3),
+            "requantize_one_by_one_GBps": round(r_bytes / (r1_ms * 1e-3) / 1e9, 1),
             "dequantize_ms": round(d_ms, 3),
             "dequantize_GBps": round(d_bytes / (d_ms * 1e-3) / 1e9, 1)}
 
@@ -733,7 +747,8 @@ def run_gpu(args):
         out["decoder"] = _decoder_measure(q, syn, device)
         out["decoder"]["frac_bf16"] = round(out["decoder"]["fwd_bwd_TFLOPs"] / peak, 4)
         ex = out["decoder"]["export"]
-        for k in ("merge", "merge_one_by_one", "requantize", "dequantize"):
+        out["decoder"]["quantize_frac_hbm"] = round(out["decoder"]["quantize_GBps"] / peaks["hbm_gbs"], 4)
+        for k in ("merge", "merge_one_by_one", "requantize", "requantize_one_by_one", "dequantize"):
             ex[f"{k}_frac_hbm"] = round(ex[f"{k}_GBps"] / peaks["hbm_gbs"], 4)
         try:
             out["merge"] = _merge_measure(q, syn, device)

@@ -36,6 +36,7 @@ from ._lib import (  # noqa: F401
     qlora_quantize,
     qlora_quantize_bf16,
     qlora_quantize_fmt,
+    qlora_quantize_many,
     qlora_quantized_sizes,
     status_string,
     workspace,

@@ -45,6 +45,7 @@ EXPORTED = (
     "qlora_merge",
     "qlora_merge_many",
     "qlora_quantize_bf16",
+    "qlora_quantize_many",
     "qlora_format_sizes",
     "qlora_quantize_fmt",
     "qlora_dequantize_fmt",
@@ -85,6 +86,10 @@ def _events(events):
             ev.record()
         handles.append(ev.cuda_event)
     return ctypes.byref(_Events(*handles))
+
+
+class _QuantJob(ctypes.Structure):
+    _fields_ = [("W", ctypes.c_void_p), ("out", ctypes.c_void_p)]   # const qlora_nf4_tensor*
 
 
 class _MergeJob(ctypes.Structure):
@@ -159,6 +164,7 @@ def lib() -> ctypes.CDLL:
         L.qlora_quantize_bf16.argtypes = [vp, tp, vp, vp]
         L.qlora_merge.argtypes = [tp, vp, vp, i32, f32, vp, vp]
         L.qlora_merge_many.argtypes = [ctypes.POINTER(_MergeJob), i32, vp]
+        L.qlora_quantize_many.argtypes = [ctypes.POINTER(_QuantJob), i32, i32, vp, vp]
         fp = ctypes.POINTER(_Format)
         L.qlora_format_sizes.argtypes = [i64, fp, sz, sz, sz]
         L.qlora_quantize_fmt.argtypes = [vp, i64, fp, vp, vp, vp, vp, vp]
@@ -264,6 +270,33 @@ def qlora_quantize(W: torch.Tensor, out: NF4Tensor | None = None, check_finite: 
     _check(lib().qlora_quantize(W.data_ptr(), ctypes.byref(st), _ptr(flag), _stream(stream)),
            "qlora_quantize")
     return out
+
+
+def qlora_quantize_many(jobs, check_finite: bool = True, stream=None) -> list:
+    """Quantise several [rows, cols] CUDA tensors, all fp32 or all bf16, in as
+    few launches as the library needs.  jobs: sequence of (W, out) with out
+    None or an NF4Tensor; returns the stored tensors in order.  check_finite
+    as qlora_quantize, for all of them together."""
+    jobs = list(jobs)
+    dtypes = {W.dtype for W, _ in jobs}
+    if len(dtypes) > 1 or not dtypes <= {torch.float32, torch.bfloat16}:
+        raise TypeError(f"qlora_quantize_many: W must be all fp32 or all bf16, got {dtypes}")
+    outs, structs = [], []
+    for W, out in jobs:
+        _need(W, W.dtype, "W")
+        rows, cols = (W.shape[0], W.shape[1]) if W.dim() == 2 else (1, W.numel())
+        out = out if out is not None else empty_nf4(rows, cols, W.device)
+        outs.append(out)
+        structs.append((W, out.c_struct()))
+    arr = (_QuantJob * max(1, len(structs)))()
+    for i, (W, st) in enumerate(structs):
+        arr[i] = _QuantJob(W.data_ptr(), ctypes.addressof(st))
+    bf16 = bool(jobs) and jobs[0][0].dtype == torch.bfloat16
+    flag = (torch.empty(1, dtype=torch.int32, device=jobs[0][0].device)
+            if check_finite and jobs else None)
+    _check(lib().qlora_quantize_many(arr, len(structs), 1 if bf16 else 0, _ptr(flag),
+                                     _stream(stream)), "qlora_quantize_many")
+    return outs
 
 
 def qlora_dequantize(w: NF4Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:

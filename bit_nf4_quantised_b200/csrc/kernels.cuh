@@ -36,6 +36,20 @@ cudaError_t launch_quantize_b64(const float* W, int64_t numel, uint8_t* packed, 
                                 float* meta, int* nonfinite_flag, const Nf4IndexLut& lut,
                                 uint32_t zero_index, int scale_fmt, cudaStream_t stream);
 
+// K1 over several weights (fp32, or bf16 when bf16 is set): up to
+// kMaxQuantizeJobs weights' whole groups per launch, each partial trailing
+// group by its own one-CTA launch.
+constexpr int kMaxQuantizeJobs = 16;
+struct QuantizeJob {
+    const void* W;
+    int64_t numel;
+    uint8_t* packed;
+    uint8_t* scale_codes;
+    float* meta;
+};
+cudaError_t launch_quantize_many(const QuantizeJob* jobs, int n, bool bf16, int* nonfinite_flag,
+                                 const Nf4IndexLut& lut, cudaStream_t stream);
+
 // K1 on a bf16 weight (the re-quantisation of a merged export).
 cudaError_t launch_quantize_bf16(const uint16_t* W, int64_t numel, uint8_t* packed,
                                  uint8_t* scale_codes, float* meta, int* nonfinite_flag,

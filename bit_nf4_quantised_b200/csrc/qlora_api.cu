@@ -8,6 +8,7 @@
 #include <limits>
 #include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "kernels.cuh"
 
@@ -507,6 +508,37 @@ int qlora_quantize_bf16(const uint16_t* W, const qlora_nf4_tensor* out, int* d_n
     if (!lut) return QLORA_ERR_UNSUPPORTED;
     st = cuda_status(launch_quantize_bf16(W, numel, out->packed, out->scale_codes,
                                           out->meta_scale, d_nonfinite_flag, *lut, s));
+    return end_checked(st, d_nonfinite_flag, s);
+}
+
+int qlora_quantize_many(const qlora_quantize_job* jobs, int n, int input_bf16,
+                        int* d_nonfinite_flag, qlora_stream_t stream) {
+    if (n < 0) return QLORA_ERR_SHAPE;
+    if (n > 0 && !jobs) return QLORA_ERR_NULL;
+    // every job is checked before anything is launched
+    std::vector<QuantizeJob> q;
+    q.reserve(static_cast<size_t>(n));
+    for (int i = 0; i < n; ++i) {
+        const qlora_nf4_tensor* o = jobs[i].out;
+        if (!o) return QLORA_ERR_NULL;
+        if (o->rows < 0 || o->cols < 0) return QLORA_ERR_SHAPE;
+        if (o->rows == 0 || o->cols == 0) continue;   // empty: W and buffers may be NULL
+        const int st = check_tensor(o);
+        if (st != QLORA_OK) return st;
+        const int64_t numel = o->rows * o->cols;
+        if (!jobs[i].W) return QLORA_ERR_NULL;
+        if (!aligned(jobs[i].W, 16)) return QLORA_ERR_ALIGN;
+        q.push_back({jobs[i].W, numel, jobs[i].out->packed, jobs[i].out->scale_codes,
+                     jobs[i].out->meta_scale});
+    }
+    if (q.empty()) return QLORA_OK;
+    const Nf4IndexLut* lut = index_lut();
+    if (!lut) return QLORA_ERR_UNSUPPORTED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int st = begin_checked(d_nonfinite_flag, s);
+    if (st != QLORA_OK) return st;
+    st = cuda_status(launch_quantize_many(q.data(), static_cast<int>(q.size()), input_bf16 != 0,
+                                          d_nonfinite_flag, *lut, s));
     return end_checked(st, d_nonfinite_flag, s);
 }
 

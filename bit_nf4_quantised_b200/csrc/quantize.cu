@@ -58,6 +58,8 @@ constexpr int kBlocksPerWarpStep = 32 / kLanesPerBlock;                         
 constexpr int kSteps = QLORA_GROUP / (kThreads / 32 * kBlocksPerWarpStep);         // 4
 constexpr int kGroupElems = QLORA_BLOCK * QLORA_GROUP;                             // 16384
 constexpr int kLutBytes = kNf4LutEntries * 32 * 8;                                  // 16 KiB
+// index 7 (the exact zero among the NF4 codes) in all eight nibbles: a zero block's word
+constexpr uint32_t kNf4ZeroWord = 0x77777777u;
 
 // eight consecutive weights of one lane
 struct W8 {
@@ -111,12 +113,13 @@ __device__ __forceinline__ uint32_t code_index(float x, uint32_t lane_lut) {
     return base + (x > __uint_as_float(thr) ? 1u : 0u);
 }
 
+// One group of 256 blocks by one CTA (the body of both kernels below).
 template <bool kFull, typename Tin>
-__global__ void __launch_bounds__(kThreads, 2)
-quantize_kernel(const Tin* __restrict__ W, int64_t numel, int64_t nblocks,
-                uint8_t* __restrict__ packed, void* __restrict__ scales,
-                float* __restrict__ meta, int* __restrict__ nonfinite_flag, Nf4IndexLut lut,
-                uint32_t zero_word, int scale_fmt) {
+__device__ __forceinline__ void quantize_group(const Tin* __restrict__ W, int64_t numel, int64_t nblocks,
+                                               uint8_t* __restrict__ packed, void* __restrict__ scales,
+                                               float* __restrict__ meta, int* __restrict__ nonfinite_flag,
+                                               const Nf4IndexLut& lut, uint32_t zero_word, int scale_fmt,
+                                               int64_t group) {
     extern __shared__ __align__(16) uint8_t smem[];                // the per-lane table
     __shared__ float sabs[QLORA_GROUP];
     __shared__ float sred[QLORA_GROUP / 32];
@@ -124,7 +127,6 @@ quantize_kernel(const Tin* __restrict__ W, int64_t numel, int64_t nblocks,
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int sub = lane & (kLanesPerBlock - 1), bq = lane / kLanesPerBlock;
-    const int64_t group = blockIdx.x;
     const int64_t gbase = group * kGroupElems;
 
     // every load of the group first
@@ -202,8 +204,36 @@ quantize_kernel(const Tin* __restrict__ W, int64_t numel, int64_t nblocks,
     }
 }
 
-// index of the exact zero among the NF4 codes: a zero block's word
-constexpr uint32_t kNf4ZeroWord = 0x77777777u;
+template <bool kFull, typename Tin>
+__global__ void __launch_bounds__(kThreads, 2)
+quantize_kernel(const Tin* __restrict__ W, int64_t numel, int64_t nblocks,
+                uint8_t* __restrict__ packed, void* __restrict__ scales,
+                float* __restrict__ meta, int* __restrict__ nonfinite_flag, Nf4IndexLut lut,
+                uint32_t zero_word, int scale_fmt) {
+    quantize_group<kFull, Tin>(W, numel, nblocks, packed, scales, meta, nonfinite_flag, lut, zero_word,
+                               scale_fmt, blockIdx.x);
+}
+
+// Several weights' whole groups in one launch: CTA x takes group
+// x - first[j] of job j, first[j] <= x < first[j + 1].
+struct QuantBatch {
+    QuantizeJob job[kMaxQuantizeJobs];
+    int64_t first[kMaxQuantizeJobs + 1];
+    int n;
+};
+
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads, 2)
+quantize_many_kernel(const __grid_constant__ QuantBatch bt, int* __restrict__ nonfinite_flag,
+                     Nf4IndexLut lut) {
+    int j = 0;
+    while (j + 1 < bt.n && bt.first[j + 1] <= int64_t(blockIdx.x)) ++j;
+    const QuantizeJob& q = bt.job[j];
+    const int64_t nblocks = (q.numel + QLORA_BLOCK - 1) / QLORA_BLOCK;
+    quantize_group<true, Tin>(static_cast<const Tin*>(q.W), q.numel, nblocks, q.packed, q.scale_codes,
+                              q.meta, nonfinite_flag, lut, kNf4ZeroWord, QLORA_SCALES_E4M3,
+                              int64_t(blockIdx.x) - bt.first[j]);
+}
 
 template <bool kFull, typename Tin>
 cudaError_t launch_one(unsigned grid, const Tin* W, int64_t numel, int64_t nblocks, uint8_t* packed,
@@ -256,6 +286,51 @@ cudaError_t launch_quantize_b64(const float* W, int64_t numel, uint8_t* packed, 
                                 uint32_t zero_index, int scale_fmt, cudaStream_t stream) {
     return quantize_any(W, numel, packed, scales, meta, nonfinite_flag, lut, zero_index * 0x11111111u,
                         scale_fmt, stream);
+}
+
+template <typename Tin>
+cudaError_t quantize_many_any(const QuantizeJob* jobs, int n, int* nonfinite_flag,
+                              const Nf4IndexLut& lut, cudaStream_t stream) {
+    for (int i0 = 0; i0 < n; i0 += kMaxQuantizeJobs) {
+        QuantBatch bt{};
+        int64_t total = 0;
+        for (int i = i0; i < n && i < i0 + kMaxQuantizeJobs; ++i) {
+            const int64_t full = jobs[i].numel / kGroupElems;
+            if (full == 0) continue;
+            bt.job[bt.n] = jobs[i];
+            bt.first[bt.n] = total;
+            total += full;
+            ++bt.n;
+        }
+        bt.first[bt.n] = total;
+        if (total > 0) {
+            if (total > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+            quantize_many_kernel<Tin><<<static_cast<unsigned>(total), kThreads, kLutBytes, stream>>>(
+                bt, nonfinite_flag, lut);
+            const cudaError_t e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        }
+        // each weight's trailing partial group, if it has one
+        for (int i = i0; i < n && i < i0 + kMaxQuantizeJobs; ++i) {
+            const QuantizeJob& q = jobs[i];
+            const int64_t full = q.numel / kGroupElems;
+            const int64_t nblocks = (q.numel + QLORA_BLOCK - 1) / QLORA_BLOCK;
+            if ((nblocks + QLORA_GROUP - 1) / QLORA_GROUP == full) continue;
+            const int64_t off = full * kGroupElems;
+            const cudaError_t e = launch_one<false>(
+                1u, static_cast<const Tin*>(q.W) + off, q.numel - off, nblocks - full * QLORA_GROUP,
+                q.packed + full * (kGroupElems / 2), q.scale_codes + full * QLORA_GROUP, q.meta + full,
+                nonfinite_flag, lut, kNf4ZeroWord, QLORA_SCALES_E4M3, stream);
+            if (e != cudaSuccess) return e;
+        }
+    }
+    return cudaSuccess;
+}
+
+cudaError_t launch_quantize_many(const QuantizeJob* jobs, int n, bool bf16, int* nonfinite_flag,
+                                 const Nf4IndexLut& lut, cudaStream_t stream) {
+    return bf16 ? quantize_many_any<uint16_t>(jobs, n, nonfinite_flag, lut, stream)
+                : quantize_many_any<float>(jobs, n, nonfinite_flag, lut, stream);
 }
 
 cudaError_t launch_quantize_bf16(const uint16_t* W, int64_t numel, uint8_t* packed,

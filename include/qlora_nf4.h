@@ -338,6 +338,38 @@ typedef struct {
 QLORA_API int qlora_merge_many(const qlora_merge_job* jobs, int n, qlora_stream_t stream);
 
 /*
+ * qlora_quantize_many -- qlora_quantize (or, with input_bf16, qlora_quantize_bf16)
+ * of several weights, e.g. every linear of a model at load time or every
+ * merged weight at export: the whole 256-block groups of up to 16 weights
+ * share one kernel launch, so small weights do not each pay a launch's ramp
+ * and tail; a weight's partial last group (numel % 16384 != 0) takes one more
+ * small launch.  Each job's stored bytes are bit for bit what qlora_quantize
+ * gives for it.
+ *   jobs  (host array of n qlora_quantize_job, read): W (device, fp32 or bf16
+ *         bits, rows*cols, read, 16-byte aligned) and out (host struct whose
+ *         buffers are written); the outputs must not overlap one another or
+ *         any input.  Empty weights (rows or cols 0) are skipped: their W
+ *         and out's buffers may be NULL.
+ *   n     >= 0 (0 launches nothing).
+ *   input_bf16  0: every W is fp32; otherwise every W is bf16.
+ *   d_nonfinite_flag (device int, nullable): as qlora_quantize, for all jobs
+ *         together: cleared first, and with a flag the call synchronises the
+ *         stream and returns QLORA_ERR_NONFINITE if any job held a NaN or an
+ *         infinity.
+ * Every job is checked before anything is launched; the first failing job's
+ * status is returned and nothing runs.
+ * Errors: QLORA_ERR_NULL, QLORA_ERR_SHAPE (n < 0, or a job's shape),
+ * QLORA_ERR_ALIGN, QLORA_ERR_NONFINITE, QLORA_ERR_CUDA.
+ */
+typedef struct {
+    const void* W;                 /* device, fp32 or bf16 (see input_bf16) */
+    const qlora_nf4_tensor* out;   /* host struct, its buffers written */
+} qlora_quantize_job;
+
+QLORA_API int qlora_quantize_many(const qlora_quantize_job* jobs, int n, int input_bf16,
+                                  int* d_nonfinite_flag, qlora_stream_t stream);
+
+/*
  * qlora_quantize_bf16 -- qlora_quantize of a bf16 weight (each value widened
  * exactly to fp32 first), the re-quantisation of a merged weight for a 4-bit
  * deployment ("QLoRA" (finetunellm.com), "What it costs you": merging into

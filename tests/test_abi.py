@@ -137,6 +137,38 @@ def _books():
             "int4": tuple(o.int4_codebook())}
 
 
+def test_quantize_many_checks_every_job_before_any_launch(q):
+    """qlora_quantize_many validates all its jobs on the host first (null or
+    misaligned weight, bad stored tensor): the failing job's status, nothing
+    launched; an empty list and empty weights (whose W may be NULL) launch
+    nothing."""
+    L = q.lib()
+    E = q._lib
+    T, J = q._lib._Tensor, q._lib._QuantJob
+    good = T(0x10000, 0x20000, 0x30000, 256, 512)
+    empty = T(0x10000, 0x20000, 0x30000, 0, 512)
+    nulled = T(0, 0x20000, 0x30000, 256, 512)
+    fake = 0x40000
+    ok = lambda: J(fake, ctypes.addressof(good))
+    assert L.qlora_quantize_many(None, 0, 0, None, None) == E.QLORA_OK
+    assert L.qlora_quantize_many(None, 1, 0, None, None) == E.QLORA_ERR_NULL
+    assert L.qlora_quantize_many(None, -1, 0, None, None) == E.QLORA_ERR_SHAPE
+    for bad, status in ((J(None, ctypes.addressof(good)), E.QLORA_ERR_NULL),
+                        (J(fake + 4, ctypes.addressof(good)), E.QLORA_ERR_ALIGN),
+                        (J(fake, ctypes.addressof(nulled)), E.QLORA_ERR_NULL),
+                        (J(fake, None), E.QLORA_ERR_NULL)):
+        arr = (J * 19)(*([ok()] * 17 + [bad] + [ok()]))
+        assert L.qlora_quantize_many(arr, 19, 0, None, None) == status
+        assert L.qlora_quantize_many(arr, 19, 1, None, None) == status
+    bare = T(0, 0, 0, 0, 16384)                 # what torch hands over for an empty tensor
+    only_empty = (J * 3)(J(fake, ctypes.addressof(empty)), J(None, ctypes.addressof(empty)),
+                         J(None, ctypes.addressof(bare)))
+    assert L.qlora_quantize_many(only_empty, 3, 0, None, None) == E.QLORA_OK
+    neg = T(0x10000, 0x20000, 0x30000, -1, 64)
+    assert L.qlora_quantize_many((J * 1)(J(fake, ctypes.addressof(neg))), 1, 0, None,
+                                 None) == E.QLORA_ERR_SHAPE
+
+
 def test_merge_many_checks_every_job_before_any_launch(q):
     """qlora_merge_many validates all its jobs on the host first: one bad job
     (rank 12, a misaligned output, a null adapter) fails the whole call with

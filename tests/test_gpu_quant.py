@@ -142,3 +142,42 @@ def test_nonfinite_is_reported(q):
     with pytest.raises(q.QloraError):
         q.qlora_quantize(W)
     q.qlora_quantize(torch.ones(4, 128, device="cuda"))      # finite: no error
+
+
+def _digests(w):
+    return [t.cpu().numpy().tobytes() for t in (w.packed, w.scale_codes, w.meta_scale)]
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_quantize_many_equals_one_by_one(q, bf16):
+    """qlora_quantize_many over 18 weights (two launches of at most 16; ragged
+    last groups and blocks; one empty weight): every stored byte equals the
+    single call's for that weight, fp32 and bf16 inputs alike."""
+    rng = np.random.default_rng(31 + bf16)
+    shapes = [(64, 256 * 64), (3, 100), (1024, 4096), (17, 1000), (2, 64 * 256 * 2 + 70),
+              (256, 512), (1, 64), (4096, 96)] * 2 + [(512, 1024)]
+    Ws = []
+    for r, c in shapes:
+        W = torch.from_numpy((rng.standard_normal((r, c)) * 0.02).astype(np.float32)).cuda()
+        W.view(-1)[:64] = 0.0                          # a zero block
+        Ws.append(W.bfloat16() if bf16 else W)
+    Ws.append(Ws[0][:0])                               # empty: torch gives it a NULL pointer
+    many = q.qlora_quantize_many([(W, None) for W in Ws])
+    torch.cuda.synchronize()
+    assert many[-1].packed.numel() == 0
+    for i, (W, w) in enumerate(zip(Ws[:-1], many)):
+        one = q.qlora_quantize_bf16(W) if bf16 else q.qlora_quantize(W)
+        torch.cuda.synchronize()
+        assert _digests(w) == _digests(one), f"job {i} {tuple(W.shape)}"
+
+
+def test_quantize_many_nonfinite(q):
+    """One non-finite weight among several: the call reports it with
+    QLORA_ERR_NONFINITE; without it the same call succeeds."""
+    Ws = [torch.ones(64, 512, device="cuda") * 0.01 for _ in range(5)]
+    Ws[3][7, 300] = float("inf")
+    with pytest.raises(q.QloraError) as ei:
+        q.qlora_quantize_many([(W, None) for W in Ws])
+    assert ei.value.status == q._lib.QLORA_ERR_NONFINITE
+    Ws[3][7, 300] = 0.5
+    q.qlora_quantize_many([(W, None) for W in Ws])
