@@ -399,17 +399,18 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
     asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
     if (blockIdx.x < a.t_ctas) {
         // a share of this slice's T = X A^T: CTA x of the first t_ctas takes
-        // an equal run of the slice's 16-wide k-steps, spread over its warps;
-        // reduced in the first reduction buffer, then written as one partial
+        // an equal run of the slice's 16-wide k-steps, spread over its warps.
+        // Per round of 32 columns of T, each warp with k-steps stores its
+        // [M][32] partial in its own slot of the reduction buffers (16 M 32
+        // floats fill them exactly); the slots are then added in warp order
+        // and written as this CTA's partial, so T is the same on every run.
         const int ksteps = kslab / 16;
         const int x = blockIdx.x;
         const int s0 = static_cast<int>(int64_t(ksteps) * x / a.t_ctas);
         const int s1 = static_cast<int>(int64_t(ksteps) * (x + 1) / a.t_ctas);
-        // [M][r] fp32, inside the reduction buffers (M r <= 2048 M floats)
-        const uint32_t tred = sp.red;
-        for (int e = warp * 32 + lane; e < a.M * a.r; e += kConsumerWarps * 32)
-            asm volatile("st.shared.b32 [%0], %1;" ::"r"(tred + e * 4), "r"(0u) : "memory");
-        asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+        const int nw = min(kConsumerWarps, s1 - s0);           // warps holding partials
+        float* tp = a.Tpart + (int64_t(slice) * a.t_ctas + x) * a.M * a.r;
+        const uint32_t slot = sp.red + static_cast<uint32_t>(warp * xrows * 32) * 4;
         // four 8-column tiles of T at a time keep the accumulators small
         for (int jg = 0; jg * 8 < a.r; jg += 4) {
             float tacc[4][4];
@@ -431,30 +432,35 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_packed, GemvArgs a) {
                     }
                 }
             }
-            if (s0 + warp < s1) {
+            if (warp < nw) {
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    if ((jg + j) * 8 < a.r) {
-                        const int col = (jg + j) * 8 + 2 * c;
-                        if (g < xrows) {
-                            const uint32_t r0 = tred + (g * a.r + col) * 4;
-                            asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(r0), "f"(tacc[j][0]) : "memory");
-                            asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(r0 + 4), "f"(tacc[j][1]) : "memory");
-                        }
-                        if (g + 8 < xrows) {
-                            const uint32_t r1 = tred + ((g + 8) * a.r + col) * 4;
-                            asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(r1), "f"(tacc[j][2]) : "memory");
-                            asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(r1 + 4), "f"(tacc[j][3]) : "memory");
-                        }
+                    const int col = j * 8 + 2 * c;                  // within the round
+                    if (g < xrows) {
+                        const uint32_t r0 = slot + (g * 32 + col) * 4;
+                        asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(r0), "f"(tacc[j][0]),
+                                     "f"(tacc[j][1]) : "memory");
+                    }
+                    if (g + 8 < xrows) {
+                        const uint32_t r1 = slot + ((g + 8) * 32 + col) * 4;
+                        asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(r1), "f"(tacc[j][2]),
+                                     "f"(tacc[j][3]) : "memory");
                     }
                 }
             }
+            asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+            const int cols = min(32, a.r - jg * 8);
+            for (int e = tid; e < xrows * 32; e += kConsumerWarps * 32) {
+                const int m = e >> 5, col = e & 31;
+                if (col < cols) {
+                    float t = 0.f;
+                    for (int w = 0; w < nw; ++w)
+                        t += __uint_as_float(lds32(sp.red + static_cast<uint32_t>((w * xrows + m) * 32 + col) * 4));
+                    tp[m * a.r + jg * 8 + col] = t;
+                }
+            }
+            asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
         }
-        asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
-        float* tp = a.Tpart + (int64_t(slice) * a.t_ctas + x) * a.M * a.r;
-        for (int e = warp * 32 + lane; e < a.M * a.r; e += kConsumerWarps * 32)
-            tp[e] = __uint_as_float(lds32(tred + e * 4));
-        asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
     }
 
     // Main loop.  Warp w takes row group rq = w / D (tile rows 16 rq + g and

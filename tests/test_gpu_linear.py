@@ -90,6 +90,42 @@ def test_forward_backward(q, M, N, K, r):
     assert_close("dB", dB, dBr)
 
 
+@pytest.mark.parametrize("M,N,K,r", [(1, 1000, 2048, 16), (4, 512, 4352, 16), (16, 1024, 2048, 128),
+                                     (9, 256, 4096, 64), (200, 264, 320, 16), (4608, 2200, 2304, 16)])
+def test_same_inputs_same_bytes(q, M, N, K, r):
+    """Every result is reproducible: three forward + backward calls on the
+    same inputs give the same bytes of Y, T, dX, dA and dB (no reduction
+    depends on the order in which warps or CTAs finish)."""
+    lin = syn.Linear("case", M, N, K, r, alpha=2.0 * r, outliers=True, seed=M + N + K + r)
+    d = syn.make_layer(lin)
+    g = _gpu_inputs(d)
+    w = q.qlora_quantize(torch.from_numpy(d["W"]).cuda())
+    outs = []
+    for _ in range(3):
+        T = torch.empty(M, r, dtype=torch.float32, device="cuda")
+        Y = q.qlora_linear_forward(g["X"], w, g["A"], g["B"], lin.gamma, T_save=T)
+        dX, dA, dB = q.qlora_linear_backward(g["dY"], g["X"], w, g["A"], g["B"], lin.gamma,
+                                             T_saved=T)
+        torch.cuda.synchronize()
+        outs.append([t.view(torch.int16 if t.dtype == torch.bfloat16 else torch.int32).cpu()
+                     for t in (Y, T, dX, dA, dB)])
+    for other in outs[1:]:
+        for name, a, b in zip(("Y", "T", "dX", "dA", "dB"), outs[0], other):
+            assert torch.equal(a, b), name
+
+
+def test_decode_same_bytes_full_size(q):
+    """The decode GEMV with 16 tokens over 8192 x 28672 (many CTAs share T):
+    the same Y bytes on every call."""
+    lin = syn.WORKLOADS["decode_gemv_8192x28672_m16"].layers[0]
+    d = syn.make_layer(lin, with_grad=False)
+    g = _gpu_inputs(d)
+    w = q.qlora_quantize(torch.from_numpy(d["W"]).cuda())
+    Ys = [q.qlora_linear_forward(g["X"], w, g["A"], g["B"], lin.gamma).view(torch.int16).cpu()
+          for _ in range(4)]
+    assert all(torch.equal(Ys[0], y) for y in Ys[1:])
+
+
 def test_recompute_T_accumulate_and_no_dX(q):
     lin = syn.Linear("case", 96, 264, 384, 16, alpha=32.0, seed=3)
     d, w, Y, T, dX, dA, dB = _run(q, lin, with_T=False, accumulate=True, want_dX=False)
