@@ -42,8 +42,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 LAUNCHES_PER_STEP = 2 + 4
 # ncu DRAM traffic (read + write bytes) of one dequant-GEMM launch of this
 # workload, valid only for the sources it was captured on (_source_sha).
-GEMM_TRAFFIC = {"source_sha": "e1cb81df73c9acac", "fwd_bytes": (44.599552 + 6.562304) * 1e6,
-                "dx_bytes": (44.409344 + 3.521536) * 1e6}
+GEMM_TRAFFIC = {"source_sha": "210d254a6052a1e8", "fwd_bytes": (44.583680 + 8.124672) * 1e6,
+                "dx_bytes": (44.357120 + 3.887104) * 1e6}
 
 
 def _peaks():
