@@ -118,6 +118,21 @@ class Clocks:
     def mark(self, t0: float, t1: float):
         self.window = (t0, t1)
 
+    def window_summary(self, t0: float, t1: float):
+        """Median SM clock and the reasons seen between two host times (call
+        after stop())."""
+        if self.error or self._thread is None:
+            return None
+        sel = [x for x in self.samples if t0 <= x[0] <= t1]
+        reasons = set()
+        for _, _, rs in sel:
+            for name, const in self.REASONS:
+                bit = getattr(self._nvml, const, 0)
+                if bit and (rs & bit):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median([m for _, m, _ in sel]) if sel else None,
+                "reasons": sorted(reasons), "samples": len(sel)}
+
     def stop(self):
         if self.error or self._thread is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.error or "not started"]}
@@ -186,6 +201,13 @@ def allreduce_adapter_grads(dA: torch.Tensor, dB: torch.Tensor) -> None:
     sums over its shard; the exchange is one sum over ranks."""
     torch.distributed.all_reduce(dA)
     torch.distributed.all_reduce(dB)
+
+
+def _hold_gpu(ms):
+    """Occupy the current stream for about `ms` milliseconds (torch's spin
+    kernel, at the maximum SM clock) so that the launches queued behind it
+    run back to back; nothing of it is inside a timed region."""
+    torch.cuda._sleep(int(ms * 1e-3 * 1.965e9))
 
 
 def _barrier(world):
@@ -676,8 +698,12 @@ def run_gpu(args):
         if world > 1:
             allreduce_adapter_grads(bufs["dA"], bufs["dB"])
 
+    hw = time.perf_counter()
     for i in range(args.warmup):
         one(i)
+    # hold long enough for the host to queue all K steps (from the warm-up's
+    # enqueue rate, which includes first-call costs, so it errs long)
+    hold_ms = min(2000.0, max(20.0, 1.5 * K * (time.perf_counter() - hw) * 1e3 / max(1, args.warmup)))
     _barrier(world)
     if q.device_error_word(ws) != 0:
         raise RuntimeError("device error word set during warm-up")
@@ -686,11 +712,16 @@ def run_gpu(args):
     _barrier(world)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    # A spin kernel holds the GPU while the host queues the steps, and the
+    # timing starts after it: the timed region then measures the GPU's work
+    # from a full queue, not the host's launch rate.
+    _hold_gpu(hold_ms)
     h0 = time.perf_counter()
     t0.record()
     for i in range(K):
         one(i)
     t1.record()
+    h_enq = time.perf_counter() - h0
     _barrier(world)
     clocks.mark(h0, time.perf_counter())
     # The GEMM kernels' own durations come from the same K steps run again
@@ -698,10 +729,15 @@ def run_gpu(args):
     # the streams they run on.  They are not recorded inside the timed steps:
     # an event between the LoRA kernel and the forward GEMM would stop the
     # GEMM from starting as the LoRA kernel's programmatic dependent.
+    _hold_gpu(hold_ms)
+    h2 = time.perf_counter()
     for i in range(K):
         one(i, evs[i])
+    h_enq_ev = time.perf_counter() - h2
     _barrier(world)
+    h3 = time.perf_counter()
     clk = clocks.stop()
+    gemm_clk = clocks.window_summary(h2, h3)
     ms = _max_over_ranks(t0.elapsed_time(t1), world) / K
     fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
     dx_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / K
@@ -731,9 +767,12 @@ def run_gpu(args):
                      "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} bf16 burst",
                      "traffic": traffic, "fwd_us": round(fwd_ms * 1e3, 2),
-                     "dx_us": round(dx_ms * 1e3, 2),
+                     "dx_us": round(dx_ms * 1e3, 2), "clocks": gemm_clk,
                      "timing": "CUDA events around each GEMM launch, the same steps rerun "
                                "right after the timed region"},
+        "host_enqueue_ms_per_step": {"timed": round(h_enq * 1e3 / K, 4),
+                                     "gemm_events_pass": round(h_enq_ev * 1e3 / K, 4),
+                                     "held_ms": round(hold_ms, 1)},
         "gpu_launches": LAUNCHES_PER_STEP * K,
         "clocks": clk,
     }

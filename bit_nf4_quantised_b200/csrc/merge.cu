@@ -81,6 +81,10 @@ struct MergeBatch {
     int rp_max;
 };
 
+// kMulti: the batch may hold several weights.  A one-weight launch indexes
+// job 0 at compile time, so its arguments stay constant-bank operands; a
+// batch copies the current job's arguments into registers once per unit.
+template <bool kMulti>
 __global__ void __launch_bounds__(kThreads)
 merge_kernel(const __grid_constant__ MergeBatch bt, Nf4Table tab) {
     extern __shared__ __align__(16) uint8_t smem[];
@@ -109,8 +113,9 @@ merge_kernel(const __grid_constant__ MergeBatch bt, Nf4Table tab) {
     const int64_t total = bt.first[bt.n];
     const int64_t u_begin = total * blockIdx.x / gridDim.x;
     const int64_t u_end = total * (blockIdx.x + 1) / gridDim.x;
-    auto rows_of = [&](int j) { return (static_cast<int>(bt.job[j].N) + kTileRows - 1) / kTileRows; };
-    auto cblocks_of = [&](int j) { return (static_cast<int>(bt.job[j].K) / kStrip + kWarps - 1) / kWarps; };
+    auto job = [&](int j) -> MergeArgs { return bt.job[kMulti ? j : 0]; };
+    auto rows_of = [&](int j) { return (static_cast<int>(job(j).N) + kTileRows - 1) / kTileRows; };
+    auto cblocks_of = [&](int j) { return (static_cast<int>(job(j).K) / kStrip + kWarps - 1) / kWarps; };
 
     // The slab position lane l fills: A's physical columns 2l, 2l+1 are
     // logical columns p0, p0 + 1 of the strip (see the column map above).
@@ -132,7 +137,7 @@ merge_kernel(const __grid_constant__ MergeBatch bt, Nf4Table tab) {
     // Unit (job j, column block cb, row tile rt); units advance row tile
     // first, then column block, then job.
     auto load_unit = [&](int j, int cb, int rt, WeightRegs& wr) {
-        const MergeArgs& a = bt.job[j];
+        const MergeArgs a = job(j);
         const int N = static_cast<int>(a.N), K = static_cast<int>(a.K);
         const int kblocks = K / kStrip;
         const int strip = cb * kWarps + warp;
@@ -166,7 +171,8 @@ merge_kernel(const __grid_constant__ MergeBatch bt, Nf4Table tab) {
     };
 
     int j = 0;
-    while (j + 1 < bt.n && bt.first[j + 1] <= u_begin) ++j;
+    if (kMulti)
+        while (j + 1 < bt.n && bt.first[j + 1] <= u_begin) ++j;
     int cb, rt;
     {
         const int64_t local = u_begin - bt.first[j];
@@ -192,7 +198,7 @@ merge_kernel(const __grid_constant__ MergeBatch bt, Nf4Table tab) {
     for (int64_t u = u_begin; u < u_end; ++u) {
         if (u + 1 < u_end) load_unit(nj, ncb, nrt, nxt);
         exchange(cur);
-        const MergeArgs& a = bt.job[j];
+        const MergeArgs a = job(j);
         const int N = static_cast<int>(a.N), K = static_cast<int>(a.K);
         const int kblocks = K / kStrip;
         const int strip = cb * kWarps + warp;
@@ -301,16 +307,16 @@ cudaError_t launch_merge(const MergeArgs* jobs, int n, const Nf4Table& tab, int 
     bt.first[bt.n] = total;
     if (total == 0) return cudaSuccess;
     const int smem = merge_smem_bytes(bt.rp_max);
-    cudaError_t e = cudaFuncSetAttribute(merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         smem);
+    const auto kernel = bt.n > 1 ? merge_kernel<true> : merge_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, merge_kernel, kThreads, smem);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, smem);
     if (e != cudaSuccess) return e;
     if (per_sm < 1) per_sm = 1;
     int64_t grid = int64_t(num_sms) * per_sm;
     if (grid > total) grid = total;                               // at least one unit per CTA
-    merge_kernel<<<dim3(static_cast<unsigned>(grid)), kThreads, smem, stream>>>(bt, tab);
+    kernel<<<dim3(static_cast<unsigned>(grid)), kThreads, smem, stream>>>(bt, tab);
     return cudaGetLastError();
 }
 
