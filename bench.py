@@ -203,6 +203,10 @@ def allreduce_adapter_grads(dA: torch.Tensor, dB: torch.Tensor) -> None:
     torch.distributed.all_reduce(dB)
 
 
+# hold before the short-kernel loops: their reps queue in well under this
+SHORT_HOLD_MS = 20.0
+
+
 def _hold_gpu(ms):
     """Occupy the current stream for about `ms` milliseconds (torch's spin
     kernel, at the maximum SM clock) so that the launches queued behind it
@@ -234,6 +238,7 @@ def _gemv_measure(q, syn, device, reps=20):
     torch.cuda.synchronize()
     call_b = torch.cuda.Event(enable_timing=True)
     call_e = torch.cuda.Event(enable_timing=True)
+    _hold_gpu(SHORT_HOLD_MS)
     call_b.record()
     for i in range(reps):
         q.qlora_linear_forward(X, copies[i % 3], A, B, lin.gamma, Y=Y, ws=ws, events=evs[i])
@@ -258,6 +263,7 @@ def _quantize_measure(q, syn, device, reps=5):
         q.qlora_quantize(W[i], out=outs[i], check_finite=False)
     torch.cuda.synchronize()
     b, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _hold_gpu(SHORT_HOLD_MS)
     b.record()
     for i in range(reps):
         q.qlora_quantize(W[i % 3], out=outs[i % 3], check_finite=False)
@@ -289,6 +295,7 @@ def _merge_measure(q, syn, device, reps=10):
         torch.cuda.synchronize()
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(reps)]
+        _hold_gpu(SHORT_HOLD_MS)
         for i in range(reps):
             evs[i][0].record()
             fn(i)
@@ -322,6 +329,7 @@ def _adam8_measure(q, syn, device, reps=10):
         q.qlora_adamw8_step(p, g, st, 2e-4, weight_decay=0.01, p_bf16=pb)
     torch.cuda.synchronize()
     b, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _hold_gpu(SHORT_HOLD_MS)
     b.record()
     for _ in range(reps):
         q.qlora_adamw8_step(p, g, st, 2e-4, weight_decay=0.01, p_bf16=pb)
@@ -359,6 +367,7 @@ def _format_measure(q, device, reps=10):
             fn()
             torch.cuda.synchronize()
             b, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            _hold_gpu(SHORT_HOLD_MS)
             b.record()
             for _ in range(reps):
                 fn()
@@ -399,6 +408,7 @@ def _gemv_sweep(q, syn, device, reps=10):
             evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                    for _ in range(reps)]
             torch.cuda.synchronize()
+            _hold_gpu(SHORT_HOLD_MS)
             for i in range(reps):
                 q.qlora_linear_forward(X, copies[i % 3], A, B, lin.gamma, Y=Y, ws=ws,
                                        events=evs[i])
