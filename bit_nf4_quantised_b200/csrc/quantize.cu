@@ -226,8 +226,12 @@ template <typename Tin>
 __global__ void __launch_bounds__(kThreads, 2)
 quantize_many_kernel(const __grid_constant__ QuantBatch bt, int* __restrict__ nonfinite_flag,
                      Nf4IndexLut lut) {
-    int j = 0;
-    while (j + 1 < bt.n && bt.first[j + 1] <= int64_t(blockIdx.x)) ++j;
+    // this CTA's job: the last whose first group is at or below blockIdx.x
+    // (first[] rises strictly: jobs without whole groups are left out), one
+    // lane per job, counted by a ballot
+    const int lane = threadIdx.x & 31;
+    const bool le = lane < bt.n && bt.first[lane] <= int64_t(blockIdx.x);
+    const int j = __popc(__ballot_sync(0xffffffffu, le)) - 1;
     const QuantizeJob& q = bt.job[j];
     const int64_t nblocks = (q.numel + QLORA_BLOCK - 1) / QLORA_BLOCK;
     quantize_group<true, Tin>(static_cast<const Tin*>(q.W), q.numel, nblocks, q.packed, q.scale_codes,

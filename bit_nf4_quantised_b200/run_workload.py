@@ -2,13 +2,14 @@
 profilers such as ncu, which want a short process around the kernels).
 
   python -m bit_nf4_quantised_b200.run_workload --workload NAME [--calls 2]
-         [--forward-only | --merge | --quantize]
+         [--forward-only | --merge | --quantize | --quantize-many N]
 
 NAME is a key of synthetic.WORKLOADS; for a multi-layer workload only its
 first layer runs.  Each call is one forward (and, unless --forward-only, one
 backward) of that layer on cuda:0; with --merge, one merge of the layer's
 weight and adapter into a bf16 weight instead; with --quantize, one
-quantisation of the layer's fp32 weight.
+quantisation of the layer's fp32 weight; with --quantize-many N, one
+qlora_quantize_many call over N separate copies of that weight.
 """
 from __future__ import annotations
 
@@ -28,6 +29,7 @@ def main() -> None:
     ap.add_argument("--forward-only", action="store_true")
     ap.add_argument("--merge", action="store_true")
     ap.add_argument("--quantize", action="store_true")
+    ap.add_argument("--quantize-many", type=int, default=0, metavar="N")
     args = ap.parse_args()
     lin = syn.WORKLOADS[args.workload].layers[0]
     if args.quantize:
@@ -37,6 +39,16 @@ def main() -> None:
             q.qlora_quantize(W)
         torch.cuda.synchronize()
         print(f"{args.workload}: {args.calls} quantise call(s)")
+        return
+    if args.quantize_many > 0:
+        rng = np.random.default_rng(lin.seed)
+        W = torch.from_numpy(syn.make_weight(lin, rng)).cuda()
+        jobs = [(W.clone(), q.empty_nf4(lin.N, lin.K)) for _ in range(args.quantize_many)]
+        del W
+        for _ in range(args.calls):
+            q.qlora_quantize_many(jobs)
+        torch.cuda.synchronize()
+        print(f"{args.workload}: {args.calls} qlora_quantize_many call(s) of {args.quantize_many}")
         return
     d = syn.make_layer(lin, with_grad=not (args.forward_only or args.merge))
     w = q.qlora_quantize(torch.from_numpy(d["W"]).cuda())
