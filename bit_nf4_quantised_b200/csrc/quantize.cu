@@ -137,14 +137,16 @@ __device__ __forceinline__ void quantize_group(const Tin* __restrict__ W, int64_
         const int64_t e0 = gbase + int64_t(blk) * QLORA_BLOCK + sub * kPerLane;
         v[step] = kFull ? load8(W, e0) : load8_tail(W, e0, numel);
     }
-    // table entry e for lane l at byte 256 e + 8 l: thread t writes entry
-    // t / 8 for lanes 4 (t mod 8) .. + 3
-    {
-        const int e = tid >> 3, l0 = (tid & 7) * 4;
-        const uint32_t a = smem_u32(smem) + e * 256 + l0 * 8;
+    // table entry e for lane l at byte 256 e + 8 l, written as 16-byte
+    // chunks c = 16 e + l / 2 (two lanes each) by thread c mod 512: a warp's
+    // stores cover 512 contiguous bytes, free of bank conflicts
+    static_assert(kLutBytes / 16 == 2 * kThreads, "two chunks per thread");
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const int c = tid + k * kThreads, e = c >> 4;
         const uint32_t t = lut.thr[e], b = lut.base[e];
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %1, %2};" ::"r"(a), "r"(t), "r"(b) : "memory");
-        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %1, %2};" ::"r"(a + 16), "r"(t), "r"(b) : "memory");
+        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %1, %2};" ::"r"(smem_u32(smem) + c * 16), "r"(t), "r"(b)
+                     : "memory");
     }
     __syncthreads();
     const uint32_t lane_lut = smem_u32(smem) + lane * 8 - (0x1000u << 8);
